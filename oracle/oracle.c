@@ -1,0 +1,211 @@
+/*
+ * Float64 CPU oracle for linear attention with the feature map phi(x) = elu(x) + 1.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load this
+ * file: only the tests, the smoke check and the CPU-baseline leg of the benchmark use it.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (page "Efficient Transformers: Linear Attention and Flash Attention",
+ * section "Linear attention: reordering the matmuls, not shrinking them", the
+ * kernelised attention formula):
+ *
+ *     out_i = phi(q_i) . sum_j phi(k_j) v_j^T  /  phi(q_i) . sum_j phi(k_j)
+ *
+ * non-causal: j runs over all tokens; causal: j <= i, the diagonal included, as in the
+ * same page's section "The recurrent view: attention as an RNN", where the state after
+ * token t already holds token t and the output at t reads that state:
+ *
+ *     S_t = S_{t-1} + phi(k_t) v_t^T,   z_t = z_{t-1} + phi(k_t),
+ *     out_t = phi(q_t) S_t / phi(q_t) . z_t.
+ *
+ * The oracle follows those two statements literally: the non-causal mode forms S and z
+ * over all tokens in token order, then reads every row out; the causal mode runs the
+ * token recurrence, one token at a time.  No chunking, no blocking, no reordering.
+ *
+ * Readings where the pages are silent:
+ *   - elu has alpha = 1 (the page writes elu(x)+1 with no parameter);
+ *   - no 1/sqrt(d) scale inside the method (the formula has none; inputs may be
+ *     pre-scaled by the caller);
+ *   - no epsilon in the denominator (phi > 0 keeps it positive, page's answer A4);
+ *   - the feature dimension D equals d and the value dimension equals d.
+ *
+ * Layouts: q, k, v, out are row-major [B][H][n][d]; S is [..][D][d] with row r the
+ * feature index and column c the value index; z is [..][D].
+ *
+ * PHI_IDENTITY selects phi(x) = x, which the page's worked example ("Worked example:
+ * the reassociation trick, by hand") uses on non-negative inputs.  It exists only so
+ * that example can pin this code; it is not part of the method.
+ *
+ * Compile-time ORACLE_PLANT=1..5 plants one deliberate mistake each.  Only the test
+ * that shows the pins catch such mistakes builds those variants.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef ORACLE_PLANT
+#define ORACLE_PLANT 0
+#endif
+
+enum { PHI_ELU1 = 0, PHI_IDENTITY = 1 };
+
+/* phi(x) = elu(x) + 1: x + 1 for x > 0 and exp(x) for x <= 0 (alpha = 1). */
+double oracle_phi(double x, int phi_kind)
+{
+    if (phi_kind == PHI_IDENTITY) return x;
+#if ORACLE_PLANT == 4
+    return x > 0.0 ? x : exp(x); /* planted: dropped the +1 on the positive branch */
+#else
+    return x > 0.0 ? x + 1.0 : exp(x);
+#endif
+}
+
+/* Rank-1 update of one head's state by one token: S += phi(k) v^T, z += phi(k). */
+static void state_add_token(double *S, double *z, const double *k, const double *v,
+                            int64_t d, int phi_kind)
+{
+    for (int64_t r = 0; r < d; ++r) {
+        double pk = oracle_phi(k[r], phi_kind);
+        for (int64_t c = 0; c < d; ++c) {
+#if ORACLE_PLANT == 2
+            S[c * d + r] += pk * v[c]; /* planted: transposed state */
+#else
+            S[r * d + c] += pk * v[c];
+#endif
+        }
+        z[r] += pk;
+    }
+}
+
+/* out = phi(q) S / (phi(q) . z) for one token and one head. */
+static void readout_token(const double *S, const double *z, const double *q, double *out,
+                          int64_t d, int phi_kind, double *pq_scratch)
+{
+    double den = 0.0;
+    for (int64_t r = 0; r < d; ++r) {
+        pq_scratch[r] = oracle_phi(q[r], phi_kind);
+#if ORACLE_PLANT != 3
+        den += pq_scratch[r] * z[r];
+#endif
+    }
+#if ORACLE_PLANT == 3
+    den = 1.0; /* planted: normaliser dropped */
+#endif
+    for (int64_t c = 0; c < d; ++c) {
+        double num = 0.0;
+        for (int64_t r = 0; r < d; ++r) num += pq_scratch[r] * S[r * d + c];
+        out[c] = num / den;
+    }
+}
+
+/* Forward pass over B*H independent heads; causal selects the token recurrence. */
+void oracle_forward_f64(const double *q, const double *k, const double *v, double *out,
+                        int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                        int phi_kind)
+{
+    const int64_t heads = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        double *S = (double *)calloc((size_t)(d * d), sizeof(double));
+        double *z = (double *)calloc((size_t)d, sizeof(double));
+        double *pq = (double *)malloc((size_t)d * sizeof(double));
+        const int64_t base = bh * n * d;
+        if (!causal) {
+            for (int64_t t = 0; t < n; ++t)
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+            for (int64_t t = 0; t < n; ++t)
+                readout_token(S, z, q + base + t * d, out + base + t * d, d, phi_kind, pq);
+        } else {
+            for (int64_t t = 0; t < n; ++t) {
+#if ORACLE_PLANT == 1
+                /* planted: diagonal excluded (read before adding token t) */
+                readout_token(S, z, q + base + t * d, out + base + t * d, d, phi_kind, pq);
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+#else
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+                readout_token(S, z, q + base + t * d, out + base + t * d, d, phi_kind, pq);
+#endif
+            }
+        }
+        free(S);
+        free(z);
+        free(pq);
+    }
+}
+
+/* Causal forward for selected rows only: runs the whole recurrence of each head but
+ * writes only the rows listed in rows[0..nrows) (ascending) to out[bh][nrows][d].
+ * Used for sampled checks at sizes where the full output would not fit in a test. */
+void oracle_forward_rows_f64(const double *q, const double *k, const double *v, double *out,
+                             int64_t heads, int64_t n, int64_t d, int causal,
+                             const int64_t *rows, int64_t nrows, int phi_kind)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        double *S = (double *)calloc((size_t)(d * d), sizeof(double));
+        double *z = (double *)calloc((size_t)d, sizeof(double));
+        double *pq = (double *)malloc((size_t)d * sizeof(double));
+        const int64_t base = bh * n * d;
+        if (!causal) {
+            for (int64_t t = 0; t < n; ++t)
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+            for (int64_t s = 0; s < nrows; ++s)
+                readout_token(S, z, q + base + rows[s] * d, out + (bh * nrows + s) * d, d,
+                              phi_kind, pq);
+        } else {
+            int64_t s = 0;
+            for (int64_t t = 0; t < n && s < nrows; ++t) {
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+                while (s < nrows && rows[s] == t) {
+                    readout_token(S, z, q + base + t * d, out + (bh * nrows + s) * d, d,
+                                  phi_kind, pq);
+                    ++s;
+                }
+            }
+        }
+        free(S);
+        free(z);
+        free(pq);
+    }
+}
+
+/* Final state of a causal pass: S = sum_j phi(k_j) v_j^T, z = sum_j phi(k_j), per head.
+ * This is the state the recurrent view carries after the last token. */
+void oracle_state_f64(const double *k, const double *v, double *S, double *z,
+                      int64_t heads, int64_t n, int64_t d, int phi_kind)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        double *Sh = S + bh * d * d;
+        double *zh = z + bh * d;
+        memset(Sh, 0, (size_t)(d * d) * sizeof(double));
+        memset(zh, 0, (size_t)d * sizeof(double));
+        for (int64_t t = 0; t < n; ++t)
+            state_add_token(Sh, zh, k + (bh * n + t) * d, v + (bh * n + t) * d, d, phi_kind);
+    }
+}
+
+/* One recurrent decode step for Bseq*H independent states, updated in place:
+ * S += phi(k) v^T, z += phi(k), then out = phi(q) S / phi(q) . z with the updated state. */
+void oracle_decode_step_f64(double *S, double *z, const double *q, const double *k,
+                            const double *v, double *out, int64_t Bseq, int64_t H, int64_t d,
+                            int phi_kind)
+{
+    const int64_t heads = Bseq * H;
+#pragma omp parallel for schedule(static)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        double *pq = (double *)malloc((size_t)d * sizeof(double));
+#if ORACLE_PLANT == 5
+        /* planted: output read from the state before the update */
+        readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, phi_kind, pq);
+        state_add_token(S + bh * d * d, z + bh * d, k + bh * d, v + bh * d, d, phi_kind);
+#else
+        state_add_token(S + bh * d * d, z + bh * d, k + bh * d, v + bh * d, d, phi_kind);
+        readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, phi_kind, pq);
+#endif
+        free(pq);
+    }
+}
+
+int oracle_plant(void) { return ORACLE_PLANT; }
