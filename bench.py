@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark: linear-attention forward tokens/s and achieved HBM GB/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-extras]
+
+Default workload (one step = one pass of the whole forward path, phi feature map, chunk
+aggregates, inter-chunk prefix and intra-chunk output, over one batch): the long-context
+causal forward, B=1, H=32, n=131072, d=D=128, bf16 I/O, fp32 state, inputs N(0,1)/sqrt(d)
+seed 3.  Inputs (3.2 GB) and output (1.1 GB) are larger than the 126 MB L2, so no flush
+is needed between timed steps.
+
+Multi-GPU (torchrun, one process per GPU): heads are independent, so each rank runs its
+own batch element of the workload (batch index = rank) with no data-path collective;
+value = all ranks' tokens / the max over ranks of the device time ("scaling": "weak").
+
+At N=1 the line also carries the decode step (256 x 32 states, d = 128, 512 steps), the
+batched 8x16x8192x64 forward (both modes) and the small latency cases under "extras", and
+the oracle's throughput on a bounded sample under "cpu_baseline".
+
+``--impl reference`` times the float64 CPU oracle (the reference implementation for
+this library) on the same workload and metric, each step a bounded sample, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_linattn_b200 import inputs  # noqa: E402
+
+METRIC = "linear-attention fwd tokens/sec and achieved HBM GB/s (fraction of B200 peak)"
+MAIN = "longctx_1x32x131072x128_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ accounting
+def forward_bytes(B, H, n, d, elem):
+    """Algorithmic bytes of one forward: read q, k, v and write out once (4 n d per head)."""
+    return 4 * B * H * n * d * elem
+
+
+def decode_bytes(heads, d, elem=2):
+    """Algorithmic bytes of one decode step: fp32 state (D*d + D) read and written once, plus
+    q, k, v read and out written (4 token vectors)."""
+    return heads * (2 * (d * d + d) * 4 + 4 * d * elem)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained",
+                                                     j["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sms:
+            return None
+        return {"sm_mhz": float(np.median(sms)), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ timing helpers
+def time_steps(fn, steps, warmup, world, clocks=None):
+    """W untimed steps, then K steps between barrier+synchronize; returns (ms per step
+    (max over ranks), per-step device ms list).  Events are on the launching stream."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    ev[0].record(stream)
+    for i in range(steps):
+        fn()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if clocks:
+        time.sleep(0.2)
+    barrier(world)
+    torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total = ev[0].elapsed_time(ev[steps])
+    return max_over_ranks(total / steps, world), per
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_sample(workload: str, target_s: float = 12.0):
+    """Times the float64 oracle on a bounded sample of the workload (host cores)."""
+    import oracle
+    w = inputs.WORKLOADS[workload]
+    cores = os.cpu_count() or 1
+    causal = True if True in w.causal else False
+    # calibrate on one head of 4096 tokens
+    q, k, v = inputs.forward_qkv(w.seed, 1, 1, min(w.n, 4096), w.d, w.scaled)
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, causal)
+    per_head_token = (time.perf_counter() - t0) / min(w.n, 4096)
+    heads = min(w.B * w.H, cores)
+    n_s = int(max(256, min(w.n, target_s / max(per_head_token, 1e-9))))
+    q, k, v = inputs.forward_qkv(w.seed, 1, heads, n_s, w.d, w.scaled)
+    if "bf16" in w.dtypes:
+        q, k, v = (inputs.round_bf16(x) for x in (q, k, v))
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, causal)
+    dt = time.perf_counter() - t0
+    # tokens in the workload's unit: a token carries all H heads of its batch element
+    tokens = heads * n_s / w.H
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+            "threads": int(os.environ.get("OMP_NUM_THREADS", cores)),
+            "sample": f"{heads} heads x {n_s} tokens of the {workload} workload "
+                      f"({'causal' if causal else 'non-causal'}), float64, {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(args.workload, target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+        if i >= args.warmup:
+            vals.append(r["value"])
+    v = float(np.median(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": w.tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+                       "causal": True in w.causal, "global_batch": w.B, "seq_len": w.n,
+                       "parallelism": "host cores (OpenMP over heads)"},
+            "cpu_baseline": dict(r, value=v),
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def main_forward(args, world, rank, local):
+    import torch
+
+    import linear_attention_linattn_b200 as la
+    w = inputs.WORKLOADS[args.workload]
+    causal = True in w.causal
+    dtype = "bf16" if "bf16" in w.dtypes else "f32"
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    elem = 2 if dtype == "bf16" else 4
+    # this rank's batch element of the workload: b = rank (weak scaling over ranks)
+    q, k, v = inputs.forward_qkv(w.seed, w.B * world, w.H, w.n, w.d, w.scaled,
+                                 heads=[(rank * w.B + b, h) for b in range(w.B)
+                                        for h in range(w.H)])
+    shape = (w.B, w.H, w.n, w.d)
+    qh = torch.from_numpy(q.reshape(shape)).to(tdt).pin_memory()
+    kh = torch.from_numpy(k.reshape(shape)).to(tdt).pin_memory()
+    vh = torch.from_numpy(v.reshape(shape)).to(tdt).pin_memory()
+    del q, k, v
+    qd, kd, vd = qh.cuda(), kh.cuda(), vh.cuda()
+    out = torch.empty_like(qd)
+
+    def step():
+        la.forward(qd, kd, vd, causal, out=out)
+
+    clocks = ClockSampler(local)
+    l0 = la.linattn_launch_count()
+    ms, per = time_steps(step, args.steps, args.warmup, world, clocks=clocks)
+    launches = (la.linattn_launch_count() - l0) // (args.steps + args.warmup) * args.steps
+    clk = clocks.stop()
+    assert la.device_error() == la.LINATTN_OK
+
+    tokens_rank = w.B * w.n
+    value = tokens_rank * world / (ms * 1e-3)
+    pk = peaks()
+    alg = forward_bytes(w.B, w.H, w.n, w.d, elem)
+    kernel_ms = float(np.mean(per))
+    achieved = alg / (kernel_ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host -> device, forward, device -> host
+    outh = torch.empty_like(qh).pin_memory()
+
+    def e2e_step():
+        a, b_, c = (x.to("cuda", non_blocking=True) for x in (qh, kh, vh))
+        o = la.forward(a, b_, c, causal)
+        outh.copy_(o, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 3))
+    e2e_ms, _ = time_steps(e2e_step, e2e_steps, 1, world)
+    e2e = {"value": tokens_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": 3 * qh.numel() * elem, "d2h_bytes_per_step": outh.numel() * elem}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+        "data": "synthetic (seeded N(0,1)/sqrt(d), see DESIGN.md input recipe)",
+        "config": {"workload": args.workload, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+                   "causal": causal, "global_batch": w.B * world, "seq_len": w.n,
+                   "parallelism": f"dp{world} (independent heads, no collective)",
+                   "l2": "inputs larger than L2 (no flush needed)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "peak_source": pk["source"], "algorithmic_bytes": alg,
+                     "kernel": "whole forward pass (all launches of one step)",
+                     "kernel_ms": kernel_ms},
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    return line
+
+
+def extras(args):
+    """Other workloads at N=1: decode, batched forward, small latency cases."""
+    import torch
+
+    import linear_attention_linattn_b200 as la
+    from linear_attention_linattn_b200 import workloads
+    pk = peaks()
+    res = {}
+    # decode: 512 steps of 256 x 32 states, d = 128
+    S, z, qs, ks, vs = workloads.decode_inputs("decode_256x32x128")
+    T = qs.shape[0]
+    out = torch.empty_like(qs[0])
+    for t in range(3):
+        la.decode_step(S, z, qs[t], ks[t], vs[t], out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(T):
+        la.decode_step(S, z, qs[t], ks[t], vs[t], out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / T
+    b = decode_bytes(256 * 32, 128)
+    res["decode_256x32x128"] = {"ms_per_step": ms, "tokens_per_s": 256 / (ms * 1e-3),
+                                "head_states_per_s": 256 * 32 / (ms * 1e-3),
+                                "gbs": b / (ms * 1e-3) / 1e9,
+                                "frac_hbm": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                "algorithmic_bytes_per_step": b, "steps": T}
+    del S, z, qs, ks, vs
+    torch.cuda.empty_cache()
+    # batched forward, both modes
+    name = "batched_8x16x8192x64_bf16"
+    w = inputs.WORKLOADS[name]
+    q, k, v = workloads.forward_inputs(name, "bf16")
+    o = torch.empty_like(q)
+    for causal in (False, True):
+        ms, _ = time_steps(lambda: la.forward(q, k, v, causal, out=o), 20, 3, 1)
+        alg = forward_bytes(w.B, w.H, w.n, w.d, 2)
+        res[f"{name}_{'causal' if causal else 'noncausal'}"] = {
+            "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
+            "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    del q, k, v, o
+    # latency cases
+    for name, dtypes in (("noncausal_1x1x512x64_f32", ("f32",)),
+                         ("causal_1x1x4096x64", ("f32", "bf16"))):
+        w = inputs.WORKLOADS[name]
+        for dt in dtypes:
+            q, k, v = workloads.forward_inputs(name, dt)
+            o = torch.empty_like(q)
+            causal = True in w.causal
+            ms, _ = time_steps(lambda: la.forward(q, k, v, causal, out=o), 50, 5, 1)
+            res[f"{name}_{dt}"] = {"us": ms * 1e3, "tokens_per_s": w.B * w.n / (ms * 1e-3)}
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=MAIN, choices=[k for k, w in inputs.WORKLOADS.items()
+                                                         if w.kind == "forward"])
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+
+    import torch
+    torch.cuda.set_device(local)
+    line = main_forward(args, world, rank, local)
+    if world == 1 and rank == 0:
+        if not args.no_extras:
+            line["extras"] = extras(args)
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(args.workload)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,133 @@
+/*
+ * linattn: linear attention with the feature map phi(x) = elu(x) + 1 on NVIDIA B200
+ * (sm_100a).  C ABI; every entry point is asynchronous on the caller's CUDA stream.
+ *
+ * The method (page "Efficient Transformers: Linear Attention and Flash Attention",
+ * section "Linear attention: reordering the matmuls, not shrinking them", the kernelised
+ * attention formula):
+ *
+ *     out_i = phi(q_i) S / (phi(q_i) . z),   S = sum_j phi(k_j) v_j^T (D x d),
+ *                                            z = sum_j phi(k_j)       (D)
+ *
+ * computed in the associativity-reordered order, so the n x n matrix is never formed.
+ * Causal attention sums over j <= i, the current token included, as in the same page's
+ * section "The recurrent view: attention as an RNN" (S_t = S_{t-1} + phi(k_t) v_t^T and
+ * the output at t reads S_t).  phi(x) = x + 1 for x > 0 and exp(x) for x <= 0.
+ * There is no 1/sqrt(d) scale and no epsilon inside the method: callers pre-scale
+ * their inputs if they want one, and phi > 0 keeps the denominator positive.
+ *
+ * Dimensions: the feature dimension D equals the head dimension d (phi is elementwise)
+ * and the value dimension equals d.  Supported d: 64 and 128.
+ *
+ * Memory: every pointer is caller-owned DEVICE memory, 16-byte aligned.  The library
+ * keeps no pointer after a call returns.  Outputs must not alias inputs.  Temporary
+ * workspace is taken from a library-owned stream-ordered pool on the caller's stream
+ * and released on the same stream.
+ *
+ * Errors: every argument is checked before anything is launched; a failed check
+ * returns LINATTN_ERR_INVALID_ARG or LINATTN_ERR_UNSUPPORTED and launches nothing.
+ * A CUDA error at launch returns LINATTN_ERR_CUDA.  Kernels never trap: a bounded wait
+ * that gives up sets a per-device error flag, which linattn_device_error() reports as
+ * LINATTN_ERR_TIMEOUT after synchronising the stream.
+ */
+#ifndef LINATTN_H
+#define LINATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's stream handle type (cudaStream_t is a typedef of this pointer). */
+struct CUstream_st;
+typedef struct CUstream_st *linattn_stream_t;
+
+typedef enum {
+    LINATTN_OK = 0,
+    LINATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size <= 0, bad flag or dtype */
+    LINATTN_ERR_UNSUPPORTED = 2, /* d outside {64, 128} */
+    LINATTN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    LINATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait gave up (see linattn_device_error) */
+} linattn_status;
+
+typedef enum {
+    LINATTN_F32 = 0, /* float32 I/O: computed in fp32 on the CUDA cores */
+    LINATTN_BF16 = 1 /* bfloat16 I/O: bf16 tensor-core products, fp32 accumulation and state */
+} linattn_dtype;
+
+/*
+ * Forward pass over B*H independent heads.
+ *   q, k, v : [B][H][n][d] row-major, element type `dtype`, read only.
+ *   out     : [B][H][n][d] row-major, element type `dtype`, written.
+ *   causal  : 0 = every query sees every key (the formula above);
+ *             1 = query i sees keys j <= i (the recurrent view's running state).
+ * Any n >= 1 is accepted.  Accumulation is fp32; the output is rounded once to `dtype`
+ * (bf16: round to nearest even).  The causal mode runs as chunked prefix sums of (S, z).
+ * Returns LINATTN_OK after enqueuing the kernels on `stream`.
+ */
+linattn_status linattn_forward(const void *q, const void *k, const void *v, void *out,
+                               int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                               linattn_dtype dtype, linattn_stream_t stream);
+
+/*
+ * One recurrent decode step for Bseq*H independent states (the recurrent view):
+ *   S' = S + phi(k) v^T,  z' = z + phi(k),  out = phi(q) S' / (phi(q) . z').
+ * The output reads the UPDATED state (the current token is included).
+ *   state_S : [Bseq][H][D][d] float32, row r = feature index, column c = value index;
+ *             read and written in place.
+ *   state_z : [Bseq][H][D] float32, read and written in place.
+ *   q, k, v : [Bseq][H][d] bfloat16, read only.   out : [Bseq][H][d] bfloat16, written.
+ * The state is the caller's: keeping the two buffers is all a pause/resume needs.
+ */
+linattn_status linattn_decode_step(float *state_S, float *state_z, const void *q,
+                                   const void *k, const void *v, void *out, int64_t Bseq,
+                                   int64_t H, int64_t d, linattn_stream_t stream);
+
+/*
+ * The state a causal pass leaves after its last token, per head:
+ *   state_S[b][h] = sum_j phi(k_j) v_j^T  ([D][d] float32),
+ *   state_z[b][h] = sum_j phi(k_j)        ([D] float32),
+ * with k, v : [B][H][n][d] of type `dtype`.  This is the prefill that hands a sequence
+ * over to linattn_decode_step (the recurrent view's S_n, z_n).  Overwrites both outputs.
+ */
+linattn_status linattn_forward_state(const void *k, const void *v, float *state_S,
+                                     float *state_z, int64_t B, int64_t H, int64_t n,
+                                     int64_t d, linattn_dtype dtype, linattn_stream_t stream);
+
+/*
+ * linattn_forward with a chosen segment length: the number of tokens one work item of
+ * the chunked causal pass covers (a multiple of the chunk size; 0 picks the default).
+ * The result does not depend on it beyond rounding order; tests use it to move the
+ * segment boundaries.  Other arguments as in linattn_forward.
+ */
+linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, void *out,
+                                  int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                  linattn_dtype dtype, int64_t segment_len,
+                                  linattn_stream_t stream);
+
+/* Bytes of one head's state, D*d*4 + D*4 (fp32 S and z), independent of n
+ * (page "Linear Attention > Memory Efficiency": 16,640 bytes at d = D = 64). */
+size_t linattn_state_bytes(int64_t d);
+
+/* Static text for a status code. */
+const char *linattn_status_string(linattn_status status);
+
+/* Synchronises `stream`, then reports and clears the current device's kernel error flag:
+ * LINATTN_ERR_TIMEOUT if a bounded wait gave up since the last call, else LINATTN_OK
+ * (or LINATTN_ERR_CUDA if synchronising failed). */
+linattn_status linattn_device_error(linattn_stream_t stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int linattn_version(void);
+
+/* Number of kernels (and device memsets) this library has enqueued in this process, on
+ * every device.  Benchmarks read it before and after a timed region. */
+uint64_t linattn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LINATTN_H */

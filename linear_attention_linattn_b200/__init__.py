@@ -1,0 +1,173 @@
+"""linattn for B200: linear attention (phi = elu + 1) as hand-written sm_100a CUDA kernels.
+
+The compute path is the C-ABI library ``liblinattn.so`` built from ``csrc/`` (declared in
+``include/linattn.h``).  This module only marshals arguments: it passes device pointers,
+sizes and the current CUDA stream of PyTorch tensors to the C entry points of the same
+names.  There is no fallback: if the library is missing or fails to load, every call
+raises.
+
+Raw C entry points (pointers as ints):
+    linattn_forward, linattn_forward_ex, linattn_forward_state, linattn_decode_step,
+    linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
+    linattn_launch_count
+
+Tensor helpers: ``forward``, ``forward_state``, ``decode_step``, ``device_error``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblinattn.so")
+
+LINATTN_OK = 0
+LINATTN_ERR_INVALID_ARG = 1
+LINATTN_ERR_UNSUPPORTED = 2
+LINATTN_ERR_CUDA = 3
+LINATTN_ERR_TIMEOUT = 4
+LINATTN_F32 = 0
+LINATTN_BF16 = 1
+
+# Every symbol include/linattn.h declares, with its ctypes signature.
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+SIGNATURES = {
+    "linattn_forward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int,
+                                       ctypes.c_int, _vp]),
+    "linattn_forward_ex": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                          ctypes.c_int, ctypes.c_int, _i64, _vp]),
+    "linattn_forward_state": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                             ctypes.c_int, _vp]),
+    "linattn_decode_step": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "linattn_state_bytes": (ctypes.c_size_t, [_i64]),
+    "linattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "linattn_device_error": (ctypes.c_int, [_vp]),
+    "linattn_version": (ctypes.c_int, []),
+    "linattn_launch_count": (ctypes.c_uint64, []),
+}
+
+_lib = None
+
+
+class LinattnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Loads liblinattn.so (raises if it is missing: build it with
+    ``python -m linear_attention_linattn_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"liblinattn.so not found at {p}; build it with "
+                           "`python -m linear_attention_linattn_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().linattn_status_string(int(status)).decode()
+
+
+def __getattr__(name):  # raw C entry points: linear_attention_linattn_b200.linattn_forward(...)
+    if name in SIGNATURES:
+        return getattr(load_library(), name)
+    raise AttributeError(name)
+
+
+# ------------------------------------------------------------------ tensor helpers
+def _stream_ptr(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return LINATTN_F32
+    if t.dtype == torch.bfloat16:
+        return LINATTN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _check(status: int, what: str):
+    if status != LINATTN_OK:
+        raise LinattnError(status, what)
+
+
+def _dev(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def forward(q, k, v, causal: bool, out=None, segment_len: int = 0, stream=None):
+    """q, k, v: [B, H, n, d] CUDA tensors (float32 or bfloat16).  Returns out (same shape)."""
+    import torch
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, nm)
+    if not (q.shape == k.shape == v.shape and q.dim() == 4 and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share one [B, H, n, d] shape and dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out")
+    B, H, n, d = q.shape
+    lib = load_library()
+    st = lib.linattn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                B, H, n, d, int(bool(causal)), _dtype_code(q), int(segment_len),
+                                _stream_ptr(stream))
+    _check(st, "linattn_forward")
+    return out
+
+
+def forward_state(k, v, S=None, z=None, stream=None):
+    """Final causal state of k, v [B, H, n, d]: S [B, H, d, d] and z [B, H, d] (float32)."""
+    import torch
+    _dev(k, "k")
+    _dev(v, "v")
+    B, H, n, d = k.shape
+    if S is None:
+        S = torch.empty((B, H, d, d), dtype=torch.float32, device=k.device)
+    if z is None:
+        z = torch.empty((B, H, d), dtype=torch.float32, device=k.device)
+    lib = load_library()
+    st = lib.linattn_forward_state(k.data_ptr(), v.data_ptr(), S.data_ptr(), z.data_ptr(),
+                                   B, H, n, d, _dtype_code(k), _stream_ptr(stream))
+    _check(st, "linattn_forward_state")
+    return S, z
+
+
+def decode_step(S, z, q, k, v, out=None, stream=None):
+    """One step in place on S [Bseq, H, d, d], z [Bseq, H, d] (float32) with bf16 q, k, v
+    [Bseq, H, d].  Returns out [Bseq, H, d] (bfloat16)."""
+    import torch
+    for t, nm in ((S, "S"), (z, "z"), (q, "q"), (k, "k"), (v, "v")):
+        _dev(t, nm)
+    if S.dtype != torch.float32 or z.dtype != torch.float32:
+        raise TypeError("the decode state is float32")
+    if not (q.dtype == k.dtype == v.dtype == torch.bfloat16):
+        raise TypeError("decode q, k, v are bfloat16")
+    Bseq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    lib = load_library()
+    st = lib.linattn_decode_step(S.data_ptr(), z.data_ptr(), q.data_ptr(), k.data_ptr(),
+                                 v.data_ptr(), out.data_ptr(), Bseq, H, d, _stream_ptr(stream))
+    _check(st, "linattn_decode_step")
+    return out
+
+
+def device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the kernels' error status."""
+    return load_library().linattn_device_error(_stream_ptr(stream))

@@ -1,0 +1,227 @@
+// C ABI of linattn (see include/linattn.h): argument checks, workspace, dispatch.
+//
+// Dispatch is by I/O type only: float32 I/O runs the CUDA-core kernels (simt_forward.cu),
+// bfloat16 I/O runs the tensor-core kernels (tc_forward.cu).  There is no host fallback:
+// every step of the pass runs in this library's kernels on the caller's stream.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "linattn.h"
+
+namespace linattn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t init_err = cudaSuccess;
+  int *err_word = nullptr;     // kernels' error word (device memory)
+  cudaMemPool_t pool = nullptr;  // stream-ordered workspace pool
+};
+DeviceState g_dev[kMaxDevices];
+
+// Per-device set-up on first use: the kernels' error word and a workspace pool that keeps
+// its memory between calls (so steady-state calls do not go back to the driver).
+cudaError_t device_state(DeviceState **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceState &s = g_dev[dev];
+  std::call_once(s.once, [&]() {
+    cudaError_t r = cudaMalloc(&s.err_word, sizeof(int));
+    if (r == cudaSuccess) r = cudaMemset(s.err_word, 0, sizeof(int));
+    if (r == cudaSuccess) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.handleTypes = cudaMemHandleTypeNone;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      r = cudaMemPoolCreate(&s.pool, &props);
+    }
+    if (r == cudaSuccess) {
+      uint64_t keep = ~0ull;
+      r = cudaMemPoolSetAttribute(s.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    if (r == cudaSuccess) r = cudaDeviceSynchronize();
+    s.init_err = r;
+  });
+  if (s.init_err != cudaSuccess) return s.init_err;
+  *out = &s;
+  return cudaSuccess;
+}
+
+// Stream-ordered scratch: allocated on `st` before the kernels, released on `st` after.
+struct Workspace {
+  void *ptr = nullptr;
+  cudaStream_t st = nullptr;
+  ~Workspace() {
+    if (ptr) cudaFreeAsync(ptr, st);
+  }
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+linattn_status to_status(cudaError_t e) { return e == cudaSuccess ? LINATTN_OK : LINATTN_ERR_CUDA; }
+
+// Checks shared by the forward entry points.  Limits keep every grid and TMA coordinate
+// inside 32 bits: n < 2^31, B*H < 2^24, total elements < 2^40.
+linattn_status check_forward_shape(int64_t B, int64_t H, int64_t n, int64_t d) {
+  if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return LINATTN_ERR_INVALID_ARG;
+  if (B > (1 << 24) || H > (1 << 24) || n >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
+  const int64_t heads = B * H;
+  if (heads > (1 << 24)) return LINATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
+  if (heads * n > (int64_t(1) << 40) / d) return LINATTN_ERR_INVALID_ARG;
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  if (nchunks * heads >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
+  return LINATTN_OK;
+}
+
+linattn_status forward_simt(const void *q, const void *k, const void *v, void *out,
+                            int64_t heads, int64_t n, int d, int causal, int is_bf16,
+                            DeviceState *ds, cudaStream_t st) {
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  const int64_t per = (int64_t)d * d + d;
+  // causal: one state per chunk; non-causal: chunk states plus one total per head
+  const size_t bytes = (size_t)(heads * nchunks * per + (causal ? 0 : heads * per)) * 4;
+  Workspace ws;
+  ws.st = st;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws.ptr, bytes, ds->pool, st);
+  if (e != cudaSuccess) return LINATTN_ERR_CUDA;
+  float *w = static_cast<float *>(ws.ptr);
+  e = launch_simt_chunk_state(k, v, w, heads, n, d, is_bf16, st);
+  if (e != cudaSuccess) return LINATTN_ERR_CUDA;
+  if (causal) {
+    e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, nullptr, st);
+    if (e != cudaSuccess) return LINATTN_ERR_CUDA;
+    e = launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
+                              nchunks * per, heads, n, d, 1, is_bf16, st);
+  } else {
+    float *tot = w + heads * nchunks * per;
+    float *tot_z = tot + heads * (int64_t)d * d;
+    e = launch_scan_states(w, heads, nchunks, d, 1, tot, tot_z, st);
+    if (e != cudaSuccess) return LINATTN_ERR_CUDA;
+    e = launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, (int64_t)d * d, 0, d, heads, n, d, 0,
+                              is_bf16, st);
+  }
+  return to_status(e);
+}
+
+}  // namespace
+}  // namespace linattn
+
+using namespace linattn;
+
+extern "C" {
+
+linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, void *out,
+                                  int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                  linattn_dtype dtype, int64_t segment_len,
+                                  linattn_stream_t stream) {
+  if (!q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return LINATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  if (segment_len < 0) return LINATTN_ERR_INVALID_ARG;
+  linattn_status s = check_forward_shape(B, H, n, d);
+  if (s != LINATTN_OK) return s;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, dtype == LINATTN_BF16, ds, st);
+}
+
+linattn_status linattn_forward(const void *q, const void *k, const void *v, void *out, int64_t B,
+                               int64_t H, int64_t n, int64_t d, int causal, linattn_dtype dtype,
+                               linattn_stream_t stream) {
+  return linattn_forward_ex(q, k, v, out, B, H, n, d, causal, dtype, 0, stream);
+}
+
+linattn_status linattn_forward_state(const void *k, const void *v, float *state_S,
+                                     float *state_z, int64_t B, int64_t H, int64_t n, int64_t d,
+                                     linattn_dtype dtype, linattn_stream_t stream) {
+  if (!k || !v || !state_S || !state_z) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(state_S) || !aligned16(state_z))
+    return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  linattn_status s = check_forward_shape(B, H, n, d);
+  if (s != LINATTN_OK) return s;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t heads = B * H;
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  const int64_t per = d * d + d;
+  Workspace ws;
+  ws.st = st;
+  if (cudaMallocFromPoolAsync(&ws.ptr, (size_t)(heads * nchunks * per) * 4, ds->pool, st) !=
+      cudaSuccess)
+    return LINATTN_ERR_CUDA;
+  float *w = static_cast<float *>(ws.ptr);
+  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, dtype == LINATTN_BF16, st);
+  if (e == cudaSuccess) e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, state_z, st);
+  return to_status(e);
+}
+
+linattn_status linattn_decode_step(float *state_S, float *state_z, const void *q, const void *k,
+                                   const void *v, void *out, int64_t Bseq, int64_t H, int64_t d,
+                                   linattn_stream_t stream) {
+  if (!state_S || !state_z || !q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(state_S) || !aligned16(state_z) || !aligned16(q) || !aligned16(k) ||
+      !aligned16(v) || !aligned16(out))
+    return LINATTN_ERR_INVALID_ARG;
+  if (Bseq <= 0 || H <= 0 || d <= 0) return LINATTN_ERR_INVALID_ARG;
+  if (Bseq > (1 << 24) || H > (1 << 24) || Bseq * H >= (int64_t(1) << 31))
+    return LINATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return to_status(launch_decode_step(state_S, state_z, q, k, v, out, Bseq * H, (int)d, st));
+}
+
+size_t linattn_state_bytes(int64_t d) {
+  if (d <= 0) return 0;
+  return (size_t)(d * d * 4 + d * 4);
+}
+
+const char *linattn_status_string(linattn_status status) {
+  switch (status) {
+    case LINATTN_OK: return "ok";
+    case LINATTN_ERR_INVALID_ARG: return "invalid argument";
+    case LINATTN_ERR_UNSUPPORTED: return "unsupported head dimension (d must be 64 or 128)";
+    case LINATTN_ERR_CUDA: return "CUDA error";
+    case LINATTN_ERR_TIMEOUT: return "a kernel's bounded wait gave up";
+  }
+  return "unknown status";
+}
+
+linattn_status linattn_device_error(linattn_stream_t stream) {
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LINATTN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ds->err_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LINATTN_ERR_CUDA;
+  if (word == 0) return LINATTN_OK;
+  if (cudaMemset(ds->err_word, 0, sizeof(int)) != cudaSuccess) return LINATTN_ERR_CUDA;
+  return LINATTN_ERR_TIMEOUT;
+}
+
+int linattn_version(void) { return 100; }
+
+uint64_t linattn_launch_count(void) { return linattn::launches_total(); }
+
+}  // extern "C"
+
+namespace linattn {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+uint64_t launches_total() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace linattn

@@ -1,0 +1,48 @@
+// Host-side declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace linattn {
+
+// Launch accounting for linattn_launch_count(): every launcher adds the kernels it enqueued.
+void count_launches(uint64_t n);
+uint64_t launches_total();
+
+// Tokens per chunk of the fp32 (CUDA-core) path.
+constexpr int kSimtChunk = 64;
+
+// ---- CUDA-core path (simt_forward.cu); is_bf16 selects bf16 I/O, else fp32 ------------
+// Chunk aggregates into ws[head][chunk][D*D + D] (S row-major, then z).
+cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int64_t heads,
+                                    int64_t n, int d, int is_bf16, cudaStream_t st);
+// In-place exclusive prefix over the chunks of each head (mode 0), or the per-head total
+// written to (S_out [heads][D][d], z_out [heads][D]) (mode 1).
+cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
+                               float *S_out, float *z_out, cudaStream_t st);
+// Outputs from per-chunk prefixes (causal) or the per-head totals (non-causal).
+cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, void *out,
+                                  const float *S, const float *z, int64_t S_chunk_stride,
+                                  int64_t S_head_stride, int64_t z_chunk_stride,
+                                  int64_t z_head_stride, int64_t heads, int64_t n, int d,
+                                  int causal, int is_bf16, cudaStream_t st);
+
+// ---- decode (decode.cu) ----------------------------------------------------------------
+cudaError_t launch_decode_step(float *S, float *z, const void *q, const void *k, const void *v,
+                               void *out, int64_t heads, int d, cudaStream_t st);
+
+// ---- bf16 I/O, tensor cores (tc_forward.cu) ----------------------------------------------
+// Chunk length of the tensor-core path.
+constexpr int kTcChunk = 64;
+// Default tokens per work item (segment) of the tensor-core path.
+int64_t tc_default_segment(int64_t heads, int64_t n, int d);
+// Workspace bytes the tensor-core forward needs.
+size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int causal);
+cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
+                       int64_t n, int d, int causal, int64_t seg, void *ws, cudaStream_t st);
+cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
+                             int64_t heads, int64_t n, int d, int64_t seg, void *ws,
+                             cudaStream_t st);
+
+}  // namespace linattn

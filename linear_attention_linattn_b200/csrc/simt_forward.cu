@@ -1,0 +1,339 @@
+// fp32-I/O forward pass on the CUDA cores (float32 FFMA end to end).
+//
+// Kernelised attention (page "Efficient Transformers: Linear Attention and Flash
+// Attention", section "Linear attention: reordering the matmuls, not shrinking them"),
+// causal as the chunked form of the running state of that page's section "The recurrent
+// view: attention as an RNN":
+//
+//   K1  chunk aggregates  S_c = phi(K_c)^T V_c,  z_c = sum_{j in c} phi(k_j)
+//   K2  exclusive prefix  S_<c = sum_{c' < c} S_c'   (or the per-head total)
+//   K3  chunk outputs     num_i = phi(q_i) S_<c + sum_{j <= i, j in c} (phi(q_i).phi(k_j)) v_j
+//                         den_i = phi(q_i).z_<c + sum_{j <= i, j in c}  phi(q_i).phi(k_j)
+//                         out_i = num_i / den_i
+//
+// Non-causal runs K1, K2 (total) and K3 with the total state and no in-chunk term.
+// This path serves float32 I/O, where the bf16 tensor-core products would not hold
+// a 1e-4 relative error.  Tokens beyond n in the last chunk are masked.
+#include "common.cuh"
+#include "internal.h"
+
+namespace linattn {
+namespace {
+
+constexpr int C = kSimtChunk;
+constexpr int kThreads = 256;
+
+// Four consecutive elements as floats.
+__device__ __forceinline__ float4 load4(const float *p) {
+  return *reinterpret_cast<const float4 *>(p);
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+}
+__device__ __forceinline__ void store1(float *p, float x) { *p = x; }
+__device__ __forceinline__ void store1(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+
+// Loads rows [t0, t0 + C) of one head into shared memory as floats (zero beyond n);
+// applies phi when `apply_phi`, and leaves masked rows at zero either way.
+template <int D, typename T>
+__device__ __forceinline__ void load_rows(float *dst, const T *src, int valid, bool apply_phi) {
+  for (int i = threadIdx.x; i < C * D / 4; i += kThreads) {
+    const int row = i / (D / 4);
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < valid) {
+      x = load4(src + 4 * i);
+      if (apply_phi) {
+        x.x = phi(x.x);
+        x.y = phi(x.y);
+        x.z = phi(x.z);
+        x.w = phi(x.w);
+      }
+    }
+    reinterpret_cast<float4 *>(dst)[i] = x;
+  }
+}
+
+// K1: one CTA per (chunk, head).  Each thread owns a (D/16) x (D/16) block of S_c with
+// rows r = tr + 16a and columns c = tc + 16b, so a warp reads consecutive columns.
+template <int D, typename T>
+__global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__restrict__ k,
+                                                                    const T *__restrict__ v,
+                                                                    float *__restrict__ ws,
+                                                                    int64_t n, int64_t nchunks) {
+  extern __shared__ float4 smem_f4[];
+  float *sK = reinterpret_cast<float *>(smem_f4);  // phi(K_c) [C][D]
+  float *sV = sK + C * D;                          // V_c [C][D]
+  const int64_t chunk = blockIdx.x % nchunks;
+  const int64_t head = blockIdx.x / nchunks;
+  const int64_t t0 = chunk * C;
+  const int valid = n - t0 < C ? static_cast<int>(n - t0) : C;
+  load_rows<D, T>(sK, k + (head * n + t0) * D, valid, true);
+  load_rows<D, T>(sV, v + (head * n + t0) * D, valid, false);
+  __syncthreads();
+
+  constexpr int R = D / 16;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  float acc[R][R];
+#pragma unroll
+  for (int a = 0; a < R; ++a)
+#pragma unroll
+    for (int b = 0; b < R; ++b) acc[a][b] = 0.f;
+  for (int t = 0; t < valid; ++t) {
+    float kr[R], vc[R];
+#pragma unroll
+    for (int a = 0; a < R; ++a) kr[a] = sK[t * D + tr + 16 * a];
+#pragma unroll
+    for (int b = 0; b < R; ++b) vc[b] = sV[t * D + tc + 16 * b];
+#pragma unroll
+    for (int a = 0; a < R; ++a)
+#pragma unroll
+      for (int b = 0; b < R; ++b) acc[a][b] = fmaf(kr[a], vc[b], acc[a][b]);
+  }
+  float *out = ws + (head * nchunks + chunk) * (int64_t)(D * D + D);
+#pragma unroll
+  for (int a = 0; a < R; ++a)
+#pragma unroll
+    for (int b = 0; b < R; ++b) out[(tr + 16 * a) * D + tc + 16 * b] = acc[a][b];
+  if (threadIdx.x < D) {
+    float zs = 0.f;
+    for (int t = 0; t < valid; ++t) zs += sK[t * D + threadIdx.x];
+    out[D * D + threadIdx.x] = zs;
+  }
+}
+
+// K2: per head, a sequential sweep over the segments for each state element.
+//   mode 0: ws[h][s] <- sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
+//   mode 1: S_out[h], z_out[h] <- sum_s ws[h][s] (the total)
+__global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws, int64_t nseg,
+                                                          int d, int mode,
+                                                          float *__restrict__ S_out,
+                                                          float *__restrict__ z_out) {
+  const int64_t per = (int64_t)d * d + d;
+  const int64_t blocks_per_head = (per + blockDim.x - 1) / blockDim.x;
+  const int64_t head = blockIdx.x / blocks_per_head;
+  const int64_t e = (blockIdx.x % blocks_per_head) * (int64_t)blockDim.x + threadIdx.x;
+  if (e >= per) return;
+  float *base = ws + head * nseg * per + e;
+  float run = 0.f;
+  if (mode == 0) {
+    for (int64_t s = 0; s < nseg; ++s) {
+      const float x = base[s * per];
+      base[s * per] = run;
+      run += x;
+    }
+  } else {
+    for (int64_t s = 0; s < nseg; ++s) run += base[s * per];
+    if (e < (int64_t)d * d)
+      S_out[head * d * d + e] = run;
+    else
+      z_out[head * d + (e - (int64_t)d * d)] = run;
+  }
+}
+
+// K3: one CTA per (chunk, head).  Thread (ti, tc) owns rows i = ti + 16a (a < 4) and
+// columns c = tc + 16b (b < D/16) of the chunk's output.
+template <int D, bool CAUSAL, typename T>
+__global__ void __launch_bounds__(kThreads) simt_chunk_out_kernel(
+    const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+    T *__restrict__ out, const float *__restrict__ S, const float *__restrict__ z,
+    int64_t S_chunk_stride, int64_t S_head_stride, int64_t z_chunk_stride,
+    int64_t z_head_stride, int64_t n, int64_t nchunks) {
+  extern __shared__ float4 smem_f4[];
+  float *sQ = reinterpret_cast<float *>(smem_f4);  // phi(Q_c) [C][D]
+  float *sS = sQ + C * D;                          // S_<c [D][D]
+  float *sz = sS + D * D;                          // z_<c [D]
+  float *sDen = sz + D;                            // [C]
+  float *sK = sDen + C;                            // phi(K_c)^T [D][C] (causal)
+  float *sV = sK + C * D;                          // V_c [C][D]        (causal)
+  float *sP = sV + C * D;                          // masked scores [C][C + 1] (causal)
+  const int64_t chunk = blockIdx.x % nchunks;
+  const int64_t head = blockIdx.x / nchunks;
+  const int64_t t0 = chunk * C;
+  const int valid = n - t0 < C ? static_cast<int>(n - t0) : C;
+  const int64_t row0 = (head * n + t0) * D;
+
+  load_rows<D, T>(sQ, q + row0, valid, true);
+  const float *Sg = S + head * S_head_stride + chunk * S_chunk_stride;
+  const float *zg = z + head * z_head_stride + chunk * z_chunk_stride;
+  for (int i = threadIdx.x; i < D * D / 4; i += kThreads)
+    reinterpret_cast<float4 *>(sS)[i] = reinterpret_cast<const float4 *>(Sg)[i];
+  if (threadIdx.x < D) sz[threadIdx.x] = zg[threadIdx.x];
+  if (CAUSAL) {
+    // phi(K_c) transposed, sK[r][j], so the score loop below reads consecutive j
+    for (int i = threadIdx.x; i < C * D / 4; i += kThreads) {
+      const int t = i % C, cg = i / C;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < valid) {
+        x = load4(k + row0 + (int64_t)t * D + 4 * cg);
+        x.x = phi(x.x);
+        x.y = phi(x.y);
+        x.z = phi(x.z);
+        x.w = phi(x.w);
+      }
+      sK[(4 * cg + 0) * C + t] = x.x;
+      sK[(4 * cg + 1) * C + t] = x.y;
+      sK[(4 * cg + 2) * C + t] = x.z;
+      sK[(4 * cg + 3) * C + t] = x.w;
+    }
+    load_rows<D, T>(sV, v + row0, valid, false);
+  }
+  __syncthreads();
+
+  if (CAUSAL) {
+    // scores P[i][j] = phi(q_i).phi(k_j) for j <= i, 0 above the diagonal
+    for (int e = threadIdx.x; e < C * C; e += kThreads) {
+      const int i = e / C, j = e % C;
+      float s = 0.f;
+      if (j <= i) {
+#pragma unroll 8
+        for (int r = 0; r < D; ++r) s = fmaf(sQ[i * D + r], sK[r * C + j], s);
+      }
+      sP[i * (C + 1) + j] = s;
+    }
+  }
+  // denominators: phi(q_i).z_<c + sum_{j<=i} P[i][j]
+  if (threadIdx.x < C) {
+    const int i = threadIdx.x;
+    float den = 0.f;
+    for (int r = 0; r < D; ++r) den = fmaf(sQ[i * D + r], sz[r], den);
+    sDen[i] = den;
+  }
+  __syncthreads();
+  if (CAUSAL && threadIdx.x < C) {
+    const int i = threadIdx.x;
+    float add = 0.f;
+    for (int j = 0; j <= i; ++j) add += sP[i * (C + 1) + j];
+    sDen[i] += add;
+  }
+
+  constexpr int RB = D / 16;
+  const int ti = threadIdx.x / 16, tc = threadIdx.x % 16;
+  float acc[4][RB];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < RB; ++b) acc[a][b] = 0.f;
+  for (int r = 0; r < D; ++r) {
+    float qa[4], sb[RB];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) qa[a] = sQ[(ti + 16 * a) * D + r];
+#pragma unroll
+    for (int b = 0; b < RB; ++b) sb[b] = sS[r * D + tc + 16 * b];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < RB; ++b) acc[a][b] = fmaf(qa[a], sb[b], acc[a][b]);
+  }
+  if (CAUSAL) {
+    for (int j = 0; j < valid; ++j) {
+      float pa[4], vb[RB];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) pa[a] = sP[(ti + 16 * a) * (C + 1) + j];
+#pragma unroll
+      for (int b = 0; b < RB; ++b) vb[b] = sV[j * D + tc + 16 * b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < RB; ++b) acc[a][b] = fmaf(pa[a], vb[b], acc[a][b]);
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = ti + 16 * a;
+    if (i < valid) {
+      const float inv = 1.f / sDen[i];
+#pragma unroll
+      for (int b = 0; b < RB; ++b) store1(out + row0 + (int64_t)i * D + tc + 16 * b, acc[a][b] * inv);
+    }
+  }
+}
+
+template <int D>
+size_t chunk_out_smem(bool causal) {
+  size_t f = (size_t)C * D + (size_t)D * D + D + C;
+  if (causal) f += 2 * (size_t)C * D + (size_t)C * (C + 1);
+  return f * sizeof(float);
+}
+
+template <int D, typename T>
+cudaError_t chunk_state_impl(const void *k, const void *v, float *ws, int64_t heads, int64_t n,
+                             cudaStream_t st) {
+  const int64_t nchunks = (n + C - 1) / C;
+  const size_t smem = 2 * (size_t)C * D * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(simt_chunk_state_kernel<D, T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  simt_chunk_state_kernel<D, T><<<(unsigned)(nchunks * heads), kThreads, smem, st>>>(
+      static_cast<const T *>(k), static_cast<const T *>(v), ws, n, nchunks);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int D, bool CAUSAL, typename T>
+cudaError_t chunk_out_impl(const void *q, const void *k, const void *v, void *out,
+                           const float *S, const float *z, int64_t Scs, int64_t Shs,
+                           int64_t zcs, int64_t zhs, int64_t heads, int64_t n, cudaStream_t st) {
+  const int64_t nchunks = (n + C - 1) / C;
+  const size_t smem = chunk_out_smem<D>(CAUSAL);
+  cudaError_t e = cudaFuncSetAttribute(simt_chunk_out_kernel<D, CAUSAL, T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  simt_chunk_out_kernel<D, CAUSAL, T><<<(unsigned)(nchunks * heads), kThreads, smem, st>>>(
+      static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
+      static_cast<T *>(out), S, z, Scs, Shs, zcs, zhs, n, nchunks);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t chunk_state_t(const void *k, const void *v, float *ws, int64_t heads, int64_t n,
+                          int d, cudaStream_t st) {
+  return d == 64 ? chunk_state_impl<64, T>(k, v, ws, heads, n, st)
+                 : chunk_state_impl<128, T>(k, v, ws, heads, n, st);
+}
+
+template <typename T>
+cudaError_t chunk_out_t(const void *q, const void *k, const void *v, void *out, const float *S,
+                        const float *z, int64_t Scs, int64_t Shs, int64_t zcs, int64_t zhs,
+                        int64_t heads, int64_t n, int d, int causal, cudaStream_t st) {
+  if (d == 64)
+    return causal ? chunk_out_impl<64, true, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads,
+                                                n, st)
+                  : chunk_out_impl<64, false, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads,
+                                                 n, st);
+  return causal ? chunk_out_impl<128, true, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n,
+                                               st)
+                : chunk_out_impl<128, false, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n,
+                                                st);
+}
+
+}  // namespace
+
+cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int64_t heads,
+                                    int64_t n, int d, int is_bf16, cudaStream_t st) {
+  return is_bf16 ? chunk_state_t<__nv_bfloat16>(k, v, ws, heads, n, d, st)
+                 : chunk_state_t<float>(k, v, ws, heads, n, d, st);
+}
+
+cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
+                               float *S_out, float *z_out, cudaStream_t st) {
+  const int64_t per = (int64_t)d * d + d;
+  scan_states_kernel<<<(unsigned)(((per + 255) / 256) * heads), 256, 0, st>>>(ws, nseg, d, mode,
+                                                                              S_out, z_out);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, void *out,
+                                  const float *S, const float *z, int64_t Scs, int64_t Shs,
+                                  int64_t zcs, int64_t zhs, int64_t heads, int64_t n, int d,
+                                  int causal, int is_bf16, cudaStream_t st) {
+  return is_bf16 ? chunk_out_t<__nv_bfloat16>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n,
+                                               d, causal, st)
+                 : chunk_out_t<float>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n, d,
+                                      causal, st);
+}
+
+}  // namespace linattn

@@ -1,0 +1,37 @@
+"""Shared helpers for the parity tests: device transfer and the error metric.
+
+Error metric: per row i, ||out_i - ref_i||_2 / ||ref_i||_2, maximised over every row of
+every head (and every decode step).  Bars: 1e-4 for float32 I/O, 2e-2 for bfloat16 I/O.
+"""
+import numpy as np
+
+from linear_attention_linattn_b200 import inputs
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def max_row_rel_err(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    d = got.shape[-1]
+    num = np.linalg.norm((got - ref).reshape(-1, d), axis=1)
+    den = np.linalg.norm(ref.reshape(-1, d), axis=1)
+    assert np.all(den > 0)
+    return float(np.max(num / den))
+
+
+def as_io(x: np.ndarray, dtype: str) -> np.ndarray:
+    """The values the device sees for float32 input x under the given I/O dtype."""
+    return inputs.round_bf16(x) if dtype == "bf16" else np.ascontiguousarray(x, np.float32)
+
+
+def to_dev(x: np.ndarray, dtype: str):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16)
+    return t.cuda()
+
+
+def to_host(t) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)

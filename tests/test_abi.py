@@ -1,0 +1,84 @@
+"""The C-ABI library loads without a GPU, exports every declared symbol, and rejects bad
+arguments before it touches a device (no compute call is made here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import linear_attention_linattn_b200 as la
+from linear_attention_linattn_b200 import build as labuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(linattn_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if labuild.needs_build():
+        labuild.build()
+    return la.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_symbols()
+    assert {"linattn_forward", "linattn_decode_step"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(la.SIGNATURES), "binding and header disagree"
+
+
+def test_state_bytes_closed_form(lib):
+    # D*d*4 + D*4 bytes: 16,640 at d = D = 64 (page "Linear Attention > Memory Efficiency")
+    assert lib.linattn_state_bytes(64) == 16640
+    assert lib.linattn_state_bytes(128) == 66048
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.linattn_status_string(s)
+    assert lib.linattn_version() >= 100
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: the checks return first
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, FAKE, FAKE, FAKE, 1, 1, 8, 64, 0, 1), la.LINATTN_ERR_INVALID_ARG),   # null q
+    ((FAKE + 4, FAKE, FAKE, FAKE, 1, 1, 8, 64, 0, 1), la.LINATTN_ERR_INVALID_ARG),  # misaligned
+    ((FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 64, 0, 1), la.LINATTN_ERR_INVALID_ARG),  # B = 0
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, 0, 1), la.LINATTN_ERR_INVALID_ARG),  # n = 0
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 2, 1), la.LINATTN_ERR_INVALID_ARG),  # causal = 2
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 0, 7), la.LINATTN_ERR_INVALID_ARG),  # dtype
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 0, 1), la.LINATTN_ERR_UNSUPPORTED),  # d = 96
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 1 << 31, 64, 0, 1), la.LINATTN_ERR_INVALID_ARG),  # n too big
+])
+def test_forward_argument_checks(lib, args, want):
+    assert lib.linattn_forward(*args, None) == want
+
+
+def test_decode_and_state_argument_checks(lib):
+    assert lib.linattn_decode_step(0, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 64, None) == \
+        la.LINATTN_ERR_INVALID_ARG
+    assert lib.linattn_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 32, None) == \
+        la.LINATTN_ERR_UNSUPPORTED
+    assert lib.linattn_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 1, 64, None) == \
+        la.LINATTN_ERR_INVALID_ARG
+    assert lib.linattn_forward_state(FAKE, FAKE, FAKE, 0, 1, 1, 8, 64, 1, None) == \
+        la.LINATTN_ERR_INVALID_ARG
+    assert lib.linattn_forward_ex(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1, 1, -64, None) == \
+        la.LINATTN_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError):
+        la.load_library(str(tmp_path / "nope.so"))

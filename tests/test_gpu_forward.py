@@ -1,0 +1,157 @@
+"""Parity of the CUDA forward pass (through the C ABI) with the float64 oracle.
+
+Small cases span several chunks and segments with ragged tails; the five measured
+workloads run at full size in the launch configuration the benchmark times, compared
+on sampled heads and rows that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from linear_attention_linattn_b200 import inputs
+from tests.helpers import TOL, as_io, max_row_rel_err, to_dev, to_host
+
+torch = pytest.importorskip("torch")
+la = pytest.importorskip("linear_attention_linattn_b200")
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, k, v, causal, dtype, segment_len=0):
+    qd, kd, vd = to_dev(q, dtype), to_dev(k, dtype), to_dev(v, dtype)
+    out = la.forward(qd, kd, vd, causal, segment_len=segment_len)
+    assert la.device_error() == la.LINATTN_OK
+    return to_host(out)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,H,n", [(1, 1, 1), (1, 2, 2), (2, 1, 63), (1, 3, 65), (2, 2, 200),
+                                   (1, 1, 1000), (1, 2, 4097)])
+def test_small_shapes(dtype, causal, d, B, H, n):
+    q, k, v = inputs.forward_qkv(100 + n, B, H, n, d, scaled=True)
+    q, k, v = as_io(q, dtype), as_io(k, dtype), as_io(v, dtype)
+    got = _run(q, k, v, causal, dtype)
+    ref = oracle.forward(q, k, v, causal)
+    assert max_row_rel_err(got, ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("seg", [0, 64, 128, 512, 1024])
+def test_segment_length_invariance(dtype, seg):
+    B, H, n, d = 1, 2, 3000, 128
+    q, k, v = inputs.forward_qkv(7, B, H, n, d, scaled=True)
+    q, k, v = as_io(q, dtype), as_io(k, dtype), as_io(v, dtype)
+    got = _run(q, k, v, True, dtype, segment_len=seg)
+    ref = oracle.forward(q, k, v, True)
+    assert max_row_rel_err(got, ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_invariants_on_device(dtype, d):
+    rng = np.random.default_rng(5)
+    B, H, n = 1, 2, 777
+    q, k, v = (as_io(rng.standard_normal((B, H, n, d)).astype(np.float32) / np.sqrt(d), dtype)
+               for _ in range(3))
+    # constant values come back unchanged (the weights are a convex combination)
+    c = as_io(rng.standard_normal(d).astype(np.float32), dtype)
+    vc = np.broadcast_to(c, (B, H, n, d)).copy()
+    for causal in (False, True):
+        got = _run(q, k, vc, causal, dtype)
+        assert max_row_rel_err(got, np.broadcast_to(c, got.shape)) <= TOL[dtype]
+    # a single token returns its own value
+    got1 = _run(q[:, :, :1], k[:, :, :1], v[:, :, :1], True, dtype)
+    assert max_row_rel_err(got1, v[:, :, :1]) <= TOL[dtype]
+    # the last causal row sees every key: it equals the non-causal row
+    nc = _run(q, k, v, False, dtype)
+    ca = _run(q, k, v, True, dtype)
+    assert max_row_rel_err(ca[:, :, -1], nc[:, :, -1]) <= 2 * TOL[dtype]
+
+
+def test_output_canary_untouched():
+    """Nothing is written outside out: guard regions on both sides keep their pattern."""
+    B, H, n, d = 1, 2, 130, 64
+    q, k, v = inputs.forward_qkv(3, B, H, n, d, scaled=True)
+    for dtype in ("f32", "bf16"):
+        qd, kd, vd = to_dev(as_io(q, dtype), dtype), to_dev(as_io(k, dtype), dtype), \
+            to_dev(as_io(v, dtype), dtype)
+        pad = 4096
+        buf = torch.full((2 * pad + qd.numel(),), 12345.0, dtype=qd.dtype, device="cuda")
+        out = buf[pad:pad + qd.numel()].view(qd.shape)
+        for causal in (False, True):
+            la.forward(qd, kd, vd, causal, out=out)
+            torch.cuda.synchronize()
+            assert bool((buf[:pad] == 12345.0).all()) and bool((buf[-pad:] == 12345.0).all())
+
+
+def test_forward_state_matches_oracle():
+    for dtype in ("f32", "bf16"):
+        for d in (64, 128):
+            B, H, n = 2, 2, 1500
+            _, k, v = inputs.forward_qkv(11, B, H, n, d, scaled=True)
+            k, v = as_io(k, dtype), as_io(v, dtype)
+            S, z = la.forward_state(to_dev(k, dtype), to_dev(v, dtype))
+            assert la.device_error() == la.LINATTN_OK
+            S_ref, z_ref = oracle.state(k, v)
+            S, z = to_host(S), to_host(z)
+            for b in range(B):
+                for h in range(H):
+                    e = np.linalg.norm(S[b, h] - S_ref[b, h]) / np.linalg.norm(S_ref[b, h])
+                    assert e <= 1e-5, (dtype, d, e)
+                    assert np.max(np.abs(z[b, h] - z_ref[b, h]) / z_ref[b, h]) <= 1e-5
+
+
+# ------------------------------------------------------------------ the measured workloads
+def test_workload_noncausal_1x1x512x64_f32():
+    w = inputs.WORKLOADS["noncausal_1x1x512x64_f32"]
+    q, k, v = inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled)
+    got = _run(q, k, v, False, "f32")
+    assert max_row_rel_err(got, oracle.forward(q, k, v, False)) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_workload_causal_1x1x4096x64(dtype):
+    w = inputs.WORKLOADS["causal_1x1x4096x64"]
+    q, k, v = (as_io(x, dtype) for x in inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled))
+    got = _run(q, k, v, True, dtype)
+    assert max_row_rel_err(got, oracle.forward(q, k, v, True)) <= TOL[dtype]
+
+
+def _sample_rows(n, extra, seed):
+    rng = np.random.default_rng(seed)
+    rows = {0, 1, 2, 63, 64, 65, 127, 128, n // 2, n - 2, n - 1}
+    rows |= {r for m in (512, 1024, 2048, 4096) for r in (m - 1, m) if r < n}
+    rows |= set(rng.integers(0, n, size=extra).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < n), dtype=np.int64)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_workload_batched_8x16x8192x64_bf16(causal):
+    w = inputs.WORKLOADS["batched_8x16x8192x64_bf16"]
+    q, k, v = inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled)
+    q, k, v = (inputs.round_bf16(x) for x in (q, k, v))
+    got = _run(q, k, v, causal, "bf16")
+    heads = [(0, 0), (3, 7), (7, 15)]
+    rows = _sample_rows(w.n, 64, 1)
+    qs = np.stack([q[b, h] for b, h in heads])
+    ks = np.stack([k[b, h] for b, h in heads])
+    vs = np.stack([v[b, h] for b, h in heads])
+    ref = oracle.forward_rows(qs, ks, vs, rows, causal)
+    gs = np.stack([got[b, h][rows] for b, h in heads])
+    assert max_row_rel_err(gs, ref) <= TOL["bf16"]
+    assert np.all(np.isfinite(got))
+
+
+def test_workload_longctx_1x32x131072x128_bf16():
+    w = inputs.WORKLOADS["longctx_1x32x131072x128_bf16"]
+    q, k, v = inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled)
+    q, k, v = (inputs.round_bf16(x) for x in (q, k, v))
+    got = _run(q, k, v, True, "bf16")
+    assert np.all(np.isfinite(got))
+    heads = [0, 17, 31]
+    rows = _sample_rows(w.n, 48, 2)
+    ref = oracle.forward_rows(q[0, heads], k[0, heads], v[0, heads], rows, True)
+    gs = np.stack([got[0, h][rows] for h in heads])
+    assert max_row_rel_err(gs, ref) <= TOL["bf16"]
