@@ -81,6 +81,18 @@ linattn_status check_forward_shape(int64_t B, int64_t H, int64_t n, int64_t d) {
   return LINATTN_OK;
 }
 
+linattn_status forward_tc(const void *q, const void *k, const void *v, void *out,
+                          int64_t heads, int64_t n, int d, int causal, int64_t seg,
+                          DeviceState *ds, cudaStream_t st) {
+  if (seg == 0) seg = tc_default_segment(heads, n, d);
+  Workspace ws;
+  ws.st = st;
+  if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, d, seg, causal), ds->pool,
+                              st) != cudaSuccess)
+    return LINATTN_ERR_CUDA;
+  return to_status(tc_forward(q, k, v, out, heads, n, d, causal, seg, ws.ptr, ds->err_word, st));
+}
+
 linattn_status forward_simt(const void *q, const void *k, const void *v, void *out,
                             int64_t heads, int64_t n, int d, int causal, int is_bf16,
                             DeviceState *ds, cudaStream_t st) {
@@ -96,14 +108,14 @@ linattn_status forward_simt(const void *q, const void *k, const void *v, void *o
   e = launch_simt_chunk_state(k, v, w, heads, n, d, is_bf16, st);
   if (e != cudaSuccess) return LINATTN_ERR_CUDA;
   if (causal) {
-    e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, nullptr, st);
+    e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, 0, nullptr, 0, st);
     if (e != cudaSuccess) return LINATTN_ERR_CUDA;
     e = launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
                               nchunks * per, heads, n, d, 1, is_bf16, st);
   } else {
     float *tot = w + heads * nchunks * per;
     float *tot_z = tot + heads * (int64_t)d * d;
-    e = launch_scan_states(w, heads, nchunks, d, 1, tot, tot_z, st);
+    e = launch_scan_states(w, heads, nchunks, d, 1, tot, (int64_t)d * d, tot_z, d, st);
     if (e != cudaSuccess) return LINATTN_ERR_CUDA;
     e = launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, (int64_t)d * d, 0, d, heads, n, d, 0,
                               is_bf16, st);
@@ -127,13 +139,15 @@ linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, v
     return LINATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
   if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  if (segment_len < 0) return LINATTN_ERR_INVALID_ARG;
+  if (segment_len < 0 || segment_len % kTcChunk != 0) return LINATTN_ERR_INVALID_ARG;
   linattn_status s = check_forward_shape(B, H, n, d);
   if (s != LINATTN_OK) return s;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, dtype == LINATTN_BF16, ds, st);
+  if (dtype == LINATTN_BF16)
+    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, segment_len, ds, st);
+  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, ds, st);
 }
 
 linattn_status linattn_forward(const void *q, const void *k, const void *v, void *out, int64_t B,
@@ -155,16 +169,25 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t heads = B * H;
-  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
-  const int64_t per = d * d + d;
   Workspace ws;
   ws.st = st;
+  if (dtype == LINATTN_BF16) {
+    const int64_t seg = tc_default_segment(heads, n, (int)d);
+    if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, (int)d, seg, 1), ds->pool,
+                                st) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
+    return to_status(tc_forward_state(k, v, state_S, state_z, heads, n, (int)d, seg, ws.ptr,
+                                      ds->err_word, st));
+  }
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  const int64_t per = d * d + d;
   if (cudaMallocFromPoolAsync(&ws.ptr, (size_t)(heads * nchunks * per) * 4, ds->pool, st) !=
       cudaSuccess)
     return LINATTN_ERR_CUDA;
   float *w = static_cast<float *>(ws.ptr);
-  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, dtype == LINATTN_BF16, st);
-  if (e == cudaSuccess) e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, state_z, st);
+  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, 0, st);
+  if (e == cudaSuccess)
+    e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, d * d, state_z, d, st);
   return to_status(e);
 }
 

@@ -104,11 +104,11 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__r
 
 // K2: per head, a sequential sweep over the segments for each state element.
 //   mode 0: ws[h][s] <- sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
-//   mode 1: S_out[h], z_out[h] <- sum_s ws[h][s] (the total)
+//   mode 1: S_out + h*S_hs, z_out + h*z_hs <- sum_s ws[h][s] (the total)
 __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws, int64_t nseg,
                                                           int d, int mode,
-                                                          float *__restrict__ S_out,
-                                                          float *__restrict__ z_out) {
+                                                          float *__restrict__ S_out, int64_t S_hs,
+                                                          float *__restrict__ z_out, int64_t z_hs) {
   const int64_t per = (int64_t)d * d + d;
   const int64_t blocks_per_head = (per + blockDim.x - 1) / blockDim.x;
   const int64_t head = blockIdx.x / blocks_per_head;
@@ -125,9 +125,9 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
   } else {
     for (int64_t s = 0; s < nseg; ++s) run += base[s * per];
     if (e < (int64_t)d * d)
-      S_out[head * d * d + e] = run;
+      S_out[head * S_hs + e] = run;
     else
-      z_out[head * d + (e - (int64_t)d * d)] = run;
+      z_out[head * z_hs + (e - (int64_t)d * d)] = run;
   }
 }
 
@@ -318,10 +318,11 @@ cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int
 }
 
 cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
-                               float *S_out, float *z_out, cudaStream_t st) {
+                               float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
+                               cudaStream_t st) {
   const int64_t per = (int64_t)d * d + d;
-  scan_states_kernel<<<(unsigned)(((per + 255) / 256) * heads), 256, 0, st>>>(ws, nseg, d, mode,
-                                                                              S_out, z_out);
+  scan_states_kernel<<<(unsigned)(((per + 255) / 256) * heads), 256, 0, st>>>(
+      ws, nseg, d, mode, S_out, S_hs, z_out, z_hs);
   count_launches(1);
   return cudaGetLastError();
 }

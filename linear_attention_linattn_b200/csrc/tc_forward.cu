@@ -1,0 +1,675 @@
+// bf16-I/O forward pass on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// The method (page "Efficient Transformers: Linear Attention and Flash Attention",
+// sections "Linear attention: reordering the matmuls, not shrinking them" and "The
+// recurrent view: attention as an RNN"):
+//     out_i = phi(q_i) S / phi(q_i).z,  S = sum_j phi(k_j) v_j^T,  z = sum_j phi(k_j)
+// with j <= i in the causal mode.  Causal work is split into chunks of C = 64 tokens:
+//     num_c = phi(Q_c) S_<c + mask(phi(Q_c) phi(K_c)^T) V_c
+//     den_c = phi(Q_c) z_<c + mask(phi(Q_c) phi(K_c)^T) 1
+//     S_<c+1 = S_<c + phi(K_c)^T V_c,   z_<c+1 = z_<c + phi(K_c)^T 1
+// and chunks are grouped into segments (one CTA each).  Three kernel modes:
+//   kState        segment aggregates (S_s, z_s) -> fp32 workspace       (K1)
+//   kCausalOut    outputs of a segment from its exclusive prefix state   (K3)
+//   kNoncausalOut outputs phi(Q) S / phi(Q).z from the per-head total    (K3, no mask)
+// The exclusive prefix over segments (K2) is the scan kernel in simt_forward.cu.
+//
+// Every product is a tcgen05.mma (kind::f16, bf16 operands, fp32 accumulator in TMEM):
+//   P     = phi(Q_c) phi(K_c)^T        M=64  N=64  K=d   (A: Q K-major, B: K K-major)
+//   O     = phi(Q_c) S_<c              M=64  N=d   K=d   (B: S bf16, MN-major)
+//   Oden  = phi(Q_c) [z 0..0]          M=64  N=16  K=d
+//   O    += P V_c                      M=64  N=d   K=64  (A: P bf16 K-major, B: V MN-major)
+//   Oden += P [1 0..0]                 M=64  N=16  K=64
+//   S    += phi(K_c)^T V_c             M=d   N=d   K=64  (A: K MN-major)
+//   z    += phi(K_c)^T [1 0..0]        M=d   N=16  K=64
+// The normaliser rides along as a 16-column block whose first column is z (or ones), so the
+// numerator and the denominator see the same rounded weights.
+//
+// Warp roles (448 threads, one CTA per SM):
+//   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of Q/K/V chunks into a
+//              ring of stages; no multicast.
+//   warp 1     TMEM allocation and the single MMA-issuing thread.
+//   warps 2-5  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
+//              n zeroed, then handed to the tensor cores.
+//   warps 6-13 TMEM epilogue: mask and round P, round S_<c+1 and z into the next chunk's
+//              operands, divide O by its denominator and TMA-store the output tile.
+// Every wait is bounded (2 s); a wait that gives up records LINATTN_ERR_TIMEOUT and the
+// CTA drains and exits without trapping.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace linattn {
+namespace {
+
+constexpr int C = kTcChunk;       // tokens per chunk (64)
+constexpr int kAtom = C * 128;    // one [64 rows][64 bf16] 128B-swizzled atom: 8 KB
+constexpr int kZAtom = 16 * 128;  // one [16 rows][64 bf16] atom: 2 KB
+
+enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
+
+constexpr int kWarpTMA = 0;
+constexpr int kWarpMMA = 1;
+constexpr int kWarpXform0 = 2;
+constexpr int kNumXformWarps = 4;
+constexpr int kWarpEpi0 = kWarpXform0 + kNumXformWarps;  // 6
+constexpr int kNumEpiWarps = 8;
+constexpr int kThreads = (kWarpEpi0 + kNumEpiWarps) * 32;  // 448
+constexpr int kXformThreads = kNumXformWarps * 32;
+constexpr int kEpiThreads = kNumEpiWarps * 32;
+constexpr int kMaxSmem = 227 * 1024;
+constexpr uint32_t kTmemCols = 512;
+
+// TMEM column map.
+constexpr uint32_t kColP = 0;    // P: 64 columns
+constexpr uint32_t kColO = 64;   // O: d columns, then the 16-column denominator block
+constexpr uint32_t kColS = 256;  // S: d columns, then the 16-column z block
+
+template <int D, int MODE>
+struct Cfg {
+  static constexpr int A = D / 64;          // 64-column atoms per [64][D] tile
+  static constexpr int TILE = A * kAtom;    // bytes of a bf16 [64][D] tile
+  static constexpr bool LQ = MODE != kState;
+  static constexpr bool LKV = MODE != kNoncausalOut;
+  static constexpr int STAGE = TILE * ((LQ ? 1 : 0) + (LKV ? 2 : 0));
+  static constexpr int S_BYTES = A * D * 128;  // bf16 S, MN-major [A][D rows][128 B]
+  static constexpr int Z_BYTES = A * kZAtom;   // bf16 [16][D], K-major, row 0 = z
+  static constexpr int ONES_BYTES = kZAtom;    // bf16 [16][64], K-major, row 0 = 1
+  static constexpr int P_BYTES = kAtom;        // bf16 [64][64], K-major
+  static constexpr int OUT_BYTES = TILE;       // bf16 output staging, TMA-store layout
+  static constexpr int FIXED = S_BYTES + Z_BYTES + ONES_BYTES + P_BYTES + OUT_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int NS_FIT = (kMaxSmem - 1024 - BAR_BYTES - FIXED) / STAGE;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static constexpr int OFF_STAGES = 0;
+  static constexpr int OFF_S = NS * STAGE;
+  static constexpr int OFF_Z = OFF_S + S_BYTES;
+  static constexpr int OFF_ONES = OFF_Z + Z_BYTES;
+  static constexpr int OFF_P = OFF_ONES + ONES_BYTES;
+  static constexpr int OFF_OUT = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_OUT + OUT_BYTES;
+  static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+  static_assert(NS >= 2, "at least two pipeline stages");
+  static_assert(SMEM <= kMaxSmem, "shared memory budget");
+  static_assert(OFF_S % 1024 == 0 && OFF_Z % 1024 == 0 && OFF_ONES % 1024 == 0 &&
+                    OFF_P % 1024 == 0 && OFF_OUT % 1024 == 0 && STAGE % 1024 == 0,
+                "128B-swizzled operands need 1024-byte alignment");
+};
+
+struct Bars {
+  uint64_t full[8], ready[8], empty[8];
+  uint64_t p_full, p_ready, s_full, s_ready, o_full, o_empty, fin;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block");
+
+// K-major operand descriptor for K-step ks of a [rows][D] tile made of 64-column atoms
+// of `atom_bytes` each: 4 K-steps of 32 bytes inside one 128-byte swizzle row.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int ks, uint32_t atom_bytes) {
+  return make_sw128_desc(base + (ks >> 2) * atom_bytes + (ks & 3) * 32, 16, 1024);
+}
+// MN-major operand descriptor for K-step ks (16 K-rows = two 8-row groups of 1024 B);
+// `lbo` is the byte stride between 64-wide M/N atoms.
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks, uint32_t lbo) {
+  return make_sw128_desc(base + ks * 2048, lbo, 1024);
+}
+
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t u) {
+  return pack_bf16x2(phi_fast(bf16_lo(u)), phi_fast(bf16_hi(u)));
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const float *__restrict__ init_state, int64_t init_head_stride,
+              int64_t init_seg_stride, float *__restrict__ out_state, int64_t n, int64_t seg_len,
+              int64_t nseg, int *err) {
+  using G = Cfg<D, MODE>;
+  constexpr int NS = G::NS;
+  constexpr int KSD = D / 16;  // K-steps over the feature dimension
+  constexpr int KSC = C / 16;  // K-steps over the chunk's tokens
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  Bars &bar = *reinterpret_cast<Bars *>(smem + G::OFF_BAR);
+  volatile int *abort = &bar.abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t head = blockIdx.x / nseg;
+  const int64_t seg = blockIdx.x % nseg;
+  const int64_t t_begin = seg * seg_len;
+  const int64_t t_end = n < t_begin + seg_len ? n : t_begin + seg_len;
+  const int nchunks = static_cast<int>((t_end - t_begin + C - 1) / C);
+
+  // ---- set-up: barriers, constant operand blocks, TMEM
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar.full[s], 1);
+      mbar_init(&bar.ready[s], kXformThreads);
+      mbar_init(&bar.empty[s], 1);
+    }
+    mbar_init(&bar.p_full, 1);
+    mbar_init(&bar.p_ready, kEpiThreads);
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.s_ready, kEpiThreads);
+    mbar_init(&bar.o_full, 1);
+    mbar_init(&bar.o_empty, kEpiThreads);
+    mbar_init(&bar.fin, 1);
+    bar.abort = 0;
+    fence_barrier_init();
+  }
+  {
+    // ones block: row 0 = 1.0, rows 1..15 = 0; z block: all zero (row 0 is rewritten)
+    uint32_t *ones = reinterpret_cast<uint32_t *>(smem + G::OFF_ONES);
+    for (int i = threadIdx.x; i < G::ONES_BYTES / 4; i += kThreads)
+      ones[i] = i < 32 ? 0x3F803F80u : 0u;  // first 128-byte row: 64 x bf16(1.0)
+    uint32_t *zb = reinterpret_cast<uint32_t *>(smem + G::OFF_Z);
+    for (int i = threadIdx.x; i < G::Z_BYTES / 4; i += kThreads) zb[i] = 0u;
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(&bar.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTMA && lane == 0) {
+    if (G::LQ) prefetch_tmap(&tmQ);
+    if (G::LKV) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+    if (MODE != kState) prefetch_tmap(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+
+  if (warp == kWarpTMA) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS;
+        const uint32_t it = c / NS;
+        if (c >= NS && !mbar_wait(&bar.empty[s], (it - 1) & 1, abort, err)) break;
+        mbar_arrive_expect_tx(&bar.full[s], G::STAGE);
+        uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+        const int y = static_cast<int>(t_begin + (int64_t)c * C);
+        const int zc = static_cast<int>(head);
+        if (G::LQ) {
+#pragma unroll
+          for (int a = 0; a < G::A; ++a) tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
+          st += G::TILE;
+        }
+        if (G::LKV) {
+#pragma unroll
+          for (int a = 0; a < G::A; ++a) tma_load_3d(st + a * kAtom, &tmK, &bar.full[s], a * 64, y, zc, pol);
+#pragma unroll
+          for (int a = 0; a < G::A; ++a)
+            tma_load_3d(st + G::TILE + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
+        }
+        issued = c + 1;
+      }
+      // drain: every issued load has landed before the CTA may exit
+      for (int c = (issued > NS ? issued - NS : 0); c < issued; ++c)
+        mbar_wait(&bar.full[c % NS], (c / NS) & 1, abort, err);
+    }
+  } else if (warp == kWarpMMA) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t I_P = make_idesc_bf16(64, 64, false, false);
+      constexpr uint32_t I_O = make_idesc_bf16(64, D, false, true);
+      constexpr uint32_t I_DEN = make_idesc_bf16(64, 16, false, false);
+      constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);
+      constexpr uint32_t I_Z = make_idesc_bf16(D, 16, true, false);
+      const uint32_t tP = tmem + kColP, tO = tmem + kColO, tOd = tmem + kColO + D;
+      const uint32_t tS = tmem + kColS, tSz = tmem + kColS + D;
+      const uint32_t sS = smem_u32(smem + G::OFF_S), sZ = smem_u32(smem + G::OFF_Z);
+      const uint32_t sOnes = smem_u32(smem + G::OFF_ONES), sP = smem_u32(smem + G::OFF_P);
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NS;
+        const uint32_t it = c / NS;
+        if (!mbar_wait(&bar.ready[s], it & 1, abort, err)) break;
+        const uint32_t st = smem_u32(smem + G::OFF_STAGES + s * G::STAGE);
+        const uint32_t sQ = st;
+        const uint32_t sK = st + (G::LQ ? G::TILE : 0);
+        const uint32_t sV = sK + G::TILE;
+        if (MODE == kState) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks) {
+            const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
+            const uint64_t a = desc_mnmajor(sK, ks, kAtom);
+            mma_bf16_ss(tS, a, desc_mnmajor(sV, ks, kAtom), I_S, acc);
+            mma_bf16_ss(tSz, a, desc_kmajor(sOnes, ks, kZAtom), I_Z, acc);
+          }
+          mma_commit(&bar.empty[s]);
+          continue;
+        }
+        // S_<c and z_<c are in shared memory; O is free again
+        if (MODE == kCausalOut || c == 0)
+          if (!mbar_wait(&bar.s_ready, MODE == kCausalOut ? (c & 1) : 0, abort, err)) break;
+        if (c > 0 && !mbar_wait(&bar.o_empty, (c - 1) & 1, abort, err)) break;
+        tc_fence_after();
+        if (MODE == kCausalOut) {
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tP, desc_kmajor(sQ, ks, kAtom), desc_kmajor(sK, ks, kAtom), I_P,
+                        ks > 0 ? 1u : 0u);
+          mma_commit(&bar.p_full);
+        }
+#pragma unroll
+        for (int ks = 0; ks < KSD; ++ks) {
+          const uint64_t a = desc_kmajor(sQ, ks, kAtom);
+          mma_bf16_ss(tO, a, desc_mnmajor(sS, ks, D * 128), I_O, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(tOd, a, desc_kmajor(sZ, ks, kZAtom), I_DEN, ks > 0 ? 1u : 0u);
+        }
+        if (MODE == kCausalOut) {
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks) {
+            const uint64_t a = desc_mnmajor(sK, ks, kAtom);
+            mma_bf16_ss(tS, a, desc_mnmajor(sV, ks, kAtom), I_S, 1u);
+            mma_bf16_ss(tSz, a, desc_kmajor(sOnes, ks, kZAtom), I_Z, 1u);
+          }
+          mma_commit(&bar.s_full);
+          if (!mbar_wait(&bar.p_ready, c & 1, abort, err)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks) {
+            const uint64_t a = desc_kmajor(sP, ks, kAtom);
+            mma_bf16_ss(tO, a, desc_mnmajor(sV, ks, kAtom), I_O, 1u);
+            mma_bf16_ss(tOd, a, desc_kmajor(sOnes, ks, kZAtom), I_DEN, 1u);
+          }
+        }
+        mma_commit(&bar.o_full);
+        mma_commit(&bar.empty[s]);
+      }
+      if (MODE == kState) mma_commit(&bar.s_full);
+      // every MMA this CTA issued has finished before TMEM is released
+      mma_commit(&bar.fin);
+      mbar_wait(&bar.fin, 0, abort, err);
+    }
+  } else if (warp < kWarpEpi0) {
+    // ================================================================ feature map
+    const int xt = threadIdx.x - kWarpXform0 * 32;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % NS;
+      if (!mbar_wait(&bar.full[s], (c / NS) & 1, abort, err)) break;
+      uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+      const int64_t left = t_end - (t_begin + (int64_t)c * C);
+      const int valid = left < C ? static_cast<int>(left) : C;
+      if (G::LQ) {
+        uint4 *p = reinterpret_cast<uint4 *>(st);
+        for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
+          uint4 x = p[i];
+          x.x = phi_bf16x2(x.x);
+          x.y = phi_bf16x2(x.y);
+          x.z = phi_bf16x2(x.z);
+          x.w = phi_bf16x2(x.w);
+          p[i] = x;
+        }
+        st += G::TILE;
+      }
+      if (G::LKV) {
+        uint4 *p = reinterpret_cast<uint4 *>(st);
+        for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
+          const int row = (i % (kAtom / 16)) >> 3;  // 8 x 16 B per 128-byte row
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (row < valid) {
+            x = p[i];
+            x.x = phi_bf16x2(x.x);
+            x.y = phi_bf16x2(x.y);
+            x.z = phi_bf16x2(x.z);
+            x.w = phi_bf16x2(x.w);
+          }
+          p[i] = x;
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar.ready[s]);
+    }
+  } else {
+    // ================================================================ TMEM epilogue
+    // Control flow is uniform across the 8 warps: lane 0 of each warp does the mbarrier
+    // waits and broadcasts the outcome, and after a give-up the loop still runs through every
+    // named barrier (doing no work), so no warp is ever left at a barrier alone.
+    const int et = threadIdx.x - kWarpEpi0 * 32;  // 0..255
+    const int sp = warp & 3;                      // TMEM sub-partition of this warp
+    const int h = (warp - kWarpEpi0) >> 2;        // which half of the columns
+    const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
+    const bool v64 = lane < 16;                   // lanes holding rows of an M=64 tile
+    const int r64 = 16 * sp + lane;               // row of an M=64 tile
+    const int rS = D == 128 ? 32 * sp + lane : r64;  // row of the S accumulator (M = D)
+    const bool vS = D == 128 ? true : v64;
+    constexpr int SC = D / 2;  // S / O columns per thread (one half)
+    uint8_t *sS = smem + G::OFF_S;
+    uint8_t *sZ = smem + G::OFF_Z;
+    bool ok = true;
+    auto warp_wait = [&](uint64_t *b, uint32_t parity) {
+      int r = 1;
+      if (lane == 0) r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
+      r = __shfl_sync(0xffffffffu, r, 0);
+      ok = ok && (r != 0);
+      return ok;
+    };
+
+    // S (fp32 values in registers) -> bf16 MN-major operand, z -> z block row 0
+    auto store_S_operand = [&](const float *vals, float zval) {
+      if (!vS) return;
+#pragma unroll
+      for (int j = 0; j < SC / 8; ++j) {
+        const int col = h * SC + 8 * j;  // first of 8 columns
+        uint4 u;
+        u.x = pack_bf16x2(vals[8 * j + 0], vals[8 * j + 1]);
+        u.y = pack_bf16x2(vals[8 * j + 2], vals[8 * j + 3]);
+        u.z = pack_bf16x2(vals[8 * j + 4], vals[8 * j + 5]);
+        u.w = pack_bf16x2(vals[8 * j + 6], vals[8 * j + 7]);
+        uint8_t *dst = sS + (col >> 6) * (D * 128) + sw128_offset(rS, col & 63);
+        *reinterpret_cast<uint4 *>(dst) = u;
+      }
+      if (h == 0) {
+        const __nv_bfloat16 zb = __float2bfloat16_rn(zval);
+        *reinterpret_cast<__nv_bfloat16 *>(sZ + (rS >> 6) * kZAtom + sw128_offset(0, rS & 63)) =
+            zb;
+      }
+    };
+
+    if (MODE != kState) {
+      // starting state: exclusive prefix (causal) or the head's total (non-causal)
+      const float *src = init_state + head * init_head_stride + seg * init_seg_stride;
+      float vals[SC];
+      float zval = 0.f;
+      if (vS) {
+#pragma unroll
+        for (int j = 0; j < SC / 4; ++j) {
+          const float4 f =
+              *reinterpret_cast<const float4 *>(src + (int64_t)rS * D + h * SC + 4 * j);
+          vals[4 * j + 0] = f.x;
+          vals[4 * j + 1] = f.y;
+          vals[4 * j + 2] = f.z;
+          vals[4 * j + 3] = f.w;
+        }
+        zval = src[(int64_t)D * D + rS];
+      } else {
+#pragma unroll
+        for (int j = 0; j < SC; ++j) vals[j] = 0.f;
+      }
+      if (MODE == kCausalOut) {
+        // the running state starts from the prefix: write it into the S accumulator
+#pragma unroll
+        for (int j = 0; j < SC / 16; ++j) {
+          uint32_t r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(vals[16 * j + e]);
+          tmem_st16(tmem + lane_off + kColS + h * SC + 16 * j, r);
+        }
+        if (h == 0) tmem_st1(tmem + lane_off + kColS + D, __float_as_uint(zval));
+        tmem_st_wait();
+      }
+      store_S_operand(vals, zval);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar.s_ready);
+    }
+
+    const uint64_t pol_out = policy_evict_first();
+    for (int c = 0; c < (MODE == kState ? 0 : nchunks); ++c) {
+      if (MODE == kCausalOut) {
+        // ---- P: mask j <= i, round to bf16, K-major A operand of P V
+        if (warp_wait(&bar.p_full, c & 1)) {
+          tc_fence_after();
+          uint32_t p0[16], p1[16];
+          tmem_ld16(tmem + lane_off + kColP + 32 * h, p0);
+          tmem_ld16(tmem + lane_off + kColP + 32 * h + 16, p1);
+          if (v64) {
+            uint8_t *sP = smem + G::OFF_P;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int col = 32 * h + 8 * j + e;
+                const uint32_t bits = (8 * j + e) < 16 ? p0[8 * j + e] : p1[8 * j + e - 16];
+                f[e] = col <= r64 ? __uint_as_float(bits) : 0.f;
+              }
+              uint4 u;
+              u.x = pack_bf16x2(f[0], f[1]);
+              u.y = pack_bf16x2(f[2], f[3]);
+              u.z = pack_bf16x2(f[4], f[5]);
+              u.w = pack_bf16x2(f[6], f[7]);
+              *reinterpret_cast<uint4 *>(sP + sw128_offset(r64, 32 * h + 8 * j)) = u;
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bar.p_ready);
+        }
+        // ---- S_<c+1, z_<c+1: the operands of the next chunk
+        if (warp_wait(&bar.s_full, c & 1)) {
+          tc_fence_after();
+          float vals[SC];
+#pragma unroll
+          for (int j = 0; j < SC / 16; ++j) {
+            uint32_t r[16];
+            tmem_ld16(tmem + lane_off + kColS + h * SC + 16 * j, r);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) vals[16 * j + e] = __uint_as_float(r[e]);
+          }
+          const float zval = __uint_as_float(tmem_ld1(tmem + lane_off + kColS + D));
+          store_S_operand(vals, zval);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bar.s_ready);
+        }
+      }
+
+      // ---- O / den -> bf16 output tile -> TMA store
+      float o[SC];
+      float inv = 0.f;
+      if (warp_wait(&bar.o_full, c & 1)) {
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < SC / 16; ++j) {
+          uint32_t r[16];
+          tmem_ld16(tmem + lane_off + kColO + h * SC + 16 * j, r);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[16 * j + e] = __uint_as_float(r[e]);
+        }
+        inv = 1.f / __uint_as_float(tmem_ld1(tmem + lane_off + kColO + D));
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty);
+      }
+      if (et == 0) tma_store_wait_read<0>();  // the staging tile is free again
+      named_barrier_sync(1, kEpiThreads);
+      if (ok && v64) {
+        uint8_t *so = smem + G::OFF_OUT;
+#pragma unroll
+        for (int j = 0; j < SC / 8; ++j) {
+          const int col = h * SC + 8 * j;
+          uint4 u;
+          u.x = pack_bf16x2(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+          u.y = pack_bf16x2(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+          u.z = pack_bf16x2(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+          u.w = pack_bf16x2(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+          *reinterpret_cast<uint4 *>(so + (col >> 6) * kAtom + sw128_offset(r64, col & 63)) = u;
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1, kEpiThreads);
+      if (et == 0 && !*abort) {
+        const int y = static_cast<int>(t_begin + (int64_t)c * C);
+#pragma unroll
+        for (int a = 0; a < G::A; ++a)
+          tma_store_3d(&tmO, smem + G::OFF_OUT + a * kAtom, a * 64, y, static_cast<int>(head),
+                       pol_out);
+        tma_store_commit();
+      }
+    }
+
+    if (MODE == kState) {
+      // segment aggregate -> fp32 workspace [D][d] then z[D]
+      if (warp_wait(&bar.s_full, 0)) {
+        tc_fence_after();
+        float *dst = out_state + (head * nseg + seg) * (int64_t)(D * D + D);
+#pragma unroll
+        for (int j = 0; j < SC / 16; ++j) {
+          uint32_t r[16];
+          tmem_ld16(tmem + lane_off + kColS + h * SC + 16 * j, r);
+          if (vS) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<float4 *>(dst + (int64_t)rS * D + h * SC + 16 * j + e) =
+                  make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                              __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+          }
+        }
+        const uint32_t zr = tmem_ld1(tmem + lane_off + kColS + D);
+        if (vS && h == 0) dst[(int64_t)D * D + rS] = __uint_as_float(zr);
+      }
+    }
+    if (et == 0) tma_store_wait_all<0>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [heads][n][d] bf16 as a 3-D tensor (d innermost), 64 x 64 boxes, 128-byte swizzle.
+// Rows beyond n read as zero and are never written.
+cudaError_t make_tmap(CUtensorMap *m, const void *ptr, int64_t heads, int64_t n, int d) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)C, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D, int MODE>
+cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                      const CUtensorMap &o, const float *init, int64_t ihs, int64_t iss,
+                      float *out_state, int64_t heads, int64_t n, int64_t seg, int64_t nseg,
+                      int *err, cudaStream_t st) {
+  using G = Cfg<D, MODE>;
+  auto kern = tc_kernel<D, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)(heads * nseg), kThreads, G::SMEM, st>>>(q, k, v, o, init, ihs, iss, out_state,
+                                                           n, seg, nseg, err);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out, int64_t heads,
+                         int64_t n, int causal, int64_t seg, void *ws, int *err, cudaStream_t st) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  const int64_t per = (int64_t)D * D + D;
+  CUtensorMap tq, tk, tv, to;
+  cudaError_t e;
+  if ((e = make_tmap(&tq, q, heads, n, D)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
+  if ((e = make_tmap(&to, out, heads, n, D)) != cudaSuccess) return e;
+  float *w = static_cast<float *>(ws);
+  e = launch_tc<D, kState>(tq, tk, tv, to, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
+  if (e != cudaSuccess) return e;
+  if (causal) {
+    e = launch_scan_states(w, heads, nseg, D, 0, nullptr, 0, nullptr, 0, st);
+    if (e != cudaSuccess) return e;
+    return launch_tc<D, kCausalOut>(tq, tk, tv, to, w, nseg * per, per, nullptr, heads, n, seg,
+                                    nseg, err, st);
+  }
+  // per-head totals, packed as [heads][D*D + D] (S row-major, then z)
+  float *tot = w + heads * nseg * per;
+  e = launch_scan_states(w, heads, nseg, D, 1, tot, per, tot + (int64_t)D * D, per, st);
+  if (e != cudaSuccess) return e;
+  return launch_tc<D, kNoncausalOut>(tq, tk, tv, to, tot, per, 0, nullptr, heads, n, seg, nseg,
+                                     err, st);
+}
+
+}  // namespace
+
+int64_t tc_default_segment(int64_t heads, int64_t n, int d) {
+  (void)d;
+  // smallest tail loss over whole waves of 148 SMs (one CTA each), preferring long segments
+  const int64_t sms = 148;
+  int64_t best = 64, best_score = -1;
+  for (int64_t seg = 4096; seg >= 256; seg -= 256) {
+    const int64_t nseg = (n + seg - 1) / seg;
+    const int64_t ctas = heads * nseg;
+    const int64_t waves = (ctas + sms - 1) / sms;
+    // efficiency in 1/1000 units; prefer longer segments on ties
+    const int64_t eff = ctas * 1000 / (waves * sms);
+    if (eff > best_score + 30 || (best_score < 0)) {
+      best_score = eff;
+      best = seg;
+    }
+  }
+  const int64_t nrounded = ((n + C - 1) / C) * C;
+  return best > nrounded ? nrounded : best;
+}
+
+size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int causal) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  const int64_t per = (int64_t)d * d + d;
+  return (size_t)(heads * nseg * per + (causal ? 0 : heads * per)) * sizeof(float);
+}
+
+cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
+                       int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
+                       cudaStream_t st) {
+  return d == 64 ? tc_forward_d<64>(q, k, v, out, heads, n, causal, seg, ws, err, st)
+                 : tc_forward_d<128>(q, k, v, out, heads, n, causal, seg, ws, err, st);
+}
+
+template <int D>
+cudaError_t tc_state_d(const void *k, const void *v, float *S_out, float *z_out, int64_t heads,
+                       int64_t n, int64_t seg, void *ws, int *err, cudaStream_t st) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  CUtensorMap tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
+  float *w = static_cast<float *>(ws);
+  e = launch_tc<D, kState>(tk, tk, tv, tv, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
+  if (e != cudaSuccess) return e;
+  return launch_scan_states(w, heads, nseg, D, 1, S_out, (int64_t)D * D, z_out, D, st);
+}
+
+cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
+                             int64_t heads, int64_t n, int d, int64_t seg, void *ws, int *err,
+                             cudaStream_t st) {
+  return d == 64 ? tc_state_d<64>(k, v, S_out, z_out, heads, n, seg, ws, err, st)
+                 : tc_state_d<128>(k, v, S_out, z_out, heads, n, seg, ws, err, st);
+}
+
+}  // namespace linattn

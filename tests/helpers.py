@@ -8,6 +8,10 @@ import numpy as np
 from linear_attention_linattn_b200 import inputs
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
+# States from bf16 I/O: the tensor-core path multiplies bf16-rounded phi(k) (relative
+# rounding 2^-9 per element), so the fp32 state carries ~2e-3 relative error; the bar is
+# the per-(sequence, head) Frobenius relative error.
+STATE_TOL_BF16 = 1e-2
 
 
 def max_row_rel_err(got, ref) -> float:

@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 from linear_attention_linattn_b200 import inputs
-from tests.helpers import TOL, max_row_rel_err, to_dev, to_host
+from tests.helpers import STATE_TOL_BF16, TOL, max_row_rel_err, to_dev, to_host
 
 torch = pytest.importorskip("torch")
 la = pytest.importorskip("linear_attention_linattn_b200")
@@ -60,9 +60,10 @@ def test_decode_replay_equals_causal_forward(d):
     ref = oracle.forward(q, k, v, True)
     assert max_row_rel_err(rep, ref) <= TOL["bf16"]
     assert max_row_rel_err(rep, fwd) <= 2 * TOL["bf16"]
-    # the state left by the replay is the forward_state of the same tokens
+    # the state left by the replay is the forward_state of the same tokens (the bf16
+    # forward_state rounds phi(k) to bf16 for the tensor cores: STATE_TOL_BF16)
     S2, z2 = la.forward_state(kd, vd)
-    assert _state_err(to_host(S), to_host(S2)) <= 1e-5
+    assert _state_err(to_host(S), to_host(S2)) <= STATE_TOL_BF16
 
 
 def test_workload_decode_256x32x128():
@@ -92,4 +93,5 @@ def test_workload_decode_256x32x128():
     for t in range(T):
         S_ref, z_ref, ref[t] = oracle.decode_step(S_ref, z_ref, sq[t], sk[t], sv[t])
     assert max_row_rel_err(to_host(outs), ref) <= TOL["bf16"]
-    assert _state_err(to_host(S[idx_s, idx_h]), S_ref) <= 1e-4
+    # the starting state came from the bf16 tensor-core prefill
+    assert _state_err(to_host(S[idx_s, idx_h]), S_ref) <= STATE_TOL_BF16
