@@ -148,9 +148,16 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_heads(B: int, H: int, rank: int):
+    """(batch, head) pairs rank `rank` owns: batch elements [rank*B, (rank+1)*B) of the
+    global batch (weak scaling: every rank runs one copy of the workload's shape)."""
+    return [(rank * B + b, h) for b in range(B) for h in range(H)]
 
 
 # ------------------------------------------------------------------ timing helpers
@@ -240,14 +247,16 @@ def main_forward(args, world, rank, local):
 
     import linear_attention_linattn_b200 as la
     w = inputs.WORKLOADS[args.workload]
+    if args.max_heads and args.max_heads < w.H:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.max_heads)
     causal = True in w.causal
     dtype = "bf16" if "bf16" in w.dtypes else "f32"
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     elem = 2 if dtype == "bf16" else 4
     # this rank's batch element of the workload: b = rank (weak scaling over ranks)
     q, k, v = inputs.forward_qkv(w.seed, w.B * world, w.H, w.n, w.d, w.scaled,
-                                 heads=[(rank * w.B + b, h) for b in range(w.B)
-                                        for h in range(w.H)])
+                                 heads=rank_heads(w.B, w.H, rank))
     shape = (w.B, w.H, w.n, w.d)
     qh = torch.from_numpy(q.reshape(shape)).to(tdt).pin_memory()
     kh = torch.from_numpy(k.reshape(shape)).to(tdt).pin_memory()
@@ -281,17 +290,21 @@ def main_forward(args, world, rank, local):
         o = la.forward(a, b_, c, causal)
         outh.copy_(o, non_blocking=True)
 
-    e2e_steps = max(1, min(args.steps, 3))
-    e2e_ms, _ = time_steps(e2e_step, e2e_steps, 1, world)
-    e2e = {"value": tokens_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-           "h2d_bytes_per_step": 3 * qh.numel() * elem, "d2h_bytes_per_step": outh.numel() * elem}
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 3))
+        e2e_ms, _ = time_steps(e2e_step, e2e_steps, 1, world)
+        e2e = {"value": tokens_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": 3 * qh.numel() * elem,
+               "d2h_bytes_per_step": outh.numel() * elem}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
         "data": "synthetic (seeded N(0,1)/sqrt(d), see DESIGN.md input recipe)",
-        "config": {"workload": args.workload, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+        "config": {"workload": args.workload + (f" (first {w.H} heads)" if args.max_heads else ""),
+                   "B": w.B, "H": w.H, "n": w.n, "d": w.d,
                    "causal": causal, "global_batch": w.B * world, "seq_len": w.n,
                    "parallelism": f"dp{world} (independent heads, no collective)",
                    "l2": "inputs larger than L2 (no flush needed)"},
@@ -372,6 +385,9 @@ def main():
                                                          if w.kind == "forward"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--max-heads", type=int, default=0,
+                    help="profiling aid: run only the first N heads of the workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

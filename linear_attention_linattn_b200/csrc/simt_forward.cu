@@ -115,15 +115,24 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
   const int64_t e = (blockIdx.x % blocks_per_head) * (int64_t)blockDim.x + threadIdx.x;
   if (e >= per) return;
   float *base = ws + head * nseg * per + e;
+  constexpr int kBatch = 16;  // independent loads in flight per thread
   float run = 0.f;
-  if (mode == 0) {
-    for (int64_t s = 0; s < nseg; ++s) {
-      const float x = base[s * per];
-      base[s * per] = run;
-      run += x;
+  for (int64_t s0 = 0; s0 < nseg; s0 += kBatch) {
+    float x[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) x[i] = s0 + i < nseg ? base[(s0 + i) * per] : 0.f;
+    if (mode == 0) {
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        if (s0 + i < nseg) base[(s0 + i) * per] = run;
+        run += x[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) run += x[i];
     }
-  } else {
-    for (int64_t s = 0; s < nseg; ++s) run += base[s * per];
+  }
+  if (mode != 0) {
     if (e < (int64_t)d * d)
       S_out[head * S_hs + e] = run;
     else

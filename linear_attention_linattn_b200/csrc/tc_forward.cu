@@ -25,14 +25,16 @@
 // The normaliser rides along as a 16-column block whose first column is z (or ones), so the
 // numerator and the denominator see the same rounded weights.
 //
-// Warp roles (448 threads, one CTA per SM):
+// Warp roles (576 threads, one CTA per SM):
 //   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of Q/K/V chunks into a
 //              ring of stages; no multicast.
 //   warp 1     TMEM allocation and the single MMA-issuing thread.
-//   warps 2-5  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
-//              n zeroed, then handed to the tensor cores.
-//   warps 6-13 TMEM epilogue: mask and round P, round S_<c+1 and z into the next chunk's
-//              operands, divide O by its denominator and TMA-store the output tile.
+//   warps 2-9  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
+//              n zeroed, then handed to the tensor cores (two warps per SM sub-partition:
+//              the exponentials are the busiest part of the kernel).
+//   warps 10-13 conversion: mask and round P; round S_<c+1 and z into the next chunk's
+//              operands; the starting state; the segment aggregate.
+//   warps 14-17 output: divide O by its denominator and TMA-store the bf16 tile.
 // Every wait is bounded (2 s); a wait that gives up records LINATTN_ERR_TIMEOUT and the
 // CTA drains and exits without trapping.
 #include <cuda.h>
@@ -55,19 +57,25 @@ enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
 constexpr int kWarpTMA = 0;
 constexpr int kWarpMMA = 1;
 constexpr int kWarpXform0 = 2;
-constexpr int kNumXformWarps = 4;
-constexpr int kWarpEpi0 = kWarpXform0 + kNumXformWarps;  // 6
-constexpr int kNumEpiWarps = 8;
-constexpr int kThreads = (kWarpEpi0 + kNumEpiWarps) * 32;  // 448
+constexpr int kNumXformWarps = 8;
+constexpr int kWarpConv0 = kWarpXform0 + kNumXformWarps;  // 10: P and S conversion group
+constexpr int kWarpOut0 = kWarpConv0 + 4;                 // 14: output group
+constexpr int kThreads = (kWarpOut0 + 4) * 32;             // 576
 constexpr int kXformThreads = kNumXformWarps * 32;
-constexpr int kEpiThreads = kNumEpiWarps * 32;
+constexpr int kGroupThreads = 128;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr uint32_t kTmemCols = 512;
 
-// TMEM column map.
-constexpr uint32_t kColP = 0;    // P: 64 columns
-constexpr uint32_t kColO = 64;   // O: d columns, then the 16-column denominator block
-constexpr uint32_t kColS = 256;  // S: d columns, then the 16-column z block
+// TMEM column map: P (64 columns), two O buffers and S, each of the last three being d value
+// columns followed by a 16-column block whose first column is the denominator / z.
+constexpr uint32_t kColP = 0;
+template <int D>
+struct TmemMap {
+  static constexpr uint32_t O0 = 64;
+  static constexpr uint32_t O1 = O0 + D + 16;
+  static constexpr uint32_t S = O1 + D + 16;
+  static_assert(S + D + 16 <= kTmemCols, "TMEM budget");
+};
 
 template <int D, int MODE>
 struct Cfg {
@@ -76,11 +84,11 @@ struct Cfg {
   static constexpr bool LQ = MODE != kState;
   static constexpr bool LKV = MODE != kNoncausalOut;
   static constexpr int STAGE = TILE * ((LQ ? 1 : 0) + (LKV ? 2 : 0));
-  static constexpr int S_BYTES = A * D * 128;  // bf16 S, MN-major [A][D rows][128 B]
-  static constexpr int Z_BYTES = A * kZAtom;   // bf16 [16][D], K-major, row 0 = z
-  static constexpr int ONES_BYTES = kZAtom;    // bf16 [16][64], K-major, row 0 = 1
-  static constexpr int P_BYTES = kAtom;        // bf16 [64][64], K-major
-  static constexpr int OUT_BYTES = TILE;       // bf16 output staging, TMA-store layout
+  static constexpr int S_BYTES = MODE == kState ? 0 : A * D * 128;  // bf16 S, MN-major
+  static constexpr int Z_BYTES = MODE == kState ? 0 : A * kZAtom;   // bf16 [16][D], row 0 = z
+  static constexpr int ONES_BYTES = kZAtom;                         // bf16 [16][64], row 0 = 1
+  static constexpr int P_BYTES = MODE == kCausalOut ? kAtom : 0;    // bf16 [64][64], K-major
+  static constexpr int OUT_BYTES = MODE == kState ? 0 : 2 * TILE;   // two output staging tiles
   static constexpr int FIXED = S_BYTES + Z_BYTES + ONES_BYTES + P_BYTES + OUT_BYTES;
   static constexpr int BAR_BYTES = 512;
   static constexpr int NS_FIT = (kMaxSmem - 1024 - BAR_BYTES - FIXED) / STAGE;
@@ -102,7 +110,7 @@ struct Cfg {
 
 struct Bars {
   uint64_t full[8], ready[8], empty[8];
-  uint64_t p_full, p_ready, s_full, s_ready, o_full, o_empty, fin;
+  uint64_t p_full, p_ready, s_full, s_ready, o_full[2], o_empty[2], fin;
   uint32_t tmem_base;
   int abort;
 };
@@ -119,9 +127,51 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks, uint32_t
   return make_sw128_desc(base + ks * 2048, lbo, 1024);
 }
 
+// phi on two packed bf16 values: exp(min(x, 0)) + max(x, 0), which is x + 1 above zero and
+// exp(x) at or below zero.  Everything is packed bf16 arithmetic:
+//   t = min(x, 0) * log2(e), with log2(e) split into a bf16 head and tail so that the product
+//       is rounded once (fma of the head onto the tail's product);
+//   e = 2^t with the packed bf16 exponential (one MUFU operation for two elements);
+//   phi = e + max(x, 0)  (above zero e = 1 exactly, so this is 1 + x rounded once).
+// The bf16 rounding of t perturbs exp(x) by at most |x| * 2^-9 relative; over the sums of
+// the method this stays far below the bf16 I/O tolerance (modelled and tested).
 __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t u) {
-  return pack_bf16x2(phi_fast(bf16_lo(u)), phi_fast(bf16_hi(u)));
+  const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&u);
+  const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+  const __nv_bfloat162 log2e_hi = __float2bfloat162_rn(1.4453125f);          // bf16(log2 e)
+  const __nv_bfloat162 log2e_lo = __float2bfloat162_rn(-0.0026174592f);      // log2 e - head
+  const __nv_bfloat162 m = __hmin2(x, zero);
+  const __nv_bfloat162 p = __hmax2(x, zero);
+  const __nv_bfloat162 t = __hfma2(m, log2e_hi, __hmul2(m, log2e_lo));
+  uint32_t e;
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(*reinterpret_cast<const uint32_t *>(&t)));
+  const __nv_bfloat162 r = __hadd2(*reinterpret_cast<const __nv_bfloat162 *>(&e), p);
+  return *reinterpret_cast<const uint32_t *>(&r);
 }
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+  uint4 u;
+  u.x = pack_bf16x2(f[0], f[1]);
+  u.y = pack_bf16x2(f[2], f[3]);
+  u.z = pack_bf16x2(f[4], f[5]);
+  u.w = pack_bf16x2(f[6], f[7]);
+  return u;
+}
+
+// Lane-0 mbarrier wait whose outcome the whole warp shares (warp-uniform control flow).
+struct WarpWaiter {
+  volatile int *abort;
+  int *err;
+  int lane;
+  bool ok = true;
+  __device__ __forceinline__ bool operator()(uint64_t *b, uint32_t parity) {
+    int r = 1;
+    if (lane == 0) r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
+    r = __shfl_sync(0xffffffffu, r, 0);
+    ok = ok && (r != 0);
+    return ok;
+  }
+};
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -131,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               int64_t init_seg_stride, float *__restrict__ out_state, int64_t n, int64_t seg_len,
               int64_t nseg, int *err) {
   using G = Cfg<D, MODE>;
+  using TM = TmemMap<D>;
   constexpr int NS = G::NS;
   constexpr int KSD = D / 16;  // K-steps over the feature dimension
   constexpr int KSC = C / 16;  // K-steps over the chunk's tokens
@@ -156,11 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.empty[s], 1);
     }
     mbar_init(&bar.p_full, 1);
-    mbar_init(&bar.p_ready, kEpiThreads);
+    mbar_init(&bar.p_ready, kGroupThreads);
     mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.s_ready, kEpiThreads);
-    mbar_init(&bar.o_full, 1);
-    mbar_init(&bar.o_empty, kEpiThreads);
+    mbar_init(&bar.s_ready, kGroupThreads);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.o_full[b], 1);
+      mbar_init(&bar.o_empty[b], kGroupThreads);
+    }
     mbar_init(&bar.fin, 1);
     bar.abort = 0;
     fence_barrier_init();
@@ -206,12 +259,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int zc = static_cast<int>(head);
         if (G::LQ) {
 #pragma unroll
-          for (int a = 0; a < G::A; ++a) tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
+          for (int a = 0; a < G::A; ++a)
+            tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
           st += G::TILE;
         }
         if (G::LKV) {
 #pragma unroll
-          for (int a = 0; a < G::A; ++a) tma_load_3d(st + a * kAtom, &tmK, &bar.full[s], a * 64, y, zc, pol);
+          for (int a = 0; a < G::A; ++a)
+            tma_load_3d(st + a * kAtom, &tmK, &bar.full[s], a * 64, y, zc, pol);
 #pragma unroll
           for (int a = 0; a < G::A; ++a)
             tma_load_3d(st + G::TILE + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
@@ -230,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t I_DEN = make_idesc_bf16(64, 16, false, false);
       constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);
       constexpr uint32_t I_Z = make_idesc_bf16(D, 16, true, false);
-      const uint32_t tP = tmem + kColP, tO = tmem + kColO, tOd = tmem + kColO + D;
-      const uint32_t tS = tmem + kColS, tSz = tmem + kColS + D;
+      const uint32_t tP = tmem + kColP;
+      const uint32_t tS = tmem + TM::S, tSz = tmem + TM::S + D;
       const uint32_t sS = smem_u32(smem + G::OFF_S), sZ = smem_u32(smem + G::OFF_Z);
       const uint32_t sOnes = smem_u32(smem + G::OFF_ONES), sP = smem_u32(smem + G::OFF_P);
       for (int c = 0; c < nchunks; ++c) {
@@ -242,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sQ = st;
         const uint32_t sK = st + (G::LQ ? G::TILE : 0);
         const uint32_t sV = sK + G::TILE;
+        tc_fence_after();
         if (MODE == kState) {
-          tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < KSC; ++ks) {
             const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
@@ -254,18 +309,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bar.empty[s]);
           continue;
         }
-        // S_<c and z_<c are in shared memory; O is free again
-        if (MODE == kCausalOut || c == 0)
-          if (!mbar_wait(&bar.s_ready, MODE == kCausalOut ? (c & 1) : 0, abort, err)) break;
-        if (c > 0 && !mbar_wait(&bar.o_empty, (c - 1) & 1, abort, err)) break;
-        tc_fence_after();
+        const int ob = c & 1;
+        const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0), tOd = tO + D;
         if (MODE == kCausalOut) {
+          // scores of this chunk first: the conversion warps can start on them at once
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tP, desc_kmajor(sQ, ks, kAtom), desc_kmajor(sK, ks, kAtom), I_P,
                         ks > 0 ? 1u : 0u);
           mma_commit(&bar.p_full);
         }
+        // S_<c, z_<c in shared memory; this O buffer drained
+        if (MODE == kCausalOut || c == 0)
+          if (!mbar_wait(&bar.s_ready, MODE == kCausalOut ? (c & 1) : 0, abort, err)) break;
+        if (c >= 2 && !mbar_wait(&bar.o_empty[ob], ((c >> 1) - 1) & 1, abort, err)) break;
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < KSD; ++ks) {
           const uint64_t a = desc_kmajor(sQ, ks, kAtom);
@@ -289,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ss(tOd, a, desc_kmajor(sOnes, ks, kZAtom), I_DEN, 1u);
           }
         }
-        mma_commit(&bar.o_full);
+        mma_commit(&bar.o_full[ob]);
         mma_commit(&bar.empty[s]);
       }
       if (MODE == kState) mma_commit(&bar.s_full);
@@ -297,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bar.fin);
       mbar_wait(&bar.fin, 0, abort, err);
     }
-  } else if (warp < kWarpEpi0) {
+  } else if (warp < kWarpConv0) {
     // ================================================================ feature map
     const int xt = threadIdx.x - kWarpXform0 * 32;
     for (int c = 0; c < nchunks; ++c) {
@@ -308,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int valid = left < C ? static_cast<int>(left) : C;
       if (G::LQ) {
         uint4 *p = reinterpret_cast<uint4 *>(st);
+#pragma unroll 2
         for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
           uint4 x = p[i];
           x.x = phi_bf16x2(x.x);
@@ -320,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (G::LKV) {
         uint4 *p = reinterpret_cast<uint4 *>(st);
+#pragma unroll 2
         for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
           const int row = (i % (kAtom / 16)) >> 3;  // 8 x 16 B per 128-byte row
           uint4 x = make_uint4(0u, 0u, 0u, 0u);
@@ -336,116 +396,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&bar.ready[s]);
     }
-  } else {
-    // ================================================================ TMEM epilogue
-    // Control flow is uniform across the 8 warps: lane 0 of each warp does the mbarrier
-    // waits and broadcasts the outcome, and after a give-up the loop still runs through every
-    // named barrier (doing no work), so no warp is ever left at a barrier alone.
-    const int et = threadIdx.x - kWarpEpi0 * 32;  // 0..255
-    const int sp = warp & 3;                      // TMEM sub-partition of this warp
-    const int h = (warp - kWarpEpi0) >> 2;        // which half of the columns
+  } else if (warp < kWarpOut0) {
+    // ================================================================ conversion group
+    // P -> masked bf16 operand; S_<c+1, z_<c+1 -> bf16 operands of the next chunk; the
+    // starting state; the segment aggregate (state mode).  Control flow is warp-uniform:
+    // lane 0 waits and the warp shares the outcome.
+    const int sp = warp & 3;  // TMEM sub-partition of this warp
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
-    const bool v64 = lane < 16;                   // lanes holding rows of an M=64 tile
-    const int r64 = 16 * sp + lane;               // row of an M=64 tile
+    const bool v64 = lane < 16;                      // lanes holding rows of an M=64 tile
+    const int r64 = 16 * sp + lane;                  // row of an M=64 tile
     const int rS = D == 128 ? 32 * sp + lane : r64;  // row of the S accumulator (M = D)
     const bool vS = D == 128 ? true : v64;
-    constexpr int SC = D / 2;  // S / O columns per thread (one half)
+    WarpWaiter wait{abort, err, lane};
     uint8_t *sS = smem + G::OFF_S;
     uint8_t *sZ = smem + G::OFF_Z;
-    bool ok = true;
-    auto warp_wait = [&](uint64_t *b, uint32_t parity) {
-      int r = 1;
-      if (lane == 0) r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
-      r = __shfl_sync(0xffffffffu, r, 0);
-      ok = ok && (r != 0);
-      return ok;
-    };
 
-    // S (fp32 values in registers) -> bf16 MN-major operand, z -> z block row 0
-    auto store_S_operand = [&](const float *vals, float zval) {
+    // 32 consecutive S columns [c0, c0+32) of row rS (fp32 in registers) -> bf16 operand
+    auto store_S32 = [&](const uint32_t *r, int c0) {
       if (!vS) return;
 #pragma unroll
-      for (int j = 0; j < SC / 8; ++j) {
-        const int col = h * SC + 8 * j;  // first of 8 columns
-        uint4 u;
-        u.x = pack_bf16x2(vals[8 * j + 0], vals[8 * j + 1]);
-        u.y = pack_bf16x2(vals[8 * j + 2], vals[8 * j + 3]);
-        u.z = pack_bf16x2(vals[8 * j + 4], vals[8 * j + 5]);
-        u.w = pack_bf16x2(vals[8 * j + 6], vals[8 * j + 7]);
-        uint8_t *dst = sS + (col >> 6) * (D * 128) + sw128_offset(rS, col & 63);
-        *reinterpret_cast<uint4 *>(dst) = u;
+      for (int j = 0; j < 4; ++j) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * j + e]);
+        *reinterpret_cast<uint4 *>(sS + (c0 >> 6) * (D * 128) +
+                                   sw128_offset(rS, (c0 & 63) + 8 * j)) = pack8(f);
       }
-      if (h == 0) {
-        const __nv_bfloat16 zb = __float2bfloat16_rn(zval);
-        *reinterpret_cast<__nv_bfloat16 *>(sZ + (rS >> 6) * kZAtom + sw128_offset(0, rS & 63)) =
-            zb;
-      }
+    };
+    auto store_z = [&](uint32_t zbits) {
+      if (!vS) return;
+      *reinterpret_cast<__nv_bfloat16 *>(sZ + (rS >> 6) * kZAtom + sw128_offset(0, rS & 63)) =
+          __float2bfloat16_rn(__uint_as_float(zbits));
     };
 
     if (MODE != kState) {
       // starting state: exclusive prefix (causal) or the head's total (non-causal)
       const float *src = init_state + head * init_head_stride + seg * init_seg_stride;
-      float vals[SC];
-      float zval = 0.f;
-      if (vS) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
 #pragma unroll
-        for (int j = 0; j < SC / 4; ++j) {
-          const float4 f =
-              *reinterpret_cast<const float4 *>(src + (int64_t)rS * D + h * SC + 4 * j);
-          vals[4 * j + 0] = f.x;
-          vals[4 * j + 1] = f.y;
-          vals[4 * j + 2] = f.z;
-          vals[4 * j + 3] = f.w;
+        for (int j = 0; j < 8; ++j) {
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (vS) f = *reinterpret_cast<const float4 *>(src + (int64_t)rS * D + c0 + 4 * j);
+          r[4 * j + 0] = __float_as_uint(f.x);
+          r[4 * j + 1] = __float_as_uint(f.y);
+          r[4 * j + 2] = __float_as_uint(f.z);
+          r[4 * j + 3] = __float_as_uint(f.w);
         }
-        zval = src[(int64_t)D * D + rS];
-      } else {
+        if (MODE == kCausalOut) {
 #pragma unroll
-        for (int j = 0; j < SC; ++j) vals[j] = 0.f;
+          for (int j = 0; j < 2; ++j)
+            tmem_st16(tmem + lane_off + TM::S + c0 + 16 * j,
+                      *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * j));
+        }
+        store_S32(r, c0);
       }
+      const uint32_t zb = vS ? __float_as_uint(src[(int64_t)D * D + rS]) : 0u;
       if (MODE == kCausalOut) {
-        // the running state starts from the prefix: write it into the S accumulator
-#pragma unroll
-        for (int j = 0; j < SC / 16; ++j) {
-          uint32_t r[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(vals[16 * j + e]);
-          tmem_st16(tmem + lane_off + kColS + h * SC + 16 * j, r);
-        }
-        if (h == 0) tmem_st1(tmem + lane_off + kColS + D, __float_as_uint(zval));
+        tmem_st1(tmem + lane_off + TM::S + D, zb);
         tmem_st_wait();
       }
-      store_S_operand(vals, zval);
+      store_z(zb);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar.s_ready);
     }
 
-    const uint64_t pol_out = policy_evict_first();
-    for (int c = 0; c < (MODE == kState ? 0 : nchunks); ++c) {
-      if (MODE == kCausalOut) {
+    if (MODE == kCausalOut) {
+      for (int c = 0; c < nchunks; ++c) {
         // ---- P: mask j <= i, round to bf16, K-major A operand of P V
-        if (warp_wait(&bar.p_full, c & 1)) {
+        if (wait(&bar.p_full, c & 1)) {
           tc_fence_after();
-          uint32_t p0[16], p1[16];
-          tmem_ld16(tmem + lane_off + kColP + 32 * h, p0);
-          tmem_ld16(tmem + lane_off + kColP + 32 * h + 16, p1);
-          if (v64) {
-            uint8_t *sP = smem + G::OFF_P;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float f[8];
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t p[32];
+            tmem_ld16_async(tmem + lane_off + kColP + c0, p);
+            tmem_ld16_async(tmem + lane_off + kColP + c0 + 16, p + 16);
+            tmem_ld_wait();
+            tmem_reg_fence<32>(p);
+            if (v64) {
+              uint8_t *sP = smem + G::OFF_P;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int col = 32 * h + 8 * j + e;
-                const uint32_t bits = (8 * j + e) < 16 ? p0[8 * j + e] : p1[8 * j + e - 16];
-                f[e] = col <= r64 ? __uint_as_float(bits) : 0.f;
+              for (int j = 0; j < 4; ++j) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  f[e] = (c0 + 8 * j + e) <= r64 ? __uint_as_float(p[8 * j + e]) : 0.f;
+                *reinterpret_cast<uint4 *>(sP + sw128_offset(r64, c0 + 8 * j)) = pack8(f);
               }
-              uint4 u;
-              u.x = pack_bf16x2(f[0], f[1]);
-              u.y = pack_bf16x2(f[2], f[3]);
-              u.z = pack_bf16x2(f[4], f[5]);
-              u.w = pack_bf16x2(f[6], f[7]);
-              *reinterpret_cast<uint4 *>(sP + sw128_offset(r64, 32 * h + 8 * j)) = u;
             }
           }
           fence_proxy_async_smem();
@@ -453,90 +491,101 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&bar.p_ready);
         }
         // ---- S_<c+1, z_<c+1: the operands of the next chunk
-        if (warp_wait(&bar.s_full, c & 1)) {
+        if (c + 1 < nchunks && wait(&bar.s_full, c & 1)) {
           tc_fence_after();
-          float vals[SC];
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
 #pragma unroll
-          for (int j = 0; j < SC / 16; ++j) {
-            uint32_t r[16];
-            tmem_ld16(tmem + lane_off + kColS + h * SC + 16 * j, r);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) vals[16 * j + e] = __uint_as_float(r[e]);
+            for (int j = 0; j < 2; ++j)
+              tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * j, r + 16 * j);
+            tmem_ld_wait();
+            tmem_reg_fence<32>(r);
+            store_S32(r, c0);
           }
-          const float zval = __uint_as_float(tmem_ld1(tmem + lane_off + kColS + D));
-          store_S_operand(vals, zval);
+          store_z(tmem_ld1(tmem + lane_off + TM::S + D));
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bar.s_ready);
         }
       }
-
-      // ---- O / den -> bf16 output tile -> TMA store
-      float o[SC];
-      float inv = 0.f;
-      if (warp_wait(&bar.o_full, c & 1)) {
-        tc_fence_after();
-#pragma unroll
-        for (int j = 0; j < SC / 16; ++j) {
-          uint32_t r[16];
-          tmem_ld16(tmem + lane_off + kColO + h * SC + 16 * j, r);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[16 * j + e] = __uint_as_float(r[e]);
-        }
-        inv = 1.f / __uint_as_float(tmem_ld1(tmem + lane_off + kColO + D));
-        tc_fence_before();
-        mbar_arrive(&bar.o_empty);
-      }
-      if (et == 0) tma_store_wait_read<0>();  // the staging tile is free again
-      named_barrier_sync(1, kEpiThreads);
-      if (ok && v64) {
-        uint8_t *so = smem + G::OFF_OUT;
-#pragma unroll
-        for (int j = 0; j < SC / 8; ++j) {
-          const int col = h * SC + 8 * j;
-          uint4 u;
-          u.x = pack_bf16x2(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-          u.y = pack_bf16x2(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-          u.z = pack_bf16x2(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-          u.w = pack_bf16x2(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
-          *reinterpret_cast<uint4 *>(so + (col >> 6) * kAtom + sw128_offset(r64, col & 63)) = u;
-        }
-      }
-      fence_proxy_async_smem();
-      named_barrier_sync(1, kEpiThreads);
-      if (et == 0 && !*abort) {
-        const int y = static_cast<int>(t_begin + (int64_t)c * C);
-#pragma unroll
-        for (int a = 0; a < G::A; ++a)
-          tma_store_3d(&tmO, smem + G::OFF_OUT + a * kAtom, a * 64, y, static_cast<int>(head),
-                       pol_out);
-        tma_store_commit();
-      }
     }
 
     if (MODE == kState) {
       // segment aggregate -> fp32 workspace [D][d] then z[D]
-      if (warp_wait(&bar.s_full, 0)) {
+      if (wait(&bar.s_full, 0)) {
         tc_fence_after();
         float *dst = out_state + (head * nseg + seg) * (int64_t)(D * D + D);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
 #pragma unroll
-        for (int j = 0; j < SC / 16; ++j) {
-          uint32_t r[16];
-          tmem_ld16(tmem + lane_off + kColS + h * SC + 16 * j, r);
+          for (int j = 0; j < 2; ++j)
+            tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * j, r + 16 * j);
+          tmem_ld_wait();
+          tmem_reg_fence<32>(r);
           if (vS) {
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              *reinterpret_cast<float4 *>(dst + (int64_t)rS * D + h * SC + 16 * j + e) =
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(dst + (int64_t)rS * D + c0 + e) =
                   make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
                               __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
           }
         }
-        const uint32_t zr = tmem_ld1(tmem + lane_off + kColS + D);
-        if (vS && h == 0) dst[(int64_t)D * D + rS] = __uint_as_float(zr);
+        const uint32_t zr = tmem_ld1(tmem + lane_off + TM::S + D);
+        if (vS) dst[(int64_t)D * D + rS] = __uint_as_float(zr);
       }
     }
-    if (et == 0) tma_store_wait_all<0>();
+  } else {
+    // ================================================================ output group
+    // O / den -> bf16 tile in a double-buffered staging area -> TMA store.
+    const int sp = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
+    const bool v64 = lane < 16;
+    const int r64 = 16 * sp + lane;
+    const int ot = threadIdx.x - kWarpOut0 * 32;  // 0..127
+    WarpWaiter wait{abort, err, lane};
+    const uint64_t pol_out = policy_evict_first();
+    for (int c = 0; c < (MODE == kState ? 0 : nchunks); ++c) {
+      const int ob = c & 1;
+      const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
+      uint8_t *so = smem + G::OFF_OUT + ob * G::TILE;
+      if (ot == 0) tma_store_wait_read<1>();  // the store that last used this buffer is done
+      named_barrier_sync(1, kGroupThreads);
+      if (wait(&bar.o_full[ob], (c >> 1) & 1)) {
+        tc_fence_after();
+        const float inv = 1.f / __uint_as_float(tmem_ld1(tO + D));
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) tmem_ld16_async(tO + c0 + 16 * j, r + 16 * j);
+          tmem_ld_wait();
+          tmem_reg_fence<32>(r);
+          if (v64) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * j + e]) * inv;
+              *reinterpret_cast<uint4 *>(so + (c0 >> 6) * kAtom +
+                                         sw128_offset(r64, (c0 & 63) + 8 * j)) = pack8(f);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty[ob]);
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1, kGroupThreads);
+      if (ot == 0 && !*abort) {
+        const int y = static_cast<int>(t_begin + (int64_t)c * C);
+#pragma unroll
+        for (int a = 0; a < G::A; ++a)
+          tma_store_3d(&tmO, so + a * kAtom, a * 64, y, static_cast<int>(head), pol_out);
+        tma_store_commit();
+      }
+    }
+    if (ot == 0) tma_store_wait_all<0>();
   }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
