@@ -126,6 +126,32 @@ int linattn_version(void);
  * every device.  Benchmarks read it before and after a timed region. */
 uint64_t linattn_launch_count(void);
 
+/* Size of the fixed device scratch block behind linattn_forward_noalloc (32 MiB). */
+#define LINATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * linattn_forward for callers that cannot allocate memory (the pages have no counterpart:
+ * this is a deployment variant, not part of the method).  Same arguments, layouts, results
+ * and dtypes as linattn_forward; it calls no cudaMalloc, cudaFree or other allocating
+ * routine.  Its temporary state lives in one fixed block of LINATTN_NOALLOC_SCRATCH_BYTES
+ * of device memory that the library declares statically; every GPU that loads the library
+ * holds that block until the process exits.
+ *   - Work that needs more temporary state than the block holds is rejected with
+ *     LINATTN_ERR_INVALID_ARG before anything is launched (the bf16 path first lengthens
+ *     its segments to fit; it needs 66,048 B per head and segment at d = 128, 16,640 B at
+ *     d = 64; the fp32 path needs that per 64-token chunk).
+ *   - All calls on a device share the block and leave their contents in it; nothing in it
+ *     needs to start at zero.  Calls that overlap on the GPU race on it: issue them on one
+ *     stream or otherwise order them.
+ *   - The first call on each device looks up the block's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - A kernel wait that gives up is recorded in the block's first word, not in the word
+ *     linattn_device_error() reads.
+ */
+linattn_status linattn_forward_noalloc(const void *q, const void *k, const void *v, void *out,
+                                       int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                       linattn_dtype dtype, linattn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

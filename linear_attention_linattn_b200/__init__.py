@@ -9,7 +9,7 @@ raises.
 Raw C entry points (pointers as ints):
     linattn_forward, linattn_forward_ex, linattn_forward_state, linattn_decode_step,
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
-    linattn_launch_count
+    linattn_launch_count, linattn_forward_noalloc
 
 Tensor helpers: ``forward``, ``forward_state``, ``decode_step``, ``device_error``.
 """
@@ -45,6 +45,8 @@ SIGNATURES = {
     "linattn_device_error": (ctypes.c_int, [_vp]),
     "linattn_version": (ctypes.c_int, []),
     "linattn_launch_count": (ctypes.c_uint64, []),
+    "linattn_forward_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                               ctypes.c_int, ctypes.c_int, _vp]),
 }
 
 _lib = None
