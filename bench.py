@@ -320,6 +320,50 @@ def main_forward(args, world, rank, local):
     return line
 
 
+def main_decode(args, world, rank, local):
+    """Decode workload as the timed step: one linattn_decode_step over all states."""
+    import torch
+
+    import linear_attention_linattn_b200 as la
+    from linear_attention_linattn_b200 import workloads
+    w = inputs.WORKLOADS[args.workload]
+    S, z, qs, ks, vs = workloads.decode_inputs(args.workload)
+    T = qs.shape[0]
+    out = torch.empty_like(qs[0])
+    it = [0]
+
+    def step():
+        t = it[0] % T
+        la.decode_step(S, z, qs[t], ks[t], vs[t], out=out)
+        it[0] += 1
+
+    clocks = ClockSampler(local)
+    l0 = la.linattn_launch_count()
+    ms, per = time_steps(step, args.steps, args.warmup, world, clocks=clocks)
+    launches = (la.linattn_launch_count() - l0) // (args.steps + args.warmup) * args.steps
+    clk = clocks.stop()
+    assert la.device_error() == la.LINATTN_OK
+    pk = peaks()
+    alg = decode_bytes(w.B * w.H, w.d)
+    kernel_ms = float(np.mean(per))
+    achieved = alg / (kernel_ms * 1e-3) / 1e9
+    return {
+        "metric": "linear-attention decode-step tokens/sec and achieved HBM GB/s",
+        "value": w.B * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(d), prefill state from linattn_forward_state)",
+        "config": {"workload": args.workload, "Bseq": w.B, "H": w.H, "d": w.d,
+                   "parallelism": f"dp{world} (independent states, no collective)",
+                   "l2": "state (541 MB) larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "peak_source": pk["source"], "algorithmic_bytes": alg,
+                     "kernel": "decode_step_kernel<128>", "kernel_ms": kernel_ms},
+        "gpu_launches": int(launches), "clocks": clk,
+    }
+
+
 def extras(args):
     """Other workloads at N=1: decode, batched forward, small latency cases."""
     import torch
@@ -381,8 +425,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=MAIN, choices=[k for k, w in inputs.WORKLOADS.items()
-                                                         if w.kind == "forward"])
+    ap.add_argument("--workload", default=MAIN, choices=list(inputs.WORKLOADS))
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -401,7 +444,11 @@ def main():
 
     import torch
     torch.cuda.set_device(local)
-    line = main_forward(args, world, rank, local)
+    if inputs.WORKLOADS[args.workload].kind == "decode":
+        line = main_decode(args, world, rank, local)
+        args.no_extras = args.no_cpu_baseline = True
+    else:
+        line = main_forward(args, world, rank, local)
     if world == 1 and rank == 0:
         if not args.no_extras:
             line["extras"] = extras(args)

@@ -32,9 +32,11 @@
 //   warps 2-9  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
 //              n zeroed, then handed to the tensor cores (two warps per SM sub-partition:
 //              the exponentials are the busiest part of the kernel).
-//   warps 10-13 conversion: mask and round P; round S_<c+1 and z into the next chunk's
-//              operands; the starting state; the segment aggregate.
-//   warps 14-17 output: divide O by its denominator and TMA-store the bf16 tile.
+//   warps 10-13 state: round S_<c+1 and z into the next chunk's operands; the starting
+//              state; the segment aggregate.
+//   warps 14-17 scores and output: mask and round P; divide O by its denominator and
+//              TMA-store the bf16 tile.  P and S are drained by different warps, so the
+//              two conversions on each chunk's critical path run side by side.
 // Every wait is bounded (2 s); a wait that gives up records LINATTN_ERR_TIMEOUT and the
 // CTA drains and exits without trapping.
 #include <cuda.h>
@@ -50,7 +52,6 @@ namespace {
 
 constexpr int C = kTcChunk;       // tokens per chunk (64)
 constexpr int kAtom = C * 128;    // one [64 rows][64 bf16] 128B-swizzled atom: 8 KB
-constexpr int kZAtom = 16 * 128;  // one [16 rows][64 bf16] atom: 2 KB
 
 enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
 
@@ -58,73 +59,96 @@ constexpr int kWarpTMA = 0;
 constexpr int kWarpMMA = 1;
 constexpr int kWarpXform0 = 2;
 constexpr int kNumXformWarps = 8;
-constexpr int kWarpConv0 = kWarpXform0 + kNumXformWarps;  // 10: P and S conversion group
-constexpr int kWarpOut0 = kWarpConv0 + 4;                 // 14: output group
-constexpr int kThreads = (kWarpOut0 + 4) * 32;             // 576
+constexpr int kWarpState0 = kWarpXform0 + kNumXformWarps;  // 10: state group
+constexpr int kWarpOut0 = kWarpState0 + 4;                  // 14: scores and output group
+constexpr int kThreads = (kWarpOut0 + 4) * 32;              // 576
 constexpr int kXformThreads = kNumXformWarps * 32;
 constexpr int kGroupThreads = 128;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr uint32_t kTmemCols = 512;
-
-// TMEM column map: P (64 columns), two O buffers and S, each of the last three being d value
-// columns followed by a 16-column block whose first column is the denominator / z.
-constexpr uint32_t kColP = 0;
-template <int D>
-struct TmemMap {
-  static constexpr uint32_t O0 = 64;
-  static constexpr uint32_t O1 = O0 + D + 16;
-  static constexpr uint32_t S = O1 + D + 16;
-  static_assert(S + D + 16 <= kTmemCols, "TMEM budget");
-};
+constexpr int kZRows = 16;  // extra key rows carrying z (row 0) in the causal K tile
 
 template <int D, int MODE>
 struct Cfg {
   static constexpr int A = D / 64;          // 64-column atoms per [64][D] tile
-  static constexpr int TILE = A * kAtom;    // bytes of a bf16 [64][D] tile
+  static constexpr int TILE = A * kAtom;    // bytes of a bf16 [64][D] tile (Q, V)
   static constexpr bool LQ = MODE != kState;
   static constexpr bool LKV = MODE != kNoncausalOut;
-  static constexpr int STAGE = TILE * ((LQ ? 1 : 0) + (LKV ? 2 : 0));
-  static constexpr int S_BYTES = MODE == kState ? 0 : A * D * 128;  // bf16 S, MN-major
-  static constexpr int Z_BYTES = MODE == kState ? 0 : A * kZAtom;   // bf16 [16][D], row 0 = z
-  static constexpr int ONES_BYTES = kZAtom;                         // bf16 [16][64], row 0 = 1
-  static constexpr int P_BYTES = MODE == kCausalOut ? kAtom : 0;    // bf16 [64][64], K-major
-  static constexpr int OUT_BYTES = MODE == kState ? 0 : 2 * TILE;   // two output staging tiles
-  static constexpr int FIXED = S_BYTES + Z_BYTES + ONES_BYTES + P_BYTES + OUT_BYTES;
-  static constexpr int BAR_BYTES = 512;
+  // causal: each K atom carries 16 more rows after the 64 keys; row 64 holds z_<c, so the
+  // score MMA (N = 80) also yields phi(q_i).z_<c in its column 64.
+  static constexpr int KROWS = MODE == kCausalOut ? 64 + kZRows : 64;
+  static constexpr int KATOM = KROWS * 128;
+  static constexpr int KTILE = A * KATOM;
+  // a constant atom after each V tile whose column 0 is 1: the S MMA with N = D + 16 then
+  // also accumulates z = phi(K)^T 1 in its column D.
+  static constexpr int ONES = LKV ? kAtom : 0;
+  static constexpr int OFF_K = LQ ? TILE : 0;
+  static constexpr int OFF_V = OFF_K + (LKV ? KTILE : 0);
+  static constexpr int OFF_ONES = OFF_V + (LKV ? TILE : 0);
+  static constexpr int STAGE = OFF_ONES + ONES;
+  static constexpr int LOAD_BYTES = (LQ ? TILE : 0) + (LKV ? 2 * TILE : 0);
+  // bf16 S operand, MN-major [atoms][D rows][128 B]; non-causal adds an atom whose column 0
+  // is z, so O (N = D + 16) carries phi(q_i).z in its column D.
+  static constexpr int S_ATOMS = MODE == kState ? 0 : (MODE == kNoncausalOut ? A + 1 : A);
+  static constexpr int S_BYTES = S_ATOMS * D * 128;
+  static constexpr int P_BYTES = MODE == kCausalOut ? kAtom : 0;  // bf16 [64][64], K-major
+  static constexpr int FIXED = S_BYTES + P_BYTES;
+  static constexpr int BAR_BYTES = 1024;
   static constexpr int NS_FIT = (kMaxSmem - 1024 - BAR_BYTES - FIXED) / STAGE;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int OFF_STAGES = 0;
   static constexpr int OFF_S = NS * STAGE;
-  static constexpr int OFF_Z = OFF_S + S_BYTES;
-  static constexpr int OFF_ONES = OFF_Z + Z_BYTES;
-  static constexpr int OFF_P = OFF_ONES + ONES_BYTES;
-  static constexpr int OFF_OUT = OFF_P + P_BYTES;
-  static constexpr int OFF_BAR = OFF_OUT + OUT_BYTES;
+  static constexpr int OFF_P = OFF_S + S_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static_assert(NS >= 2, "at least two pipeline stages");
   static_assert(SMEM <= kMaxSmem, "shared memory budget");
-  static_assert(OFF_S % 1024 == 0 && OFF_Z % 1024 == 0 && OFF_ONES % 1024 == 0 &&
-                    OFF_P % 1024 == 0 && OFF_OUT % 1024 == 0 && STAGE % 1024 == 0,
+  static_assert(OFF_S % 1024 == 0 && OFF_P % 1024 == 0 && STAGE % 1024 == 0 &&
+                    OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_ONES % 1024 == 0 &&
+                    KATOM % 1024 == 0,
                 "128B-swizzled operands need 1024-byte alignment");
+};
+
+// TMEM column map (32-column aligned): P (80 columns, causal), two O buffers (D columns,
+// plus the 16-column denominator block in the non-causal mode), S (D + 16 columns, z in
+// column D).
+template <int D, int MODE>
+struct TmemMap {
+  static constexpr uint32_t P = 0;
+  static constexpr uint32_t OW = ((MODE == kNoncausalOut ? D + 16 : D) + 31) / 32 * 32;
+  static constexpr uint32_t O0 = MODE == kCausalOut ? 96 : 0;
+  static constexpr uint32_t O1 = O0 + OW;
+  static constexpr uint32_t S = MODE == kCausalOut ? O1 + OW : 0;  // unused when non-causal
+  static_assert((MODE == kNoncausalOut ? O1 + OW : S + D + 16) <= kTmemCols, "TMEM budget");
 };
 
 struct Bars {
   uint64_t full[8], ready[8], empty[8];
-  uint64_t p_full, p_ready, s_full, s_ready, o_full[2], o_empty[2], fin;
+  uint64_t p_full, p_ready, s_full, s_ready, z_ready, rs_ready, o_full[2], o_empty[2], fin;
+  float rowsum[2][64];  // the state group's half of P's row sums, by chunk parity
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
-// K-major operand descriptor for K-step ks of a [rows][D] tile made of 64-column atoms
-// of `atom_bytes` each: 4 K-steps of 32 bytes inside one 128-byte swizzle row.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int ks, uint32_t atom_bytes) {
-  return make_sw128_desc(base + (ks >> 2) * atom_bytes + (ks & 3) * 32, 16, 1024);
+// Shared-memory descriptors are built once per operand base (make_sw128_desc) and then
+// stepped by adding (byte offset >> 4) to the 14-bit start-address field, which never
+// carries: shared addresses stay below 2^18 bytes.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t byte_off) {
+  return desc + static_cast<uint64_t>(byte_off >> 4);
 }
-// MN-major operand descriptor for K-step ks (16 K-rows = two 8-row groups of 1024 B);
-// `lbo` is the byte stride between 64-wide M/N atoms.
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks, uint32_t lbo) {
-  return make_sw128_desc(base + ks * 2048, lbo, 1024);
+// K-major operand, K-step ks of a tile made of 64-column atoms of `atom_bytes` each: four
+// K-steps of 32 bytes inside one 128-byte swizzle row, then the next atom.
+__device__ __forceinline__ uint32_t kmajor_off(int ks, uint32_t atom_bytes) {
+  return (ks >> 2) * atom_bytes + (ks & 3) * 32;
+}
+// MN-major operand, K-step ks: 16 K-rows = two 8-row groups of 1024 bytes.
+__device__ __forceinline__ uint32_t mnmajor_off(int ks) { return ks * 2048; }
+__device__ __forceinline__ uint64_t kmajor_base(uint32_t addr) {
+  return make_sw128_desc(addr, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mnmajor_base(uint32_t addr, uint32_t lbo) {
+  return make_sw128_desc(addr, lbo, 1024);
 }
 
 // phi on two packed bf16 values: exp(min(x, 0)) + max(x, 0), which is x + 1 above zero and
@@ -138,8 +162,8 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks, uint32_t
 __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t u) {
   const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&u);
   const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
-  const __nv_bfloat162 log2e_hi = __float2bfloat162_rn(1.4453125f);          // bf16(log2 e)
-  const __nv_bfloat162 log2e_lo = __float2bfloat162_rn(-0.0026174592f);      // log2 e - head
+  const __nv_bfloat162 log2e_hi = __float2bfloat162_rn(1.4453125f);      // bf16(log2 e)
+  const __nv_bfloat162 log2e_lo = __float2bfloat162_rn(-0.0026174592f);  // log2 e - head
   const __nv_bfloat162 m = __hmin2(x, zero);
   const __nv_bfloat162 p = __hmax2(x, zero);
   const __nv_bfloat162 t = __hfma2(m, log2e_hi, __hmul2(m, log2e_lo));
@@ -156,6 +180,42 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
   u.z = pack_bf16x2(f[4], f[5]);
   u.w = pack_bf16x2(f[6], f[7]);
   return u;
+}
+// One 32-byte store (a full sector): 16 bf16 values.
+__device__ __forceinline__ void st_global_32B(void *p, uint4 a, uint4 b) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y),
+               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
+// Columns [c0, c0 + 32) of the causal score row r64 (lanes < 16 of each warp hold rows of the
+// M = 64 accumulator): mask keys after the query (j > i), round to bf16 into the K-major
+// operand of P V, and return the row's partial sum (of the unrounded fp32 scores; it differs
+// from the sum of the rounded ones by at most 2^-9 relative).
+__device__ __forceinline__ float convert_P32(uint32_t taddr, uint8_t *sP, int r64, bool v64,
+                                             int c0) {
+  uint32_t p[32];
+  tmem_ld16_async(taddr + c0, p);
+  tmem_ld16_async(taddr + c0 + 16, p + 16);
+  tmem_ld_wait();
+  tmem_reg_fence<32>(p);
+  float sum = 0.f;
+  if (v64) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = c0 + 8 * j;  // first key of this group of 8
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float x = __uint_as_float(p[8 * j + e]);
+        f[e] = (g + 7 <= r64 || g + e <= r64) ? x : 0.f;
+        sum += f[e];
+      }
+      *reinterpret_cast<uint4 *>(sP + sw128_offset(r64, g)) =
+          g > r64 ? make_uint4(0u, 0u, 0u, 0u) : pack8(f);
+    }
+  }
+  return sum;
 }
 
 // Lane-0 mbarrier wait whose outcome the whole warp shares (warp-uniform control flow).
@@ -176,12 +236,12 @@ struct WarpWaiter {
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
               const float *__restrict__ init_state, int64_t init_head_stride,
               int64_t init_seg_stride, float *__restrict__ out_state, int64_t n, int64_t seg_len,
               int64_t nseg, int *err) {
   using G = Cfg<D, MODE>;
-  using TM = TmemMap<D>;
+  using TM = TmemMap<D, MODE>;
   constexpr int NS = G::NS;
   constexpr int KSD = D / 16;  // K-steps over the feature dimension
   constexpr int KSC = C / 16;  // K-steps over the chunk's tokens
@@ -207,9 +267,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.empty[s], 1);
     }
     mbar_init(&bar.p_full, 1);
-    mbar_init(&bar.p_ready, kGroupThreads);
+    mbar_init(&bar.p_ready, 2 * kGroupThreads);
+    mbar_init(&bar.rs_ready, kGroupThreads);
     mbar_init(&bar.s_full, 1);
     mbar_init(&bar.s_ready, kGroupThreads);
+    mbar_init(&bar.z_ready, kGroupThreads);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.o_full[b], 1);
       mbar_init(&bar.o_empty[b], kGroupThreads);
@@ -218,15 +280,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     bar.abort = 0;
     fence_barrier_init();
   }
-  {
-    // ones block: row 0 = 1.0, rows 1..15 = 0; z block: all zero (row 0 is rewritten)
-    uint32_t *ones = reinterpret_cast<uint32_t *>(smem + G::OFF_ONES);
-    for (int i = threadIdx.x; i < G::ONES_BYTES / 4; i += kThreads)
-      ones[i] = i < 32 ? 0x3F803F80u : 0u;  // first 128-byte row: 64 x bf16(1.0)
-    uint32_t *zb = reinterpret_cast<uint32_t *>(smem + G::OFF_Z);
-    for (int i = threadIdx.x; i < G::Z_BYTES / 4; i += kThreads) zb[i] = 0u;
-    fence_proxy_async_smem();
+  for (int s = 0; s < NS; ++s) {
+    uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+    if (G::LKV) {
+      // ones atom: column 0 of every row is 1.0 (row r's column 0 sits in 16-byte chunk r & 7)
+      uint32_t *ones = reinterpret_cast<uint32_t *>(st + G::OFF_ONES);
+      for (int i = threadIdx.x; i < kAtom / 4; i += kThreads) {
+        const int row = i >> 5, word = i & 31;  // 32 words per 128-byte row
+        ones[i] = (word == 4 * (row & 7)) ? 0x00003F80u : 0u;
+      }
+    }
+    if (MODE == kCausalOut) {
+      // z rows of the K tile start at zero (row 64 is rewritten before every chunk)
+      for (int a = 0; a < G::A; ++a) {
+        uint32_t *zr = reinterpret_cast<uint32_t *>(st + G::OFF_K + a * G::KATOM + 64 * 128);
+        for (int i = threadIdx.x; i < kZRows * 128 / 4; i += kThreads) zr[i] = 0u;
+      }
+    }
   }
+  if (MODE == kNoncausalOut) {
+    // the z atom of the S operand: zero except column 0 (rewritten with z below)
+    uint32_t *za = reinterpret_cast<uint32_t *>(smem + G::OFF_S + G::A * D * 128);
+    for (int i = threadIdx.x; i < D * 128 / 4; i += kThreads) za[i] = 0u;
+  }
+  fence_proxy_async_smem();
   if (warp == kWarpMMA) {
     tmem_alloc(&bar.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -237,7 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
     }
-    if (MODE != kState) prefetch_tmap(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -253,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = c % NS;
         const uint32_t it = c / NS;
         if (c >= NS && !mbar_wait(&bar.empty[s], (it - 1) & 1, abort, err)) break;
-        mbar_arrive_expect_tx(&bar.full[s], G::STAGE);
+        mbar_arrive_expect_tx(&bar.full[s], G::LOAD_BYTES);
         uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
         const int y = static_cast<int>(t_begin + (int64_t)c * C);
         const int zc = static_cast<int>(head);
@@ -261,15 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int a = 0; a < G::A; ++a)
             tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
-          st += G::TILE;
         }
         if (G::LKV) {
 #pragma unroll
           for (int a = 0; a < G::A; ++a)
-            tma_load_3d(st + a * kAtom, &tmK, &bar.full[s], a * 64, y, zc, pol);
+            tma_load_3d(st + G::OFF_K + a * G::KATOM, &tmK, &bar.full[s], a * 64, y, zc, pol);
 #pragma unroll
           for (int a = 0; a < G::A; ++a)
-            tma_load_3d(st + G::TILE + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
+            tma_load_3d(st + G::OFF_V + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
         }
         issued = c + 1;
       }
@@ -280,72 +355,65 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMMA) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t I_P = make_idesc_bf16(64, 64, false, false);
-      constexpr uint32_t I_O = make_idesc_bf16(64, D, false, true);
-      constexpr uint32_t I_DEN = make_idesc_bf16(64, 16, false, false);
-      constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);
-      constexpr uint32_t I_Z = make_idesc_bf16(D, 16, true, false);
-      const uint32_t tP = tmem + kColP;
-      const uint32_t tS = tmem + TM::S, tSz = tmem + TM::S + D;
-      const uint32_t sS = smem_u32(smem + G::OFF_S), sZ = smem_u32(smem + G::OFF_Z);
-      const uint32_t sOnes = smem_u32(smem + G::OFF_ONES), sP = smem_u32(smem + G::OFF_P);
+      constexpr uint32_t I_P = make_idesc_bf16(64, 64 + kZRows, false, false);
+      constexpr uint32_t I_O = make_idesc_bf16(64, MODE == kNoncausalOut ? D + 16 : D, false, true);
+      constexpr uint32_t I_S = make_idesc_bf16(D, D + 16, true, true);
+      const uint32_t tP = tmem + TM::P, tS = tmem + TM::S;
+      const uint64_t dS = mnmajor_base(smem_u32(smem + G::OFF_S), D * 128);
+      const uint64_t dP = kmajor_base(smem_u32(smem + G::OFF_P));
+      const uint32_t st0 = smem_u32(smem + G::OFF_STAGES);
       for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS;
         const uint32_t it = c / NS;
         if (!mbar_wait(&bar.ready[s], it & 1, abort, err)) break;
-        const uint32_t st = smem_u32(smem + G::OFF_STAGES + s * G::STAGE);
-        const uint32_t sQ = st;
-        const uint32_t sK = st + (G::LQ ? G::TILE : 0);
-        const uint32_t sV = sK + G::TILE;
+        const uint32_t st = st0 + s * G::STAGE;
+        const uint64_t dQk = kmajor_base(st);                           // Q, K-major
+        const uint64_t dKk = kmajor_base(st + G::OFF_K);                // K (+z rows), K-major
+        const uint64_t dKm = mnmajor_base(st + G::OFF_K, G::KATOM);     // K, MN-major
+        const uint64_t dVm = mnmajor_base(st + G::OFF_V, kAtom);        // [V | ones], MN-major
         tc_fence_after();
         if (MODE == kState) {
 #pragma unroll
-          for (int ks = 0; ks < KSC; ++ks) {
-            const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
-            const uint64_t a = desc_mnmajor(sK, ks, kAtom);
-            mma_bf16_ss(tS, a, desc_mnmajor(sV, ks, kAtom), I_S, acc);
-            mma_bf16_ss(tSz, a, desc_kmajor(sOnes, ks, kZAtom), I_Z, acc);
-          }
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
+                        (c > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.empty[s]);
           continue;
         }
         const int ob = c & 1;
-        const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0), tOd = tO + D;
+        const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0);
         if (MODE == kCausalOut) {
-          // scores of this chunk first: the conversion warps can start on them at once
+          // [scores | phi(q).z_<c] first, as soon as z_<c sits in this chunk's K tile: the
+          // score warps start on them while the S snapshot is still being rounded
+          if (!mbar_wait(&bar.z_ready, c & 1, abort, err)) break;
+          tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
-            mma_bf16_ss(tP, desc_kmajor(sQ, ks, kAtom), desc_kmajor(sK, ks, kAtom), I_P,
-                        ks > 0 ? 1u : 0u);
+            mma_bf16_ss(tP, desc_add(dQk, kmajor_off(ks, kAtom)),
+                        desc_add(dKk, kmajor_off(ks, G::KATOM)), I_P, ks > 0 ? 1u : 0u);
           mma_commit(&bar.p_full);
         }
-        // S_<c, z_<c in shared memory; this O buffer drained
+        // S_<c (and, non-causal, z) in the S operand; this O buffer drained
         if (MODE == kCausalOut || c == 0)
           if (!mbar_wait(&bar.s_ready, MODE == kCausalOut ? (c & 1) : 0, abort, err)) break;
         if (c >= 2 && !mbar_wait(&bar.o_empty[ob], ((c >> 1) - 1) & 1, abort, err)) break;
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < KSD; ++ks) {
-          const uint64_t a = desc_kmajor(sQ, ks, kAtom);
-          mma_bf16_ss(tO, a, desc_mnmajor(sS, ks, D * 128), I_O, ks > 0 ? 1u : 0u);
-          mma_bf16_ss(tOd, a, desc_kmajor(sZ, ks, kZAtom), I_DEN, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < KSD; ++ks)
+          mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)), I_O,
+                      ks > 0 ? 1u : 0u);
         if (MODE == kCausalOut) {
 #pragma unroll
-          for (int ks = 0; ks < KSC; ++ks) {
-            const uint64_t a = desc_mnmajor(sK, ks, kAtom);
-            mma_bf16_ss(tS, a, desc_mnmajor(sV, ks, kAtom), I_S, 1u);
-            mma_bf16_ss(tSz, a, desc_kmajor(sOnes, ks, kZAtom), I_Z, 1u);
-          }
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
+                        1u);
           mma_commit(&bar.s_full);
           if (!mbar_wait(&bar.p_ready, c & 1, abort, err)) break;
           tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < KSC; ++ks) {
-            const uint64_t a = desc_kmajor(sP, ks, kAtom);
-            mma_bf16_ss(tO, a, desc_mnmajor(sV, ks, kAtom), I_O, 1u);
-            mma_bf16_ss(tOd, a, desc_kmajor(sOnes, ks, kZAtom), I_DEN, 1u);
-          }
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tO, desc_add(dP, kmajor_off(ks, kAtom)), desc_add(dVm, mnmajor_off(ks)),
+                        make_idesc_bf16(64, D, false, true), 1u);
         }
         mma_commit(&bar.o_full[ob]);
         mma_commit(&bar.empty[s]);
@@ -355,8 +423,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bar.fin);
       mbar_wait(&bar.fin, 0, abort, err);
     }
-  } else if (warp < kWarpConv0) {
+  } else if (warp < kWarpState0) {
     // ================================================================ feature map
+    // phi in place on the Q tile and on the 64 key rows of each K atom; K rows past n are
+    // zeroed (they must add nothing to S, z or the scores).
     const int xt = threadIdx.x - kWarpXform0 * 32;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % NS;
@@ -375,31 +445,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           x.w = phi_bf16x2(x.w);
           p[i] = x;
         }
-        st += G::TILE;
       }
       if (G::LKV) {
-        uint4 *p = reinterpret_cast<uint4 *>(st);
 #pragma unroll 2
         for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
-          const int row = (i % (kAtom / 16)) >> 3;  // 8 x 16 B per 128-byte row
+          const int a = i / (kAtom / 16), within = i % (kAtom / 16);
+          const int row = within >> 3;  // 8 x 16 B per 128-byte row
+          uint4 *p = reinterpret_cast<uint4 *>(st + G::OFF_K + a * G::KATOM) + within;
           uint4 x = make_uint4(0u, 0u, 0u, 0u);
           if (row < valid) {
-            x = p[i];
+            x = *p;
             x.x = phi_bf16x2(x.x);
             x.y = phi_bf16x2(x.y);
             x.z = phi_bf16x2(x.z);
             x.w = phi_bf16x2(x.w);
           }
-          p[i] = x;
+          *p = x;
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(&bar.ready[s]);
     }
   } else if (warp < kWarpOut0) {
-    // ================================================================ conversion group
-    // P -> masked bf16 operand; S_<c+1, z_<c+1 -> bf16 operands of the next chunk; the
-    // starting state; the segment aggregate (state mode).  Control flow is warp-uniform:
+    // ================================================================ state group
+    // Causal: half of each chunk's scores (columns 0..31) and their row sums; S_<c+1, z_<c+1
+    // -> bf16 operands of the next chunk (z into that chunk's K tile row 64).  Also the
+    // starting state and the segment aggregate (state mode).  Control flow is warp-uniform:
     // lane 0 waits and the warp shares the outcome.
     const int sp = warp & 3;  // TMEM sub-partition of this warp
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
@@ -409,7 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool vS = D == 128 ? true : v64;
     WarpWaiter wait{abort, err, lane};
     uint8_t *sS = smem + G::OFF_S;
-    uint8_t *sZ = smem + G::OFF_Z;
 
     // 32 consecutive S columns [c0, c0+32) of row rS (fp32 in registers) -> bf16 operand
     auto store_S32 = [&](const uint32_t *r, int c0) {
@@ -423,10 +493,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    sw128_offset(rS, (c0 & 63) + 8 * j)) = pack8(f);
       }
     };
-    auto store_z = [&](uint32_t zbits) {
+    // z_<c for chunk c: causal -> row 64 of that chunk's K atoms; non-causal -> column 0 of
+    // the S operand's z atom
+    auto store_z = [&](uint32_t zbits, int c) {
       if (!vS) return;
-      *reinterpret_cast<__nv_bfloat16 *>(sZ + (rS >> 6) * kZAtom + sw128_offset(0, rS & 63)) =
-          __float2bfloat16_rn(__uint_as_float(zbits));
+      const __nv_bfloat16 zb = __float2bfloat16_rn(__uint_as_float(zbits));
+      if (MODE == kCausalOut) {
+        uint8_t *kt = smem + G::OFF_STAGES + (c % NS) * G::STAGE + G::OFF_K;
+        *reinterpret_cast<__nv_bfloat16 *>(kt + (rS >> 6) * G::KATOM +
+                                           sw128_offset(64, rS & 63)) = zb;
+      } else {
+        *reinterpret_cast<__nv_bfloat16 *>(sS + G::A * D * 128 + sw128_offset(rS, 0)) = zb;
+      }
     };
 
     if (MODE != kState) {
@@ -456,53 +534,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st1(tmem + lane_off + TM::S + D, zb);
         tmem_st_wait();
       }
-      store_z(zb);
+      store_z(zb, 0);
       fence_proxy_async_smem();
       tc_fence_before();
+      if (MODE == kCausalOut) mbar_arrive(&bar.z_ready);
       mbar_arrive(&bar.s_ready);
     }
 
     if (MODE == kCausalOut) {
       for (int c = 0; c < nchunks; ++c) {
-        // ---- P: mask j <= i, round to bf16, K-major A operand of P V
+        // ---- this chunk's scores, columns 0..31 (the output group takes 32..63)
         if (wait(&bar.p_full, c & 1)) {
           tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < 64; c0 += 32) {
-            uint32_t p[32];
-            tmem_ld16_async(tmem + lane_off + kColP + c0, p);
-            tmem_ld16_async(tmem + lane_off + kColP + c0 + 16, p + 16);
-            tmem_ld_wait();
-            tmem_reg_fence<32>(p);
-            if (v64) {
-              uint8_t *sP = smem + G::OFF_P;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  f[e] = (c0 + 8 * j + e) <= r64 ? __uint_as_float(p[8 * j + e]) : 0.f;
-                *reinterpret_cast<uint4 *>(sP + sw128_offset(r64, c0 + 8 * j)) = pack8(f);
-              }
-            }
-          }
+          const float rs = convert_P32(tmem + lane_off + TM::P, smem + G::OFF_P, r64, v64, 0);
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bar.p_ready);
+          if (v64) bar.rowsum[c & 1][r64] = rs;
+          mbar_arrive(&bar.rs_ready);
         }
         // ---- S_<c+1, z_<c+1: the operands of the next chunk
         if (c + 1 < nchunks && wait(&bar.s_full, c & 1)) {
           tc_fence_after();
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t r[32];
+          // z_<c+1 first: the next chunk's score MMA needs only that
+          store_z(tmem_ld1(tmem + lane_off + TM::S + D), c + 1);
+          fence_proxy_async_smem();
+          mbar_arrive(&bar.z_ready);
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 64) {
+            uint32_t r[64];
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int j = 0; j < 4; ++j)
               tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * j, r + 16 * j);
             tmem_ld_wait();
-            tmem_reg_fence<32>(r);
+            tmem_reg_fence<64>(r);
             store_S32(r, c0);
+            store_S32(r + 32, c0 + 32);
           }
-          store_z(tmem_ld1(tmem + lane_off + TM::S + D));
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bar.s_ready);
@@ -535,55 +603,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ================================================================ output group
-    // O / den -> bf16 tile in a double-buffered staging area -> TMA store.
+    // ================================================================ scores and output
+    // P(c) columns 32..63 -> masked bf16 operand of P V (the state group takes 0..31), with
+    // phi(q).z_<c (column 64) and both groups' row sums -> the denominator of chunk c; then
+    // O(c-1) / den -> bf16 rows stored straight to global memory (32-byte stores; rows past
+    // n are not written).
     const int sp = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
     const bool v64 = lane < 16;
     const int r64 = 16 * sp + lane;
-    const int ot = threadIdx.x - kWarpOut0 * 32;  // 0..127
     WarpWaiter wait{abort, err, lane};
-    const uint64_t pol_out = policy_evict_first();
-    for (int c = 0; c < (MODE == kState ? 0 : nchunks); ++c) {
+
+    // Denominators of the chunks in flight, by parity.  The state group's half of the row sum
+    // is read BEFORE this group releases p_ready: the state group's next sums need this
+    // chunk's p_ready, so it never completes rs_ready's next phase (or rewrites that slot)
+    // before this wait has seen the current one.
+    float den0 = 1.f, den1 = 1.f;
+    auto convert_P = [&](int c) {
+      if (!wait(&bar.p_full, c & 1)) return;
+      tc_fence_after();
+      const float rs = convert_P32(tmem + lane_off + TM::P, smem + G::OFF_P, r64, v64, 32);
+      const float dz = __uint_as_float(tmem_ld1(tmem + lane_off + TM::P + 64));
+      const bool got = wait(&bar.rs_ready, c & 1);
+      const float d = dz + rs + (got ? bar.rowsum[c & 1][v64 ? r64 : 0] : 0.f);
+      if (c & 1) den1 = d; else den0 = d;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar.p_ready);
+    };
+
+    auto emit_O = [&](int c) {
       const int ob = c & 1;
       const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
-      uint8_t *so = smem + G::OFF_OUT + ob * G::TILE;
-      if (ot == 0) tma_store_wait_read<1>();  // the store that last used this buffer is done
-      named_barrier_sync(1, kGroupThreads);
-      if (wait(&bar.o_full[ob], (c >> 1) & 1)) {
-        tc_fence_after();
-        const float inv = 1.f / __uint_as_float(tmem_ld1(tO + D));
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t r[32];
+      if (!wait(&bar.o_full[ob], (c >> 1) & 1)) return;
+      tc_fence_after();
+      const float dd = MODE == kCausalOut ? (ob ? den1 : den0) : __uint_as_float(tmem_ld1(tO + D));
+      const float inv = 1.f / dd;
+      const int64_t t = t_begin + (int64_t)c * C + r64;
+      const bool live = v64 && t < t_end;
+      __nv_bfloat16 *orow = out + (head * n + (live ? t : 0)) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        uint32_t r[64];
 #pragma unroll
-          for (int j = 0; j < 2; ++j) tmem_ld16_async(tO + c0 + 16 * j, r + 16 * j);
-          tmem_ld_wait();
-          tmem_reg_fence<32>(r);
-          if (v64) {
+        for (int j = 0; j < 4; ++j) tmem_ld16_async(tO + c0 + 16 * j, r + 16 * j);
+        tmem_ld_wait();
+        tmem_reg_fence<64>(r);
+        if (live) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float f[8];
+          for (int j = 0; j < 4; ++j) {
+            float f[16];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * j + e]) * inv;
-              *reinterpret_cast<uint4 *>(so + (c0 >> 6) * kAtom +
-                                         sw128_offset(r64, (c0 & 63) + 8 * j)) = pack8(f);
-            }
+            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * j + e]) * inv;
+            st_global_32B(orow + c0 + 16 * j, pack8(f), pack8(f + 8));
           }
         }
-        tc_fence_before();
-        mbar_arrive(&bar.o_empty[ob]);
       }
-      fence_proxy_async_smem();
-      named_barrier_sync(1, kGroupThreads);
-      if (ot == 0 && !*abort) {
-        const int y = static_cast<int>(t_begin + (int64_t)c * C);
-#pragma unroll
-        for (int a = 0; a < G::A; ++a)
-          tma_store_3d(&tmO, so + a * kAtom, a * 64, y, static_cast<int>(head), pol_out);
-        tma_store_commit();
+      tc_fence_before();
+      mbar_arrive(&bar.o_empty[ob]);
+    };
+
+    if (MODE == kCausalOut) {
+      for (int c = 0; c < nchunks; ++c) {
+        convert_P(c);
+        if (c >= 1) emit_O(c - 1);
       }
+      if (nchunks > 0) emit_O(nchunks - 1);
+    } else if (MODE == kNoncausalOut) {
+      for (int c = 0; c < nchunks; ++c) emit_O(c);
     }
-    if (ot == 0) tma_store_wait_all<0>();
   }
 
   tc_fence_before();
@@ -624,15 +712,15 @@ cudaError_t make_tmap(CUtensorMap *m, const void *ptr, int64_t heads, int64_t n,
 
 template <int D, int MODE>
 cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
-                      const CUtensorMap &o, const float *init, int64_t ihs, int64_t iss,
+                      void *out, const float *init, int64_t ihs, int64_t iss,
                       float *out_state, int64_t heads, int64_t n, int64_t seg, int64_t nseg,
                       int *err, cudaStream_t st) {
   using G = Cfg<D, MODE>;
   auto kern = tc_kernel<D, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(heads * nseg), kThreads, G::SMEM, st>>>(q, k, v, o, init, ihs, iss, out_state,
-                                                           n, seg, nseg, err);
+  kern<<<(unsigned)(heads * nseg), kThreads, G::SMEM, st>>>(
+      q, k, v, static_cast<__nv_bfloat16 *>(out), init, ihs, iss, out_state, n, seg, nseg, err);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -642,26 +730,25 @@ cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out,
                          int64_t n, int causal, int64_t seg, void *ws, int *err, cudaStream_t st) {
   const int64_t nseg = (n + seg - 1) / seg;
   const int64_t per = (int64_t)D * D + D;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   cudaError_t e;
   if ((e = make_tmap(&tq, q, heads, n, D)) != cudaSuccess) return e;
   if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
   if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
-  if ((e = make_tmap(&to, out, heads, n, D)) != cudaSuccess) return e;
   float *w = static_cast<float *>(ws);
-  e = launch_tc<D, kState>(tq, tk, tv, to, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
+  e = launch_tc<D, kState>(tq, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
   if (e != cudaSuccess) return e;
   if (causal) {
     e = launch_scan_states(w, heads, nseg, D, 0, nullptr, 0, nullptr, 0, st);
     if (e != cudaSuccess) return e;
-    return launch_tc<D, kCausalOut>(tq, tk, tv, to, w, nseg * per, per, nullptr, heads, n, seg,
+    return launch_tc<D, kCausalOut>(tq, tk, tv, out, w, nseg * per, per, nullptr, heads, n, seg,
                                     nseg, err, st);
   }
   // per-head totals, packed as [heads][D*D + D] (S row-major, then z)
   float *tot = w + heads * nseg * per;
   e = launch_scan_states(w, heads, nseg, D, 1, tot, per, tot + (int64_t)D * D, per, st);
   if (e != cudaSuccess) return e;
-  return launch_tc<D, kNoncausalOut>(tq, tk, tv, to, tot, per, 0, nullptr, heads, n, seg, nseg,
+  return launch_tc<D, kNoncausalOut>(tq, tk, tv, out, tot, per, 0, nullptr, heads, n, seg, nseg,
                                      err, st);
 }
 
@@ -709,7 +796,7 @@ cudaError_t tc_state_d(const void *k, const void *v, float *S_out, float *z_out,
   if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
   if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
   float *w = static_cast<float *>(ws);
-  e = launch_tc<D, kState>(tk, tk, tv, tv, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
+  e = launch_tc<D, kState>(tk, tk, tv, nullptr, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
   if (e != cudaSuccess) return e;
   return launch_scan_states(w, heads, nseg, D, 1, S_out, (int64_t)D * D, z_out, D, st);
 }
