@@ -55,6 +55,26 @@ def decode_bytes(heads, d, elem=2):
     return heads * (2 * (d * d + d) * 4 + 4 * d * elem)
 
 
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from profiles/ncu_traffic.json (an ncu
+    capture, scaled to the full launch), or None when there is none or the kernel's source
+    file has changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        table = json.load(f)
+    rec = table.get(f"{kernel} | {workload}")
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return float(rec["dram_bytes_per_launch"])
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -189,6 +209,45 @@ def time_steps(fn, steps, warmup, world, clocks=None):
     return max_over_ranks(total / steps, world), per
 
 
+def time_launches(fn, steps, warmup, names):
+    """Per-launch device times of a multi-kernel call: before each timed call the library is
+    given events (linattn_profile_events) that it records after each of its launches on the
+    call's stream; returns the mean ms of each launch."""
+    import ctypes
+
+    import torch
+
+    import linear_attention_linattn_b200 as la
+    lib = la.load_library()
+    k = len(names)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(k)] for _ in range(steps)]
+    arrs = []
+    for i in range(steps):
+        for e in evs[i]:
+            e.record(stream)  # materialise the handles
+    torch.cuda.synchronize()
+    for i in range(steps):
+        arr = (ctypes.c_void_p * k)(*[e.cuda_event for e in evs[i]])
+        arrs.append(arr)
+        starts[i].record(stream)
+        lib.linattn_profile_events(arr, k)
+        fn()
+        lib.linattn_profile_events(None, 0)
+    torch.cuda.synchronize()
+    per = np.zeros(k)
+    for i in range(steps):
+        prev = starts[i]
+        for j in range(k):
+            per[j] += prev.elapsed_time(evs[i][j])
+            prev = evs[i][j]
+    return {nm: float(per[j] / steps) for j, nm in enumerate(names)}
+
+
 # ------------------------------------------------------------------ oracle baseline
 def oracle_sample(workload: str, target_s: float = 12.0):
     """Times the float64 oracle on a bounded sample of the workload (host cores)."""
@@ -251,6 +310,8 @@ def main_forward(args, world, rank, local):
         import dataclasses
         w = dataclasses.replace(w, H=args.max_heads)
     causal = True in w.causal
+    if args.mode is not None:
+        causal = args.mode == "causal"
     dtype = "bf16" if "bf16" in w.dtypes else "f32"
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     elem = 2 if dtype == "bf16" else 4
@@ -279,8 +340,20 @@ def main_forward(args, world, rank, local):
     value = tokens_rank * world / (ms * 1e-3)
     pk = peaks()
     alg = forward_bytes(w.B, w.H, w.n, w.d, elem)
-    kernel_ms = float(np.mean(per))
-    achieved = alg / (kernel_ms * 1e-3) / 1e9
+    unit = w.B * w.H * w.n * w.d * elem  # one [B,H,n,d] tensor
+    if dtype == "bf16":
+        names = ["tc_kernel<state> (segment aggregates, K1)", "scan_states_kernel (prefix, K2)",
+                 "tc_kernel<causal out> (K3)" if causal else "tc_kernel<non-causal out> (K3)"]
+        kbytes = [2 * unit, 0, 4 * unit if causal else 2 * unit]
+    else:
+        names = ["simt_chunk_state_kernel (K1)", "scan_states_kernel (K2)",
+                 "simt_chunk_out_kernel (K3)"]
+        kbytes = [2 * unit, 0, 4 * unit if causal else 2 * unit]
+    launch_ms = time_launches(step, max(3, min(args.steps, 10)), 2, names)
+    top = max(launch_ms, key=launch_ms.get)
+    kernel_ms = launch_ms[top]
+    kernel_alg = kbytes[names.index(top)]
+    achieved = kernel_alg / (kernel_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host -> device, forward, device -> host
     outh = torch.empty_like(qh).pin_memory()
@@ -303,16 +376,22 @@ def main_forward(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
         "data": "synthetic (seeded N(0,1)/sqrt(d), see DESIGN.md input recipe)",
-        "config": {"workload": args.workload + (f" (first {w.H} heads)" if args.max_heads else ""),
+        "config": {"workload": args.workload + (f" (first {w.H} heads)" if args.max_heads else "")
+                   + (f" [{args.mode}]" if args.mode else ""),
                    "B": w.B, "H": w.H, "n": w.n, "d": w.d,
                    "causal": causal, "global_batch": w.B * world, "seq_len": w.n,
                    "parallelism": f"dp{world} (independent heads, no collective)",
                    "l2": "inputs larger than L2 (no flush needed)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                     "peak_source": pk["source"], "algorithmic_bytes": alg,
-                     "kernel": "whole forward pass (all launches of one step)",
-                     "kernel_ms": kernel_ms},
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                     "traffic": kernel_traffic(top, args.workload),
+                     "peak_source": pk["source"] + " (burst copy bandwidth)",
+                     "kernel": top, "kernel_ms": kernel_ms,
+                     "algorithmic_bytes_per_launch": kernel_alg,
+                     "launch_ms": launch_ms,
+                     "whole_step": {"algorithmic_bytes": alg, "ms": ms,
+                                    "gbs": alg / (ms * 1e-3) / 1e9,
+                                    "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}},
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -429,6 +508,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mode", choices=["causal", "noncausal"], default=None,
+                    help="for a workload that has both modes (default: causal)")
     ap.add_argument("--max-heads", type=int, default=0,
                     help="profiling aid: run only the first N heads of the workload")
     args = ap.parse_args()

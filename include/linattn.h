@@ -126,6 +126,15 @@ int linattn_version(void);
  * every device.  Benchmarks read it before and after a timed region. */
 uint64_t linattn_launch_count(void);
 
+/*
+ * Measurement aid: while `count` > 0, every kernel this library enqueues on the calling
+ * thread is followed by cudaEventRecord(events[i], stream) with i = 0, 1, ... (up to
+ * count - 1), so the caller can time each launch of a multi-kernel call with
+ * cudaEventElapsedTime.  `events` holds cudaEvent_t handles created by the caller; the
+ * library keeps the pointer until the next call with count = 0.
+ */
+linattn_status linattn_profile_events(void *const *events, int count);
+
 /* Size of the fixed device scratch block behind linattn_forward_noalloc (32 MiB). */
 #define LINATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
 

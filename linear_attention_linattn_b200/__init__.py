@@ -9,7 +9,7 @@ raises.
 Raw C entry points (pointers as ints):
     linattn_forward, linattn_forward_ex, linattn_forward_state, linattn_decode_step,
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
-    linattn_launch_count, linattn_forward_noalloc
+    linattn_launch_count, linattn_forward_noalloc, linattn_profile_events
 
 Tensor helpers: ``forward``, ``forward_state``, ``decode_step``, ``device_error``.
 """
@@ -47,6 +47,7 @@ SIGNATURES = {
     "linattn_launch_count": (ctypes.c_uint64, []),
     "linattn_forward_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                                ctypes.c_int, ctypes.c_int, _vp]),
+    "linattn_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
 }
 
 _lib = None

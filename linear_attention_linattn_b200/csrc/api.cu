@@ -244,7 +244,23 @@ uint64_t linattn_launch_count(void) { return linattn::launches_total(); }
 namespace linattn {
 namespace {
 std::atomic<uint64_t> g_launches{0};
-}
+// per-thread event list of linattn_profile_events
+thread_local void *const *t_events = nullptr;
+thread_local int t_event_count = 0;
+thread_local int t_event_next = 0;
+}  // namespace
 void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 uint64_t launches_total() { return g_launches.load(std::memory_order_relaxed); }
+void record_launch_event(cudaStream_t st) {
+  if (t_event_count > 0 && t_event_next < t_event_count)
+    cudaEventRecord(static_cast<cudaEvent_t>(t_events[t_event_next++]), st);
+}
 }  // namespace linattn
+
+extern "C" linattn_status linattn_profile_events(void *const *events, int count) {
+  if (count < 0 || (count > 0 && !events)) return LINATTN_ERR_INVALID_ARG;
+  linattn::t_events = count > 0 ? events : nullptr;
+  linattn::t_event_count = count;
+  linattn::t_event_next = 0;
+  return LINATTN_OK;
+}

@@ -117,6 +117,7 @@ cudaError_t launch_decode_step(float *S, float *z, const void *q, const void *k,
   else
     decode_step_kernel<128><<<(unsigned)heads, kThreads, 0, st>>>(S, z, qb, kb, vb, ob);
   count_launches(1);
+  record_launch_event(st);
   return cudaGetLastError();
 }
 

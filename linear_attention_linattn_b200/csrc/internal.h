@@ -9,6 +9,8 @@ namespace linattn {
 // Launch accounting for linattn_launch_count(): every launcher adds the kernels it enqueued.
 void count_launches(uint64_t n);
 uint64_t launches_total();
+// Records the next caller-supplied profiling event (linattn_profile_events) on `st`.
+void record_launch_event(cudaStream_t st);
 
 // Tokens per chunk of the fp32 (CUDA-core) path.
 constexpr int kSimtChunk = 64;

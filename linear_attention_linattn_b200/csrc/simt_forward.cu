@@ -277,6 +277,7 @@ cudaError_t chunk_state_impl(const void *k, const void *v, float *ws, int64_t he
   simt_chunk_state_kernel<D, T><<<(unsigned)(nchunks * heads), kThreads, smem, st>>>(
       static_cast<const T *>(k), static_cast<const T *>(v), ws, n, nchunks);
   count_launches(1);
+  record_launch_event(st);
   return cudaGetLastError();
 }
 
@@ -293,6 +294,7 @@ cudaError_t chunk_out_impl(const void *q, const void *k, const void *v, void *ou
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
       static_cast<T *>(out), S, z, Scs, Shs, zcs, zhs, n, nchunks);
   count_launches(1);
+  record_launch_event(st);
   return cudaGetLastError();
 }
 
@@ -333,6 +335,7 @@ cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, in
   scan_states_kernel<<<(unsigned)(((per + 255) / 256) * heads), 256, 0, st>>>(
       ws, nseg, d, mode, S_out, S_hs, z_out, z_hs);
   count_launches(1);
+  record_launch_event(st);
   return cudaGetLastError();
 }
 

@@ -722,6 +722,7 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
   kern<<<(unsigned)(heads * nseg), kThreads, G::SMEM, st>>>(
       q, k, v, static_cast<__nv_bfloat16 *>(out), init, ihs, iss, out_state, n, seg, nseg, err);
   count_launches(1);
+  record_launch_event(st);
   return cudaGetLastError();
 }
 
