@@ -102,41 +102,44 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__r
   }
 }
 
-// K2: per head, a sequential sweep over the segments for each state element.
+// K2: per head, a sequential sweep over the segments for each group of 4 state elements
+// (16-byte loads and stores; d (d + 1) is a multiple of 4, so a group never straddles S and z).
 //   mode 0: ws[h][s] <- sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
 //   mode 1: S_out + h*S_hs, z_out + h*z_hs <- sum_s ws[h][s] (the total)
+// The segments are summed in order, one group of elements per thread.
 __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws, int64_t nseg,
                                                           int d, int mode,
                                                           float *__restrict__ S_out, int64_t S_hs,
                                                           float *__restrict__ z_out, int64_t z_hs) {
-  const int64_t per = (int64_t)d * d + d;
-  const int64_t blocks_per_head = (per + blockDim.x - 1) / blockDim.x;
+  const int64_t per4 = ((int64_t)d * d + d) / 4;
+  const int64_t blocks_per_head = (per4 + blockDim.x - 1) / blockDim.x;
   const int64_t head = blockIdx.x / blocks_per_head;
-  const int64_t e = (blockIdx.x % blocks_per_head) * (int64_t)blockDim.x + threadIdx.x;
-  if (e >= per) return;
-  float *base = ws + head * nseg * per + e;
-  constexpr int kBatch = 16;  // independent loads in flight per thread
-  float run = 0.f;
+  const int64_t e4 = (blockIdx.x % blocks_per_head) * (int64_t)blockDim.x + threadIdx.x;
+  if (e4 >= per4) return;
+  float4 *base = reinterpret_cast<float4 *>(ws) + head * nseg * per4 + e4;
+  constexpr int kBatch = 8;  // independent 16-byte loads in flight per thread
+  float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int64_t s0 = 0; s0 < nseg; s0 += kBatch) {
-    float x[kBatch];
+    float4 x[kBatch];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) x[i] = s0 + i < nseg ? base[(s0 + i) * per] : 0.f;
-    if (mode == 0) {
+    for (int i = 0; i < kBatch; ++i)
+      x[i] = s0 + i < nseg ? base[(s0 + i) * per4] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        if (s0 + i < nseg) base[(s0 + i) * per] = run;
-        run += x[i];
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) run += x[i];
+    for (int i = 0; i < kBatch; ++i) {
+      if (mode == 0 && s0 + i < nseg) base[(s0 + i) * per4] = run;
+      run.x += x[i].x;
+      run.y += x[i].y;
+      run.z += x[i].z;
+      run.w += x[i].w;
     }
   }
   if (mode != 0) {
-    if (e < (int64_t)d * d)
-      S_out[head * S_hs + e] = run;
-    else
-      z_out[head * z_hs + (e - (int64_t)d * d)] = run;
+    const int64_t e = e4 * 4;
+    float *dst = e < (int64_t)d * d ? S_out + head * S_hs + e : z_out + head * z_hs + (e - (int64_t)d * d);
+    dst[0] = run.x;
+    dst[1] = run.y;
+    dst[2] = run.z;
+    dst[3] = run.w;
   }
 }
 
@@ -331,8 +334,8 @@ cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int
 cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
                                cudaStream_t st) {
-  const int64_t per = (int64_t)d * d + d;
-  scan_states_kernel<<<(unsigned)(((per + 255) / 256) * heads), 256, 0, st>>>(
+  const int64_t per4 = ((int64_t)d * d + d) / 4;
+  scan_states_kernel<<<(unsigned)(((per4 + 255) / 256) * heads), 256, 0, st>>>(
       ws, nseg, d, mode, S_out, S_hs, z_out, z_hs);
   count_launches(1);
   record_launch_event(st);

@@ -25,23 +25,23 @@
 // The normaliser rides along as a 16-column block whose first column is z (or ones), so the
 // numerator and the denominator see the same rounded weights.
 //
-// Warp roles (576 threads, one CTA per SM):
+// Warp roles (one CTA per SM; 16, 22 or 18 warps in the causal, aggregate, non-causal modes):
 //   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of Q/K/V chunks into a
 //              ring of stages; no multicast.
 //   warp 1     TMEM allocation and the single MMA-issuing thread.
-//   warps 2-9  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
-//              n zeroed, then handed to the tensor cores (two warps per SM sub-partition:
-//              the exponentials are the busiest part of the kernel).
-//   warps 10-13 state: round S_<c+1 and z into the next chunk's operands; the starting
+//   next 6-12  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
+//              n zeroed, then handed to the tensor cores.
+//   next 4     state: round S_<c+1 and z into the next chunk's operands; the starting
 //              state; the segment aggregate.
-//   warps 14-17 scores and output: mask and round P; divide O by its denominator and
-//              TMA-store the bf16 tile.  P and S are drained by different warps, so the
-//              two conversions on each chunk's critical path run side by side.
+//   last 4     scores and output: mask and round P; divide O by its denominator and
+//              store the bf16 rows.  P and S are drained by different warps, so the two
+//              conversions on each chunk's critical path run side by side.
 // Every wait is bounded (2 s); a wait that gives up records LINATTN_ERR_TIMEOUT and the
 // CTA drains and exits without trapping.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -58,15 +58,25 @@ enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
 constexpr int kWarpTMA = 0;
 constexpr int kWarpMMA = 1;
 constexpr int kWarpXform0 = 2;
-constexpr int kNumXformWarps = 8;
-constexpr int kWarpState0 = kWarpXform0 + kNumXformWarps;  // 10: state group
-constexpr int kWarpOut0 = kWarpState0 + 4;                  // 14: scores and output group
-constexpr int kThreads = (kWarpOut0 + 4) * 32;              // 576
-constexpr int kXformThreads = kNumXformWarps * 32;
 constexpr int kGroupThreads = 128;
+// Warps per mode (measured on the benchmark shapes).  Causal: 6 feature-map warps, 16 warps
+// in all, so each SM sub-partition holds 4 warps and a thread may use 128 registers (the
+// score, state and output drains keep 64-column batches in registers).  Aggregate: the
+// feature map on K bounds the chunk rate, so 12 feature-map warps (22 warps, 80 registers).
+// Non-causal: 8 feature-map warps (18 warps, 96 registers).
+template <int MODE>
+struct Warps {
+  static constexpr int XFORM = MODE == kCausalOut ? 6 : (MODE == kState ? 12 : 8);
+  static constexpr int XTHREADS = XFORM * 32;
+  static constexpr int STATE0 = kWarpXform0 + XFORM;  // state group: 4 warps
+  static constexpr int OUT0 = STATE0 + 4;             // scores and output group: 4 warps
+  static constexpr int THREADS = (OUT0 + 4) * 32;
+};
 constexpr int kMaxSmem = 227 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kZRows = 16;  // extra key rows carrying z (row 0) in the causal K tile
+// causal items of at most this many chunks run on persistent CTAs
+constexpr int kPersistentCausalChunks = 32;
 
 template <int D, int MODE>
 struct Cfg {
@@ -90,7 +100,9 @@ struct Cfg {
   // bf16 S operand, MN-major [atoms][D rows][128 B]; non-causal adds an atom whose column 0
   // is z, so O (N = D + 16) carries phi(q_i).z in its column D.
   static constexpr int S_ATOMS = MODE == kState ? 0 : (MODE == kNoncausalOut ? A + 1 : A);
-  static constexpr int S_BYTES = S_ATOMS * D * 128;
+  static constexpr int S_BUF = S_ATOMS * D * 128;  // one S operand
+  // non-causal: two S operands, so the next item's total is rounded while this one runs
+  static constexpr int S_BYTES = (MODE == kNoncausalOut ? 2 : 1) * S_BUF;
   static constexpr int P_BYTES = MODE == kCausalOut ? kAtom : 0;  // bf16 [64][64], K-major
   static constexpr int FIXED = S_BYTES + P_BYTES;
   static constexpr int BAR_BYTES = 1024;
@@ -111,7 +123,8 @@ struct Cfg {
 
 // TMEM column map (32-column aligned): P (80 columns, causal), two O buffers (D columns,
 // plus the 16-column denominator block in the non-causal mode), S (D + 16 columns, z in
-// column D).
+// column D).  The state mode keeps two S accumulators, one per item parity, so one item's
+// aggregate is written out while the next one accumulates.
 template <int D, int MODE>
 struct TmemMap {
   static constexpr uint32_t P = 0;
@@ -119,12 +132,17 @@ struct TmemMap {
   static constexpr uint32_t O0 = MODE == kCausalOut ? 96 : 0;
   static constexpr uint32_t O1 = O0 + OW;
   static constexpr uint32_t S = MODE == kCausalOut ? O1 + OW : 0;  // unused when non-causal
-  static_assert((MODE == kNoncausalOut ? O1 + OW : S + D + 16) <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t S1 = MODE == kState ? kTmemCols / 2 : S;
+  static_assert((MODE == kNoncausalOut ? O1 + OW : S1 + D + 16) <= kTmemCols, "TMEM budget");
 };
 
 struct Bars {
   uint64_t full[8], ready[8], empty[8];
   uint64_t p_full, p_ready, s_full, s_ready, z_ready, rs_ready, o_full[2], o_empty[2], fin;
+  // per item parity: state mode, S accumulator complete (MMA -> state group) / written out
+  // (state group -> MMA); non-causal, S operand rounded (state group -> MMA) / no longer read
+  // (MMA -> state group)
+  uint64_t item_full[2], item_empty[2];
   float rowsum[2][64];  // the state group's half of P's row sums, by chunk parity
   uint32_t tmem_base;
   int abort;
@@ -233,15 +251,36 @@ struct WarpWaiter {
   }
 };
 
+// One work item: tokens [t_begin, t_end) of one head (one segment).
+struct Item {
+  int64_t head, seg, t_begin, t_end;
+  int nchunks;
+};
+__device__ __forceinline__ Item item_at(int64_t it, int64_t n, int64_t seg_len, int64_t nseg) {
+  Item I;
+  I.head = it / nseg;
+  I.seg = it % nseg;
+  I.t_begin = I.seg * seg_len;
+  I.t_end = n < I.t_begin + seg_len ? n : I.t_begin + seg_len;
+  I.nchunks = static_cast<int>((I.t_end - I.t_begin + C - 1) / C);
+  return I;
+}
+
+// CTA b takes the items b, b + gridDim.x, b + 2 gridDim.x, ... (one item when the grid
+// covers them all; several on persistent CTAs).  Every role walks the same sequence of
+// chunks, and g counts them across items, so the stage ring, the barrier phases and the O
+// buffers run on from one item into the next: the loads of an item's first chunks overlap
+// the previous item's last ones.
 template <int D, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
               const float *__restrict__ init_state, int64_t init_head_stride,
               int64_t init_seg_stride, float *__restrict__ out_state, int64_t n, int64_t seg_len,
-              int64_t nseg, int *err) {
+              int64_t nseg, int64_t nitems, int *err) {
   using G = Cfg<D, MODE>;
   using TM = TmemMap<D, MODE>;
+  using W = Warps<MODE>;
   constexpr int NS = G::NS;
   constexpr int KSD = D / 16;  // K-steps over the feature dimension
   constexpr int KSC = C / 16;  // K-steps over the chunk's tokens
@@ -253,17 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t head = blockIdx.x / nseg;
-  const int64_t seg = blockIdx.x % nseg;
-  const int64_t t_begin = seg * seg_len;
-  const int64_t t_end = n < t_begin + seg_len ? n : t_begin + seg_len;
-  const int nchunks = static_cast<int>((t_end - t_begin + C - 1) / C);
+  const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
   // ---- set-up: barriers, constant operand blocks, TMEM
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar.full[s], 1);
-      mbar_init(&bar.ready[s], kXformThreads);
+      mbar_init(&bar.ready[s], W::XTHREADS);
       mbar_init(&bar.empty[s], 1);
     }
     mbar_init(&bar.p_full, 1);
@@ -275,6 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.o_full[b], 1);
       mbar_init(&bar.o_empty[b], kGroupThreads);
+      mbar_init(&bar.item_full[b], MODE == kNoncausalOut ? kGroupThreads : 1);
+      mbar_init(&bar.item_empty[b], MODE == kState ? kGroupThreads : 1);
     }
     mbar_init(&bar.fin, 1);
     bar.abort = 0;
@@ -285,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (G::LKV) {
       // ones atom: column 0 of every row is 1.0 (row r's column 0 sits in 16-byte chunk r & 7)
       uint32_t *ones = reinterpret_cast<uint32_t *>(st + G::OFF_ONES);
-      for (int i = threadIdx.x; i < kAtom / 4; i += kThreads) {
+      for (int i = threadIdx.x; i < kAtom / 4; i += W::THREADS) {
         const int row = i >> 5, word = i & 31;  // 32 words per 128-byte row
         ones[i] = (word == 4 * (row & 7)) ? 0x00003F80u : 0u;
       }
@@ -294,14 +331,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // z rows of the K tile start at zero (row 64 is rewritten before every chunk)
       for (int a = 0; a < G::A; ++a) {
         uint32_t *zr = reinterpret_cast<uint32_t *>(st + G::OFF_K + a * G::KATOM + 64 * 128);
-        for (int i = threadIdx.x; i < kZRows * 128 / 4; i += kThreads) zr[i] = 0u;
+        for (int i = threadIdx.x; i < kZRows * 128 / 4; i += W::THREADS) zr[i] = 0u;
       }
     }
   }
   if (MODE == kNoncausalOut) {
-    // the z atom of the S operand: zero except column 0 (rewritten with z below)
-    uint32_t *za = reinterpret_cast<uint32_t *>(smem + G::OFF_S + G::A * D * 128);
-    for (int i = threadIdx.x; i < D * 128 / 4; i += kThreads) za[i] = 0u;
+    // the z atoms of the two S operands: zero except column 0 (rewritten with z per item)
+    for (int b = 0; b < 2; ++b) {
+      uint32_t *za = reinterpret_cast<uint32_t *>(smem + G::OFF_S + b * G::S_BUF + G::A * D * 128);
+      for (int i = threadIdx.x; i < D * 128 / 4; i += W::THREADS) za[i] = 0u;
+    }
   }
   fence_proxy_async_smem();
   if (warp == kWarpMMA) {
@@ -324,33 +363,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ TMA producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int issued = 0;
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % NS;
-        const uint32_t it = c / NS;
-        if (c >= NS && !mbar_wait(&bar.empty[s], (it - 1) & 1, abort, err)) break;
-        mbar_arrive_expect_tx(&bar.full[s], G::LOAD_BYTES);
-        uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
-        const int y = static_cast<int>(t_begin + (int64_t)c * C);
-        const int zc = static_cast<int>(head);
-        if (G::LQ) {
+      int g = 0;  // chunks issued
+      bool ok = true;
+      for (int64_t it = it0; ok && it < nitems; it += istep) {
+        const Item I = item_at(it, n, seg_len, nseg);
+        const int zc = static_cast<int>(I.head);
+        for (int c = 0; c < I.nchunks; ++c, ++g) {
+          const int s = g % NS;
+          const uint32_t ph = g / NS;
+          if (g >= NS && !mbar_wait(&bar.empty[s], (ph - 1) & 1, abort, err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar.full[s], G::LOAD_BYTES);
+          uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+          const int y = static_cast<int>(I.t_begin + (int64_t)c * C);
+          if (G::LQ) {
 #pragma unroll
-          for (int a = 0; a < G::A; ++a)
-            tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
+            for (int a = 0; a < G::A; ++a)
+              tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
+          }
+          if (G::LKV) {
+#pragma unroll
+            for (int a = 0; a < G::A; ++a)
+              tma_load_3d(st + G::OFF_K + a * G::KATOM, &tmK, &bar.full[s], a * 64, y, zc, pol);
+#pragma unroll
+            for (int a = 0; a < G::A; ++a)
+              tma_load_3d(st + G::OFF_V + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
+          }
         }
-        if (G::LKV) {
-#pragma unroll
-          for (int a = 0; a < G::A; ++a)
-            tma_load_3d(st + G::OFF_K + a * G::KATOM, &tmK, &bar.full[s], a * 64, y, zc, pol);
-#pragma unroll
-          for (int a = 0; a < G::A; ++a)
-            tma_load_3d(st + G::OFF_V + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
-        }
-        issued = c + 1;
       }
       // drain: every issued load has landed before the CTA may exit
-      for (int c = (issued > NS ? issued - NS : 0); c < issued; ++c)
-        mbar_wait(&bar.full[c % NS], (c / NS) & 1, abort, err);
+      for (int gg = (g > NS ? g - NS : 0); gg < g; ++gg)
+        mbar_wait(&bar.full[gg % NS], (gg / NS) & 1, abort, err);
     }
   } else if (warp == kWarpMMA) {
     // ================================================================ MMA issuer
@@ -358,120 +403,160 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t I_P = make_idesc_bf16(64, 64 + kZRows, false, false);
       constexpr uint32_t I_O = make_idesc_bf16(64, MODE == kNoncausalOut ? D + 16 : D, false, true);
       constexpr uint32_t I_S = make_idesc_bf16(D, D + 16, true, true);
-      const uint32_t tP = tmem + TM::P, tS = tmem + TM::S;
-      const uint64_t dS = mnmajor_base(smem_u32(smem + G::OFF_S), D * 128);
+      const uint32_t tP = tmem + TM::P;
       const uint64_t dP = kmajor_base(smem_u32(smem + G::OFF_P));
       const uint32_t st0 = smem_u32(smem + G::OFF_STAGES);
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % NS;
-        const uint32_t it = c / NS;
-        if (!mbar_wait(&bar.ready[s], it & 1, abort, err)) break;
-        const uint32_t st = st0 + s * G::STAGE;
-        const uint64_t dQk = kmajor_base(st);                           // Q, K-major
-        const uint64_t dKk = kmajor_base(st + G::OFF_K);                // K (+z rows), K-major
-        const uint64_t dKm = mnmajor_base(st + G::OFF_K, G::KATOM);     // K, MN-major
-        const uint64_t dVm = mnmajor_base(st + G::OFF_V, kAtom);        // [V | ones], MN-major
-        tc_fence_after();
-        if (MODE == kState) {
+      int g = 0;
+      int j = 0;  // items of this CTA
+      bool ok = true;
+      for (int64_t it = it0; ok && it < nitems; it += istep, ++j) {
+        const Item I = item_at(it, n, seg_len, nseg);
+        const int b = j & 1;
+        const uint32_t tS = tmem + (b ? TM::S1 : TM::S);
+        const uint64_t dS =
+            mnmajor_base(smem_u32(smem + G::OFF_S + (MODE == kNoncausalOut ? b * G::S_BUF : 0)),
+                         D * 128);
+        // state mode: this S accumulator written out (item j - 2); non-causal: the head's
+        // total rounded into this S operand
+        if (MODE == kState && j >= 2 && !mbar_wait(&bar.item_empty[b], ((j >> 1) - 1) & 1, abort, err))
+          break;
+        if (MODE == kNoncausalOut && !mbar_wait(&bar.item_full[b], (j >> 1) & 1, abort, err)) break;
+        for (int c = 0; c < I.nchunks; ++c, ++g) {
+          const int s = g % NS;
+          if (!mbar_wait(&bar.ready[s], (g / NS) & 1, abort, err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = st0 + s * G::STAGE;
+          const uint64_t dQk = kmajor_base(st);                        // Q, K-major
+          const uint64_t dKk = kmajor_base(st + G::OFF_K);             // K (+z rows), K-major
+          const uint64_t dKm = mnmajor_base(st + G::OFF_K, G::KATOM);  // K, MN-major
+          const uint64_t dVm = mnmajor_base(st + G::OFF_V, kAtom);     // [V | ones], MN-major
+          tc_fence_after();
+          if (MODE == kState) {
 #pragma unroll
-          for (int ks = 0; ks < KSC; ++ks)
-            mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
-                        (c > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&bar.empty[s]);
-          continue;
-        }
-        const int ob = c & 1;
-        const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0);
-        if (MODE == kCausalOut) {
-          // [scores | phi(q).z_<c] first, as soon as z_<c sits in this chunk's K tile: the
-          // score warps start on them while the S snapshot is still being rounded
-          if (!mbar_wait(&bar.z_ready, c & 1, abort, err)) break;
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)),
+                          I_S, (c > 0 || ks > 0) ? 1u : 0u);
+            mma_commit(&bar.empty[s]);
+            continue;
+          }
+          const int ob = g & 1;
+          const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0);
+          if (MODE == kCausalOut) {
+            // [scores | phi(q).z_<c] first, as soon as z_<c sits in this chunk's K tile: the
+            // score warps start on them while the S snapshot is still being rounded
+            if (!mbar_wait(&bar.z_ready, g & 1, abort, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < KSD; ++ks)
+              mma_bf16_ss(tP, desc_add(dQk, kmajor_off(ks, kAtom)),
+                          desc_add(dKk, kmajor_off(ks, G::KATOM)), I_P, ks > 0 ? 1u : 0u);
+            mma_commit(&bar.p_full);
+            // S_<c in the S operand
+            if (!mbar_wait(&bar.s_ready, g & 1, abort, err)) {
+              ok = false;
+              break;
+            }
+          }
+          // this O buffer drained
+          if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
-            mma_bf16_ss(tP, desc_add(dQk, kmajor_off(ks, kAtom)),
-                        desc_add(dKk, kmajor_off(ks, G::KATOM)), I_P, ks > 0 ? 1u : 0u);
-          mma_commit(&bar.p_full);
+            mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
+                        I_O, ks > 0 ? 1u : 0u);
+          if (MODE == kCausalOut) {
+#pragma unroll
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)),
+                          I_S, 1u);
+            mma_commit(&bar.s_full);
+            if (!mbar_wait(&bar.p_ready, g & 1, abort, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tO, desc_add(dP, kmajor_off(ks, kAtom)), desc_add(dVm, mnmajor_off(ks)),
+                          make_idesc_bf16(64, D, false, true), 1u);
+          }
+          mma_commit(&bar.o_full[ob]);
+          mma_commit(&bar.empty[s]);
         }
-        // S_<c (and, non-causal, z) in the S operand; this O buffer drained
-        if (MODE == kCausalOut || c == 0)
-          if (!mbar_wait(&bar.s_ready, MODE == kCausalOut ? (c & 1) : 0, abort, err)) break;
-        if (c >= 2 && !mbar_wait(&bar.o_empty[ob], ((c >> 1) - 1) & 1, abort, err)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < KSD; ++ks)
-          mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)), I_O,
-                      ks > 0 ? 1u : 0u);
-        if (MODE == kCausalOut) {
-#pragma unroll
-          for (int ks = 0; ks < KSC; ++ks)
-            mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
-                        1u);
-          mma_commit(&bar.s_full);
-          if (!mbar_wait(&bar.p_ready, c & 1, abort, err)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < KSC; ++ks)
-            mma_bf16_ss(tO, desc_add(dP, kmajor_off(ks, kAtom)), desc_add(dVm, mnmajor_off(ks)),
-                        make_idesc_bf16(64, D, false, true), 1u);
-        }
-        mma_commit(&bar.o_full[ob]);
-        mma_commit(&bar.empty[s]);
+        if (!ok) break;
+        if (MODE == kState) mma_commit(&bar.item_full[b]);        // aggregate complete
+        if (MODE == kNoncausalOut) mma_commit(&bar.item_empty[b]);  // S operand no longer read
       }
-      if (MODE == kState) mma_commit(&bar.s_full);
       // every MMA this CTA issued has finished before TMEM is released
       mma_commit(&bar.fin);
       mbar_wait(&bar.fin, 0, abort, err);
     }
-  } else if (warp < kWarpState0) {
+  } else if (warp < W::STATE0) {
     // ================================================================ feature map
-    // phi in place on the Q tile and on the 64 key rows of each K atom; K rows past n are
-    // zeroed (they must add nothing to S, z or the scores).
+    // phi in place on the Q tile and on the 64 key rows of each K atom; K rows past the
+    // item's end are zeroed (they must add nothing to S, z or the scores).
     const int xt = threadIdx.x - kWarpXform0 * 32;
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c % NS;
-      if (!mbar_wait(&bar.full[s], (c / NS) & 1, abort, err)) break;
-      uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
-      const int64_t left = t_end - (t_begin + (int64_t)c * C);
-      const int valid = left < C ? static_cast<int>(left) : C;
-      if (G::LQ) {
-        uint4 *p = reinterpret_cast<uint4 *>(st);
-#pragma unroll 2
-        for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
-          uint4 x = p[i];
-          x.x = phi_bf16x2(x.x);
-          x.y = phi_bf16x2(x.y);
-          x.z = phi_bf16x2(x.z);
-          x.w = phi_bf16x2(x.w);
-          p[i] = x;
+    int g = 0;
+    bool ok = true;
+    for (int64_t it = it0; ok && it < nitems; it += istep) {
+      const Item I = item_at(it, n, seg_len, nseg);
+      for (int c = 0; c < I.nchunks; ++c, ++g) {
+        const int s = g % NS;
+        if (!mbar_wait(&bar.full[s], (g / NS) & 1, abort, err)) {
+          ok = false;
+          break;
         }
-      }
-      if (G::LKV) {
+        uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+        const int64_t left = I.t_end - (I.t_begin + (int64_t)c * C);
+        const int valid = left < C ? static_cast<int>(left) : C;
+        if (G::LQ) {
+          uint4 *p = reinterpret_cast<uint4 *>(st);
 #pragma unroll 2
-        for (int i = xt; i < G::TILE / 16; i += kXformThreads) {
-          const int a = i / (kAtom / 16), within = i % (kAtom / 16);
-          const int row = within >> 3;  // 8 x 16 B per 128-byte row
-          uint4 *p = reinterpret_cast<uint4 *>(st + G::OFF_K + a * G::KATOM) + within;
-          uint4 x = make_uint4(0u, 0u, 0u, 0u);
-          if (row < valid) {
-            x = *p;
+          for (int i = xt; i < G::TILE / 16; i += W::XTHREADS) {
+            uint4 x = p[i];
             x.x = phi_bf16x2(x.x);
             x.y = phi_bf16x2(x.y);
             x.z = phi_bf16x2(x.z);
             x.w = phi_bf16x2(x.w);
+            p[i] = x;
           }
-          *p = x;
         }
+        if (G::LKV) {
+#pragma unroll 2
+          for (int i = xt; i < G::TILE / 16; i += W::XTHREADS) {
+            const int a = i / (kAtom / 16), within = i % (kAtom / 16);
+            const int row = within >> 3;  // 8 x 16 B per 128-byte row
+            uint4 *p = reinterpret_cast<uint4 *>(st + G::OFF_K + a * G::KATOM) + within;
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);
+            if (row < valid) {
+              x = *p;
+              x.x = phi_bf16x2(x.x);
+              x.y = phi_bf16x2(x.y);
+              x.z = phi_bf16x2(x.z);
+              x.w = phi_bf16x2(x.w);
+            }
+            *p = x;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bar.ready[s]);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&bar.ready[s]);
     }
-  } else if (warp < kWarpOut0) {
+  } else if (warp < W::OUT0) {
     // ================================================================ state group
     // Causal: half of each chunk's scores (columns 0..31) and their row sums; S_<c+1, z_<c+1
-    // -> bf16 operands of the next chunk (z into that chunk's K tile row 64).  Also the
-    // starting state and the segment aggregate (state mode).  Control flow is warp-uniform:
-    // lane 0 waits and the warp shares the outcome.
+    // -> bf16 operands of the next chunk (z into that chunk's K tile row 64); each item's
+    // starting state.  Non-causal: each item's head total -> one of the two S operands.
+    // State mode: each item's aggregate.  Control flow is warp-uniform: lane 0 waits and the
+    // warp shares the outcome.
     const int sp = warp & 3;  // TMEM sub-partition of this warp
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
     const bool v64 = lane < 16;                      // lanes holding rows of an M=64 tile
@@ -479,10 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rS = D == 128 ? 32 * sp + lane : r64;  // row of the S accumulator (M = D)
     const bool vS = D == 128 ? true : v64;
     WarpWaiter wait{abort, err, lane};
-    uint8_t *sS = smem + G::OFF_S;
 
-    // 32 consecutive S columns [c0, c0+32) of row rS (fp32 in registers) -> bf16 operand
-    auto store_S32 = [&](const uint32_t *r, int c0) {
+    // 32 consecutive S columns [c0, c0+32) of row rS (fp32 in registers) -> bf16 operand sS
+    auto store_S32 = [&](uint8_t *sS, const uint32_t *r, int c0) {
       if (!vS) return;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -493,23 +577,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    sw128_offset(rS, (c0 & 63) + 8 * j)) = pack8(f);
       }
     };
-    // z_<c for chunk c: causal -> row 64 of that chunk's K atoms; non-causal -> column 0 of
-    // the S operand's z atom
-    auto store_z = [&](uint32_t zbits, int c) {
+    // z_< for chunk gg: causal -> row 64 of that chunk's K atoms; non-causal -> column 0 of
+    // the z atom of the S operand sS
+    auto store_z = [&](uint8_t *sS, uint32_t zbits, int gg) {
       if (!vS) return;
       const __nv_bfloat16 zb = __float2bfloat16_rn(__uint_as_float(zbits));
       if (MODE == kCausalOut) {
-        uint8_t *kt = smem + G::OFF_STAGES + (c % NS) * G::STAGE + G::OFF_K;
+        uint8_t *kt = smem + G::OFF_STAGES + (gg % NS) * G::STAGE + G::OFF_K;
         *reinterpret_cast<__nv_bfloat16 *>(kt + (rS >> 6) * G::KATOM +
                                            sw128_offset(64, rS & 63)) = zb;
       } else {
         *reinterpret_cast<__nv_bfloat16 *>(sS + G::A * D * 128 + sw128_offset(rS, 0)) = zb;
       }
     };
-
-    if (MODE != kState) {
-      // starting state: exclusive prefix (causal) or the head's total (non-causal)
-      const float *src = init_state + head * init_head_stride + seg * init_seg_stride;
+    // an item's starting state (exclusive prefix, causal; the head's total, non-causal) ->
+    // TMEM S (causal) and the bf16 operand sS; z for the item's first chunk gg
+    auto load_start = [&](const Item &I, uint8_t *sS, int gg) {
+      const float *src = init_state + I.head * init_head_stride + I.seg * init_seg_stride;
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t r[32];
 #pragma unroll
@@ -527,79 +611,112 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tmem + lane_off + TM::S + c0 + 16 * j,
                       *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * j));
         }
-        store_S32(r, c0);
+        store_S32(sS, r, c0);
       }
       const uint32_t zb = vS ? __float_as_uint(src[(int64_t)D * D + rS]) : 0u;
       if (MODE == kCausalOut) {
         tmem_st1(tmem + lane_off + TM::S + D, zb);
         tmem_st_wait();
       }
-      store_z(zb, 0);
+      store_z(sS, zb, gg);
       fence_proxy_async_smem();
-      tc_fence_before();
-      if (MODE == kCausalOut) mbar_arrive(&bar.z_ready);
-      mbar_arrive(&bar.s_ready);
-    }
+    };
 
     if (MODE == kCausalOut) {
-      for (int c = 0; c < nchunks; ++c) {
+      // One flat loop over this CTA's chunks; only the chunk counter, the chunks left in
+      // the current item and the next item's index stay live across it.
+      uint8_t *sS = smem + G::OFF_S;
+      int64_t it = it0;
+      int left = 0;
+#pragma unroll 1
+      for (int g = 0;; ++g) {
+        if (left == 0) {
+          // ---- an item's starting state, once the previous item's last S and O products
+          // are done with TMEM S and the S operand
+          if (it >= nitems) break;
+          const Item I = item_at(it, n, seg_len, nseg);
+          it += istep;
+          left = I.nchunks;
+          if (g == 0 || wait(&bar.s_full, (g - 1) & 1)) {
+            tc_fence_after();
+            load_start(I, sS, g);
+            tc_fence_before();
+          }
+          mbar_arrive(&bar.z_ready);
+          mbar_arrive(&bar.s_ready);
+        }
         // ---- this chunk's scores, columns 0..31 (the output group takes 32..63)
-        if (wait(&bar.p_full, c & 1)) {
+        if (wait(&bar.p_full, g & 1)) {
           tc_fence_after();
           const float rs = convert_P32(tmem + lane_off + TM::P, smem + G::OFF_P, r64, v64, 0);
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bar.p_ready);
-          if (v64) bar.rowsum[c & 1][r64] = rs;
+          if (v64) bar.rowsum[g & 1][r64] = rs;
           mbar_arrive(&bar.rs_ready);
         }
-        // ---- S_<c+1, z_<c+1: the operands of the next chunk
-        if (c + 1 < nchunks && wait(&bar.s_full, c & 1)) {
+        // ---- S_<c+1, z_<c+1: the operands of the item's next chunk
+        if (--left > 0 && wait(&bar.s_full, g & 1)) {
           tc_fence_after();
           // z_<c+1 first: the next chunk's score MMA needs only that
-          store_z(tmem_ld1(tmem + lane_off + TM::S + D), c + 1);
+          store_z(sS, tmem_ld1(tmem + lane_off + TM::S + D), g + 1);
           fence_proxy_async_smem();
           mbar_arrive(&bar.z_ready);
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 64) {
             uint32_t r[64];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * j, r + 16 * j);
+            for (int q = 0; q < 4; ++q)
+              tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * q, r + 16 * q);
             tmem_ld_wait();
             tmem_reg_fence<64>(r);
-            store_S32(r, c0);
-            store_S32(r + 32, c0 + 32);
+            store_S32(sS, r, c0);
+            store_S32(sS, r + 32, c0 + 32);
           }
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bar.s_ready);
         }
       }
-    }
-
-    if (MODE == kState) {
-      // segment aggregate -> fp32 workspace [D][d] then z[D]
-      if (wait(&bar.s_full, 0)) {
-        tc_fence_after();
-        float *dst = out_state + (head * nseg + seg) * (int64_t)(D * D + D);
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t r[32];
+    } else if (MODE == kNoncausalOut) {
+      int j = 0;
+      for (int64_t it = it0; it < nitems; it += istep, ++j) {
+        const Item I = item_at(it, n, seg_len, nseg);
+        const int b = j & 1;
+        uint8_t *sS = smem + G::OFF_S + b * G::S_BUF;
+        // the MMAs of item j - 2 no longer read this S operand
+        if (j < 2 || wait(&bar.item_empty[b], ((j >> 1) - 1) & 1)) load_start(I, sS, 0);
+        mbar_arrive(&bar.item_full[b]);
+      }
+    } else {
+      // segment aggregates -> fp32 workspace [D][d] then z[D]
+      int j = 0;
+      for (int64_t it = it0; it < nitems; it += istep, ++j) {
+        const Item I = item_at(it, n, seg_len, nseg);
+        const int b = j & 1;
+        const uint32_t tS = tmem + lane_off + (b ? TM::S1 : TM::S);
+        if (wait(&bar.item_full[b], (j >> 1) & 1)) {
+          tc_fence_after();
+          float *dst = out_state + (I.head * nseg + I.seg) * (int64_t)(D * D + D);
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * j, r + 16 * j);
-          tmem_ld_wait();
-          tmem_reg_fence<32>(r);
-          if (vS) {
+            for (int q = 0; q < 2; ++q) tmem_ld16_async(tS + c0 + 16 * q, r + 16 * q);
+            tmem_ld_wait();
+            tmem_reg_fence<32>(r);
+            if (vS) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4 *>(dst + (int64_t)rS * D + c0 + e) =
-                  make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                              __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4 *>(dst + (int64_t)rS * D + c0 + e) =
+                    make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+            }
           }
+          const uint32_t zr = tmem_ld1(tS + D);
+          if (vS) dst[(int64_t)D * D + rS] = __uint_as_float(zr);
         }
-        const uint32_t zr = tmem_ld1(tmem + lane_off + TM::S + D);
-        if (vS) dst[(int64_t)D * D + rS] = __uint_as_float(zr);
+        tc_fence_before();
+        mbar_arrive(&bar.item_empty[b]);
       }
     }
   } else {
@@ -607,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P(c) columns 32..63 -> masked bf16 operand of P V (the state group takes 0..31), with
     // phi(q).z_<c (column 64) and both groups' row sums -> the denominator of chunk c; then
     // O(c-1) / den -> bf16 rows stored straight to global memory (32-byte stores; rows past
-    // n are not written).
+    // the item's end are not written).
     const int sp = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
     const bool v64 = lane < 16;
@@ -619,43 +736,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     // chunk's p_ready, so it never completes rs_ready's next phase (or rewrites that slot)
     // before this wait has seen the current one.
     float den0 = 1.f, den1 = 1.f;
-    auto convert_P = [&](int c) {
-      if (!wait(&bar.p_full, c & 1)) return;
+    auto convert_P = [&](int gg) {
+      if (!wait(&bar.p_full, gg & 1)) return;
       tc_fence_after();
       const float rs = convert_P32(tmem + lane_off + TM::P, smem + G::OFF_P, r64, v64, 32);
       const float dz = __uint_as_float(tmem_ld1(tmem + lane_off + TM::P + 64));
-      const bool got = wait(&bar.rs_ready, c & 1);
-      const float d = dz + rs + (got ? bar.rowsum[c & 1][v64 ? r64 : 0] : 0.f);
-      if (c & 1) den1 = d; else den0 = d;
+      const bool got = wait(&bar.rs_ready, gg & 1);
+      const float d = dz + rs + (got ? bar.rowsum[gg & 1][v64 ? r64 : 0] : 0.f);
+      if (gg & 1) den1 = d; else den0 = d;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar.p_ready);
     };
 
-    auto emit_O = [&](int c) {
-      const int ob = c & 1;
+    // O of chunk gg (chunk c of item I)
+    auto emit_O = [&](int gg, const Item &I, int c) {
+      const int ob = gg & 1;
       const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
-      if (!wait(&bar.o_full[ob], (c >> 1) & 1)) return;
+      if (!wait(&bar.o_full[ob], (gg >> 1) & 1)) return;
       tc_fence_after();
       const float dd = MODE == kCausalOut ? (ob ? den1 : den0) : __uint_as_float(tmem_ld1(tO + D));
       const float inv = 1.f / dd;
-      const int64_t t = t_begin + (int64_t)c * C + r64;
-      const bool live = v64 && t < t_end;
-      __nv_bfloat16 *orow = out + (head * n + (live ? t : 0)) * D;
+      const int64_t t = I.t_begin + (int64_t)c * C + r64;
+      const bool live = v64 && t < I.t_end;
+      __nv_bfloat16 *orow = out + (I.head * n + (live ? t : 0)) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 64) {
         uint32_t r[64];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld16_async(tO + c0 + 16 * j, r + 16 * j);
+        for (int q = 0; q < 4; ++q) tmem_ld16_async(tO + c0 + 16 * q, r + 16 * q);
         tmem_ld_wait();
         tmem_reg_fence<64>(r);
         if (live) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int q = 0; q < 4; ++q) {
             float f[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * j + e]) * inv;
-            st_global_32B(orow + c0 + 16 * j, pack8(f), pack8(f + 8));
+            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
+            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8));
           }
         }
       }
@@ -664,13 +782,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if (MODE == kCausalOut) {
-      for (int c = 0; c < nchunks; ++c) {
-        convert_P(c);
-        if (c >= 1) emit_O(c - 1);
+      int g = 0;
+      Item prev{};
+      int prev_c = 0;
+      for (int64_t it = it0; it < nitems; it += istep) {
+        const Item I = item_at(it, n, seg_len, nseg);
+        for (int c = 0; c < I.nchunks; ++c, ++g) {
+          convert_P(g);
+          if (g >= 1) emit_O(g - 1, prev, prev_c);
+          prev = I;
+          prev_c = c;
+        }
       }
-      if (nchunks > 0) emit_O(nchunks - 1);
+      if (g > 0) emit_O(g - 1, prev, prev_c);
     } else if (MODE == kNoncausalOut) {
-      for (int c = 0; c < nchunks; ++c) emit_O(c);
+      int g = 0;
+      for (int64_t it = it0; it < nitems; it += istep) {
+        const Item I = item_at(it, n, seg_len, nseg);
+        for (int c = 0; c < I.nchunks; ++c, ++g) emit_O(g, I, c);
+      }
     }
   }
 
@@ -710,6 +840,21 @@ cudaError_t make_tmap(CUtensorMap *m, const void *ptr, int64_t heads, int64_t n,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
 template <int D, int MODE>
 cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                       void *out, const float *init, int64_t ihs, int64_t iss,
@@ -719,8 +864,19 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
   auto kern = tc_kernel<D, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(heads * nseg), kThreads, G::SMEM, st>>>(
-      q, k, v, static_cast<__nv_bfloat16 *>(out), init, ihs, iss, out_state, n, seg, nseg, err);
+  // One CTA holds a whole SM's shared memory and TMEM.  Persistent CTAs (one per SM, items
+  // dealt round-robin) save each item the CTA start-up and pipeline fill and drain; they
+  // pay off for the aggregate and non-causal kernels and for short causal items.  Long
+  // causal items run one CTA each: there the hardware's dynamic placement of CTAs on SMs
+  // evens out the few per cent by which SMs differ in speed, and a fresh CTA hides the load
+  // of its starting state behind its first TMA loads.
+  const int64_t nitems = heads * nseg;
+  const int64_t sms = sm_count();
+  const bool persistent = MODE != kCausalOut || seg <= kPersistentCausalChunks * C;
+  const int64_t want = persistent ? sms : nitems;
+  const unsigned grid = static_cast<unsigned>(nitems < want ? nitems : want);
+  kern<<<grid, Warps<MODE>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out), init, ihs,
+                                        iss, out_state, n, seg, nseg, nitems, err);
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();
