@@ -370,6 +370,17 @@ def main_forward(args, world, rank, local):
         e2e = {"value": tokens_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": 3 * qh.numel() * elem,
                "d2h_bytes_per_step": outh.numel() * elem}
+        # the host link's own rate on one input tensor, for context
+        t0, t1, t2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        t0.record()
+        tmp = qh.to("cuda", non_blocking=True)
+        t1.record()
+        outh.copy_(tmp, non_blocking=True)
+        t2.record()
+        torch.cuda.synchronize()
+        e2e["h2d_gbs"] = qh.numel() * elem / (t0.elapsed_time(t1) * 1e-3) / 1e9
+        e2e["d2h_gbs"] = qh.numel() * elem / (t1.elapsed_time(t2) * 1e-3) / 1e9
+        del tmp
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -493,8 +504,14 @@ def extras(args):
             q, k, v = workloads.forward_inputs(name, dt)
             o = torch.empty_like(q)
             causal = True in w.causal
-            ms, _ = time_steps(lambda: la.forward(q, k, v, causal, out=o), 50, 5, 1)
-            res[f"{name}_{dt}"] = {"us": ms * 1e3, "tokens_per_s": w.B * w.n / (ms * 1e-3)}
+            fn = lambda: la.forward(q, k, v, causal, out=o)  # noqa: E731
+            ms, _ = time_steps(fn, 50, 5, 1)
+            # back-to-back calls of a small problem measure the host's call rate; the device
+            # time of one call is the sum of its launches
+            dev = time_launches(fn, 20, 5, ["K1", "K2", "K3"])
+            dev_us = sum(dev.values()) * 1e3
+            res[f"{name}_{dt}"] = {"us": ms * 1e3, "device_us": dev_us,
+                                   "tokens_per_s": w.B * w.n / (ms * 1e-3)}
     return res
 
 

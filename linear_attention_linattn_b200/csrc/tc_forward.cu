@@ -403,6 +403,9 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
       constexpr uint32_t I_P = make_idesc_bf16(64, 64 + kZRows, false, false);
       constexpr uint32_t I_O = make_idesc_bf16(64, MODE == kNoncausalOut ? D + 16 : D, false, true);
       constexpr uint32_t I_S = make_idesc_bf16(D, D + 16, true, true);
+      constexpr uint32_t I_OV = make_idesc_bf16(64, D, false, true);
+      uint64_t dVprev = 0;  // causal: [V | ones] of the previous chunk (its P V is still due)
+      int sprev = 0;        // and that chunk's stage
       const uint32_t tP = tmem + TM::P;
       const uint64_t dP = kmajor_base(smem_u32(smem + G::OFF_P));
       const uint32_t st0 = smem_u32(smem + G::OFF_STAGES);
@@ -444,23 +447,56 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
           const int ob = g & 1;
           const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0);
           if (MODE == kCausalOut) {
-            // [scores | phi(q).z_<c] first, as soon as z_<c sits in this chunk's K tile: the
-            // score warps start on them while the S snapshot is still being rounded
+            // The previous chunk's P V (its scores rounded by now) interleaved with this
+            // chunk's [scores | phi(q).z_<c]: different accumulators, so the tensor pipe
+            // overlaps the two chains instead of running them back to back.
             if (!mbar_wait(&bar.z_ready, g & 1, abort, err)) {
               ok = false;
               break;
             }
+            if (g >= 1 && !mbar_wait(&bar.p_ready, (g - 1) & 1, abort, err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
+            const uint32_t tOp = tmem + (((g - 1) & 1) ? TM::O1 : TM::O0);  // O of chunk g - 1
 #pragma unroll
-            for (int ks = 0; ks < KSD; ++ks)
+            for (int ks = 0; ks < KSD; ++ks) {
+              if (g >= 1 && ks < KSC)
+                mma_bf16_ss(tOp, desc_add(dP, kmajor_off(ks, kAtom)),
+                            desc_add(dVprev, mnmajor_off(ks)), I_OV, 1u);
               mma_bf16_ss(tP, desc_add(dQk, kmajor_off(ks, kAtom)),
                           desc_add(dKk, kmajor_off(ks, G::KATOM)), I_P, ks > 0 ? 1u : 0u);
+              if (g >= 1 && ks == KSC - 1) {
+                mma_commit(&bar.o_full[(g - 1) & 1]);
+                mma_commit(&bar.empty[sprev]);
+              }
+            }
             mma_commit(&bar.p_full);
-            // S_<c in the S operand
+            // S_<c in the S operand; this O buffer drained
             if (!mbar_wait(&bar.s_ready, g & 1, abort, err)) {
               ok = false;
               break;
             }
+            if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // phi(Q_c) S_<c, then S += phi(K_c)^T [V_c | 1] (interleaving these two measured
+            // no faster)
+#pragma unroll
+            for (int ks = 0; ks < KSD; ++ks)
+              mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
+                          I_O, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
+                          1u);
+            mma_commit(&bar.s_full);
+            dVprev = dVm;  // P V of this chunk goes with the next chunk's scores
+            sprev = s;
+            continue;
           }
           // this O buffer drained
           if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
@@ -472,28 +508,25 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
                         I_O, ks > 0 ? 1u : 0u);
-          if (MODE == kCausalOut) {
-#pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)),
-                          I_S, 1u);
-            mma_commit(&bar.s_full);
-            if (!mbar_wait(&bar.p_ready, g & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tO, desc_add(dP, kmajor_off(ks, kAtom)), desc_add(dVm, mnmajor_off(ks)),
-                          make_idesc_bf16(64, D, false, true), 1u);
-          }
           mma_commit(&bar.o_full[ob]);
           mma_commit(&bar.empty[s]);
         }
         if (!ok) break;
         if (MODE == kState) mma_commit(&bar.item_full[b]);        // aggregate complete
         if (MODE == kNoncausalOut) mma_commit(&bar.item_empty[b]);  // S operand no longer read
+      }
+      if (MODE == kCausalOut && ok && g > 0) {
+        // the last chunk's P V
+        if (mbar_wait(&bar.p_ready, (g - 1) & 1, abort, err)) {
+          tc_fence_after();
+          const uint32_t tOp = tmem + (((g - 1) & 1) ? TM::O1 : TM::O0);
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tOp, desc_add(dP, kmajor_off(ks, kAtom)), desc_add(dVprev, mnmajor_off(ks)),
+                        I_OV, 1u);
+          mma_commit(&bar.o_full[(g - 1) & 1]);
+          mma_commit(&bar.empty[sprev]);
+        }
       }
       // every MMA this CTA issued has finished before TMEM is released
       mma_commit(&bar.fin);
