@@ -156,3 +156,48 @@ def test_workload_longctx_1x32x131072x128_bf16():
     ref = oracle.forward_rows(q[0, heads], k[0, heads], v[0, heads], rows, True)
     gs = np.stack([got[0, h][rows] for h in heads])
     assert max_row_rel_err(gs, ref) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ persistent work items
+# The tensor-core kernels walk a list of (head, segment) items per CTA (one per SM); these
+# cases put several items of different lengths on each CTA, and ragged final segments.
+def _sampled_parity(q, k, v, causal, segment_len, heads_to_check, seed):
+    got = _run(q, k, v, causal, "bf16", segment_len=segment_len)
+    assert np.all(np.isfinite(got))
+    B, H, n, d = q.shape
+    rows = _sample_rows(n, 24, seed)
+    qs = np.stack([q[b, h] for b, h in heads_to_check])
+    ks = np.stack([k[b, h] for b, h in heads_to_check])
+    vs = np.stack([v[b, h] for b, h in heads_to_check])
+    ref = oracle.forward_rows(qs, ks, vs, rows, causal)
+    gs = np.stack([got[b, h][rows] for b, h in heads_to_check])
+    assert max_row_rel_err(gs, ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_persistent_many_heads_ragged_items(causal, d):
+    """400 heads of 200 tokens: more items than SMs, each ending in a partial chunk."""
+    B, H, n = 4, 100, 200
+    q, k, v = (inputs.round_bf16(x) for x in inputs.forward_qkv(21, B, H, n, d, scaled=True))
+    _sampled_parity(q, k, v, causal, 0, [(0, 0), (1, 37), (2, 63), (3, 99)], 3)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("seg", [256, 2304])
+def test_persistent_segments_of_unequal_length(causal, seg):
+    """160 heads split into segments whose last one is shorter (n = 4500): the items of one
+    CTA differ in length.  seg = 256 runs the causal items on persistent CTAs (4 chunks
+    each), seg = 2304 runs them one CTA per item (36 chunks)."""
+    B, H, n, d = 2, 80, 4500, 64
+    q, k, v = (inputs.round_bf16(x) for x in inputs.forward_qkv(22, B, H, n, d, scaled=True))
+    _sampled_parity(q, k, v, causal, seg, [(0, 0), (0, 79), (1, 5), (1, 79)], 4)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fewer_items_than_sms(causal):
+    """3 heads x 2 segments: a grid of 6 CTAs, one item each."""
+    B, H, n, d = 1, 3, 700, 128
+    q, k, v = (inputs.round_bf16(x) for x in inputs.forward_qkv(23, B, H, n, d, scaled=True))
+    got = _run(q, k, v, causal, "bf16", segment_len=384)
+    assert max_row_rel_err(got, oracle.forward(q, k, v, causal)) <= TOL["bf16"]
