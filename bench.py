@@ -2,7 +2,7 @@
 """Benchmark: linear-attention forward tokens/s and achieved HBM GB/s on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-extras]
+                    [--workload NAME] [--shard heads|seq] [--no-extras]
 
 Default workload (one step = one pass of the whole forward path, phi feature map, chunk
 aggregates, inter-chunk prefix and intra-chunk output, over one batch): the long-context
@@ -13,6 +13,9 @@ is needed between timed steps.
 Multi-GPU (torchrun, one process per GPU): heads are independent, so each rank runs its
 own batch element of the workload (batch index = rank) with no data-path collective;
 value = all ranks' tokens / the max over ranks of the device time ("scaling": "weak").
+``--shard seq`` instead splits one sequence per head over the ranks: each rank computes its
+block's state, the ranks all-gather the block states once, and each continues its block
+from the states before it ("scaling": "strong"; linear_attention_linattn_b200.seqshard).
 
 At N=1 the line also carries the decode step (256 x 32 states, d = 128, 512 steps), the
 batched 8x16x8192x64 forward (both modes) and the small latency cases under "extras", and
@@ -36,7 +39,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from linear_attention_linattn_b200 import inputs  # noqa: E402
+from linear_attention_linattn_b200 import inputs, seqshard  # noqa: E402
 
 METRIC = "linear-attention fwd tokens/sec and achieved HBM GB/s (fraction of B200 peak)"
 MAIN = "longctx_1x32x131072x128_bf16"
@@ -315,10 +318,21 @@ def main_forward(args, world, rank, local):
     dtype = "bf16" if "bf16" in w.dtypes else "f32"
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     elem = 2 if dtype == "bf16" else 4
-    # this rank's batch element of the workload: b = rank (weak scaling over ranks)
-    q, k, v = inputs.forward_qkv(w.seed, w.B * world, w.H, w.n, w.d, w.scaled,
-                                 heads=rank_heads(w.B, w.H, rank))
-    shape = (w.B, w.H, w.n, w.d)
+    seq = args.shard == "seq"
+    if seq:
+        # one sequence per head split over the ranks: rank r holds tokens
+        # [r*n/N, (r+1)*n/N) of every head (strong scaling, one all-gather of block states)
+        if w.n % (world * 64) != 0:
+            raise SystemExit(f"--shard seq needs n divisible by 64 * ranks (n = {w.n})")
+        blk = w.n // world
+        q, k, v = inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled)
+        q, k, v = (np.ascontiguousarray(x[:, :, rank * blk:(rank + 1) * blk]) for x in (q, k, v))
+        shape = (w.B, w.H, blk, w.d)
+    else:
+        # this rank's batch element of the workload: b = rank (weak scaling over ranks)
+        q, k, v = inputs.forward_qkv(w.seed, w.B * world, w.H, w.n, w.d, w.scaled,
+                                     heads=rank_heads(w.B, w.H, rank))
+        shape = (w.B, w.H, w.n, w.d)
     qh = torch.from_numpy(q.reshape(shape)).to(tdt).pin_memory()
     kh = torch.from_numpy(k.reshape(shape)).to(tdt).pin_memory()
     vh = torch.from_numpy(v.reshape(shape)).to(tdt).pin_memory()
@@ -327,7 +341,10 @@ def main_forward(args, world, rank, local):
     out = torch.empty_like(qd)
 
     def step():
-        la.forward(qd, kd, vd, causal, out=out)
+        if seq:
+            seqshard.forward_sequence_sharded(qd, kd, vd, causal)
+        else:
+            la.forward(qd, kd, vd, causal, out=out)
 
     clocks = ClockSampler(local)
     l0 = la.linattn_launch_count()
@@ -336,11 +353,11 @@ def main_forward(args, world, rank, local):
     clk = clocks.stop()
     assert la.device_error() == la.LINATTN_OK
 
-    tokens_rank = w.B * w.n
+    tokens_rank = w.B * shape[2]
     value = tokens_rank * world / (ms * 1e-3)
     pk = peaks()
-    alg = forward_bytes(w.B, w.H, w.n, w.d, elem)
-    unit = w.B * w.H * w.n * w.d * elem  # one [B,H,n,d] tensor
+    alg = forward_bytes(w.B, w.H, shape[2], w.d, elem)  # this rank's share
+    unit = w.B * w.H * shape[2] * w.d * elem  # one [B,H,n,d] tensor (this rank's share)
     if dtype == "bf16":
         names = ["tc_kernel<state> (segment aggregates, K1)", "scan_states_kernel (prefix, K2)",
                  "tc_kernel<causal out> (K3)" if causal else "tc_kernel<non-causal out> (K3)"]
@@ -349,6 +366,11 @@ def main_forward(args, world, rank, local):
         names = ["simt_chunk_state_kernel (K1)", "scan_states_kernel (K2)",
                  "simt_chunk_out_kernel (K3)"]
         kbytes = [2 * unit, 0, 4 * unit if causal else 2 * unit]
+    if seq:
+        # block state (K1, total), the start state, then the forward from it (K1, K2, K3)
+        names = ["block state: " + names[0], "block state: total (K2)",
+                 "sum_states_kernel"] + names
+        kbytes = [2 * unit, 0, 0] + kbytes
     launch_ms = time_launches(step, max(3, min(args.steps, 10)), 2, names)
     top = max(launch_ms, key=launch_ms.get)
     kernel_ms = launch_ms[top]
@@ -360,7 +382,10 @@ def main_forward(args, world, rank, local):
 
     def e2e_step():
         a, b_, c = (x.to("cuda", non_blocking=True) for x in (qh, kh, vh))
-        o = la.forward(a, b_, c, causal)
+        if seq:
+            o = seqshard.forward_sequence_sharded(a, b_, c, causal)
+        else:
+            o = la.forward(a, b_, c, causal)
         outh.copy_(o, non_blocking=True)
 
     e2e = None
@@ -385,13 +410,17 @@ def main_forward(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+        "higher_is_better": True, "scaling": "strong" if seq else "weak", "vs_baseline": None,
+        "dtype": dtype,
         "data": "synthetic (seeded N(0,1)/sqrt(d), see DESIGN.md input recipe)",
         "config": {"workload": args.workload + (f" (first {w.H} heads)" if args.max_heads else "")
                    + (f" [{args.mode}]" if args.mode else ""),
                    "B": w.B, "H": w.H, "n": w.n, "d": w.d,
-                   "causal": causal, "global_batch": w.B * world, "seq_len": w.n,
-                   "parallelism": f"dp{world} (independent heads, no collective)",
+                   "causal": causal, "global_batch": w.B if seq else w.B * world,
+                   "seq_len": w.n,
+                   "parallelism": (f"sequence split over {world} ranks (one all-gather of "
+                                   "block states)") if seq else
+                                  f"dp{world} (independent heads, no collective)",
                    "l2": "inputs larger than L2 (no flush needed)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
@@ -525,6 +554,9 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard", choices=["heads", "seq"], default="heads",
+                    help="heads: every rank runs its own batch element (weak scaling); seq: "
+                         "one sequence per head split over the ranks (strong scaling)")
     ap.add_argument("--mode", choices=["causal", "noncausal"], default=None,
                     help="for a workload that has both modes (default: causal)")
     ap.add_argument("--max-heads", type=int, default=0,

@@ -97,6 +97,39 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
                                      int64_t d, linattn_dtype dtype, linattn_stream_t stream);
 
 /*
+ * linattn_forward continued from a given state: the pass over tokens [0, n) of each head
+ * starts from (state_S[b][h] [D][d], state_z[b][h] [D], float32, device memory, read only).
+ *   causal = 1: the state is that of the tokens before this block (the recurrent view's
+ *     S_t, z_t at the block's start), so out_i = phi(q_i)(S0 + sum_{j<=i} phi(k_j) v_j^T) /
+ *     phi(q_i).(z0 + sum_{j<=i} phi(k_j)).  With state 0 this is linattn_forward.
+ *   causal = 0: the state is what the rest of the sequence contributes, so
+ *     out_i = phi(q_i)(S0 + sum_j phi(k_j) v_j^T) / phi(q_i).(z0 + sum_j phi(k_j)).
+ * This splits one sequence over several calls or devices: each block's state comes from
+ * linattn_forward_state of the other blocks, summed with linattn_sum_states.  Other
+ * arguments, layouts and errors as in linattn_forward; state_S and state_z must be 16-byte
+ * aligned.  (Pages: "Efficient Transformers: Linear Attention and Flash Attention", section
+ * "The recurrent view: attention as an RNN" — the state carries everything earlier tokens
+ * contribute.)
+ */
+linattn_status linattn_forward_init(const void *q, const void *k, const void *v, void *out,
+                                    const float *state_S, const float *state_z, int64_t B,
+                                    int64_t H, int64_t n, int64_t d, int causal,
+                                    linattn_dtype dtype, linattn_stream_t stream);
+
+/*
+ * Per-head sum of gathered states.  states: float32 device memory laid out
+ * [count][B][H][D*d + D] (each state: S row-major [D][d], then z [D]; this is what an
+ * all-gather of every rank's linattn_forward_state output, packed that way, produces).
+ * Writes state_S[b][h] = sum over i in [0, count), i != skip, of the S part of
+ * states[i][b][h] (added in order of i), and state_z likewise; zero when nothing is summed
+ * (count = 0).  skip = -1 sums every state.  All pointers 16-byte aligned; states may be
+ * null when count = 0.  d in {64, 128}.
+ */
+linattn_status linattn_sum_states(const float *states, int64_t count, int64_t skip, int64_t B,
+                                  int64_t H, int64_t d, float *state_S, float *state_z,
+                                  linattn_stream_t stream);
+
+/*
  * linattn_forward with a chosen segment length: the number of tokens one work item of
  * the chunked causal pass covers (a multiple of the chunk size; 0 picks the default).
  * The result does not depend on it beyond rounding order; tests use it to move the

@@ -9,9 +9,11 @@ raises.
 Raw C entry points (pointers as ints):
     linattn_forward, linattn_forward_ex, linattn_forward_state, linattn_decode_step,
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
-    linattn_launch_count, linattn_forward_noalloc, linattn_profile_events
+    linattn_launch_count, linattn_forward_noalloc, linattn_profile_events,
+    linattn_forward_init, linattn_sum_states
 
-Tensor helpers: ``forward``, ``forward_state``, ``decode_step``, ``device_error``.
+Tensor helpers: ``forward``, ``forward_init``, ``forward_state``, ``sum_states``,
+``decode_step``, ``device_error``; ``seqshard`` splits one sequence over ranks.
 """
 from __future__ import annotations
 
@@ -48,6 +50,9 @@ SIGNATURES = {
     "linattn_forward_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                                ctypes.c_int, ctypes.c_int, _vp]),
     "linattn_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
+    "linattn_forward_init": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                            _i64, ctypes.c_int, ctypes.c_int, _vp]),
+    "linattn_sum_states": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
 }
 
 _lib = None
@@ -132,6 +137,50 @@ def forward(q, k, v, causal: bool, out=None, segment_len: int = 0, stream=None):
                                 _stream_ptr(stream))
     _check(st, "linattn_forward")
     return out
+
+
+def forward_init(q, k, v, S0, z0, causal: bool, out=None, stream=None):
+    """forward continued from a state: S0 [B, H, d, d] and z0 [B, H, d] (float32) hold what
+    the tokens before this block (causal) or the rest of the sequence (non-causal)
+    contribute."""
+    import torch
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (S0, "S0"), (z0, "z0")):
+        _dev(t, nm)
+    if not (q.shape == k.shape == v.shape and q.dim() == 4 and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share one [B, H, n, d] shape and dtype")
+    B, H, n, d = q.shape
+    if S0.dtype != torch.float32 or z0.dtype != torch.float32 or \
+            tuple(S0.shape) != (B, H, d, d) or tuple(z0.shape) != (B, H, d):
+        raise ValueError("S0 must be float32 [B, H, d, d] and z0 float32 [B, H, d]")
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out")
+    lib = load_library()
+    st = lib.linattn_forward_init(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  S0.data_ptr(), z0.data_ptr(), B, H, n, d, int(bool(causal)),
+                                  _dtype_code(q), _stream_ptr(stream))
+    _check(st, "linattn_forward_init")
+    return out
+
+
+def sum_states(states, count: int, skip: int = -1, S=None, z=None, stream=None):
+    """states: float32 [G, B, H, d*d + d] (S row-major then z, per head).  Returns the sum of
+    states[i] over i < count, i != skip, as S [B, H, d, d] and z [B, H, d]."""
+    import torch
+    _dev(states, "states")
+    G, B, H, per = states.shape
+    d = int(round((-1 + (1 + 4 * per) ** 0.5) / 2))
+    if d * d + d != per or states.dtype != torch.float32 or not 0 <= count <= G:
+        raise ValueError("states must be float32 [G, B, H, d*d + d] and 0 <= count <= G")
+    if S is None:
+        S = torch.empty((B, H, d, d), dtype=torch.float32, device=states.device)
+    if z is None:
+        z = torch.empty((B, H, d), dtype=torch.float32, device=states.device)
+    lib = load_library()
+    st = lib.linattn_sum_states(states.data_ptr(), int(count), int(skip), B, H, d, S.data_ptr(),
+                                z.data_ptr(), _stream_ptr(stream))
+    _check(st, "linattn_sum_states")
+    return S, z
 
 
 def forward_state(k, v, S=None, z=None, stream=None):

@@ -81,21 +81,26 @@ linattn_status check_forward_shape(int64_t B, int64_t H, int64_t n, int64_t d) {
   return LINATTN_OK;
 }
 
+// init_S / init_z (nullable): the state before each head's first token (causal), or the
+// state the other tokens of the sequence contribute (non-causal).
 linattn_status forward_tc(const void *q, const void *k, const void *v, void *out,
                           int64_t heads, int64_t n, int d, int causal, int64_t seg,
-                          DeviceState *ds, cudaStream_t st) {
+                          const float *init_S, const float *init_z, DeviceState *ds,
+                          cudaStream_t st) {
   if (seg == 0) seg = tc_default_segment(heads, n, d);
   Workspace ws;
   ws.st = st;
   if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, d, seg, causal), ds->pool,
                               st) != cudaSuccess)
     return LINATTN_ERR_CUDA;
-  return to_status(tc_forward(q, k, v, out, heads, n, d, causal, seg, ws.ptr, ds->err_word, st));
+  return to_status(tc_forward(q, k, v, out, heads, n, d, causal, seg, ws.ptr, ds->err_word,
+                              init_S, init_z, st));
 }
 
 linattn_status forward_simt(const void *q, const void *k, const void *v, void *out,
                             int64_t heads, int64_t n, int d, int causal, int is_bf16,
-                            DeviceState *ds, cudaStream_t st) {
+                            const float *init_S, const float *init_z, DeviceState *ds,
+                            cudaStream_t st) {
   const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
   const int64_t per = (int64_t)d * d + d;
   // causal: one state per chunk; non-causal: chunk states plus one total per head
@@ -108,14 +113,15 @@ linattn_status forward_simt(const void *q, const void *k, const void *v, void *o
   e = launch_simt_chunk_state(k, v, w, heads, n, d, is_bf16, st);
   if (e != cudaSuccess) return LINATTN_ERR_CUDA;
   if (causal) {
-    e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, 0, nullptr, 0, st);
+    e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
     if (e != cudaSuccess) return LINATTN_ERR_CUDA;
     e = launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
                               nchunks * per, heads, n, d, 1, is_bf16, st);
   } else {
     float *tot = w + heads * nchunks * per;
     float *tot_z = tot + heads * (int64_t)d * d;
-    e = launch_scan_states(w, heads, nchunks, d, 1, tot, (int64_t)d * d, tot_z, d, st);
+    e = launch_scan_states(w, heads, nchunks, d, 1, tot, (int64_t)d * d, tot_z, d, init_S,
+                           init_z, st);
     if (e != cudaSuccess) return LINATTN_ERR_CUDA;
     e = launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, (int64_t)d * d, 0, d, heads, n, d, 0,
                               is_bf16, st);
@@ -146,8 +152,45 @@ linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, v
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == LINATTN_BF16)
-    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, segment_len, ds, st);
-  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, ds, st);
+    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, segment_len, nullptr, nullptr, ds,
+                      st);
+  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, ds, st);
+}
+
+linattn_status linattn_forward_init(const void *q, const void *k, const void *v, void *out,
+                                    const float *state_S, const float *state_z, int64_t B,
+                                    int64_t H, int64_t n, int64_t d, int causal,
+                                    linattn_dtype dtype, linattn_stream_t stream) {
+  if (!q || !k || !v || !out || !state_S || !state_z) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(state_S) || !aligned16(state_z))
+    return LINATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  linattn_status s = check_forward_shape(B, H, n, d);
+  if (s != LINATTN_OK) return s;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == LINATTN_BF16)
+    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, ds, st);
+  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, ds, st);
+}
+
+linattn_status linattn_sum_states(const float *states, int64_t count, int64_t skip, int64_t B,
+                                  int64_t H, int64_t d, float *state_S, float *state_z,
+                                  linattn_stream_t stream) {
+  if (!state_S || !state_z || (count > 0 && !states)) return LINATTN_ERR_INVALID_ARG;
+  if ((states && !aligned16(states)) || !aligned16(state_S) || !aligned16(state_z))
+    return LINATTN_ERR_INVALID_ARG;
+  if (count < 0 || count > (1 << 20) || skip < -1 || B <= 0 || H <= 0 || B > (1 << 24) ||
+      H > (1 << 24) || B * H > (1 << 24))
+    return LINATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  return to_status(launch_sum_states(states, count, skip, B * H, (int)d, state_S, state_z,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 linattn_status linattn_forward(const void *q, const void *k, const void *v, void *out, int64_t B,
@@ -187,7 +230,8 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
   float *w = static_cast<float *>(ws.ptr);
   cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, 0, st);
   if (e == cudaSuccess)
-    e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, d * d, state_z, d, st);
+    e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, d * d, state_z, d, nullptr,
+                           nullptr, st);
   return to_status(e);
 }
 

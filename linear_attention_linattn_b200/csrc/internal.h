@@ -20,10 +20,14 @@ constexpr int kSimtChunk = 64;
 cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int64_t heads,
                                     int64_t n, int d, int is_bf16, cudaStream_t st);
 // In-place exclusive prefix over the segments of each head (mode 0), or the per-head total
-// written to S_out + head*S_hs ([D][d]) and z_out + head*z_hs ([D]) (mode 1).
+// written to S_out + head*S_hs ([D][d]) and z_out + head*z_hs ([D]) (mode 1); both start
+// from the state (init_S [heads][D][d], init_z [heads][D]) when init_S is not null.
 cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
-                               cudaStream_t st);
+                               const float *init_S, const float *init_z, cudaStream_t st);
+// Per-head sum of gathered states [count][heads][D*d + D], skipping index `skip`.
+cudaError_t launch_sum_states(const float *states, int64_t count, int64_t skip, int64_t heads,
+                              int d, float *S_out, float *z_out, cudaStream_t st);
 // Outputs from per-chunk prefixes (causal) or the per-head totals (non-causal).
 cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, void *out,
                                   const float *S, const float *z, int64_t S_chunk_stride,
@@ -42,9 +46,10 @@ constexpr int kTcChunk = 64;
 int64_t tc_default_segment(int64_t heads, int64_t n, int d);
 // Workspace bytes the tensor-core forward needs.
 size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int causal);
+// init_S / init_z (nullable): the state before the first token of every head.
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
                        int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
-                       cudaStream_t st);
+                       const float *init_S, const float *init_z, cudaStream_t st);
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
                              int64_t heads, int64_t n, int d, int64_t seg, void *ws, int *err,
                              cudaStream_t st);

@@ -104,13 +104,16 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__r
 
 // K2: per head, a sequential sweep over the segments for each group of 4 state elements
 // (16-byte loads and stores; d (d + 1) is a multiple of 4, so a group never straddles S and z).
-//   mode 0: ws[h][s] <- sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
-//   mode 1: S_out + h*S_hs, z_out + h*z_hs <- sum_s ws[h][s] (the total)
-// The segments are summed in order, one group of elements per thread.
+//   mode 0: ws[h][s] <- init[h] + sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
+//   mode 1: S_out + h*S_hs, z_out + h*z_hs <- init[h] + sum_s ws[h][s] (the total)
+// init[h] is the state before the first segment: (init_S[h] [D][d], init_z[h] [D]), or zero
+// when init_S is null.  The segments are summed in order, one group of elements per thread.
 __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws, int64_t nseg,
                                                           int d, int mode,
                                                           float *__restrict__ S_out, int64_t S_hs,
-                                                          float *__restrict__ z_out, int64_t z_hs) {
+                                                          float *__restrict__ z_out, int64_t z_hs,
+                                                          const float *__restrict__ init_S,
+                                                          const float *__restrict__ init_z) {
   const int64_t per4 = ((int64_t)d * d + d) / 4;
   const int64_t blocks_per_head = (per4 + blockDim.x - 1) / blockDim.x;
   const int64_t head = blockIdx.x / blocks_per_head;
@@ -119,6 +122,11 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
   float4 *base = reinterpret_cast<float4 *>(ws) + head * nseg * per4 + e4;
   constexpr int kBatch = 8;  // independent 16-byte loads in flight per thread
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (init_S != nullptr) {
+    const int64_t e = e4 * 4, dd = (int64_t)d * d;
+    run = e < dd ? *reinterpret_cast<const float4 *>(init_S + head * dd + e)
+                 : *reinterpret_cast<const float4 *>(init_z + head * d + (e - dd));
+  }
   for (int64_t s0 = 0; s0 < nseg; s0 += kBatch) {
     float4 x[kBatch];
 #pragma unroll
@@ -333,10 +341,49 @@ cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int
 
 cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
-                               cudaStream_t st) {
+                               const float *init_S, const float *init_z, cudaStream_t st) {
   const int64_t per4 = ((int64_t)d * d + d) / 4;
   scan_states_kernel<<<(unsigned)(((per4 + 255) / 256) * heads), 256, 0, st>>>(
-      ws, nseg, d, mode, S_out, S_hs, z_out, z_hs);
+      ws, nseg, d, mode, S_out, S_hs, z_out, z_hs, init_S, init_z);
+  count_launches(1);
+  record_launch_event(st);
+  return cudaGetLastError();
+}
+
+// Sum of gathered states: for each head h, (S_out[h], z_out[h]) <- sum over i in [0, count),
+// i != skip, of states[i][h] (each [D*d + D]: S row-major then z), added in order of i; zero
+// when no state is summed.
+__global__ void __launch_bounds__(256) sum_states_kernel(const float *__restrict__ states,
+                                                         int64_t count, int64_t skip,
+                                                         int64_t heads, int d,
+                                                         float *__restrict__ S_out,
+                                                         float *__restrict__ z_out) {
+  const int64_t per4 = ((int64_t)d * d + d) / 4;
+  const int64_t blocks_per_head = (per4 + blockDim.x - 1) / blockDim.x;
+  const int64_t head = blockIdx.x / blocks_per_head;
+  const int64_t e4 = (blockIdx.x % blocks_per_head) * (int64_t)blockDim.x + threadIdx.x;
+  if (e4 >= per4) return;
+  const float4 *src = reinterpret_cast<const float4 *>(states) + head * per4 + e4;
+  float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t i = 0; i < count; ++i) {
+    if (i == skip) continue;
+    const float4 x = src[i * heads * per4];
+    run.x += x.x;
+    run.y += x.y;
+    run.z += x.z;
+    run.w += x.w;
+  }
+  const int64_t e = e4 * 4, dd = (int64_t)d * d;
+  float4 *dst = e < dd ? reinterpret_cast<float4 *>(S_out + head * dd + e)
+                       : reinterpret_cast<float4 *>(z_out + head * d + (e - dd));
+  *dst = run;
+}
+
+cudaError_t launch_sum_states(const float *states, int64_t count, int64_t skip, int64_t heads,
+                              int d, float *S_out, float *z_out, cudaStream_t st) {
+  const int64_t per4 = ((int64_t)d * d + d) / 4;
+  sum_states_kernel<<<(unsigned)(((per4 + 255) / 256) * heads), 256, 0, st>>>(
+      states, count, skip, heads, d, S_out, z_out);
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();

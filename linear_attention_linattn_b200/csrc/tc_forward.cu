@@ -917,7 +917,8 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
 
 template <int D>
 cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out, int64_t heads,
-                         int64_t n, int causal, int64_t seg, void *ws, int *err, cudaStream_t st) {
+                         int64_t n, int causal, int64_t seg, void *ws, int *err,
+                         const float *init_S, const float *init_z, cudaStream_t st) {
   const int64_t nseg = (n + seg - 1) / seg;
   const int64_t per = (int64_t)D * D + D;
   CUtensorMap tq, tk, tv;
@@ -929,14 +930,15 @@ cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out,
   e = launch_tc<D, kState>(tq, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
   if (e != cudaSuccess) return e;
   if (causal) {
-    e = launch_scan_states(w, heads, nseg, D, 0, nullptr, 0, nullptr, 0, st);
+    e = launch_scan_states(w, heads, nseg, D, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
     if (e != cudaSuccess) return e;
     return launch_tc<D, kCausalOut>(tq, tk, tv, out, w, nseg * per, per, nullptr, heads, n, seg,
                                     nseg, err, st);
   }
   // per-head totals, packed as [heads][D*D + D] (S row-major, then z)
   float *tot = w + heads * nseg * per;
-  e = launch_scan_states(w, heads, nseg, D, 1, tot, per, tot + (int64_t)D * D, per, st);
+  e = launch_scan_states(w, heads, nseg, D, 1, tot, per, tot + (int64_t)D * D, per, init_S,
+                         init_z, st);
   if (e != cudaSuccess) return e;
   return launch_tc<D, kNoncausalOut>(tq, tk, tv, out, tot, per, 0, nullptr, heads, n, seg, nseg,
                                      err, st);
@@ -972,9 +974,10 @@ size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int caus
 
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
                        int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
-                       cudaStream_t st) {
-  return d == 64 ? tc_forward_d<64>(q, k, v, out, heads, n, causal, seg, ws, err, st)
-                 : tc_forward_d<128>(q, k, v, out, heads, n, causal, seg, ws, err, st);
+                       const float *init_S, const float *init_z, cudaStream_t st) {
+  return d == 64
+             ? tc_forward_d<64>(q, k, v, out, heads, n, causal, seg, ws, err, init_S, init_z, st)
+             : tc_forward_d<128>(q, k, v, out, heads, n, causal, seg, ws, err, init_S, init_z, st);
 }
 
 template <int D>
@@ -988,7 +991,8 @@ cudaError_t tc_state_d(const void *k, const void *v, float *S_out, float *z_out,
   float *w = static_cast<float *>(ws);
   e = launch_tc<D, kState>(tk, tk, tv, nullptr, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
   if (e != cudaSuccess) return e;
-  return launch_scan_states(w, heads, nseg, D, 1, S_out, (int64_t)D * D, z_out, D, st);
+  return launch_scan_states(w, heads, nseg, D, 1, S_out, (int64_t)D * D, z_out, D, nullptr,
+                            nullptr, st);
 }
 
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
