@@ -8,6 +8,9 @@ library: the only code both sides share is the seeded input generator
 
 Contents
 --------
+* ``backward``: gradients of sum(g * out) with respect to q, k, v, by the chain rule
+  through the forward's definition as weights w_ij = phi(q_i).phi(k_j) (the pages give
+  no backward formulas; this is plain differentiation of the forward they define).
 * ``forward`` / ``forward_rows`` / ``state`` / ``decode_step``: ctypes wrappers around
   ``oracle.c`` (plain float64 loops, OpenMP over heads).  The method follows the page
   "Efficient Transformers: Linear Attention and Flash Attention", section "Linear
@@ -79,6 +82,9 @@ class Oracle:
         lib.oracle_decode_step_f64.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64,
                                                ctypes.c_int]
         lib.oracle_decode_step_f64.restype = None
+        lib.oracle_backward_f64.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64,
+                                            _i64, _i64, ctypes.c_int, ctypes.c_int]
+        lib.oracle_backward_f64.restype = None
         lib.oracle_plant.restype = ctypes.c_int
         self.lib = lib
         self.plant = lib.oracle_plant()
@@ -117,6 +123,19 @@ class Oracle:
                                          self._ptr(out), heads, n, d, int(bool(causal)),
                                          rows.ctypes.data_as(_ip), rows.size, int(phi_kind))
         return out
+
+    def backward(self, q, k, v, g, causal: bool, phi_kind: int = PHI_ELU1):
+        """Gradients of sum(g * forward(q, k, v)) with respect to q, k, v: q, k, v, g are
+        [..., n, d]; returns (dq, dk, dv) as float64 arrays of that shape."""
+        q, k, v, g = self._f64(q), self._f64(k), self._f64(v), self._f64(g)
+        assert q.shape == k.shape == v.shape == g.shape and q.ndim >= 2
+        n, d = q.shape[-2:]
+        heads = int(np.prod(q.shape[:-2], dtype=np.int64)) if q.ndim > 2 else 1
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        self.lib.oracle_backward_f64(self._ptr(q), self._ptr(k), self._ptr(v), self._ptr(g),
+                                     self._ptr(dq), self._ptr(dk), self._ptr(dv), 1, heads, n,
+                                     d, int(bool(causal)), int(phi_kind))
+        return dq, dk, dv
 
     def state(self, k, v, phi_kind: int = PHI_ELU1):
         """Final causal state per head: S [..., d, d] (row = feature, col = value), z [..., d]."""
@@ -159,7 +178,7 @@ def default() -> Oracle:
 
 
 def load_planted(plant: int) -> Oracle:
-    """Build and load a variant of the oracle with planted mistake ``plant`` (1..5)."""
+    """Build and load a variant of the oracle with planted mistake ``plant`` (1..7)."""
     tmp = tempfile.mkdtemp(prefix="oracle_plant_")
     path = build(plant=plant, out_path=os.path.join(tmp, f"liboracle_plant{plant}.so"))
     return Oracle(path)
@@ -175,6 +194,10 @@ def forward_rows(q, k, v, rows, causal: bool, phi_kind: int = PHI_ELU1) -> np.nd
 
 def state(k, v, phi_kind: int = PHI_ELU1):
     return default().state(k, v, phi_kind)
+
+
+def backward(q, k, v, g, causal: bool, phi_kind: int = PHI_ELU1):
+    return default().backward(q, k, v, g, causal, phi_kind)
 
 
 def decode_step(S, z, q, k, v, phi_kind: int = PHI_ELU1):

@@ -36,8 +36,12 @@
  * the reassociation trick, by hand") uses on non-negative inputs.  It exists only so
  * that example can pin this code; it is not part of the method.
  *
- * Compile-time ORACLE_PLANT=1..5 plants one deliberate mistake each.  Only the test
+ * Compile-time ORACLE_PLANT=1..7 plants one deliberate mistake each.  Only the test
  * that shows the pins catch such mistakes builds those variants.
+ *
+ * The backward pass (gradients of a loss through the forward pass; the pages give no
+ * formulas for it) is the chain rule through the forward's definition written as weights
+ * w_ij = phi(q_i) . phi(k_j); see oracle_backward_f64.
  */
 #include <math.h>
 #include <stdint.h>
@@ -205,6 +209,100 @@ void oracle_decode_step_f64(double *S, double *z, const double *q, const double 
         readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, phi_kind, pq);
 #endif
         free(pq);
+    }
+}
+
+/* phi'(x): 1 above zero, exp(x) at or below zero (the derivative of elu + 1, alpha = 1;
+ * both one-sided derivatives are 1 at zero). */
+static double phi_deriv(double x, int phi_kind)
+{
+    if (phi_kind == PHI_IDENTITY) return 1.0;
+#if ORACLE_PLANT == 7
+    return 1.0; /* planted: the chain rule through phi dropped on the negative branch */
+#else
+    return x > 0.0 ? 1.0 : exp(x);
+#endif
+}
+
+/*
+ * Gradients of the loss L = sum_i g_i . out_i with respect to q, k and v, per head, for
+ * the forward pass above (causal: j <= i; non-causal: all j).  The forward is written as
+ *     w_ij = phi(q_i) . phi(k_j),   den_i = sum_j w_ij,   out_i = sum_j w_ij v_j / den_i,
+ * and differentiated term by term:
+ *     dL/dw_ij      = g_i . (v_j - out_i) / den_i
+ *     dL/dv_j       = sum_i w_ij g_i / den_i
+ *     dL/dphi(q_i)  = sum_j dL/dw_ij phi(k_j)
+ *     dL/dphi(k_j)  = sum_i dL/dw_ij phi(q_i)
+ *     dL/dq = dL/dphi(q) * phi'(q),   dL/dk = dL/dphi(k) * phi'(k).
+ * Plain O(n^2 d) loops in float64; g, dq, dk, dv are [B][H][n][d] like q.
+ */
+void oracle_backward_f64(const double *q, const double *k, const double *v, const double *g,
+                         double *dq, double *dk, double *dv, int64_t B, int64_t H, int64_t n,
+                         int64_t d, int causal, int phi_kind)
+{
+    const int64_t heads = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        const int64_t base = bh * n * d;
+        double *pq = (double *)malloc((size_t)(n * d) * sizeof(double));
+        double *pk = (double *)malloc((size_t)(n * d) * sizeof(double));
+        double *den = (double *)malloc((size_t)n * sizeof(double));
+        double *gout = (double *)malloc((size_t)n * sizeof(double)); /* g_i . out_i */
+        double *out = (double *)malloc((size_t)d * sizeof(double));
+        for (int64_t t = 0; t < n * d; ++t) {
+            pq[t] = oracle_phi(q[base + t], phi_kind);
+            pk[t] = oracle_phi(k[base + t], phi_kind);
+        }
+        /* forward quantities per query row */
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t jend = causal ? i + 1 : n;
+            double s = 0.0;
+            for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+            for (int64_t j = 0; j < jend; ++j) {
+                double w = 0.0;
+                for (int64_t r = 0; r < d; ++r) w += pq[i * d + r] * pk[j * d + r];
+                s += w;
+                for (int64_t c = 0; c < d; ++c) out[c] += w * v[base + j * d + c];
+            }
+            den[i] = s;
+            double go = 0.0;
+            for (int64_t c = 0; c < d; ++c) go += g[base + i * d + c] * out[c] / s;
+            gout[i] = go;
+        }
+        for (int64_t t = 0; t < n * d; ++t) {
+            dq[base + t] = 0.0;
+            dk[base + t] = 0.0;
+            dv[base + t] = 0.0;
+        }
+        /* every (i, j) pair of the sum: dL/dw_ij feeds phi(q_i) and phi(k_j); w_ij feeds v_j */
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t jend = causal ? i + 1 : n;
+            for (int64_t j = 0; j < jend; ++j) {
+                double w = 0.0, gv = 0.0;
+                for (int64_t r = 0; r < d; ++r) w += pq[i * d + r] * pk[j * d + r];
+                for (int64_t c = 0; c < d; ++c) gv += g[base + i * d + c] * v[base + j * d + c];
+#if ORACLE_PLANT == 6
+                const double dw = gv / den[i]; /* planted: the normaliser's term dropped */
+#else
+                const double dw = (gv - gout[i]) / den[i];
+#endif
+                for (int64_t r = 0; r < d; ++r) {
+                    dq[base + i * d + r] += dw * pk[j * d + r];
+                    dk[base + j * d + r] += dw * pq[i * d + r];
+                }
+                for (int64_t c = 0; c < d; ++c)
+                    dv[base + j * d + c] += w * g[base + i * d + c] / den[i];
+            }
+        }
+        for (int64_t t = 0; t < n * d; ++t) {
+            dq[base + t] *= phi_deriv(q[base + t], phi_kind);
+            dk[base + t] *= phi_deriv(k[base + t], phi_kind);
+        }
+        free(pq);
+        free(pk);
+        free(den);
+        free(gout);
+        free(out);
     }
 }
 
