@@ -117,6 +117,25 @@ linattn_status linattn_forward_init(const void *q, const void *k, const void *v,
                                     linattn_dtype dtype, linattn_stream_t stream);
 
 /*
+ * Backward pass: the gradients of a loss L with respect to q, k and v, given
+ * dout = dL/dout for out = linattn_forward(q, k, v, causal).  All seven tensors are
+ * [B][H][n][d] of type `dtype` (dq, dk, dv written in that type); accumulation is float32
+ * on the CUDA cores.  The pages define the forward only; this is its chain rule: with
+ * w_ij = phi(q_i).phi(k_j), den_i = sum_j w_ij and a_i = dout_i / den_i,
+ * b_i = -(dout_i . out_i) / den_i,
+ *     dL/dphi(q_i) = sum_j (v_j . a_i + b_i) phi(k_j),
+ *     dL/dphi(k_j) = sum_i (v_j . a_i + b_i) phi(q_i),
+ *     dL/dv_j      = sum_i w_ij a_i,
+ * then through phi'(x) = 1 (x > 0), exp(x) (x <= 0); sums over j <= i (causal) or all.
+ * Asynchronous on `stream`; takes a stream-ordered workspace of about
+ * 2 (n/64) (d^2 + d) + n (d + 1) floats per head.  Errors as in linattn_forward.
+ */
+linattn_status linattn_backward(const void *q, const void *k, const void *v, const void *dout,
+                                void *dq, void *dk, void *dv, int64_t B, int64_t H, int64_t n,
+                                int64_t d, int causal, linattn_dtype dtype,
+                                linattn_stream_t stream);
+
+/*
  * Per-head sum of gathered states.  states: float32 device memory laid out
  * [count][B][H][D*d + D] (each state: S row-major [D][d], then z [D]; this is what an
  * all-gather of every rank's linattn_forward_state output, packed that way, produces).

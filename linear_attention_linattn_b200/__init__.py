@@ -10,10 +10,10 @@ Raw C entry points (pointers as ints):
     linattn_forward, linattn_forward_ex, linattn_forward_state, linattn_decode_step,
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
     linattn_launch_count, linattn_forward_noalloc, linattn_profile_events,
-    linattn_forward_init, linattn_sum_states
+    linattn_forward_init, linattn_sum_states, linattn_backward
 
 Tensor helpers: ``forward``, ``forward_init``, ``forward_state``, ``sum_states``,
-``decode_step``, ``device_error``; ``seqshard`` splits one sequence over ranks.
+``backward``, ``decode_step``, ``device_error``; ``seqshard`` splits one sequence over ranks.
 """
 from __future__ import annotations
 
@@ -53,6 +53,8 @@ SIGNATURES = {
     "linattn_forward_init": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                             _i64, ctypes.c_int, ctypes.c_int, _vp]),
     "linattn_sum_states": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "linattn_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                        _i64, ctypes.c_int, ctypes.c_int, _vp]),
 }
 
 _lib = None
@@ -181,6 +183,25 @@ def sum_states(states, count: int, skip: int = -1, S=None, z=None, stream=None):
                                 z.data_ptr(), _stream_ptr(stream))
     _check(st, "linattn_sum_states")
     return S, z
+
+
+def backward(q, k, v, dout, causal: bool, stream=None):
+    """Gradients (dq, dk, dv) of a loss given dout = dL/dout for out = forward(q, k, v, causal);
+    all [B, H, n, d] CUDA tensors of one dtype (float32 or bfloat16)."""
+    import torch
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _dev(t, nm)
+    if not (q.shape == k.shape == v.shape == dout.shape and q.dim() == 4 and
+            q.dtype == k.dtype == v.dtype == dout.dtype):
+        raise ValueError("q, k, v, dout must share one [B, H, n, d] shape and dtype")
+    B, H, n, d = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    lib = load_library()
+    st = lib.linattn_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, n, d,
+                              int(bool(causal)), _dtype_code(q), _stream_ptr(stream))
+    _check(st, "linattn_backward")
+    return dq, dk, dv
 
 
 def forward_state(k, v, S=None, z=None, stream=None):

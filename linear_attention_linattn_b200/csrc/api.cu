@@ -177,6 +177,31 @@ linattn_status linattn_forward_init(const void *q, const void *k, const void *v,
   return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, ds, st);
 }
 
+linattn_status linattn_backward(const void *q, const void *k, const void *v, const void *dout,
+                                void *dq, void *dk, void *dv, int64_t B, int64_t H, int64_t n,
+                                int64_t d, int causal, linattn_dtype dtype,
+                                linattn_stream_t stream) {
+  if (!q || !k || !v || !dout || !dq || !dk || !dv) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return LINATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  linattn_status s = check_forward_shape(B, H, n, d);
+  if (s != LINATTN_OK) return s;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t heads = B * H;
+  Workspace ws;
+  ws.st = st;
+  const size_t bytes = backward_workspace_floats(heads, n, (int)d, causal) * sizeof(float);
+  if (cudaMallocFromPoolAsync(&ws.ptr, bytes, ds->pool, st) != cudaSuccess)
+    return LINATTN_ERR_CUDA;
+  return to_status(backward(q, k, v, dout, dq, dk, dv, heads, n, (int)d, causal,
+                            dtype == LINATTN_BF16, static_cast<float *>(ws.ptr), st));
+}
+
 linattn_status linattn_sum_states(const float *states, int64_t count, int64_t skip, int64_t B,
                                   int64_t H, int64_t d, float *state_S, float *state_z,
                                   linattn_stream_t stream) {

@@ -22,6 +22,7 @@ cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int
 // In-place exclusive prefix over the segments of each head (mode 0), or the per-head total
 // written to S_out + head*S_hs ([D][d]) and z_out + head*z_hs ([D]) (mode 1); both start
 // from the state (init_S [heads][D][d], init_z [heads][D]) when init_S is not null.
+// Mode 2: in-place exclusive suffix (sum of the later segments; no starting state).
 cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
                                const float *init_S, const float *init_z, cudaStream_t st);
@@ -34,6 +35,13 @@ cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, v
                                   int64_t S_head_stride, int64_t z_chunk_stride,
                                   int64_t z_head_stride, int64_t heads, int64_t n, int d,
                                   int causal, int is_bf16, cudaStream_t st);
+
+// ---- backward pass (backward.cu), CUDA cores; is_bf16 selects bf16 I/O, else fp32 ------
+// Workspace floats linattn_backward needs.
+size_t backward_workspace_floats(int64_t heads, int64_t n, int d, int causal);
+cudaError_t backward(const void *q, const void *k, const void *v, const void *g, void *dq,
+                     void *dk, void *dv, int64_t heads, int64_t n, int d, int causal, int is_bf16,
+                     float *ws, cudaStream_t st);
 
 // ---- decode (decode.cu) ----------------------------------------------------------------
 cudaError_t launch_decode_step(float *S, float *z, const void *q, const void *k, const void *v,

@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__r
 // (16-byte loads and stores; d (d + 1) is a multiple of 4, so a group never straddles S and z).
 //   mode 0: ws[h][s] <- init[h] + sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
 //   mode 1: S_out + h*S_hs, z_out + h*z_hs <- init[h] + sum_s ws[h][s] (the total)
+//   mode 2: ws[h][s] <- sum_{s' > s} ws[h][s'] (exclusive suffix, in place; the backward
+//           pass's states of the later chunks)
 // init[h] is the state before the first segment: (init_S[h] [D][d], init_z[h] [D]), or zero
 // when init_S is null.  The segments are summed in order, one group of elements per thread.
 __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws, int64_t nseg,
@@ -127,21 +129,25 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
     run = e < dd ? *reinterpret_cast<const float4 *>(init_S + head * dd + e)
                  : *reinterpret_cast<const float4 *>(init_z + head * d + (e - dd));
   }
+  const bool rev = mode == 2;
   for (int64_t s0 = 0; s0 < nseg; s0 += kBatch) {
     float4 x[kBatch];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i)
-      x[i] = s0 + i < nseg ? base[(s0 + i) * per4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t s = rev ? nseg - 1 - (s0 + i) : s0 + i;
+      x[i] = s0 + i < nseg ? base[s * per4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      if (mode == 0 && s0 + i < nseg) base[(s0 + i) * per4] = run;
+      const int64_t s = rev ? nseg - 1 - (s0 + i) : s0 + i;
+      if (mode != 1 && s0 + i < nseg) base[s * per4] = run;
       run.x += x[i].x;
       run.y += x[i].y;
       run.z += x[i].z;
       run.w += x[i].w;
     }
   }
-  if (mode != 0) {
+  if (mode == 1) {
     const int64_t e = e4 * 4;
     float *dst = e < (int64_t)d * d ? S_out + head * S_hs + e : z_out + head * z_hs + (e - (int64_t)d * d);
     dst[0] = run.x;

@@ -79,6 +79,27 @@ def test_decode_and_state_argument_checks(lib):
         la.LINATTN_ERR_INVALID_ARG
 
 
+def test_backward_init_and_sum_argument_checks(lib):
+    bad = la.LINATTN_ERR_INVALID_ARG
+    # backward: null dq, misaligned dout, causal out of range, d unsupported
+    assert lib.linattn_backward(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, 1, 1, 8, 64, 1, 0,
+                                None) == bad
+    assert lib.linattn_backward(FAKE, FAKE, FAKE, FAKE + 8, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1, 0,
+                                None) == bad
+    assert lib.linattn_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 2, 0,
+                                None) == bad
+    assert lib.linattn_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 1, 0,
+                                None) == la.LINATTN_ERR_UNSUPPORTED
+    # forward from a state: the state pointers are required
+    assert lib.linattn_forward_init(FAKE, FAKE, FAKE, FAKE, 0, FAKE, 1, 1, 8, 64, 1, 1,
+                                    None) == bad
+    # state sums: negative count, skip below -1, unsupported d
+    assert lib.linattn_sum_states(FAKE, -1, -1, 1, 1, 64, FAKE, FAKE, None) == bad
+    assert lib.linattn_sum_states(FAKE, 2, -2, 1, 1, 64, FAKE, FAKE, None) == bad
+    assert lib.linattn_sum_states(FAKE, 2, -1, 1, 1, 80, FAKE, FAKE, None) == \
+        la.LINATTN_ERR_UNSUPPORTED
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError):
         la.load_library(str(tmp_path / "nope.so"))

@@ -1,0 +1,61 @@
+"""Parity of the CUDA backward pass (through the C ABI) with the float64 oracle's gradients.
+
+Metric: per row, ||got_i - ref_i|| / max(||ref_i||, mean_i ||ref_i||), maximised over the rows
+of dq, dk and dv.  The floor at the mean row norm is needed because some gradient rows
+vanish exactly (causal: the first token's dq is zero, its output being v_0 whatever q_0 is),
+where a plain per-row ratio would divide rounding by zero.  Bars: 1e-4 for float32 I/O,
+2e-2 for bfloat16 I/O (the gradients are rounded to bf16 once).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from linear_attention_linattn_b200 import inputs
+from tests.helpers import TOL, as_io, to_dev, to_host
+
+torch = pytest.importorskip("torch")
+la = pytest.importorskip("linear_attention_linattn_b200")
+
+pytestmark = pytest.mark.gpu
+
+
+def grad_err(got, ref) -> float:
+    d = ref.shape[-1]
+    g = np.asarray(got, np.float64).reshape(-1, d)
+    r = np.asarray(ref, np.float64).reshape(-1, d)
+    rn = np.linalg.norm(r, axis=1)
+    floor = max(rn.mean(), 1e-30)
+    return float(np.max(np.linalg.norm(g - r, axis=1) / np.maximum(rn, floor)))
+
+
+def _check(B, H, n, d, causal, dtype, seed):
+    q, k, v, g = (as_io(x, dtype) for x in inputs.forward_qkv(seed, B, H, n, d, scaled=True))
+    g = as_io(inputs.forward_qkv(seed + 1000, B, H, n, d, scaled=True)[0], dtype)
+    dq, dk, dv = la.backward(*(to_dev(x, dtype) for x in (q, k, v, g)), causal)
+    assert la.device_error() == la.LINATTN_OK
+    ref = oracle.backward(q, k, v, g, causal)
+    errs = [grad_err(to_host(a), b) for a, b in zip((dq, dk, dv), ref)]
+    assert max(errs) <= TOL[dtype], errs
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,H,n", [(1, 2, 2), (2, 1, 63), (1, 2, 65), (1, 3, 200), (1, 1, 1000)])
+def test_backward_small_shapes(dtype, causal, d, B, H, n):
+    _check(B, H, n, d, causal, dtype, 300 + n)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_longer_sequence(dtype, causal):
+    _check(1, 2, 4096, 64, causal, dtype, 7)
+
+
+def test_value_gradients_sum_to_output_gradients_on_gpu():
+    """sum_j dL/dv_j = sum_i dL/dout_i: each output row is a convex combination of values."""
+    B, H, n, d = 2, 2, 700, 64
+    q, k, v, g = (to_dev(x, "f32") for x in inputs.forward_qkv(9, B, H, n, d, scaled=True))
+    for causal in (True, False):
+        _, _, dv = la.backward(q, k, v, g, causal)
+        assert torch.allclose(dv.double().sum(2), g.double().sum(2), rtol=1e-4, atol=1e-4)
