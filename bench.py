@@ -524,7 +524,15 @@ def extras(args):
         res[f"{name}_{'causal' if causal else 'noncausal'}"] = {
             "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
             "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
-    del q, k, v, o
+    # backward pass on the same shape (causal): reads q, k, v, dout and writes dq, dk, dv
+    dout = torch.randn_like(o)
+    ms, _ = time_steps(lambda: la.backward(q, k, v, dout, True), 5, 3, 1)
+    alg = 7 * w.B * w.H * w.n * w.d * 2
+    res[f"backward_{name}_causal"] = {
+        "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
+        "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
+        "path": "CUDA cores (float32 FFMA), 6 launches"}
+    del q, k, v, o, dout
     # latency cases
     for name, dtypes in (("noncausal_1x1x512x64_f32", ("f32",)),
                          ("causal_1x1x4096x64", ("f32", "bf16"))):
