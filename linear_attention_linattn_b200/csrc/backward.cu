@@ -81,6 +81,43 @@ __device__ __forceinline__ void load_state_t(float *dst, const float *S) {
   }
 }
 
+// W[i][j] = sum_r X[i][r] Y[j][r] + add[i] for j <= i, zero above the diagonal (X, Y: [C][D+1]
+// tiles; add may be null).  Each thread computes a 4 x 4 block, rows ti + 16a and columns
+// tj + 16b, so a sweep over r loads 8 values for 16 FMAs.
+template <int D>
+__device__ __forceinline__ void masked_products(float *W, const float *X, const float *Y,
+                                                const float *add) {
+  constexpr int PD = D + 1;
+  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+  for (int r = 0; r < D; ++r) {
+    float x[4], y[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) x[a] = X[(ti + 16 * a) * PD + r];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) y[b] = Y[(tj + 16 * b) * PD + r];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(x[a], y[b], acc[a][b]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = ti + 16 * a;
+    const float ad = add ? add[i] : 0.f;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = tj + 16 * b;
+      W[i * (C + 1) + j] = j <= i ? acc[a][b] + ad : 0.f;
+    }
+  }
+}
+
 template <int D>
 constexpr size_t bwd_smem_floats(bool causal) {
   // four [C][D+1] tiles, one transposed state [D][D+1], z or r [D], [C] den and b,
@@ -125,16 +162,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(
   __syncthreads();
 
   if (CAUSAL) {
-    // P[i][j] = phi(q_i).phi(k_j) for j <= i
-    for (int e = threadIdx.x; e < C * C; e += kThreads) {
-      const int i = e / C, j = e % C;
-      float s = 0.f;
-      if (j <= i) {
-#pragma unroll 8
-        for (int r = 0; r < D; ++r) s = fmaf(sQ[i * PD + r], sK[j * PD + r], s);
-      }
-      sW[i * (C + 1) + j] = s;
-    }
+    masked_products<D>(sW, sQ, sK, nullptr);  // P[i][j] = phi(q_i).phi(k_j), j <= i
     __syncthreads();
   }
   if (threadIdx.x < C) {
@@ -217,17 +245,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(
   __syncthreads();
 
   if (CAUSAL) {
-    // dL/dw[i][j] = v_j . a_i + b_i for j <= i
-    for (int e = threadIdx.x; e < C * C; e += kThreads) {
-      const int i = e / C, j = e % C;
-      float s = 0.f;
-      if (j <= i) {
-#pragma unroll 8
-        for (int c = 0; c < D; ++c) s = fmaf(sA[i * PD + c], sV[j * PD + c], s);
-        s += sB[i];
-      }
-      sW[i * (C + 1) + j] = s;
-    }
+    masked_products<D>(sW, sA, sV, sB);  // dL/dw[i][j] = v_j . a_i + b_i, j <= i
     __syncthreads();
   }
 
@@ -377,16 +395,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(
   constexpr int RB = D / 16;
   const int tj = threadIdx.x / 16, tx = threadIdx.x % 16;
   if (CAUSAL) {
-    // P[i][j] = phi(q_i).phi(k_j) for i >= j
-    for (int e = threadIdx.x; e < C * C; e += kThreads) {
-      const int i = e / C, j = e % C;
-      float s = 0.f;
-      if (j <= i) {
-#pragma unroll 8
-        for (int r = 0; r < D; ++r) s = fmaf(sQ[i * PD + r], sK[j * PD + r], s);
-      }
-      sW[i * (C + 1) + j] = s;
-    }
+    masked_products<D>(sW, sQ, sK, nullptr);  // P[i][j] = phi(q_i).phi(k_j), i >= j
     __syncthreads();
   }
   // dv_j[c] = sum_r R[r][c] phi(k_j)[r] + sum_{i >= j} P[i][j] a_i[c]
@@ -431,17 +440,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(
   }
   if (CAUSAL) {
     __syncthreads();  // every thread is done with P
-    // dL/dw[i][j] = v_j . a_i + b_i for i >= j
-    for (int e = threadIdx.x; e < C * C; e += kThreads) {
-      const int i = e / C, j = e % C;
-      float s = 0.f;
-      if (j <= i) {
-#pragma unroll 8
-        for (int c = 0; c < D; ++c) s = fmaf(sA[i * PD + c], sV[j * PD + c], s);
-        s += sB[i];
-      }
-      sW[i * (C + 1) + j] = s;
-    }
+    masked_products<D>(sW, sA, sV, sB);  // dL/dw[i][j] = v_j . a_i + b_i, i >= j
     __syncthreads();
   }
   // dphi(k_j)[r] = sum_c R[r][c] v_j[c] + r[r] + sum_{i >= j} dL/dw[i][j] phi(q_i)[r]
