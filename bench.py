@@ -58,11 +58,23 @@ def decode_bytes(heads, d, elem=2):
     return heads * (2 * (d * d + d) * 4 + 4 * d * elem)
 
 
+def code_hash(path: str) -> str:
+    """sha256 of a C/CUDA source with its comments, trailing blanks and empty lines removed, so
+    that only a change of the code itself changes it."""
+    import hashlib
+    import re
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    lines = [ln.rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
 def kernel_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` on `workload` from profiles/ncu_traffic.json (an ncu
-    capture, scaled to the full launch), or None when there is none or the kernel's source
-    file has changed since the counters were taken."""
-    import hashlib
+    capture, scaled to the full launch), or None when there is none or the code of the
+    kernel's source file has changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -71,10 +83,8 @@ def kernel_traffic(kernel: str, workload: str):
     rec = table.get(f"{kernel} | {workload}")
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-            return None
+    if code_hash(os.path.join(ROOT, rec["source"])) != rec["source_code_sha256"]:
+        return None
     return float(rec["dram_bytes_per_launch"])
 
 

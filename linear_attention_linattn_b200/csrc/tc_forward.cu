@@ -8,22 +8,23 @@
 //     num_c = phi(Q_c) S_<c + mask(phi(Q_c) phi(K_c)^T) V_c
 //     den_c = phi(Q_c) z_<c + mask(phi(Q_c) phi(K_c)^T) 1
 //     S_<c+1 = S_<c + phi(K_c)^T V_c,   z_<c+1 = z_<c + phi(K_c)^T 1
-// and chunks are grouped into segments (one CTA each).  Three kernel modes:
+// and chunks are grouped into segments, the work items of the CTAs.  Three kernel modes:
 //   kState        segment aggregates (S_s, z_s) -> fp32 workspace       (K1)
 //   kCausalOut    outputs of a segment from its exclusive prefix state   (K3)
 //   kNoncausalOut outputs phi(Q) S / phi(Q).z from the per-head total    (K3, no mask)
 // The exclusive prefix over segments (K2) is the scan kernel in simt_forward.cu.
 //
 // Every product is a tcgen05.mma (kind::f16, bf16 operands, fp32 accumulator in TMEM):
-//   P     = phi(Q_c) phi(K_c)^T        M=64  N=64  K=d   (A: Q K-major, B: K K-major)
-//   O     = phi(Q_c) S_<c              M=64  N=d   K=d   (B: S bf16, MN-major)
-//   Oden  = phi(Q_c) [z 0..0]          M=64  N=16  K=d
-//   O    += P V_c                      M=64  N=d   K=64  (A: P bf16 K-major, B: V MN-major)
-//   Oden += P [1 0..0]                 M=64  N=16  K=64
-//   S    += phi(K_c)^T V_c             M=d   N=d   K=64  (A: K MN-major)
-//   z    += phi(K_c)^T [1 0..0]        M=d   N=16  K=64
-// The normaliser rides along as a 16-column block whose first column is z (or ones), so the
-// numerator and the denominator see the same rounded weights.
+//   [P | phi(Q_c).z_<c] = phi(Q_c) [phi(K_c); z_<c]^T   M=64 N=80    K=d   (causal; A: Q, B: K,
+//                          both K-major; the K tile carries 16 more rows, row 64 = z_<c)
+//   O  = phi(Q_c) S_<c                                   M=64 N=d     K=d   (B: S bf16 MN-major;
+//                          non-causal N=d+16: an extra atom holds z, column d = denominator)
+//   O += mask(P) V_c                                     M=64 N=d     K=64  (A: P bf16 K-major,
+//                          B: V MN-major)
+//   [S | z] += phi(K_c)^T [V_c | 1]                      M=d  N=d+16  K=64  (A: K MN-major; a
+//                          constant ones atom after each V tile puts z in column d)
+// The causal denominator is column 64 of the score block plus the masked row sum of the
+// scores (taken while they are rounded), so numerator and denominator weigh the same keys.
 //
 // Warp roles (one CTA per SM; 16, 22 or 18 warps in the causal, aggregate, non-causal modes):
 //   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of Q/K/V chunks into a
