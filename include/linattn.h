@@ -54,7 +54,8 @@ typedef enum {
 
 typedef enum {
     LINATTN_F32 = 0, /* float32 I/O: computed in fp32 on the CUDA cores */
-    LINATTN_BF16 = 1 /* bfloat16 I/O: bf16 tensor-core products, fp32 accumulation and state */
+    LINATTN_BF16 = 1 /* bfloat16 I/O: the forward runs bf16 tensor-core products with fp32
+                        accumulation and state; the backward runs on the CUDA cores in fp32 */
 } linattn_dtype;
 
 /*

@@ -11,6 +11,9 @@ Contents
 * ``backward``: gradients of sum(g * out) with respect to q, k, v, by the chain rule
   through the forward's definition as weights w_ij = phi(q_i).phi(k_j) (the pages give
   no backward formulas; this is plain differentiation of the forward they define).
+* ``favor_features``: Performer's positive random features exp(W x - |x|^2/2)/sqrt(m), whose
+  dot products approximate exp(q . k) (named on the same page); with them ``forward(...,
+  phi_kind=PHI_IDENTITY)`` is FAVOR+ linear attention.
 * ``forward`` / ``forward_rows`` / ``state`` / ``decode_step``: ctypes wrappers around
   ``oracle.c`` (plain float64 loops, OpenMP over heads).  The method follows the page
   "Efficient Transformers: Linear Attention and Flash Attention", section "Linear
@@ -85,6 +88,8 @@ class Oracle:
         lib.oracle_backward_f64.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64,
                                             _i64, _i64, ctypes.c_int, ctypes.c_int]
         lib.oracle_backward_f64.restype = None
+        lib.oracle_favor_features_f64.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64]
+        lib.oracle_favor_features_f64.restype = None
         lib.oracle_plant.restype = ctypes.c_int
         self.lib = lib
         self.plant = lib.oracle_plant()
@@ -137,6 +142,17 @@ class Oracle:
                                      d, int(bool(causal)), int(phi_kind))
         return dq, dk, dv
 
+    def favor_features(self, x, W):
+        """x: [..., d]; W: [m, d].  Returns exp(W x - |x|^2 / 2) / sqrt(m): [..., m]."""
+        x, W = self._f64(x), self._f64(W)
+        d = x.shape[-1]
+        m = W.shape[0]
+        assert W.shape == (m, d)
+        rows = int(np.prod(x.shape[:-1], dtype=np.int64)) if x.ndim > 1 else 1
+        out = np.empty(x.shape[:-1] + (m,), dtype=np.float64)
+        self.lib.oracle_favor_features_f64(self._ptr(x), self._ptr(W), self._ptr(out), rows, d, m)
+        return out
+
     def state(self, k, v, phi_kind: int = PHI_ELU1):
         """Final causal state per head: S [..., d, d] (row = feature, col = value), z [..., d]."""
         k, v = self._f64(k), self._f64(v)
@@ -178,7 +194,7 @@ def default() -> Oracle:
 
 
 def load_planted(plant: int) -> Oracle:
-    """Build and load a variant of the oracle with planted mistake ``plant`` (1..7)."""
+    """Build and load a variant of the oracle with planted mistake ``plant`` (1..8)."""
     tmp = tempfile.mkdtemp(prefix="oracle_plant_")
     path = build(plant=plant, out_path=os.path.join(tmp, f"liboracle_plant{plant}.so"))
     return Oracle(path)
@@ -198,6 +214,10 @@ def state(k, v, phi_kind: int = PHI_ELU1):
 
 def backward(q, k, v, g, causal: bool, phi_kind: int = PHI_ELU1):
     return default().backward(q, k, v, g, causal, phi_kind)
+
+
+def favor_features(x, W):
+    return default().favor_features(x, W)
 
 
 def decode_step(S, z, q, k, v, phi_kind: int = PHI_ELU1):

@@ -36,7 +36,7 @@
  * the reassociation trick, by hand") uses on non-negative inputs.  It exists only so
  * that example can pin this code; it is not part of the method.
  *
- * Compile-time ORACLE_PLANT=1..7 plants one deliberate mistake each.  Only the test
+ * Compile-time ORACLE_PLANT=1..8 plants one deliberate mistake each.  Only the test
  * that shows the pins catch such mistakes builds those variants.
  *
  * The backward pass (gradients of a loss through the forward pass; the pages give no
@@ -303,6 +303,35 @@ void oracle_backward_f64(const double *q, const double *k, const double *v, cons
         free(den);
         free(gout);
         free(out);
+    }
+}
+
+/*
+ * Positive random features of Performer's FAVOR+ (named on the page "Efficient Transformers:
+ * Linear Attention and Flash Attention", section "Linear attention: reordering the matmuls,
+ * not shrinking them", as random features whose dot products approximate the softmax
+ * kernel exp(q . k); the page gives no formula, and this is the positive-feature form of
+ * that method):
+ *     phi(x)_i = exp(w_i . x - |x|^2 / 2) / sqrt(m),   i = 0 .. m-1,
+ * for random rows w_i of W [m][d] (the caller draws them, typically N(0, I_d)), so that
+ * E_w[phi(q) . phi(k)] = exp(q . k).  x: [rows][d]; out: [rows][m].
+ */
+void oracle_favor_features_f64(const double *x, const double *W, double *out, int64_t rows,
+                               int64_t d, int64_t m)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < rows; ++t) {
+        double sq = 0.0;
+        for (int64_t r = 0; r < d; ++r) sq += x[t * d + r] * x[t * d + r];
+        for (int64_t i = 0; i < m; ++i) {
+            double dot = 0.0;
+            for (int64_t r = 0; r < d; ++r) dot += W[i * d + r] * x[t * d + r];
+#if ORACLE_PLANT == 8
+            out[t * m + i] = exp(dot) / sqrt((double)m); /* planted: the -|x|^2/2 term dropped */
+#else
+            out[t * m + i] = exp(dot - 0.5 * sq) / sqrt((double)m);
+#endif
+        }
     }
 }
 
