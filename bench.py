@@ -542,6 +542,15 @@ def extras(args):
         "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
         "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
         "path": "CUDA cores (float32 FFMA), 6 launches"}
+    # FAVOR+ (Performer's positive random features, m = d) on the same shape, causal:
+    # features of q and k, then the pass on them
+    W = torch.randn(w.d, w.d, device="cuda")
+    ms, _ = time_steps(lambda: la.forward_favor(q, k, v, W, True), 10, 3, 1)
+    alg = 4 * w.B * w.H * w.n * w.d * 2 + 2 * 2 * w.B * w.H * w.n * w.d * 2  # + features out/in
+    res[f"favor_{name}_causal"] = {
+        "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
+        "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
+        "path": "features on CUDA cores, then the tensor-core pass (identity feature map)"}
     del q, k, v, o, dout
     # latency cases
     for name, dtypes in (("noncausal_1x1x512x64_f32", ("f32",)),

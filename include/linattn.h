@@ -118,6 +118,33 @@ linattn_status linattn_forward_init(const void *q, const void *k, const void *v,
                                     linattn_dtype dtype, linattn_stream_t stream);
 
 /*
+ * Performer's FAVOR+ positive random features (named on the page "Efficient Transformers:
+ * Linear Attention and Flash Attention", section "Linear attention: reordering the matmuls,
+ * not shrinking them", as features whose dot products approximate the softmax kernel
+ * exp(q . k); the page gives no formula, this is the positive-feature form):
+ *     out[t][i] = exp(W[i] . x[t] - |x[t]|^2 / 2) / sqrt(m),   m = d features,
+ * so that E_W[phi(q) . phi(k)] = exp(q . k) for W with i.i.d. N(0, 1) entries.
+ *   x   : [rows][d] of type `dtype` (for attention: q or k, already scaled as wanted).
+ *   W   : [d][d] float32, the random projection (row i = w_i), drawn by the caller.
+ *   out : [rows][d] of type `dtype`, written.
+ * d in {64, 128}.  Feed the features of q and k to linattn_forward_features.
+ */
+linattn_status linattn_favor_features(const void *x, const float *W, void *out, int64_t rows,
+                                      int64_t d, linattn_dtype dtype, linattn_stream_t stream);
+
+/*
+ * linattn_forward on features the caller has computed: phi_q and phi_k ([B][H][n][d], type
+ * `dtype`) are used as phi(q) and phi(k) directly, with no feature map applied:
+ *     out_i = phi_q_i S / phi_q_i . z,   S = sum_j phi_k_j v_j^T,   z = sum_j phi_k_j.
+ * The features must be non-negative with positive denominators (FAVOR+ features are).
+ * Other arguments, layouts and errors as in linattn_forward.
+ */
+linattn_status linattn_forward_features(const void *phi_q, const void *phi_k, const void *v,
+                                        void *out, int64_t B, int64_t H, int64_t n, int64_t d,
+                                        int causal, linattn_dtype dtype,
+                                        linattn_stream_t stream);
+
+/*
  * Backward pass: the gradients of a loss L with respect to q, k and v, given
  * dout = dL/dout for out = linattn_forward(q, k, v, causal).  All seven tensors are
  * [B][H][n][d] of type `dtype` (dq, dk, dv written in that type); accumulation is float32

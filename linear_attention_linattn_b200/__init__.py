@@ -10,10 +10,12 @@ Raw C entry points (pointers as ints):
     linattn_forward, linattn_forward_ex, linattn_forward_state, linattn_decode_step,
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
     linattn_launch_count, linattn_forward_noalloc, linattn_profile_events,
-    linattn_forward_init, linattn_sum_states, linattn_backward
+    linattn_forward_init, linattn_sum_states, linattn_backward, linattn_favor_features,
+    linattn_forward_features
 
 Tensor helpers: ``forward``, ``forward_init``, ``forward_state``, ``sum_states``,
-``backward``, ``decode_step``, ``device_error``; ``seqshard`` splits one sequence over ranks.
+``backward``, ``favor_features``, ``forward_features``, ``forward_favor``, ``decode_step``,
+``device_error``; ``seqshard`` splits one sequence over ranks.
 """
 from __future__ import annotations
 
@@ -55,6 +57,9 @@ SIGNATURES = {
     "linattn_sum_states": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
     "linattn_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                         _i64, ctypes.c_int, ctypes.c_int, _vp]),
+    "linattn_favor_features": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]),
+    "linattn_forward_features": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                                ctypes.c_int, ctypes.c_int, _vp]),
 }
 
 _lib = None
@@ -183,6 +188,51 @@ def sum_states(states, count: int, skip: int = -1, S=None, z=None, stream=None):
                                 z.data_ptr(), _stream_ptr(stream))
     _check(st, "linattn_sum_states")
     return S, z
+
+
+def favor_features(x, W, out=None, stream=None):
+    """FAVOR+ positive random features exp(W x - |x|^2/2) / sqrt(d) of x [..., d] (float32 or
+    bfloat16 CUDA tensor); W: float32 [d, d] CUDA tensor of random rows.  Returns [..., d]."""
+    import torch
+    _dev(x, "x")
+    _dev(W, "W")
+    d = x.shape[-1]
+    if W.dtype != torch.float32 or tuple(W.shape) != (d, d):
+        raise ValueError("W must be a float32 [d, d] tensor")
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(out, "out")
+    lib = load_library()
+    st = lib.linattn_favor_features(x.data_ptr(), W.data_ptr(), out.data_ptr(), x.numel() // d, d,
+                                    _dtype_code(x), _stream_ptr(stream))
+    _check(st, "linattn_favor_features")
+    return out
+
+
+def forward_features(phi_q, phi_k, v, causal: bool, out=None, stream=None):
+    """forward with caller-computed non-negative features phi_q, phi_k [B, H, n, d]."""
+    import torch
+    for t, nm in ((phi_q, "phi_q"), (phi_k, "phi_k"), (v, "v")):
+        _dev(t, nm)
+    if not (phi_q.shape == phi_k.shape == v.shape and v.dim() == 4 and
+            phi_q.dtype == phi_k.dtype == v.dtype):
+        raise ValueError("phi_q, phi_k, v must share one [B, H, n, d] shape and dtype")
+    if out is None:
+        out = torch.empty_like(v)
+    _dev(out, "out")
+    B, H, n, d = v.shape
+    lib = load_library()
+    st = lib.linattn_forward_features(phi_q.data_ptr(), phi_k.data_ptr(), v.data_ptr(),
+                                      out.data_ptr(), B, H, n, d, int(bool(causal)),
+                                      _dtype_code(v), _stream_ptr(stream))
+    _check(st, "linattn_forward_features")
+    return out
+
+
+def forward_favor(q, k, v, W, causal: bool, stream=None):
+    """FAVOR+ linear attention: the forward pass on favor_features(q, W), favor_features(k, W)."""
+    return forward_features(favor_features(q, W, stream=stream), favor_features(k, W, stream=stream),
+                            v, causal, stream=stream)
 
 
 def backward(q, k, v, dout, causal: bool, stream=None):

@@ -85,8 +85,8 @@ linattn_status check_forward_shape(int64_t B, int64_t H, int64_t n, int64_t d) {
 // state the other tokens of the sequence contribute (non-causal).
 linattn_status forward_tc(const void *q, const void *k, const void *v, void *out,
                           int64_t heads, int64_t n, int d, int causal, int64_t seg,
-                          const float *init_S, const float *init_z, DeviceState *ds,
-                          cudaStream_t st) {
+                          const float *init_S, const float *init_z, int features,
+                          DeviceState *ds, cudaStream_t st) {
   if (seg == 0) seg = tc_default_segment(heads, n, d);
   Workspace ws;
   ws.st = st;
@@ -94,13 +94,13 @@ linattn_status forward_tc(const void *q, const void *k, const void *v, void *out
                               st) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   return to_status(tc_forward(q, k, v, out, heads, n, d, causal, seg, ws.ptr, ds->err_word,
-                              init_S, init_z, st));
+                              init_S, init_z, features, st));
 }
 
 linattn_status forward_simt(const void *q, const void *k, const void *v, void *out,
                             int64_t heads, int64_t n, int d, int causal, int is_bf16,
-                            const float *init_S, const float *init_z, DeviceState *ds,
-                            cudaStream_t st) {
+                            const float *init_S, const float *init_z, int features,
+                            DeviceState *ds, cudaStream_t st) {
   const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
   const int64_t per = (int64_t)d * d + d;
   // causal: one state per chunk; non-causal: chunk states plus one total per head
@@ -110,13 +110,13 @@ linattn_status forward_simt(const void *q, const void *k, const void *v, void *o
   cudaError_t e = cudaMallocFromPoolAsync(&ws.ptr, bytes, ds->pool, st);
   if (e != cudaSuccess) return LINATTN_ERR_CUDA;
   float *w = static_cast<float *>(ws.ptr);
-  e = launch_simt_chunk_state(k, v, w, heads, n, d, is_bf16, st);
+  e = launch_simt_chunk_state(k, v, w, heads, n, d, is_bf16, features, st);
   if (e != cudaSuccess) return LINATTN_ERR_CUDA;
   if (causal) {
     e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
     if (e != cudaSuccess) return LINATTN_ERR_CUDA;
     e = launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
-                              nchunks * per, heads, n, d, 1, is_bf16, st);
+                              nchunks * per, heads, n, d, 1, is_bf16, features, st);
   } else {
     float *tot = w + heads * nchunks * per;
     float *tot_z = tot + heads * (int64_t)d * d;
@@ -124,7 +124,7 @@ linattn_status forward_simt(const void *q, const void *k, const void *v, void *o
                            init_z, st);
     if (e != cudaSuccess) return LINATTN_ERR_CUDA;
     e = launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, (int64_t)d * d, 0, d, heads, n, d, 0,
-                              is_bf16, st);
+                              is_bf16, features, st);
   }
   return to_status(e);
 }
@@ -152,9 +152,9 @@ linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, v
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == LINATTN_BF16)
-    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, segment_len, nullptr, nullptr, ds,
-                      st);
-  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, ds, st);
+    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, segment_len, nullptr, nullptr, 0,
+                      ds, st);
+  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, 0, ds, st);
 }
 
 linattn_status linattn_forward_init(const void *q, const void *k, const void *v, void *out,
@@ -173,8 +173,43 @@ linattn_status linattn_forward_init(const void *q, const void *k, const void *v,
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == LINATTN_BF16)
-    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, ds, st);
-  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, ds, st);
+    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, 0, ds, st);
+  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, 0, ds, st);
+}
+
+linattn_status linattn_forward_features(const void *phi_q, const void *phi_k, const void *v,
+                                        void *out, int64_t B, int64_t H, int64_t n, int64_t d,
+                                        int causal, linattn_dtype dtype,
+                                        linattn_stream_t stream) {
+  if (!phi_q || !phi_k || !v || !out) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(phi_q) || !aligned16(phi_k) || !aligned16(v) || !aligned16(out))
+    return LINATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  linattn_status s = check_forward_shape(B, H, n, d);
+  if (s != LINATTN_OK) return s;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == LINATTN_BF16)
+    return forward_tc(phi_q, phi_k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, 1, ds,
+                      st);
+  return forward_simt(phi_q, phi_k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, 1, ds,
+                      st);
+}
+
+linattn_status linattn_favor_features(const void *x, const float *W, void *out, int64_t rows,
+                                      int64_t d, linattn_dtype dtype, linattn_stream_t stream) {
+  if (!x || !W || !out) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W) || !aligned16(out)) return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  if (rows <= 0 || d <= 0) return LINATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
+  if (rows > (int64_t(1) << 40) / d) return LINATTN_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  return to_status(launch_favor_features(x, W, out, rows, (int)d, dtype == LINATTN_BF16,
+                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
 linattn_status linattn_backward(const void *q, const void *k, const void *v, const void *dout,
@@ -253,7 +288,7 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
       cudaSuccess)
     return LINATTN_ERR_CUDA;
   float *w = static_cast<float *>(ws.ptr);
-  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, 0, st);
+  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, 0, 0, st);
   if (e == cudaSuccess)
     e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, d * d, state_z, d, nullptr,
                            nullptr, st);

@@ -512,7 +512,8 @@ cudaError_t backward_impl(const T *q, const T *k, const T *v, const T *g, T *dq,
   if ((e = set_smem(bwd_state_kernel<D, T>, smem_state)) != cudaSuccess) return e;
 
   // K1 + K2: the forward states of the chunks (prefix) or the head (total)
-  e = launch_simt_chunk_state(k, v, Sf, heads, n, D, std::is_same<T, __nv_bfloat16>::value, st);
+  e = launch_simt_chunk_state(k, v, Sf, heads, n, D, std::is_same<T, __nv_bfloat16>::value, 0,
+                              st);
   if (e != cudaSuccess) return e;
   int64_t Scs = per, Shs = nchunks * per;
   const float *Sbase = Sf;

@@ -16,9 +16,11 @@ void record_launch_event(cudaStream_t st);
 constexpr int kSimtChunk = 64;
 
 // ---- CUDA-core path (simt_forward.cu); is_bf16 selects bf16 I/O, else fp32 ------------
-// Chunk aggregates into ws[head][chunk][D*D + D] (S row-major, then z).
+// Chunk aggregates into ws[head][chunk][D*D + D] (S row-major, then z).  features != 0:
+// k holds non-negative features already (no phi applied), likewise q below.
 cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int64_t heads,
-                                    int64_t n, int d, int is_bf16, cudaStream_t st);
+                                    int64_t n, int d, int is_bf16, int features,
+                                    cudaStream_t st);
 // In-place exclusive prefix over the segments of each head (mode 0), or the per-head total
 // written to S_out + head*S_hs ([D][d]) and z_out + head*z_hs ([D]) (mode 1); both start
 // from the state (init_S [heads][D][d], init_z [heads][D]) when init_S is not null.
@@ -34,7 +36,11 @@ cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, v
                                   const float *S, const float *z, int64_t S_chunk_stride,
                                   int64_t S_head_stride, int64_t z_chunk_stride,
                                   int64_t z_head_stride, int64_t heads, int64_t n, int d,
-                                  int causal, int is_bf16, cudaStream_t st);
+                                  int causal, int is_bf16, int features, cudaStream_t st);
+// FAVOR+ positive random features: out[t][i] = exp(W[i] . x[t] - |x[t]|^2 / 2) / sqrt(d)
+// for rows t < rows; W [d][d] float32 (m = d features); x, out of type bf16 or fp32.
+cudaError_t launch_favor_features(const void *x, const float *W, void *out, int64_t rows, int d,
+                                  int is_bf16, cudaStream_t st);
 
 // ---- backward pass (backward.cu), CUDA cores; is_bf16 selects bf16 I/O, else fp32 ------
 // Workspace floats linattn_backward needs.
@@ -55,9 +61,11 @@ int64_t tc_default_segment(int64_t heads, int64_t n, int d);
 // Workspace bytes the tensor-core forward needs.
 size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int causal);
 // init_S / init_z (nullable): the state before the first token of every head.
+// features != 0: q and k are non-negative features already (no phi applied).
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
                        int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
-                       const float *init_S, const float *init_z, cudaStream_t st);
+                       const float *init_S, const float *init_z, int features,
+                       cudaStream_t st);
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
                              int64_t heads, int64_t n, int d, int64_t seg, void *ws, int *err,
                              cudaStream_t st);

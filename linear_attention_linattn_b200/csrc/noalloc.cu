@@ -114,16 +114,16 @@ extern "C" linattn_status linattn_forward_noalloc(const void *q, const void *k, 
 
   cudaError_t e;
   if (dtype == LINATTN_BF16) {
-    e = tc_forward(q, k, v, out, heads, n, di, causal, seg, ws, status_word, nullptr, nullptr,
+    e = tc_forward(q, k, v, out, heads, n, di, causal, seg, ws, status_word, nullptr, nullptr, 0,
                    st);
   } else {
-    e = launch_simt_chunk_state(k, v, ws, heads, n, di, 0, st);
+    e = launch_simt_chunk_state(k, v, ws, heads, n, di, 0, 0, st);
     if (e == cudaSuccess && causal) {
       e = launch_scan_states(ws, heads, nseg, di, 0, nullptr, 0, nullptr, 0, nullptr, nullptr,
                              st);
       if (e == cudaSuccess)
         e = launch_simt_chunk_out(q, k, v, out, ws, ws + d * d, per, nseg * per, per,
-                                  nseg * per, heads, n, di, 1, 0, st);
+                                  nseg * per, heads, n, di, 1, 0, 0, st);
     } else if (e == cudaSuccess) {
       float *tot = ws + heads * nseg * per;
       float *tot_z = tot + heads * d * d;
@@ -131,7 +131,7 @@ extern "C" linattn_status linattn_forward_noalloc(const void *q, const void *k, 
                              st);
       if (e == cudaSuccess)
         e = launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, d * d, 0, d, heads, n, di, 0, 0,
-                                  st);
+                                  0, st);
     }
   }
   return e == cudaSuccess ? LINATTN_OK : LINATTN_ERR_CUDA;

@@ -60,7 +60,8 @@ template <int D, typename T>
 __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__restrict__ k,
                                                                     const T *__restrict__ v,
                                                                     float *__restrict__ ws,
-                                                                    int64_t n, int64_t nchunks) {
+                                                                    int64_t n, int64_t nchunks,
+                                                                    int apply_phi) {
   extern __shared__ float4 smem_f4[];
   float *sK = reinterpret_cast<float *>(smem_f4);  // phi(K_c) [C][D]
   float *sV = sK + C * D;                          // V_c [C][D]
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__r
   const int64_t head = blockIdx.x / nchunks;
   const int64_t t0 = chunk * C;
   const int valid = n - t0 < C ? static_cast<int>(n - t0) : C;
-  load_rows<D, T>(sK, k + (head * n + t0) * D, valid, true);
+  load_rows<D, T>(sK, k + (head * n + t0) * D, valid, apply_phi != 0);
   load_rows<D, T>(sV, v + (head * n + t0) * D, valid, false);
   __syncthreads();
 
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_out_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     T *__restrict__ out, const float *__restrict__ S, const float *__restrict__ z,
     int64_t S_chunk_stride, int64_t S_head_stride, int64_t z_chunk_stride,
-    int64_t z_head_stride, int64_t n, int64_t nchunks) {
+    int64_t z_head_stride, int64_t n, int64_t nchunks, int apply_phi) {
   extern __shared__ float4 smem_f4[];
   float *sQ = reinterpret_cast<float *>(smem_f4);  // phi(Q_c) [C][D]
   float *sS = sQ + C * D;                          // S_<c [D][D]
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_out_kernel(
   const int valid = n - t0 < C ? static_cast<int>(n - t0) : C;
   const int64_t row0 = (head * n + t0) * D;
 
-  load_rows<D, T>(sQ, q + row0, valid, true);
+  load_rows<D, T>(sQ, q + row0, valid, apply_phi != 0);
   const float *Sg = S + head * S_head_stride + chunk * S_chunk_stride;
   const float *zg = z + head * z_head_stride + chunk * z_chunk_stride;
   for (int i = threadIdx.x; i < D * D / 4; i += kThreads)
@@ -192,10 +193,12 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_out_kernel(
       float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
       if (t < valid) {
         x = load4(k + row0 + (int64_t)t * D + 4 * cg);
-        x.x = phi(x.x);
-        x.y = phi(x.y);
-        x.z = phi(x.z);
-        x.w = phi(x.w);
+        if (apply_phi) {
+          x.x = phi(x.x);
+          x.y = phi(x.y);
+          x.z = phi(x.z);
+          x.w = phi(x.w);
+        }
       }
       sK[(4 * cg + 0) * C + t] = x.x;
       sK[(4 * cg + 1) * C + t] = x.y;
@@ -285,14 +288,14 @@ size_t chunk_out_smem(bool causal) {
 
 template <int D, typename T>
 cudaError_t chunk_state_impl(const void *k, const void *v, float *ws, int64_t heads, int64_t n,
-                             cudaStream_t st) {
+                             int apply_phi, cudaStream_t st) {
   const int64_t nchunks = (n + C - 1) / C;
   const size_t smem = 2 * (size_t)C * D * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(simt_chunk_state_kernel<D, T>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   simt_chunk_state_kernel<D, T><<<(unsigned)(nchunks * heads), kThreads, smem, st>>>(
-      static_cast<const T *>(k), static_cast<const T *>(v), ws, n, nchunks);
+      static_cast<const T *>(k), static_cast<const T *>(v), ws, n, nchunks, apply_phi);
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();
@@ -301,7 +304,8 @@ cudaError_t chunk_state_impl(const void *k, const void *v, float *ws, int64_t he
 template <int D, bool CAUSAL, typename T>
 cudaError_t chunk_out_impl(const void *q, const void *k, const void *v, void *out,
                            const float *S, const float *z, int64_t Scs, int64_t Shs,
-                           int64_t zcs, int64_t zhs, int64_t heads, int64_t n, cudaStream_t st) {
+                           int64_t zcs, int64_t zhs, int64_t heads, int64_t n, int apply_phi,
+                           cudaStream_t st) {
   const int64_t nchunks = (n + C - 1) / C;
   const size_t smem = chunk_out_smem<D>(CAUSAL);
   cudaError_t e = cudaFuncSetAttribute(simt_chunk_out_kernel<D, CAUSAL, T>,
@@ -309,7 +313,7 @@ cudaError_t chunk_out_impl(const void *q, const void *k, const void *v, void *ou
   if (e != cudaSuccess) return e;
   simt_chunk_out_kernel<D, CAUSAL, T><<<(unsigned)(nchunks * heads), kThreads, smem, st>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
-      static_cast<T *>(out), S, z, Scs, Shs, zcs, zhs, n, nchunks);
+      static_cast<T *>(out), S, z, Scs, Shs, zcs, zhs, n, nchunks, apply_phi);
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();
@@ -317,32 +321,34 @@ cudaError_t chunk_out_impl(const void *q, const void *k, const void *v, void *ou
 
 template <typename T>
 cudaError_t chunk_state_t(const void *k, const void *v, float *ws, int64_t heads, int64_t n,
-                          int d, cudaStream_t st) {
-  return d == 64 ? chunk_state_impl<64, T>(k, v, ws, heads, n, st)
-                 : chunk_state_impl<128, T>(k, v, ws, heads, n, st);
+                          int d, int apply_phi, cudaStream_t st) {
+  return d == 64 ? chunk_state_impl<64, T>(k, v, ws, heads, n, apply_phi, st)
+                 : chunk_state_impl<128, T>(k, v, ws, heads, n, apply_phi, st);
 }
 
 template <typename T>
 cudaError_t chunk_out_t(const void *q, const void *k, const void *v, void *out, const float *S,
                         const float *z, int64_t Scs, int64_t Shs, int64_t zcs, int64_t zhs,
-                        int64_t heads, int64_t n, int d, int causal, cudaStream_t st) {
+                        int64_t heads, int64_t n, int d, int causal, int apply_phi,
+                        cudaStream_t st) {
   if (d == 64)
     return causal ? chunk_out_impl<64, true, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads,
-                                                n, st)
+                                                n, apply_phi, st)
                   : chunk_out_impl<64, false, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads,
-                                                 n, st);
+                                                 n, apply_phi, st);
   return causal ? chunk_out_impl<128, true, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n,
-                                               st)
+                                               apply_phi, st)
                 : chunk_out_impl<128, false, T>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n,
-                                                st);
+                                                apply_phi, st);
 }
 
 }  // namespace
 
 cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int64_t heads,
-                                    int64_t n, int d, int is_bf16, cudaStream_t st) {
-  return is_bf16 ? chunk_state_t<__nv_bfloat16>(k, v, ws, heads, n, d, st)
-                 : chunk_state_t<float>(k, v, ws, heads, n, d, st);
+                                    int64_t n, int d, int is_bf16, int features,
+                                    cudaStream_t st) {
+  return is_bf16 ? chunk_state_t<__nv_bfloat16>(k, v, ws, heads, n, d, !features, st)
+                 : chunk_state_t<float>(k, v, ws, heads, n, d, !features, st);
 }
 
 cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
@@ -398,11 +404,11 @@ cudaError_t launch_sum_states(const float *states, int64_t count, int64_t skip, 
 cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, void *out,
                                   const float *S, const float *z, int64_t Scs, int64_t Shs,
                                   int64_t zcs, int64_t zhs, int64_t heads, int64_t n, int d,
-                                  int causal, int is_bf16, cudaStream_t st) {
+                                  int causal, int is_bf16, int features, cudaStream_t st) {
   return is_bf16 ? chunk_out_t<__nv_bfloat16>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n,
-                                               d, causal, st)
+                                               d, causal, !features, st)
                  : chunk_out_t<float>(q, k, v, out, S, z, Scs, Shs, zcs, zhs, heads, n, d,
-                                      causal, st);
+                                      causal, !features, st);
 }
 
 }  // namespace linattn

@@ -272,7 +272,9 @@ __device__ __forceinline__ Item item_at(int64_t it, int64_t n, int64_t seg_len, 
 // chunks, and g counts them across items, so the stage ring, the barrier phases and the O
 // buffers run on from one item into the next: the loads of an item's first chunks overlap
 // the previous item's last ones.
-template <int D, int MODE>
+// PHI: apply phi = elu + 1 to Q and K (the method); false takes Q and K as given,
+// non-negative features (FAVOR+ features computed by favor_features_kernel).
+template <int D, int MODE, bool PHI>
 __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
@@ -551,7 +553,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
         uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
         const int64_t left = I.t_end - (I.t_begin + (int64_t)c * C);
         const int valid = left < C ? static_cast<int>(left) : C;
-        if (G::LQ) {
+        if (G::LQ && PHI) {
           uint4 *p = reinterpret_cast<uint4 *>(st);
 #pragma unroll 2
           for (int i = xt; i < G::TILE / 16; i += W::XTHREADS) {
@@ -572,10 +574,12 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
             uint4 x = make_uint4(0u, 0u, 0u, 0u);
             if (row < valid) {
               x = *p;
-              x.x = phi_bf16x2(x.x);
-              x.y = phi_bf16x2(x.y);
-              x.z = phi_bf16x2(x.z);
-              x.w = phi_bf16x2(x.w);
+              if (PHI) {
+                x.x = phi_bf16x2(x.x);
+                x.y = phi_bf16x2(x.y);
+                x.z = phi_bf16x2(x.z);
+                x.w = phi_bf16x2(x.w);
+              }
             }
             *p = x;
           }
@@ -889,13 +893,13 @@ int sm_count() {
   return v;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool PHI = true>
 cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                       void *out, const float *init, int64_t ihs, int64_t iss,
                       float *out_state, int64_t heads, int64_t n, int64_t seg, int64_t nseg,
                       int *err, cudaStream_t st) {
   using G = Cfg<D, MODE>;
-  auto kern = tc_kernel<D, MODE>;
+  auto kern = tc_kernel<D, MODE, PHI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   // One CTA holds a whole SM's shared memory and TMEM.  Persistent CTAs (one per SM, items
@@ -916,7 +920,7 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool PHI>
 cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out, int64_t heads,
                          int64_t n, int causal, int64_t seg, void *ws, int *err,
                          const float *init_S, const float *init_z, cudaStream_t st) {
@@ -928,21 +932,21 @@ cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out,
   if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
   if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
   float *w = static_cast<float *>(ws);
-  e = launch_tc<D, kState>(tq, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
+  e = launch_tc<D, kState, PHI>(tq, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
   if (e != cudaSuccess) return e;
   if (causal) {
     e = launch_scan_states(w, heads, nseg, D, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
     if (e != cudaSuccess) return e;
-    return launch_tc<D, kCausalOut>(tq, tk, tv, out, w, nseg * per, per, nullptr, heads, n, seg,
-                                    nseg, err, st);
+    return launch_tc<D, kCausalOut, PHI>(tq, tk, tv, out, w, nseg * per, per, nullptr, heads, n,
+                                         seg, nseg, err, st);
   }
   // per-head totals, packed as [heads][D*D + D] (S row-major, then z)
   float *tot = w + heads * nseg * per;
   e = launch_scan_states(w, heads, nseg, D, 1, tot, per, tot + (int64_t)D * D, per, init_S,
                          init_z, st);
   if (e != cudaSuccess) return e;
-  return launch_tc<D, kNoncausalOut>(tq, tk, tv, out, tot, per, 0, nullptr, heads, n, seg, nseg,
-                                     err, st);
+  return launch_tc<D, kNoncausalOut, PHI>(tq, tk, tv, out, tot, per, 0, nullptr, heads, n, seg,
+                                          nseg, err, st);
 }
 
 }  // namespace
@@ -975,10 +979,17 @@ size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int caus
 
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
                        int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
-                       const float *init_S, const float *init_z, cudaStream_t st) {
-  return d == 64
-             ? tc_forward_d<64>(q, k, v, out, heads, n, causal, seg, ws, err, init_S, init_z, st)
-             : tc_forward_d<128>(q, k, v, out, heads, n, causal, seg, ws, err, init_S, init_z, st);
+                       const float *init_S, const float *init_z, int features,
+                       cudaStream_t st) {
+  if (features)
+    return d == 64 ? tc_forward_d<64, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                             init_z, st)
+                   : tc_forward_d<128, false>(q, k, v, out, heads, n, causal, seg, ws, err,
+                                              init_S, init_z, st);
+  return d == 64 ? tc_forward_d<64, true>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                          init_z, st)
+                 : tc_forward_d<128, true>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                           init_z, st);
 }
 
 template <int D>
