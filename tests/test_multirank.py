@@ -32,7 +32,7 @@ def _worker(rank, world, port, out):
 def test_two_ranks_partition_heads_and_take_max():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)

@@ -89,7 +89,7 @@ def _worker(rank, world, port, causal, out):
 def test_two_gloo_ranks_match_whole_sequence(causal):
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, causal, out), nprocs=world,
                            start_method="spawn")
