@@ -199,6 +199,12 @@ const char *linattn_status_string(linattn_status status);
  * (or LINATTN_ERR_CUDA if synchronising failed). */
 linattn_status linattn_device_error(linattn_stream_t stream);
 
+/* Self-test of the failure path: launches one thread that waits, with the kernels' bounded
+ * wait, on a barrier nothing ever completes.  It gives up after the wait limit (2 s) without
+ * trapping; the next linattn_device_error() then returns LINATTN_ERR_TIMEOUT (and clears it),
+ * and the context stays usable. */
+linattn_status linattn_selftest_wait_timeout(linattn_stream_t stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int linattn_version(void);
 

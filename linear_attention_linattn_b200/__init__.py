@@ -11,7 +11,7 @@ Raw C entry points (pointers as ints):
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
     linattn_launch_count, linattn_forward_noalloc, linattn_profile_events,
     linattn_forward_init, linattn_sum_states, linattn_backward, linattn_favor_features,
-    linattn_forward_features
+    linattn_forward_features, linattn_selftest_wait_timeout
 
 Tensor helpers: ``forward``, ``forward_init``, ``forward_state``, ``sum_states``,
 ``backward``, ``favor_features``, ``forward_features``, ``forward_favor``, ``decode_step``,
@@ -58,6 +58,7 @@ SIGNATURES = {
     "linattn_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                         _i64, ctypes.c_int, ctypes.c_int, _vp]),
     "linattn_favor_features": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]),
+    "linattn_selftest_wait_timeout": (ctypes.c_int, [_vp]),
     "linattn_forward_features": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                                 ctypes.c_int, ctypes.c_int, _vp]),
 }

@@ -129,12 +129,36 @@ linattn_status forward_simt(const void *q, const void *k, const void *v, void *o
   return to_status(e);
 }
 
+// Failure-path self-test: one thread waits, with the kernels' own bounded wait, on an mbarrier
+// that nothing ever arrives at.  The wait gives up after its limit and records
+// LINATTN_ERR_TIMEOUT in the device's error word, exactly as a stalled kernel would.
+__global__ void wait_timeout_selftest_kernel(int *err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err);
+}
+
 }  // namespace
 }  // namespace linattn
 
 using namespace linattn;
 
 extern "C" {
+
+linattn_status linattn_selftest_wait_timeout(linattn_stream_t stream) {
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      ds->err_word);
+  count_launches(1);
+  return to_status(cudaGetLastError());
+}
 
 linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, void *out,
                                   int64_t B, int64_t H, int64_t n, int64_t d, int causal,
