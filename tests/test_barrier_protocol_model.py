@@ -1,0 +1,197 @@
+"""A model of the tensor-core kernel's barrier protocol (tc_forward.cu), checked on the CPU.
+
+Every warp role (TMA producer, feature map, MMA issuer, state group, scores/output group) is
+written as the sequence of mbarrier waits (with the phase index it waits for) and arrivals it
+performs, for the three modes (0 aggregate, 1 causal output, 2 non-causal output) and any list
+of work items of 1..16 chunks walked by one CTA.  A random scheduler interleaves the roles. The
+test fails on a deadlock (no role can move) or on parity aliasing (a wait for a phase two or more
+phases behind its barrier, which the hardware's parity test cannot tell from a pending one).
+Each role's arrivals count as one (the kernel's thread counts are per role).  This model mirrors
+the kernel's code by hand: change both together.
+"""
+import random
+import sys
+
+import pytest
+
+
+class Barrier:
+    def __init__(self, count):
+        self.count, self.pending, self.completed = count, 0, 0
+
+
+def roles(mode, NS, items):
+    """Generators of ('w', barrier, phase) and ('a', barrier) events, one per warp role."""
+
+    def tma():
+        g = 0
+        for nc in items:
+            for _ in range(nc):
+                s = g % NS
+                if g >= NS:
+                    yield ("w", f"empty[{s}]", g // NS - 1)
+                yield ("a", f"full[{s}]")
+                g += 1
+        for gg in range(max(0, g - NS), g):  # drain: every load has landed
+            yield ("w", f"full[{gg % NS}]", gg // NS)
+
+    def feature_map():
+        g = 0
+        for nc in items:
+            for _ in range(nc):
+                s = g % NS
+                yield ("w", f"full[{s}]", g // NS)
+                yield ("a", f"ready[{s}]")
+                g += 1
+
+    def mma():
+        g = 0
+        for j, nc in enumerate(items):
+            b = j & 1
+            if mode == 0 and j >= 2:
+                yield ("w", f"item_empty[{b}]", (j >> 1) - 1)
+            if mode == 2:
+                yield ("w", f"item_full[{b}]", j >> 1)
+            for _ in range(nc):
+                s = g % NS
+                yield ("w", f"ready[{s}]", g // NS)
+                if mode == 0:
+                    yield ("a", f"empty[{s}]")
+                elif mode == 1:
+                    yield ("w", "z_ready", g)
+                    if g >= 1:  # the previous chunk's P V, interleaved with this chunk's scores
+                        yield ("w", "p_ready", g - 1)
+                        yield ("a", f"o_full[{(g - 1) & 1}]")
+                        yield ("a", f"empty[{(g - 1) % NS}]")
+                    yield ("a", "p_full")
+                    yield ("w", "s_ready", g)
+                    if g >= 2:
+                        yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
+                    yield ("a", "s_full")
+                else:
+                    if g >= 2:
+                        yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
+                    yield ("a", f"o_full[{g & 1}]")
+                    yield ("a", f"empty[{s}]")
+                g += 1
+            if mode == 0:
+                yield ("a", f"item_full[{b}]")
+            if mode == 2:
+                yield ("a", f"item_empty[{b}]")
+        if mode == 1 and g > 0:  # the last chunk's P V
+            yield ("w", "p_ready", g - 1)
+            yield ("a", f"o_full[{(g - 1) & 1}]")
+            yield ("a", f"empty[{(g - 1) % NS}]")
+        yield ("a", "fin")
+        yield ("w", "fin", 0)
+
+    def state_group():
+        if mode == 1:
+            g = 0
+            for j, nc in enumerate(items):
+                if j > 0:  # the previous item's last S and O products are done
+                    yield ("w", "s_full", g - 1)
+                yield ("a", "z_ready")
+                yield ("a", "s_ready")
+                for c in range(nc):
+                    yield ("w", "p_full", g)
+                    yield ("a", "p_ready")
+                    yield ("a", "rs_ready")
+                    if c + 1 < nc:
+                        yield ("w", "s_full", g)
+                        yield ("a", "z_ready")
+                        yield ("a", "s_ready")
+                    g += 1
+        elif mode == 2:
+            for j in range(len(items)):
+                b = j & 1
+                if j >= 2:
+                    yield ("w", f"item_empty[{b}]", (j >> 1) - 1)
+                yield ("a", f"item_full[{b}]")
+        else:
+            for j in range(len(items)):
+                b = j & 1
+                yield ("w", f"item_full[{b}]", j >> 1)
+                yield ("a", f"item_empty[{b}]")
+
+    def output_group():
+        g = 0
+        if mode == 1:
+            for nc in items:
+                for _ in range(nc):
+                    yield ("w", "p_full", g)
+                    yield ("w", "rs_ready", g)
+                    yield ("a", "p_ready")
+                    if g >= 1:
+                        yield ("w", f"o_full[{(g - 1) & 1}]", (g - 1) >> 1)
+                        yield ("a", f"o_empty[{(g - 1) & 1}]")
+                    g += 1
+            if g > 0:
+                yield ("w", f"o_full[{(g - 1) & 1}]", (g - 1) >> 1)
+                yield ("a", f"o_empty[{(g - 1) & 1}]")
+        elif mode == 2:
+            for nc in items:
+                for _ in range(nc):
+                    yield ("w", f"o_full[{g & 1}]", g >> 1)
+                    yield ("a", f"o_empty[{g & 1}]")
+                    g += 1
+
+    return [tma(), feature_map(), mma(), state_group(), output_group()]
+
+
+def run(mode, NS, items, rng):
+    counts = {"p_ready": 2}  # arrivals per phase: both drain groups release p_ready
+    bars = {}
+
+    def bar(name):
+        if name not in bars:
+            bars[name] = Barrier(counts.get(name.split("[")[0], 1))
+        return bars[name]
+
+    gens = roles(mode, NS, items)
+    cur = [next(gen, None) for gen in gens]
+    while True:
+        runnable = []
+        for r, ev in enumerate(cur):
+            if ev is None:
+                continue
+            if ev[0] == "a":
+                runnable.append(r)
+                continue
+            b, phase = bar(ev[1]), ev[2]
+            assert b.completed < phase + 2, f"parity aliasing: {ev}, mode {mode}, items {items}"
+            if b.completed > phase:  # the waited-for phase has completed
+                runnable.append(r)
+        if not runnable:
+            assert all(ev is None for ev in cur), f"deadlock at {cur}, mode {mode}, items {items}"
+            return True
+        r = rng.choice(runnable)
+        if cur[r][0] == "a":
+            b = bar(cur[r][1])
+            b.pending += 1
+            if b.pending == b.count:
+                b.pending, b.completed = 0, b.completed + 1
+        cur[r] = next(gens[r], None)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_protocol_has_no_deadlock_or_aliasing(mode):
+    rng = random.Random(1000 + mode)
+    for _ in range(1500):
+        NS = rng.choice([2, 3, 5, 6, 8])
+        items = [rng.choice([1, 1, 2, 3, 5, 16]) for _ in range(rng.randint(1, 9))]
+        assert run(mode, NS, items, rng)
+
+
+def test_model_catches_a_missing_arrival(monkeypatch):
+    """The check has teeth: a state group that never releases p_ready deadlocks the model."""
+    original = roles
+
+    def broken(mode, NS, items):
+        gens = original(mode, NS, items)
+        gens[3] = (ev for ev in gens[3] if ev != ("a", "p_ready"))
+        return gens
+
+    monkeypatch.setattr(sys.modules[__name__], "roles", broken)
+    with pytest.raises(AssertionError, match="deadlock"):
+        run(1, 3, [4, 2], random.Random(0))
