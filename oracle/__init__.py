@@ -77,6 +77,9 @@ class Oracle:
         lib.oracle_forward_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
                                            ctypes.c_int, ctypes.c_int]
         lib.oracle_forward_f64.restype = None
+        lib.oracle_forward_dkv_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
+                                               ctypes.c_int, ctypes.c_int]
+        lib.oracle_forward_dkv_f64.restype = None
         lib.oracle_forward_rows_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64,
                                                 ctypes.c_int, _ip, _i64, ctypes.c_int]
         lib.oracle_forward_rows_f64.restype = None
@@ -91,6 +94,9 @@ class Oracle:
         lib.oracle_favor_features_f64.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64]
         lib.oracle_favor_features_f64.restype = None
         lib.oracle_plant.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = None
+        lib.oracle_get_threads.restype = ctypes.c_int
         self.lib = lib
         self.plant = lib.oracle_plant()
 
@@ -106,8 +112,19 @@ class Oracle:
         return self.lib.oracle_phi(float(x), int(phi_kind))
 
     def forward(self, q, k, v, causal: bool, phi_kind: int = PHI_ELU1) -> np.ndarray:
-        """q, k, v: [..., n, d] (any number of leading head axes).  Returns float64 out."""
+        """q, k, v: [..., n, d] (any number of leading head axes).  Returns float64 out.
+        q and k may have their own last dimension m (features, e.g. FAVOR+ with
+        phi_kind=PHI_IDENTITY): then S is m x d and out has v's shape."""
         q, k, v = self._f64(q), self._f64(k), self._f64(v)
+        if q.shape[-1] != v.shape[-1]:
+            assert q.shape == k.shape and q.shape[:-1] == v.shape[:-1] and q.ndim >= 2
+            n, m, d = q.shape[-2], q.shape[-1], v.shape[-1]
+            heads = int(np.prod(q.shape[:-2], dtype=np.int64)) if q.ndim > 2 else 1
+            out = np.empty_like(v)
+            self.lib.oracle_forward_dkv_f64(self._ptr(q), self._ptr(k), self._ptr(v),
+                                            self._ptr(out), heads, n, m, d, int(bool(causal)),
+                                            int(phi_kind))
+            return out
         assert q.shape == k.shape == v.shape and q.ndim >= 2
         n, d = q.shape[-2:]
         heads = int(np.prod(q.shape[:-2], dtype=np.int64)) if q.ndim > 2 else 1
@@ -226,6 +243,15 @@ def decode_step(S, z, q, k, v, phi_kind: int = PHI_ELU1):
 
 def phi(x: float, phi_kind: int = PHI_ELU1) -> float:
     return default().phi(x, phi_kind)
+
+
+def set_threads(threads: int) -> None:
+    """Threads of the oracle's OpenMP loops (for timing; results do not depend on it)."""
+    default().lib.oracle_set_threads(int(threads))
+
+
+def get_threads() -> int:
+    return int(default().lib.oracle_get_threads())
 
 
 # --------------------------------------------------------------------------------------

@@ -44,6 +44,9 @@
  * w_ij = phi(q_i) . phi(k_j); see oracle_backward_f64.
  */
 #include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -65,29 +68,30 @@ double oracle_phi(double x, int phi_kind)
 #endif
 }
 
-/* Rank-1 update of one head's state by one token: S += phi(k) v^T, z += phi(k). */
+/* Rank-1 update of one head's state by one token: S += phi(k) v^T, z += phi(k).
+ * k has dk entries (the feature dimension D), v has dv (the value dimension d); S is [dk][dv]. */
 static void state_add_token(double *S, double *z, const double *k, const double *v,
-                            int64_t d, int phi_kind)
+                            int64_t dk, int64_t dv, int phi_kind)
 {
-    for (int64_t r = 0; r < d; ++r) {
+    for (int64_t r = 0; r < dk; ++r) {
         double pk = oracle_phi(k[r], phi_kind);
-        for (int64_t c = 0; c < d; ++c) {
+        for (int64_t c = 0; c < dv; ++c) {
 #if ORACLE_PLANT == 2
-            S[c * d + r] += pk * v[c]; /* planted: transposed state */
+            S[c * dk + r] += pk * v[c]; /* planted: transposed state */
 #else
-            S[r * d + c] += pk * v[c];
+            S[r * dv + c] += pk * v[c];
 #endif
         }
         z[r] += pk;
     }
 }
 
-/* out = phi(q) S / (phi(q) . z) for one token and one head. */
+/* out = phi(q) S / (phi(q) . z) for one token and one head (q: dk entries, out: dv). */
 static void readout_token(const double *S, const double *z, const double *q, double *out,
-                          int64_t d, int phi_kind, double *pq_scratch)
+                          int64_t dk, int64_t dv, int phi_kind, double *pq_scratch)
 {
     double den = 0.0;
-    for (int64_t r = 0; r < d; ++r) {
+    for (int64_t r = 0; r < dk; ++r) {
         pq_scratch[r] = oracle_phi(q[r], phi_kind);
 #if ORACLE_PLANT != 3
         den += pq_scratch[r] * z[r];
@@ -96,9 +100,9 @@ static void readout_token(const double *S, const double *z, const double *q, dou
 #if ORACLE_PLANT == 3
     den = 1.0; /* planted: normaliser dropped */
 #endif
-    for (int64_t c = 0; c < d; ++c) {
+    for (int64_t c = 0; c < dv; ++c) {
         double num = 0.0;
-        for (int64_t r = 0; r < d; ++r) num += pq_scratch[r] * S[r * d + c];
+        for (int64_t r = 0; r < dk; ++r) num += pq_scratch[r] * S[r * dv + c];
         out[c] = num / den;
     }
 }
@@ -117,19 +121,52 @@ void oracle_forward_f64(const double *q, const double *k, const double *v, doubl
         const int64_t base = bh * n * d;
         if (!causal) {
             for (int64_t t = 0; t < n; ++t)
-                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, d, phi_kind);
             for (int64_t t = 0; t < n; ++t)
-                readout_token(S, z, q + base + t * d, out + base + t * d, d, phi_kind, pq);
+                readout_token(S, z, q + base + t * d, out + base + t * d, d, d, phi_kind, pq);
         } else {
             for (int64_t t = 0; t < n; ++t) {
 #if ORACLE_PLANT == 1
                 /* planted: diagonal excluded (read before adding token t) */
-                readout_token(S, z, q + base + t * d, out + base + t * d, d, phi_kind, pq);
-                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+                readout_token(S, z, q + base + t * d, out + base + t * d, d, d, phi_kind, pq);
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, d, phi_kind);
 #else
-                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
-                readout_token(S, z, q + base + t * d, out + base + t * d, d, phi_kind, pq);
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, d, phi_kind);
+                readout_token(S, z, q + base + t * d, out + base + t * d, d, d, phi_kind, pq);
 #endif
+            }
+        }
+        free(S);
+        free(z);
+        free(pq);
+    }
+}
+
+/* Forward pass on features of their own dimension: q, k [heads][n][dk] (taken through
+ * phi_kind, normally the identity: caller-computed features such as FAVOR+), v and out
+ * [heads][n][dv].  The same order as oracle_forward_f64: S = sum_j phi(k_j) v_j^T is dk x dv
+ * and z = sum_j phi(k_j) has dk entries (page "Linear Attention > Memory Efficiency" writes
+ * the state as D x d with D the feature dimension). */
+void oracle_forward_dkv_f64(const double *q, const double *k, const double *v, double *out,
+                            int64_t heads, int64_t n, int64_t dk, int64_t dv, int causal,
+                            int phi_kind)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        double *S = (double *)calloc((size_t)(dk * dv), sizeof(double));
+        double *z = (double *)calloc((size_t)dk, sizeof(double));
+        double *pq = (double *)malloc((size_t)dk * sizeof(double));
+        const double *qh = q + bh * n * dk, *kh = k + bh * n * dk, *vh = v + bh * n * dv;
+        double *oh = out + bh * n * dv;
+        if (!causal) {
+            for (int64_t t = 0; t < n; ++t)
+                state_add_token(S, z, kh + t * dk, vh + t * dv, dk, dv, phi_kind);
+            for (int64_t t = 0; t < n; ++t)
+                readout_token(S, z, qh + t * dk, oh + t * dv, dk, dv, phi_kind, pq);
+        } else {
+            for (int64_t t = 0; t < n; ++t) {
+                state_add_token(S, z, kh + t * dk, vh + t * dv, dk, dv, phi_kind);
+                readout_token(S, z, qh + t * dk, oh + t * dv, dk, dv, phi_kind, pq);
             }
         }
         free(S);
@@ -153,16 +190,16 @@ void oracle_forward_rows_f64(const double *q, const double *k, const double *v, 
         const int64_t base = bh * n * d;
         if (!causal) {
             for (int64_t t = 0; t < n; ++t)
-                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, d, phi_kind);
             for (int64_t s = 0; s < nrows; ++s)
-                readout_token(S, z, q + base + rows[s] * d, out + (bh * nrows + s) * d, d,
+                readout_token(S, z, q + base + rows[s] * d, out + (bh * nrows + s) * d, d, d,
                               phi_kind, pq);
         } else {
             int64_t s = 0;
             for (int64_t t = 0; t < n && s < nrows; ++t) {
-                state_add_token(S, z, k + base + t * d, v + base + t * d, d, phi_kind);
+                state_add_token(S, z, k + base + t * d, v + base + t * d, d, d, phi_kind);
                 while (s < nrows && rows[s] == t) {
-                    readout_token(S, z, q + base + t * d, out + (bh * nrows + s) * d, d,
+                    readout_token(S, z, q + base + t * d, out + (bh * nrows + s) * d, d, d,
                                   phi_kind, pq);
                     ++s;
                 }
@@ -186,7 +223,7 @@ void oracle_state_f64(const double *k, const double *v, double *S, double *z,
         memset(Sh, 0, (size_t)(d * d) * sizeof(double));
         memset(zh, 0, (size_t)d * sizeof(double));
         for (int64_t t = 0; t < n; ++t)
-            state_add_token(Sh, zh, k + (bh * n + t) * d, v + (bh * n + t) * d, d, phi_kind);
+            state_add_token(Sh, zh, k + (bh * n + t) * d, v + (bh * n + t) * d, d, d, phi_kind);
     }
 }
 
@@ -202,11 +239,11 @@ void oracle_decode_step_f64(double *S, double *z, const double *q, const double 
         double *pq = (double *)malloc((size_t)d * sizeof(double));
 #if ORACLE_PLANT == 5
         /* planted: output read from the state before the update */
-        readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, phi_kind, pq);
-        state_add_token(S + bh * d * d, z + bh * d, k + bh * d, v + bh * d, d, phi_kind);
+        readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, d, phi_kind, pq);
+        state_add_token(S + bh * d * d, z + bh * d, k + bh * d, v + bh * d, d, d, phi_kind);
 #else
-        state_add_token(S + bh * d * d, z + bh * d, k + bh * d, v + bh * d, d, phi_kind);
-        readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, phi_kind, pq);
+        state_add_token(S + bh * d * d, z + bh * d, k + bh * d, v + bh * d, d, d, phi_kind);
+        readout_token(S + bh * d * d, z + bh * d, q + bh * d, out + bh * d, d, d, phi_kind, pq);
 #endif
         free(pq);
     }
@@ -336,3 +373,20 @@ void oracle_favor_features_f64(const double *x, const double *W, double *out, in
 }
 
 int oracle_plant(void) { return ORACLE_PLANT; }
+
+/* Threads the OpenMP loops above use from now on (timing only; results do not depend on it). */
+void oracle_set_threads(int threads) {
+#ifdef _OPENMP
+  if (threads > 0) omp_set_num_threads(threads);
+#else
+  (void)threads;
+#endif
+}
+
+int oracle_get_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

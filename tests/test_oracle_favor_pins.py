@@ -62,3 +62,45 @@ def test_planted_favor_mistake_is_caught():
     orc = oracle.load_planted(8)
     assert orc.plant == 8
     assert _unbiased_check(orc, 0) > 50.0
+
+
+# ------------------------------------------------------------------ features of their own size
+# The pass on m features with d-dimensional values (S is m x d; page "Linear Attention > Memory
+# Efficiency" writes the state as D x d with D the feature dimension) is pinned by the
+# quadratic form written out in numpy, which never forms S, for m < d and m > d, both modes.
+@pytest.mark.parametrize("m,d", [(3, 5), (8, 2), (16, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_on_m_features_matches_brute_force(m, d, causal):
+    rng = np.random.default_rng(10 * m + d)
+    n = 37
+    fq, fk = (np.abs(rng.standard_normal((2, n, m))) + 0.05 for _ in range(2))
+    v = rng.standard_normal((2, n, d))
+    got = oracle.forward(fq, fk, v, causal, phi_kind=oracle.PHI_IDENTITY)
+    assert got.shape == v.shape
+    for h in range(2):  # the brute force takes one head
+        ref = oracle.brute_force(fq[h], fk[h], v[h], causal, phi_kind=oracle.PHI_IDENTITY)
+        assert np.max(np.abs(got[h] - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_forward_on_m_features_reduces_to_the_square_pass():
+    """With m = d padded by zero features, the result equals the m = d pass (zero features add
+    nothing to S, z or the denominators)."""
+    rng = np.random.default_rng(11)
+    n, d = 29, 4
+    fq, fk = (np.abs(rng.standard_normal((n, d))) + 0.1 for _ in range(2))
+    v = rng.standard_normal((n, d))
+    pad = lambda x: np.concatenate([x, np.zeros((n, 3))], axis=1)  # noqa: E731
+    for causal in (False, True):
+        sq = oracle.forward(fq, fk, v, causal, phi_kind=oracle.PHI_IDENTITY)
+        wide = oracle.forward(pad(fq), pad(fk), v, causal, phi_kind=oracle.PHI_IDENTITY)
+        assert np.max(np.abs(sq - wide)) <= 1e-13
+
+
+def test_planted_transposed_state_is_caught_with_m_features():
+    orc = oracle.load_planted(2)  # S indexed as [value][feature]
+    rng = np.random.default_rng(12)
+    fq, fk = (np.abs(rng.standard_normal((20, 6))) + 0.1 for _ in range(2))
+    v = rng.standard_normal((20, 3))
+    got = orc.forward(fq, fk, v, True, phi_kind=oracle.PHI_IDENTITY)
+    ref = oracle.brute_force(fq, fk, v, True, phi_kind=oracle.PHI_IDENTITY)
+    assert np.max(np.abs(got - ref)) > 1e-3
