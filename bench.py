@@ -222,6 +222,21 @@ def time_steps(fn, steps, warmup, world, clocks=None):
     return max_over_ranks(total / steps, world), per
 
 
+def forward_launches(dtype: str, causal: bool, unit: int):
+    """Names of the launches of one forward call, in order, and the algorithmic bytes of each
+    (unit: the bytes of one [B,H,n,d] tensor)."""
+    if dtype == "bf16" and causal:
+        # the single pass: the look-back flags cleared, then one kernel reads q, k, v and
+        # writes out
+        return (["memset (look-back flags)",
+                 "tc_causal_kernel (single pass: aggregates, look-back, outputs)"], [0, 4 * unit])
+    if dtype == "bf16":
+        return (["tc_kernel<state> (segment aggregates, K1)", "scan_states_kernel (totals, K2)",
+                 "tc_kernel<non-causal out> (K3)"], [2 * unit, 0, 2 * unit])
+    return (["simt_chunk_state_kernel (K1)", "scan_states_kernel (K2)",
+             "simt_chunk_out_kernel (K3)"], [2 * unit, 0, 4 * unit if causal else 2 * unit])
+
+
 def time_launches(fn, steps, warmup, names):
     """Per-launch device times of a multi-kernel call: before each timed call the library is
     given events (linattn_profile_events) that it records after each of its launches on the
@@ -262,12 +277,14 @@ def time_launches(fn, steps, warmup, names):
 
 
 # ------------------------------------------------------------------ oracle baseline
-def oracle_sample(workload: str, target_s: float = 12.0):
-    """Times the float64 oracle on a bounded sample of the workload (host cores)."""
+def oracle_sample(workload: str, target_s: float = 12.0, one_thread_s: float = 0.0):
+    """Times the float64 oracle on a bounded sample of the workload (host cores, OpenMP over
+    heads); with one_thread_s > 0 also on one thread, on a sample of about that many seconds."""
     import oracle
     w = inputs.WORKLOADS[workload]
     cores = os.cpu_count() or 1
     causal = True if True in w.causal else False
+    oracle.set_threads(cores)
     # calibrate on one head of 4096 tokens
     q, k, v = inputs.forward_qkv(w.seed, 1, 1, min(w.n, 4096), w.d, w.scaled)
     t0 = time.perf_counter()
@@ -283,10 +300,20 @@ def oracle_sample(workload: str, target_s: float = 12.0):
     dt = time.perf_counter() - t0
     # tokens in the workload's unit: a token carries all H heads of its batch element
     tokens = heads * n_s / w.H
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
-            "threads": int(os.environ.get("OMP_NUM_THREADS", cores)),
-            "sample": f"{heads} heads x {n_s} tokens of the {workload} workload "
-                      f"({'causal' if causal else 'non-causal'}), float64, {dt:.1f} s"}
+    rec = {"value": tokens / dt, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+           "threads": int(oracle.get_threads()),
+           "sample": f"{heads} heads x {n_s} tokens of the {workload} workload "
+                     f"({'causal' if causal else 'non-causal'}), float64, {dt:.1f} s"}
+    if one_thread_s > 0:
+        n1 = int(max(256, min(w.n, one_thread_s / max(per_head_token, 1e-9))))
+        oracle.set_threads(1)
+        t0 = time.perf_counter()
+        oracle.forward(q[:, :1, :n1], k[:, :1, :n1], v[:, :1, :n1], causal)
+        dt1 = time.perf_counter() - t0
+        oracle.set_threads(cores)
+        rec["one_thread"] = {"value": n1 / w.H / dt1, "unit": "tokens/s", "threads": 1,
+                             "sample": f"1 head x {n1} tokens, float64, {dt1:.1f} s"}
+    return rec
 
 
 def run_reference(args, world, rank):
@@ -368,17 +395,10 @@ def main_forward(args, world, rank, local):
     pk = peaks()
     alg = forward_bytes(w.B, w.H, shape[2], w.d, elem)  # this rank's share
     unit = w.B * w.H * shape[2] * w.d * elem  # one [B,H,n,d] tensor (this rank's share)
-    if dtype == "bf16":
-        names = ["tc_kernel<state> (segment aggregates, K1)", "scan_states_kernel (prefix, K2)",
-                 "tc_kernel<causal out> (K3)" if causal else "tc_kernel<non-causal out> (K3)"]
-        kbytes = [2 * unit, 0, 4 * unit if causal else 2 * unit]
-    else:
-        names = ["simt_chunk_state_kernel (K1)", "scan_states_kernel (K2)",
-                 "simt_chunk_out_kernel (K3)"]
-        kbytes = [2 * unit, 0, 4 * unit if causal else 2 * unit]
+    names, kbytes = forward_launches(dtype, causal, unit)
     if seq:
-        # block state (K1, total), the start state, then the forward from it (K1, K2, K3)
-        names = ["block state: " + names[0], "block state: total (K2)",
+        # block state (aggregates, total), the start state, then the forward from it
+        names = ["block state: aggregates (K1)", "block state: total (K2)",
                  "sum_states_kernel"] + names
         kbytes = [2 * unit, 0, 0] + kbytes
     launch_ms = time_launches(step, max(3, min(args.steps, 10)), 2, names)
@@ -422,7 +442,7 @@ def main_forward(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "strong" if seq else "weak", "vs_baseline": None,
         "dtype": dtype,
-        "data": "synthetic (seeded N(0,1)/sqrt(d), see DESIGN.md input recipe)",
+        "data": "synthetic (per head default_rng([seed, b, h]) draws q, k, v N(0,1), times 1/sqrt(d); bf16-rounded)",
         "config": {"workload": args.workload + (f" (first {w.H} heads)" if args.max_heads else "")
                    + (f" [{args.mode}]" if args.mode else ""),
                    "B": w.B, "H": w.H, "n": w.n, "d": w.d,
@@ -542,15 +562,17 @@ def extras(args):
         "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
         "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
         "path": "CUDA cores (float32 FFMA), 6 launches"}
-    # FAVOR+ (Performer's positive random features, m = d) on the same shape, causal:
-    # features of q and k, then the pass on them
-    W = torch.randn(w.d, w.d, device="cuda")
-    ms, _ = time_steps(lambda: la.forward_favor(q, k, v, W, True), 10, 3, 1)
-    alg = 4 * w.B * w.H * w.n * w.d * 2 + 2 * 2 * w.B * w.H * w.n * w.d * 2  # + features out/in
-    res[f"favor_{name}_causal"] = {
-        "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
-        "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
-        "path": "features on CUDA cores, then the tensor-core pass (identity feature map)"}
+    # FAVOR+ (Performer's positive random features) on the same shape, causal: the features of
+    # q and k (m of them), then the pass on them; m = d and m = 2 d
+    for m in (w.d, 2 * w.d):
+        W = torch.randn(m, w.d, device="cuda")
+        ms, _ = time_steps(lambda: la.forward_favor(q, k, v, W, True), 10, 3, 1)
+        # q, k, v read and out written, plus the features written and read back
+        alg = 4 * w.B * w.H * w.n * w.d * 2 + 2 * 2 * w.B * w.H * w.n * m * 2
+        res[f"favor_m{m}_{name}_causal"] = {
+            "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
+            "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
+            "m": m, "path": "features and pass on the tensor cores (identity feature map)"}
     del q, k, v, o, dout
     # latency cases
     for name, dtypes in (("noncausal_1x1x512x64_f32", ("f32",)),
@@ -564,7 +586,7 @@ def extras(args):
             ms, _ = time_steps(fn, 50, 5, 1)
             # back-to-back calls of a small problem measure the host's call rate; the device
             # time of one call is the sum of its launches
-            dev = time_launches(fn, 20, 5, ["K1", "K2", "K3"])
+            dev = time_launches(fn, 20, 5, forward_launches(dt, causal, 0)[0])
             dev_us = sum(dev.values()) * 1e3
             res[f"{name}_{dt}"] = {"us": ms * 1e3, "device_us": dev_us,
                                    "tokens_per_s": w.B * w.n / (ms * 1e-3)}
@@ -610,7 +632,7 @@ def main():
         if not args.no_extras:
             line["extras"] = extras(args)
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(args.workload)
+            line["cpu_baseline"] = oracle_sample(args.workload, one_thread_s=6.0)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

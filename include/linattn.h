@@ -65,8 +65,11 @@ typedef enum {
  *   causal  : 0 = every query sees every key (the formula above);
  *             1 = query i sees keys j <= i (the recurrent view's running state).
  * Any n >= 1 is accepted.  Accumulation is fp32; the output is rounded once to `dtype`
- * (bf16: round to nearest even).  The causal mode runs as chunked prefix sums of (S, z).
- * Returns LINATTN_OK after enqueuing the kernels on `stream`.
+ * (bf16: round to nearest even).  The causal mode runs as chunked prefix sums of (S, z):
+ * with bf16 I/O in one pass, where each segment of a head publishes its aggregate state and
+ * takes its prefix from the segments before it (a look-back); with fp32 I/O as per-chunk
+ * aggregates, their scan, and the outputs.  Returns LINATTN_OK after enqueuing the work on
+ * `stream`.
  */
 linattn_status linattn_forward(const void *q, const void *k, const void *v, void *out,
                                int64_t B, int64_t H, int64_t n, int64_t d, int causal,
@@ -122,26 +125,31 @@ linattn_status linattn_forward_init(const void *q, const void *k, const void *v,
  * Linear Attention and Flash Attention", section "Linear attention: reordering the matmuls,
  * not shrinking them", as features whose dot products approximate the softmax kernel
  * exp(q . k); the page gives no formula, this is the positive-feature form):
- *     out[t][i] = exp(W[i] . x[t] - |x[t]|^2 / 2) / sqrt(m),   m = d features,
+ *     out[t][i] = exp(W[i] . x[t] - |x[t]|^2 / 2) / sqrt(m),   i < m features,
  * so that E_W[phi(q) . phi(k)] = exp(q . k) for W with i.i.d. N(0, 1) entries.
  *   x   : [rows][d] of type `dtype` (for attention: q or k, already scaled as wanted).
- *   W   : [d][d] float32, the random projection (row i = w_i), drawn by the caller.
- *   out : [rows][d] of type `dtype`, written.
- * d in {64, 128}.  Feed the features of q and k to linattn_forward_features.
+ *   W   : [m][d] float32, the random projection (row i = w_i), drawn by the caller.
+ *   out : [rows][m] of type `dtype`, written.
+ * d, m in {64, 128}; rows < 2^31.  bf16: the product X W^T runs on the tensor cores with W
+ * split into two bf16 parts (about 2^-16 relative); fp32: CUDA cores.  Feed the features of q
+ * and k to linattn_forward_features.
  */
 linattn_status linattn_favor_features(const void *x, const float *W, void *out, int64_t rows,
-                                      int64_t d, linattn_dtype dtype, linattn_stream_t stream);
+                                      int64_t d, int64_t m, linattn_dtype dtype,
+                                      linattn_stream_t stream);
 
 /*
- * linattn_forward on features the caller has computed: phi_q and phi_k ([B][H][n][d], type
- * `dtype`) are used as phi(q) and phi(k) directly, with no feature map applied:
- *     out_i = phi_q_i S / phi_q_i . z,   S = sum_j phi_k_j v_j^T,   z = sum_j phi_k_j.
+ * linattn_forward on features the caller has computed: phi_q and phi_k ([B][H][n][m], type
+ * `dtype`) are used as phi(q) and phi(k) directly, with no feature map applied, and v, out are
+ * [B][H][n][d]:
+ *     out_i = phi_q_i S / phi_q_i . z,   S = sum_j phi_k_j v_j^T (m x d),   z = sum_j phi_k_j.
  * The features must be non-negative with positive denominators (FAVOR+ features are).
- * Other arguments, layouts and errors as in linattn_forward.
+ * m, d in {64, 128}; m != d needs bf16 I/O (the fp32 CUDA-core kernels keep m = d, else
+ * LINATTN_ERR_UNSUPPORTED).  Other arguments, layouts and errors as in linattn_forward.
  */
 linattn_status linattn_forward_features(const void *phi_q, const void *phi_k, const void *v,
-                                        void *out, int64_t B, int64_t H, int64_t n, int64_t d,
-                                        int causal, linattn_dtype dtype,
+                                        void *out, int64_t B, int64_t H, int64_t n, int64_t m,
+                                        int64_t d, int causal, linattn_dtype dtype,
                                         linattn_stream_t stream);
 
 /*
@@ -178,7 +186,7 @@ linattn_status linattn_sum_states(const float *states, int64_t count, int64_t sk
 
 /*
  * linattn_forward with a chosen segment length: the number of tokens one work item of
- * the chunked causal pass covers (a multiple of the chunk size; 0 picks the default).
+ * the chunked causal pass covers (a multiple of 128 tokens; 0 picks the default).
  * The result does not depend on it beyond rounding order; tests use it to move the
  * segment boundaries.  Other arguments as in linattn_forward.
  */
@@ -194,9 +202,10 @@ size_t linattn_state_bytes(int64_t d);
 /* Static text for a status code. */
 const char *linattn_status_string(linattn_status status);
 
-/* Synchronises `stream`, then reports and clears the current device's kernel error flag:
+/* Synchronises `stream`, then reports and clears the current device's kernel error flags:
  * LINATTN_ERR_TIMEOUT if a bounded wait gave up since the last call, else LINATTN_OK
- * (or LINATTN_ERR_CUDA if synchronising failed). */
+ * (or LINATTN_ERR_CUDA if synchronising or reading a flag failed).  It covers every entry
+ * point, linattn_forward_noalloc included, and allocates nothing itself. */
 linattn_status linattn_device_error(linattn_stream_t stream);
 
 /* Self-test of the failure path: launches one thread that waits, with the kernels' bounded
@@ -213,9 +222,9 @@ int linattn_version(void);
 uint64_t linattn_launch_count(void);
 
 /*
- * Measurement aid: while `count` > 0, every kernel this library enqueues on the calling
- * thread is followed by cudaEventRecord(events[i], stream) with i = 0, 1, ... (up to
- * count - 1), so the caller can time each launch of a multi-kernel call with
+ * Measurement aid: while `count` > 0, every kernel (and device memset) this library
+ * enqueues on the calling thread is followed by cudaEventRecord(events[i], stream) with
+ * i = 0, 1, ... (up to count - 1), so the caller can time each launch of a multi-kernel call with
  * cudaEventElapsedTime.  `events` holds cudaEvent_t handles created by the caller; the
  * library keeps the pointer until the next call with count = 0.
  */
@@ -225,12 +234,14 @@ linattn_status linattn_profile_events(void *const *events, int count);
 #define LINATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /*
- * linattn_forward for callers that cannot allocate memory (the pages have no counterpart:
- * this is a deployment variant, not part of the method).  Same arguments, layouts, results
- * and dtypes as linattn_forward; it calls no cudaMalloc, cudaFree or other allocating
- * routine.  Its temporary state lives in one fixed block of LINATTN_NOALLOC_SCRATCH_BYTES
- * of device memory that the library declares statically; every GPU that loads the library
- * holds that block until the process exits.
+ * linattn_forward for callers that cannot allocate memory: hosts that reserve all device
+ * memory up front, and runtimes that own the device allocator and forbid libraries from
+ * calling it.  The pages have no counterpart; this is a deployment variant, not part of the
+ * method.  Same arguments, checks, layouts, results and dtypes as linattn_forward, through
+ * the same kernels; it calls no cudaMalloc, cudaFree or other allocating routine.  Its
+ * temporary state lives in one fixed block of LINATTN_NOALLOC_SCRATCH_BYTES of device memory
+ * that the library declares statically; every GPU that loads the library holds that block
+ * until the process exits.
  *   - Work that needs more temporary state than the block holds is rejected with
  *     LINATTN_ERR_INVALID_ARG before anything is launched (the bf16 path first lengthens
  *     its segments to fit; it needs 66,048 B per head and segment at d = 128, 16,640 B at
@@ -239,13 +250,20 @@ linattn_status linattn_profile_events(void *const *events, int count);
  *     needs to start at zero.  Calls that overlap on the GPU race on it: issue them on one
  *     stream or otherwise order them.
  *   - The first call on each device looks up the block's device address with that device
- *     current; make that first call before any stream capture.
- *   - A kernel wait that gives up is recorded in the block's first word, not in the word
- *     linattn_device_error() reads.
+ *     current; make that first call before any stream capture.  A failed look-up returns
+ *     LINATTN_ERR_CUDA and is retried by the next call.
+ *   - A kernel wait that gives up is recorded in the block's status word; linattn_device_error()
+ *     reports it (and clears it) like any other.
  */
 linattn_status linattn_forward_noalloc(const void *q, const void *k, const void *v, void *out,
                                        int64_t B, int64_t H, int64_t n, int64_t d, int causal,
                                        linattn_dtype dtype, linattn_stream_t stream);
+
+/* Self-test of linattn_forward_noalloc's failure report: the same bounded wait as
+ * linattn_selftest_wait_timeout, recording its give-up in the static block's status word.
+ * The next linattn_device_error() returns LINATTN_ERR_TIMEOUT (and clears it).  Allocates
+ * nothing. */
+linattn_status linattn_selftest_noalloc_wait_timeout(linattn_stream_t stream);
 
 #ifdef __cplusplus
 }

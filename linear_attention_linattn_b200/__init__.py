@@ -11,7 +11,8 @@ Raw C entry points (pointers as ints):
     linattn_state_bytes, linattn_status_string, linattn_device_error, linattn_version,
     linattn_launch_count, linattn_forward_noalloc, linattn_profile_events,
     linattn_forward_init, linattn_sum_states, linattn_backward, linattn_favor_features,
-    linattn_forward_features, linattn_selftest_wait_timeout
+    linattn_forward_features, linattn_selftest_wait_timeout,
+    linattn_selftest_noalloc_wait_timeout
 
 Tensor helpers: ``forward``, ``forward_init``, ``forward_state``, ``sum_states``,
 ``backward``, ``favor_features``, ``forward_features``, ``forward_favor``, ``decode_step``,
@@ -57,10 +58,12 @@ SIGNATURES = {
     "linattn_sum_states": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
     "linattn_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                         _i64, ctypes.c_int, ctypes.c_int, _vp]),
-    "linattn_favor_features": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]),
+    "linattn_favor_features": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int,
+                                              _vp]),
     "linattn_selftest_wait_timeout": (ctypes.c_int, [_vp]),
+    "linattn_selftest_noalloc_wait_timeout": (ctypes.c_int, [_vp]),
     "linattn_forward_features": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
-                                                ctypes.c_int, ctypes.c_int, _vp]),
+                                                _i64, ctypes.c_int, ctypes.c_int, _vp]),
 }
 
 _lib = None
@@ -192,46 +195,51 @@ def sum_states(states, count: int, skip: int = -1, S=None, z=None, stream=None):
 
 
 def favor_features(x, W, out=None, stream=None):
-    """FAVOR+ positive random features exp(W x - |x|^2/2) / sqrt(d) of x [..., d] (float32 or
-    bfloat16 CUDA tensor); W: float32 [d, d] CUDA tensor of random rows.  Returns [..., d]."""
+    """FAVOR+ positive random features exp(W x - |x|^2/2) / sqrt(m) of x [..., d] (float32 or
+    bfloat16 CUDA tensor); W: float32 [m, d] CUDA tensor of m random rows.  Returns [..., m]."""
     import torch
     _dev(x, "x")
     _dev(W, "W")
     d = x.shape[-1]
-    if W.dtype != torch.float32 or tuple(W.shape) != (d, d):
-        raise ValueError("W must be a float32 [d, d] tensor")
+    if W.dtype != torch.float32 or W.dim() != 2 or W.shape[1] != d:
+        raise ValueError("W must be a float32 [m, d] tensor")
+    m = W.shape[0]
     if out is None:
-        out = torch.empty_like(x)
+        out = torch.empty(tuple(x.shape[:-1]) + (m,), dtype=x.dtype, device=x.device)
     _dev(out, "out")
     lib = load_library()
-    st = lib.linattn_favor_features(x.data_ptr(), W.data_ptr(), out.data_ptr(), x.numel() // d, d,
-                                    _dtype_code(x), _stream_ptr(stream))
+    st = lib.linattn_favor_features(x.data_ptr(), W.contiguous().data_ptr(), out.data_ptr(),
+                                    x.numel() // d, d, m, _dtype_code(x), _stream_ptr(stream))
     _check(st, "linattn_favor_features")
     return out
 
 
 def forward_features(phi_q, phi_k, v, causal: bool, out=None, stream=None):
-    """forward with caller-computed non-negative features phi_q, phi_k [B, H, n, d]."""
+    """forward with caller-computed non-negative features phi_q, phi_k [B, H, n, m] and
+    values v [B, H, n, d]; returns [B, H, n, d]."""
     import torch
     for t, nm in ((phi_q, "phi_q"), (phi_k, "phi_k"), (v, "v")):
         _dev(t, nm)
-    if not (phi_q.shape == phi_k.shape == v.shape and v.dim() == 4 and
+    if not (phi_q.shape == phi_k.shape and v.dim() == 4 and phi_q.shape[:3] == v.shape[:3] and
             phi_q.dtype == phi_k.dtype == v.dtype):
-        raise ValueError("phi_q, phi_k, v must share one [B, H, n, d] shape and dtype")
+        raise ValueError("phi_q, phi_k must share one [B, H, n, m] shape, v be [B, H, n, d], "
+                         "all of one dtype")
     if out is None:
         out = torch.empty_like(v)
     _dev(out, "out")
     B, H, n, d = v.shape
+    m = phi_q.shape[-1]
     lib = load_library()
     st = lib.linattn_forward_features(phi_q.data_ptr(), phi_k.data_ptr(), v.data_ptr(),
-                                      out.data_ptr(), B, H, n, d, int(bool(causal)),
+                                      out.data_ptr(), B, H, n, m, d, int(bool(causal)),
                                       _dtype_code(v), _stream_ptr(stream))
     _check(st, "linattn_forward_features")
     return out
 
 
 def forward_favor(q, k, v, W, causal: bool, stream=None):
-    """FAVOR+ linear attention: the forward pass on favor_features(q, W), favor_features(k, W)."""
+    """FAVOR+ linear attention: the forward pass on favor_features(q, W), favor_features(k, W)
+    (m = W.shape[0] random features)."""
     return forward_features(favor_features(q, W, stream=stream), favor_features(k, W, stream=stream),
                             v, causal, stream=stream)
 

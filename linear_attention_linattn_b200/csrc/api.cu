@@ -17,6 +17,7 @@ constexpr int kMaxDevices = 64;
 
 struct DeviceState {
   std::once_flag once;
+  std::atomic<bool> ready{false};
   cudaError_t init_err = cudaSuccess;
   int *err_word = nullptr;     // kernels' error word (device memory)
   cudaMemPool_t pool = nullptr;  // stream-ordered workspace pool
@@ -48,10 +49,19 @@ cudaError_t device_state(DeviceState **out) {
     }
     if (r == cudaSuccess) r = cudaDeviceSynchronize();
     s.init_err = r;
+    s.ready.store(r == cudaSuccess, std::memory_order_release);
   });
   if (s.init_err != cudaSuccess) return s.init_err;
   *out = &s;
   return cudaSuccess;
+}
+
+// The current device's state if device_state() has set it up already, else null (no set-up,
+// so nothing is allocated).
+DeviceState *device_state_if_ready() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  return g_dev[dev].ready.load(std::memory_order_acquire) ? &g_dev[dev] : nullptr;
 }
 
 // Stream-ordered scratch: allocated on `st` before the kernels, released on `st` after.
@@ -67,66 +77,18 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 linattn_status to_status(cudaError_t e) { return e == cudaSuccess ? LINATTN_OK : LINATTN_ERR_CUDA; }
 
-// Checks shared by the forward entry points.  Limits keep every grid and TMA coordinate
-// inside 32 bits: n < 2^31, B*H < 2^24, total elements < 2^40.
-linattn_status check_forward_shape(int64_t B, int64_t H, int64_t n, int64_t d) {
-  if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return LINATTN_ERR_INVALID_ARG;
-  if (B > (1 << 24) || H > (1 << 24) || n >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
-  const int64_t heads = B * H;
-  if (heads > (1 << 24)) return LINATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
-  if (heads * n > (int64_t(1) << 40) / d) return LINATTN_ERR_INVALID_ARG;
-  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
-  if (nchunks * heads >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
-  return LINATTN_OK;
-}
-
-// init_S / init_z (nullable): the state before each head's first token (causal), or the
-// state the other tokens of the sequence contribute (non-causal).
-linattn_status forward_tc(const void *q, const void *k, const void *v, void *out,
-                          int64_t heads, int64_t n, int d, int causal, int64_t seg,
-                          const float *init_S, const float *init_z, int features,
-                          DeviceState *ds, cudaStream_t st) {
-  if (seg == 0) seg = tc_default_segment(heads, n, d);
+// Forward pass with its workspace taken from the device's pool on `st`.
+linattn_status forward_pooled(const void *q, const void *k, const void *v, void *out,
+                              int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
+                              int64_t seg_len, const float *init_S, const float *init_z,
+                              int features, DeviceState *ds, cudaStream_t st) {
+  const ForwardPlan p = plan_forward(heads, n, dk, d, causal, is_bf16, seg_len);
   Workspace ws;
   ws.st = st;
-  if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, d, seg, causal), ds->pool,
-                              st) != cudaSuccess)
+  if (cudaMallocFromPoolAsync(&ws.ptr, p.ws_bytes, ds->pool, st) != cudaSuccess)
     return LINATTN_ERR_CUDA;
-  return to_status(tc_forward(q, k, v, out, heads, n, d, causal, seg, ws.ptr, ds->err_word,
-                              init_S, init_z, features, st));
-}
-
-linattn_status forward_simt(const void *q, const void *k, const void *v, void *out,
-                            int64_t heads, int64_t n, int d, int causal, int is_bf16,
-                            const float *init_S, const float *init_z, int features,
-                            DeviceState *ds, cudaStream_t st) {
-  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
-  const int64_t per = (int64_t)d * d + d;
-  // causal: one state per chunk; non-causal: chunk states plus one total per head
-  const size_t bytes = (size_t)(heads * nchunks * per + (causal ? 0 : heads * per)) * 4;
-  Workspace ws;
-  ws.st = st;
-  cudaError_t e = cudaMallocFromPoolAsync(&ws.ptr, bytes, ds->pool, st);
-  if (e != cudaSuccess) return LINATTN_ERR_CUDA;
-  float *w = static_cast<float *>(ws.ptr);
-  e = launch_simt_chunk_state(k, v, w, heads, n, d, is_bf16, features, st);
-  if (e != cudaSuccess) return LINATTN_ERR_CUDA;
-  if (causal) {
-    e = launch_scan_states(w, heads, nchunks, d, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
-    if (e != cudaSuccess) return LINATTN_ERR_CUDA;
-    e = launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
-                              nchunks * per, heads, n, d, 1, is_bf16, features, st);
-  } else {
-    float *tot = w + heads * nchunks * per;
-    float *tot_z = tot + heads * (int64_t)d * d;
-    e = launch_scan_states(w, heads, nchunks, d, 1, tot, (int64_t)d * d, tot_z, d, init_S,
-                           init_z, st);
-    if (e != cudaSuccess) return LINATTN_ERR_CUDA;
-    e = launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, (int64_t)d * d, 0, d, heads, n, d, 0,
-                              is_bf16, features, st);
-  }
-  return to_status(e);
+  return to_status(run_forward(p, q, k, v, out, heads, n, dk, d, causal, is_bf16, init_S, init_z,
+                               features, ws.ptr, ds->err_word, st));
 }
 
 // Failure-path self-test: one thread waits, with the kernels' own bounded wait, on an mbarrier
@@ -145,6 +107,90 @@ __global__ void wait_timeout_selftest_kernel(int *err) {
 }
 
 }  // namespace
+
+linattn_status check_forward_args(const void *q, const void *k, const void *v, const void *out,
+                                  int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                  linattn_dtype dtype) {
+  if (!q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return LINATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
+  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
+  // n < 2^31, B*H < 2^24, total elements < 2^40
+  if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return LINATTN_ERR_INVALID_ARG;
+  if (B > (1 << 24) || H > (1 << 24) || n >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
+  const int64_t heads = B * H;
+  if (heads > (1 << 24)) return LINATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
+  if (heads * n > (int64_t(1) << 40) / d) return LINATTN_ERR_INVALID_ARG;
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  if (nchunks * heads >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
+  return LINATTN_OK;
+}
+
+ForwardPlan plan_forward(int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
+                         int64_t seg_len) {
+  ForwardPlan p;
+  if (is_bf16) {
+    p.seg = seg_len > 0 ? seg_len
+                        : (causal ? tc_fused_segment(heads, n, dk, d) : tc_default_segment(heads, n, d));
+    p.ws_bytes = tc_workspace_bytes(heads, n, dk, d, p.seg, causal);
+    return p;
+  }
+  // fp32 path: one state per 64-token chunk; non-causal adds one total per head
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  const int64_t per = (int64_t)d * d + d;
+  p.ws_bytes = (size_t)(heads * nchunks * per + (causal ? 0 : heads * per)) * sizeof(float);
+  return p;
+}
+
+cudaError_t run_forward(const ForwardPlan &p, const void *q, const void *k, const void *v,
+                        void *out, int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
+                        const float *init_S, const float *init_z, int features, void *ws,
+                        int *err, cudaStream_t st) {
+  if (is_bf16)
+    return tc_forward(q, k, v, out, heads, n, dk, d, causal, p.seg, ws, err, init_S, init_z,
+                      features, st);
+  if (dk != d) return cudaErrorInvalidValue;  // the CUDA-core kernels keep one dimension
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  const int64_t per = (int64_t)d * d + d;
+  float *w = static_cast<float *>(ws);
+  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, d, 0, features, st);
+  if (e != cudaSuccess) return e;
+  if (causal) {
+    e = launch_scan_states(w, heads, nchunks, d, d, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
+    if (e != cudaSuccess) return e;
+    return launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
+                                 nchunks * per, heads, n, d, 1, 0, features, st);
+  }
+  float *tot = w + heads * nchunks * per;
+  float *tot_z = tot + heads * (int64_t)d * d;
+  e = launch_scan_states(w, heads, nchunks, d, d, 1, tot, (int64_t)d * d, tot_z, d, init_S, init_z,
+                         st);
+  if (e != cudaSuccess) return e;
+  return launch_simt_chunk_out(q, k, v, out, tot, tot_z, 0, (int64_t)d * d, 0, d, heads, n, d, 0,
+                               0, features, st);
+}
+
+cudaError_t launch_wait_timeout_selftest(int *err, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(err);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return 148;  // not cached: asked again next time
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
 }  // namespace linattn
 
 using namespace linattn;
@@ -154,100 +200,77 @@ extern "C" {
 linattn_status linattn_selftest_wait_timeout(linattn_stream_t stream) {
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
-  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      ds->err_word);
-  count_launches(1);
-  return to_status(cudaGetLastError());
+  return to_status(launch_wait_timeout_selftest(ds->err_word,
+                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, void *out,
                                   int64_t B, int64_t H, int64_t n, int64_t d, int causal,
                                   linattn_dtype dtype, int64_t segment_len,
                                   linattn_stream_t stream) {
-  if (!q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return LINATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
-  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  if (segment_len < 0 || segment_len % kTcChunk != 0) return LINATTN_ERR_INVALID_ARG;
-  linattn_status s = check_forward_shape(B, H, n, d);
+  linattn_status s = check_forward_args(q, k, v, out, B, H, n, d, causal, dtype);
   if (s != LINATTN_OK) return s;
+  if (segment_len < 0 || segment_len % kTcCausalChunk != 0) return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == LINATTN_BF16)
-    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, segment_len, nullptr, nullptr, 0,
-                      ds, st);
-  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, 0, ds, st);
+  return forward_pooled(q, k, v, out, B * H, n, (int)d, (int)d, causal, dtype == LINATTN_BF16,
+                        segment_len, nullptr, nullptr, 0, ds,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 linattn_status linattn_forward_init(const void *q, const void *k, const void *v, void *out,
                                     const float *state_S, const float *state_z, int64_t B,
                                     int64_t H, int64_t n, int64_t d, int causal,
                                     linattn_dtype dtype, linattn_stream_t stream) {
-  if (!q || !k || !v || !out || !state_S || !state_z) return LINATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      !aligned16(state_S) || !aligned16(state_z))
-    return LINATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
-  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  linattn_status s = check_forward_shape(B, H, n, d);
+  linattn_status s = check_forward_args(q, k, v, out, B, H, n, d, causal, dtype);
   if (s != LINATTN_OK) return s;
+  if (!state_S || !state_z || !aligned16(state_S) || !aligned16(state_z))
+    return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == LINATTN_BF16)
-    return forward_tc(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, 0, ds, st);
-  return forward_simt(q, k, v, out, B * H, n, (int)d, causal, 0, state_S, state_z, 0, ds, st);
+  return forward_pooled(q, k, v, out, B * H, n, (int)d, (int)d, causal, dtype == LINATTN_BF16,
+                        0, state_S, state_z, 0, ds, reinterpret_cast<cudaStream_t>(stream));
 }
 
 linattn_status linattn_forward_features(const void *phi_q, const void *phi_k, const void *v,
-                                        void *out, int64_t B, int64_t H, int64_t n, int64_t d,
-                                        int causal, linattn_dtype dtype,
+                                        void *out, int64_t B, int64_t H, int64_t n, int64_t m,
+                                        int64_t d, int causal, linattn_dtype dtype,
                                         linattn_stream_t stream) {
-  if (!phi_q || !phi_k || !v || !out) return LINATTN_ERR_INVALID_ARG;
-  if (!aligned16(phi_q) || !aligned16(phi_k) || !aligned16(v) || !aligned16(out))
-    return LINATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
-  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  linattn_status s = check_forward_shape(B, H, n, d);
+  linattn_status s = check_forward_args(phi_q, phi_k, v, out, B, H, n, d, causal, dtype);
   if (s != LINATTN_OK) return s;
+  if (m <= 0) return LINATTN_ERR_INVALID_ARG;
+  if (m != 64 && m != 128) return LINATTN_ERR_UNSUPPORTED;
+  if (m != d && dtype != LINATTN_BF16) return LINATTN_ERR_UNSUPPORTED;  // fp32: m = d only
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == LINATTN_BF16)
-    return forward_tc(phi_q, phi_k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, 1, ds,
-                      st);
-  return forward_simt(phi_q, phi_k, v, out, B * H, n, (int)d, causal, 0, nullptr, nullptr, 1, ds,
-                      st);
+  return forward_pooled(phi_q, phi_k, v, out, B * H, n, (int)m, (int)d, causal,
+                        dtype == LINATTN_BF16, 0, nullptr, nullptr, 1, ds,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 linattn_status linattn_favor_features(const void *x, const float *W, void *out, int64_t rows,
-                                      int64_t d, linattn_dtype dtype, linattn_stream_t stream) {
+                                      int64_t d, int64_t m, linattn_dtype dtype,
+                                      linattn_stream_t stream) {
   if (!x || !W || !out) return LINATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(W) || !aligned16(out)) return LINATTN_ERR_INVALID_ARG;
   if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  if (rows <= 0 || d <= 0) return LINATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return LINATTN_ERR_UNSUPPORTED;
-  if (rows > (int64_t(1) << 40) / d) return LINATTN_ERR_INVALID_ARG;
+  if (rows <= 0 || d <= 0 || m <= 0) return LINATTN_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || (m != 64 && m != 128)) return LINATTN_ERR_UNSUPPORTED;
+  if (rows >= (int64_t(1) << 31) || rows > (int64_t(1) << 40) / m) return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
-  return to_status(launch_favor_features(x, W, out, rows, (int)d, dtype == LINATTN_BF16,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+  return to_status(launch_favor_features(x, W, out, rows, (int)d, (int)m, dtype == LINATTN_BF16,
+                                         ds->err_word, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 linattn_status linattn_backward(const void *q, const void *k, const void *v, const void *dout,
                                 void *dq, void *dk, void *dv, int64_t B, int64_t H, int64_t n,
                                 int64_t d, int causal, linattn_dtype dtype,
                                 linattn_stream_t stream) {
-  if (!q || !k || !v || !dout || !dq || !dk || !dv) return LINATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv))
-    return LINATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
-  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  linattn_status s = check_forward_shape(B, H, n, d);
+  linattn_status s = check_forward_args(q, k, v, dout, B, H, n, d, causal, dtype);
   if (s != LINATTN_OK) return s;
+  if (!dq || !dk || !dv || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -286,12 +309,9 @@ linattn_status linattn_forward(const void *q, const void *k, const void *v, void
 linattn_status linattn_forward_state(const void *k, const void *v, float *state_S,
                                      float *state_z, int64_t B, int64_t H, int64_t n, int64_t d,
                                      linattn_dtype dtype, linattn_stream_t stream) {
-  if (!k || !v || !state_S || !state_z) return LINATTN_ERR_INVALID_ARG;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(state_S) || !aligned16(state_z))
-    return LINATTN_ERR_INVALID_ARG;
-  if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
-  linattn_status s = check_forward_shape(B, H, n, d);
+  linattn_status s = check_forward_args(k, k, v, state_S, B, H, n, d, 0, dtype);
   if (s != LINATTN_OK) return s;
+  if (!state_z || !aligned16(state_z)) return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -300,7 +320,7 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
   ws.st = st;
   if (dtype == LINATTN_BF16) {
     const int64_t seg = tc_default_segment(heads, n, (int)d);
-    if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, (int)d, seg, 1), ds->pool,
+    if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, (int)d, (int)d, seg, 0), ds->pool,
                                 st) != cudaSuccess)
       return LINATTN_ERR_CUDA;
     return to_status(tc_forward_state(k, v, state_S, state_z, heads, n, (int)d, seg, ws.ptr,
@@ -314,7 +334,7 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
   float *w = static_cast<float *>(ws.ptr);
   cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, 0, 0, st);
   if (e == cudaSuccess)
-    e = launch_scan_states(w, heads, nchunks, (int)d, 1, state_S, d * d, state_z, d, nullptr,
+    e = launch_scan_states(w, heads, nchunks, (int)d, (int)d, 1, state_S, d * d, state_z, d, nullptr,
                            nullptr, st);
   return to_status(e);
 }
@@ -351,16 +371,20 @@ const char *linattn_status_string(linattn_status status) {
 }
 
 linattn_status linattn_device_error(linattn_stream_t stream) {
-  DeviceState *ds = nullptr;
-  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   int word = 0;
-  if (cudaMemcpy(&word, ds->err_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return LINATTN_ERR_CUDA;
-  if (word == 0) return LINATTN_OK;
-  if (cudaMemset(ds->err_word, 0, sizeof(int)) != cudaSuccess) return LINATTN_ERR_CUDA;
-  return LINATTN_ERR_TIMEOUT;
+  // the pooled entry points' word, if any of them has run on this device
+  if (DeviceState *ds = device_state_if_ready()) {
+    if (cudaMemcpy(&word, ds->err_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
+    if (word != 0 && cudaMemset(ds->err_word, 0, sizeof(int)) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
+  }
+  // linattn_forward_noalloc's word, in its static block
+  int noalloc_word = 0;
+  if (noalloc_take_status(&noalloc_word) != cudaSuccess) return LINATTN_ERR_CUDA;
+  return (word | noalloc_word) == 0 ? LINATTN_OK : LINATTN_ERR_TIMEOUT;
 }
 
 int linattn_version(void) { return 100; }

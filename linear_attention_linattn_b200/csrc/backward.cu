@@ -518,9 +518,9 @@ cudaError_t backward_impl(const T *q, const T *k, const T *v, const T *g, T *dq,
   int64_t Scs = per, Shs = nchunks * per;
   const float *Sbase = Sf;
   if (CAUSAL) {
-    e = launch_scan_states(Sf, heads, nchunks, D, 0, nullptr, 0, nullptr, 0, nullptr, nullptr, st);
+    e = launch_scan_states(Sf, heads, nchunks, D, D, 0, nullptr, 0, nullptr, 0, nullptr, nullptr, st);
   } else {
-    e = launch_scan_states(Sf, heads, nchunks, D, 1, tot, per, tot + (int64_t)D * D, per, nullptr,
+    e = launch_scan_states(Sf, heads, nchunks, D, D, 1, tot, per, tot + (int64_t)D * D, per, nullptr,
                            nullptr, st);
     Scs = 0;
     Shs = per;
@@ -541,9 +541,9 @@ cudaError_t backward_impl(const T *q, const T *k, const T *v, const T *g, T *dq,
   int64_t Rcs = per, Rhs = nchunks * per;
   const float *Rbase = Sr;
   if (CAUSAL) {
-    e = launch_scan_states(Sr, heads, nchunks, D, 2, nullptr, 0, nullptr, 0, nullptr, nullptr, st);
+    e = launch_scan_states(Sr, heads, nchunks, D, D, 2, nullptr, 0, nullptr, 0, nullptr, nullptr, st);
   } else {
-    e = launch_scan_states(Sr, heads, nchunks, D, 1, tot, per, tot + (int64_t)D * D, per, nullptr,
+    e = launch_scan_states(Sr, heads, nchunks, D, D, 1, tot, per, tot + (int64_t)D * D, per, nullptr,
                            nullptr, st);
     Rcs = 0;
     Rhs = per;

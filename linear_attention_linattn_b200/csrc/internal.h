@@ -2,9 +2,47 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
+#include "linattn.h"
+
 namespace linattn {
+
+// ---- forward dispatch shared by the entry points (api.cu) ---------------------------------
+// Checks shared by every forward entry point: pointers (non-null, 16-byte aligned), the causal
+// flag, the dtype and the sizes.  Limits keep every grid and TMA coordinate inside 32 bits.
+linattn_status check_forward_args(const void *q, const void *k, const void *v, const void *out,
+                                  int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                  linattn_dtype dtype);
+// What one forward pass needs: the tensor-core path's tokens per work item (0 on the fp32
+// path) and the bytes of temporary state.
+struct ForwardPlan {
+  int64_t seg = 0;
+  size_t ws_bytes = 0;
+};
+// dk: feature dimension of q, k (= d unless they are random features); d: value dimension.
+// seg_len: tokens per work item of the tensor-core path, a multiple of 128; 0 picks the default.
+ForwardPlan plan_forward(int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
+                         int64_t seg_len);
+// Enqueues the pass `p` describes on `st`, with the caller's workspace (at least p.ws_bytes)
+// and the word that bounded waits report a give-up in.  init_S / init_z (nullable): the state
+// before each head's first token (causal) or what the rest of the sequence contributes
+// (non-causal).  features != 0: q and k are non-negative features already.
+cudaError_t run_forward(const ForwardPlan &p, const void *q, const void *k, const void *v,
+                        void *out, int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
+                        const float *init_S, const float *init_z, int features, void *ws,
+                        int *err, cudaStream_t st);
+// The no-allocation entry point's status word (noalloc.cu): reads it for the current device
+// into *word and clears it.  *word = 0 when that entry point has not run on this device.
+cudaError_t noalloc_take_status(int *word);
+
+// Failure-path self-test: one thread waits, with the kernels' bounded wait, on a barrier that
+// nothing completes; the give-up is recorded in *err.
+cudaError_t launch_wait_timeout_selftest(int *err, cudaStream_t st);
+
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count();
 
 // Launch accounting for linattn_launch_count(): every launcher adds the kernels it enqueued.
 void count_launches(uint64_t n);
@@ -21,11 +59,12 @@ constexpr int kSimtChunk = 64;
 cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int64_t heads,
                                     int64_t n, int d, int is_bf16, int features,
                                     cudaStream_t st);
-// In-place exclusive prefix over the segments of each head (mode 0), or the per-head total
-// written to S_out + head*S_hs ([D][d]) and z_out + head*z_hs ([D]) (mode 1); both start
-// from the state (init_S [heads][D][d], init_z [heads][D]) when init_S is not null.
+// States [heads][nseg][dk*dv + dk] (S [dk][dv] row-major, then z [dk]).  In-place exclusive
+// prefix over the segments of each head (mode 0), or the per-head total written to
+// S_out + head*S_hs ([dk][dv]) and z_out + head*z_hs ([dk]) (mode 1); both start from the
+// state (init_S [heads][dk][dv], init_z [heads][dk]) when init_S is not null.
 // Mode 2: in-place exclusive suffix (sum of the later segments; no starting state).
-cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
+cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int dk, int dv, int mode,
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
                                const float *init_S, const float *init_z, cudaStream_t st);
 // Per-head sum of gathered states [count][heads][D*d + D], skipping index `skip`.
@@ -37,10 +76,11 @@ cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, v
                                   int64_t S_head_stride, int64_t z_chunk_stride,
                                   int64_t z_head_stride, int64_t heads, int64_t n, int d,
                                   int causal, int is_bf16, int features, cudaStream_t st);
-// FAVOR+ positive random features: out[t][i] = exp(W[i] . x[t] - |x[t]|^2 / 2) / sqrt(d)
-// for rows t < rows; W [d][d] float32 (m = d features); x, out of type bf16 or fp32.
+// FAVOR+ positive random features: out[t][i] = exp(W[i] . x[t] - |x[t]|^2 / 2) / sqrt(m) for
+// rows t < rows, i < m; W [m][d] float32; x [rows][d], out [rows][m] of type bf16 (tensor
+// cores) or fp32 (CUDA cores).  d, m in {64, 128}.
 cudaError_t launch_favor_features(const void *x, const float *W, void *out, int64_t rows, int d,
-                                  int is_bf16, cudaStream_t st);
+                                  int m, int is_bf16, int *err, cudaStream_t st);
 
 // ---- backward pass (backward.cu), CUDA cores; is_bf16 selects bf16 I/O, else fp32 ------
 // Workspace floats linattn_backward needs.
@@ -53,17 +93,38 @@ cudaError_t backward(const void *q, const void *k, const void *v, const void *g,
 cudaError_t launch_decode_step(float *S, float *z, const void *q, const void *k, const void *v,
                                void *out, int64_t heads, int d, cudaStream_t st);
 
-// ---- bf16 I/O, tensor cores (tc_forward.cu) ----------------------------------------------
-// Chunk length of the tensor-core path.
+// ---- bf16 I/O, tensor cores (tc_forward.cu, tc_causal.cu) ---------------------------------
+// Chunk length of the tensor-core aggregate and non-causal kernels.
 constexpr int kTcChunk = 64;
-// Default tokens per work item (segment) of the tensor-core path.
+// Chunk length of the tensor-core causal output kernel; segments are multiples of it.
+constexpr int kTcCausalChunk = 128;
+// Causal outputs from the exclusive prefix state of every segment (prefix: [heads][segments]
+// [dk*dv + dk] fp32, S row-major then z).  q, k: [heads][n][dk]; v, out: [heads][n][dv];
+// dk = dv unless features != 0 (q and k are then non-negative features already).
+// seg: a multiple of kTcCausalChunk.
+cudaError_t tc_causal_out(const void *q, const void *k, const void *v, void *out, int64_t heads,
+                          int64_t n, int dk, int dv, int64_t seg, const float *prefix,
+                          int features, int *err, cudaStream_t st);
+// The causal pass in one kernel (each segment's aggregate, a look-back over the published
+// states of the earlier segments, then its outputs).  ws: tc_fused_workspace_bytes.
+// init_S [heads][dk][dv], init_z [heads][dk] (nullable): the state before each head's first
+// token.
+int64_t tc_fused_segment(int64_t heads, int64_t n, int dk, int dv);
+size_t tc_fused_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg);
+cudaError_t tc_causal_fused(const void *q, const void *k, const void *v, void *out,
+                            int64_t heads, int64_t n, int dk, int dv, int64_t seg, void *ws,
+                            const float *init_S, const float *init_z, int features, int *err,
+                            cudaStream_t st);
+// Default tokens per work item (segment) of the tensor-core path: the aggregate and
+// non-causal kernels (causal: tc_fused_segment).
 int64_t tc_default_segment(int64_t heads, int64_t n, int d);
 // Workspace bytes the tensor-core forward needs.
-size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int causal);
-// init_S / init_z (nullable): the state before the first token of every head.
-// features != 0: q and k are non-negative features already (no phi applied).
+size_t tc_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg, int causal);
+// q, k: [heads][n][dk]; v, out: [heads][n][dv].  init_S / init_z (nullable): the state before
+// the first token of every head.  features != 0: q and k are non-negative features already
+// (no phi applied; dk may differ from dv), else dk = dv.
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
-                       int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
+                       int64_t n, int dk, int dv, int causal, int64_t seg, void *ws, int *err,
                        const float *init_S, const float *init_z, int features,
                        cudaStream_t st);
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,

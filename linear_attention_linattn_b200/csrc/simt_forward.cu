@@ -104,20 +104,23 @@ __global__ void __launch_bounds__(kThreads) simt_chunk_state_kernel(const T *__r
 }
 
 // K2: per head, a sequential sweep over the segments for each group of 4 state elements
-// (16-byte loads and stores; d (d + 1) is a multiple of 4, so a group never straddles S and z).
+// (16-byte loads and stores; a state is [dk][dv] then [dk] floats with dk, dv multiples of 4, so
+// a group never straddles S and z).  One thread per group keeps the running sum in registers:
+// the sums over segments are independent per element, so no cross-thread scan is needed, and
+// the sweep reads each aggregate once.
 //   mode 0: ws[h][s] <- init[h] + sum_{s' < s} ws[h][s'] (exclusive prefix, in place)
 //   mode 1: S_out + h*S_hs, z_out + h*z_hs <- init[h] + sum_s ws[h][s] (the total)
 //   mode 2: ws[h][s] <- sum_{s' > s} ws[h][s'] (exclusive suffix, in place; the backward
 //           pass's states of the later chunks)
-// init[h] is the state before the first segment: (init_S[h] [D][d], init_z[h] [D]), or zero
+// init[h] is the state before the first segment: (init_S[h] [dk][dv], init_z[h] [dk]), or zero
 // when init_S is null.  The segments are summed in order, one group of elements per thread.
 __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws, int64_t nseg,
-                                                          int d, int mode,
+                                                          int dk, int dv, int mode,
                                                           float *__restrict__ S_out, int64_t S_hs,
                                                           float *__restrict__ z_out, int64_t z_hs,
                                                           const float *__restrict__ init_S,
                                                           const float *__restrict__ init_z) {
-  const int64_t per4 = ((int64_t)d * d + d) / 4;
+  const int64_t per4 = ((int64_t)dk * dv + dk) / 4;
   const int64_t blocks_per_head = (per4 + blockDim.x - 1) / blockDim.x;
   const int64_t head = blockIdx.x / blocks_per_head;
   const int64_t e4 = (blockIdx.x % blocks_per_head) * (int64_t)blockDim.x + threadIdx.x;
@@ -126,9 +129,9 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
   constexpr int kBatch = 8;  // independent 16-byte loads in flight per thread
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
   if (init_S != nullptr) {
-    const int64_t e = e4 * 4, dd = (int64_t)d * d;
+    const int64_t e = e4 * 4, dd = (int64_t)dk * dv;
     run = e < dd ? *reinterpret_cast<const float4 *>(init_S + head * dd + e)
-                 : *reinterpret_cast<const float4 *>(init_z + head * d + (e - dd));
+                 : *reinterpret_cast<const float4 *>(init_z + head * dk + (e - dd));
   }
   const bool rev = mode == 2;
   for (int64_t s0 = 0; s0 < nseg; s0 += kBatch) {
@@ -150,7 +153,8 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
   }
   if (mode == 1) {
     const int64_t e = e4 * 4;
-    float *dst = e < (int64_t)d * d ? S_out + head * S_hs + e : z_out + head * z_hs + (e - (int64_t)d * d);
+    const int64_t dd = (int64_t)dk * dv;
+    float *dst = e < dd ? S_out + head * S_hs + e : z_out + head * z_hs + (e - dd);
     dst[0] = run.x;
     dst[1] = run.y;
     dst[2] = run.z;
@@ -351,12 +355,12 @@ cudaError_t launch_simt_chunk_state(const void *k, const void *v, float *ws, int
                  : chunk_state_t<float>(k, v, ws, heads, n, d, !features, st);
 }
 
-cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int d, int mode,
+cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int dk, int dv, int mode,
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
                                const float *init_S, const float *init_z, cudaStream_t st) {
-  const int64_t per4 = ((int64_t)d * d + d) / 4;
+  const int64_t per4 = ((int64_t)dk * dv + dk) / 4;
   scan_states_kernel<<<(unsigned)(((per4 + 255) / 256) * heads), 256, 0, st>>>(
-      ws, nseg, d, mode, S_out, S_hs, z_out, z_hs, init_S, init_z);
+      ws, nseg, dk, dv, mode, S_out, S_hs, z_out, z_hs, init_S, init_z);
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();

@@ -1,271 +1,127 @@
-// bf16-I/O forward pass on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+// bf16-I/O forward pass on the 5th-generation tensor cores (tcgen05, TMEM, TMA): the segment
+// aggregates and the non-causal outputs, and the host side of the whole tensor-core pass.
 //
 // The method (page "Efficient Transformers: Linear Attention and Flash Attention",
 // sections "Linear attention: reordering the matmuls, not shrinking them" and "The
 // recurrent view: attention as an RNN"):
 //     out_i = phi(q_i) S / phi(q_i).z,  S = sum_j phi(k_j) v_j^T,  z = sum_j phi(k_j)
-// with j <= i in the causal mode.  Causal work is split into chunks of C = 64 tokens:
-//     num_c = phi(Q_c) S_<c + mask(phi(Q_c) phi(K_c)^T) V_c
-//     den_c = phi(Q_c) z_<c + mask(phi(Q_c) phi(K_c)^T) 1
-//     S_<c+1 = S_<c + phi(K_c)^T V_c,   z_<c+1 = z_<c + phi(K_c)^T 1
-// and chunks are grouped into segments, the work items of the CTAs.  Three kernel modes:
-//   kState        segment aggregates (S_s, z_s) -> fp32 workspace       (K1)
-//   kCausalOut    outputs of a segment from its exclusive prefix state   (K3)
-//   kNoncausalOut outputs phi(Q) S / phi(Q).z from the per-head total    (K3, no mask)
-// The exclusive prefix over segments (K2) is the scan kernel in simt_forward.cu.
+// with j <= i in the causal mode.  A head's tokens are split into segments, the work items of
+// the CTAs, and segments into chunks of C = 64 tokens.  The pass runs as three kernels:
+//   K1  this file, mode kState: each segment's aggregate (S_s, z_s) -> fp32 workspace;
+//   K2  simt_forward.cu: exclusive prefix over the segments (causal) or the per-head total;
+//   K3  causal: tc_causal.cu (128-token chunks from each segment's prefix);
+//       non-causal: this file, mode kNoncausalOut, out = phi(Q) S / phi(Q).z.
 //
-// Every product is a tcgen05.mma (kind::f16, bf16 operands, fp32 accumulator in TMEM):
-//   [P | phi(Q_c).z_<c] = phi(Q_c) [phi(K_c); z_<c]^T   M=64 N=80    K=d   (causal; A: Q, B: K,
-//                          both K-major; the K tile carries 16 more rows, row 64 = z_<c)
-//   O  = phi(Q_c) S_<c                                   M=64 N=d     K=d   (B: S bf16 MN-major;
-//                          non-causal N=d+16: an extra atom holds z, column d = denominator)
-//   O += mask(P) V_c                                     M=64 N=d     K=64  (A: P bf16 K-major,
-//                          B: V MN-major)
-//   [S | z] += phi(K_c)^T [V_c | 1]                      M=d  N=d+16  K=64  (A: K MN-major; a
-//                          constant ones atom after each V tile puts z in column d)
-// The causal denominator is column 64 of the score block plus the masked row sum of the
-// scores (taken while they are rounded), so numerator and denominator weigh the same keys.
+// Products (tcgen05.mma kind::f16, bf16 operands, fp32 accumulators in TMEM):
+//   [S | z] += phi(K_c)^T [V_c | 1]   M=DK N=DV+16 K=64   (A: K MN-major; a constant ones atom
+//                                      after each V tile puts z in column DV)
+//   [O | den] = phi(Q_c) [S | z]      M=64 N=DV+16 K=DK   (B: the bf16 total, MN-major, an
+//                                      extra atom holds z, so column DV is the denominator)
+// DK is the feature dimension of phi(q), phi(k) (the head dimension for phi = elu + 1, m for
+// random features), DV the value dimension; each 64 or 128.
 //
-// Warp roles (one CTA per SM; 16, 22 or 18 warps in the causal, aggregate, non-causal modes):
-//   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of Q/K/V chunks into a
-//              ring of stages; no multicast.
+// Warp roles (one CTA per SM; 22 warps in the aggregate mode, 18 in the non-causal mode):
+//   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of the chunks into a ring of
+//              stages; no multicast.
 //   warp 1     TMEM allocation and the single MMA-issuing thread.
-//   next 6-12  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
-//              n zeroed, then handed to the tensor cores.
-//   next 4     state: round S_<c+1 and z into the next chunk's operands; the starting
-//              state; the segment aggregate.
-//   last 4     scores and output: mask and round P; divide O by its denominator and
-//              store the bf16 rows.  P and S are drained by different warps, so the two
-//              conversions on each chunk's critical path run side by side.
+//   next 12/8  feature map: phi applied in place to the K (aggregate) or Q (non-causal) tiles
+//              (packed bf16), K rows beyond the item's end zeroed.
+//   next 4     state: the item's aggregate out of TMEM (aggregate); the head's total rounded
+//              into the bf16 S operand (non-causal).
+//   last 4     output: O / den -> bf16 rows stored straight to global memory (non-causal).
 // Every wait is bounded (2 s); a wait that gives up records LINATTN_ERR_TIMEOUT and the
 // CTA drains and exits without trapping.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace linattn {
 namespace {
 
-constexpr int C = kTcChunk;       // tokens per chunk (64)
-constexpr int kAtom = C * 128;    // one [64 rows][64 bf16] 128B-swizzled atom: 8 KB
+using namespace tc;
 
-enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
+constexpr int C = kTcChunk;     // tokens per chunk (64)
+constexpr int kAtom = C * 128;  // one [64 rows][64 bf16] 128B-swizzled atom: 8 KB
+
+enum Mode : int { kState = 0, kNoncausalOut = 2 };
 
 constexpr int kWarpTMA = 0;
 constexpr int kWarpMMA = 1;
 constexpr int kWarpXform0 = 2;
 constexpr int kGroupThreads = 128;
-// Warps per mode (measured on the benchmark shapes).  Causal: 6 feature-map warps, 16 warps
-// in all, so each SM sub-partition holds 4 warps and a thread may use 128 registers (the
-// score, state and output drains keep 64-column batches in registers).  Aggregate: the
-// feature map on K bounds the chunk rate, so 12 feature-map warps (22 warps, 80 registers).
-// Non-causal: 8 feature-map warps (18 warps, 96 registers).
+// Warps per mode (measured on the benchmark shapes).  Aggregate: the feature map on K bounds
+// the chunk rate, so 12 feature-map warps (22 warps, 80 registers).  Non-causal: 8 feature-map
+// warps (18 warps, 96 registers).
 template <int MODE>
 struct Warps {
-  static constexpr int XFORM = MODE == kCausalOut ? 6 : (MODE == kState ? 12 : 8);
+  static constexpr int XFORM = MODE == kState ? 12 : 8;
   static constexpr int XTHREADS = XFORM * 32;
   static constexpr int STATE0 = kWarpXform0 + XFORM;  // state group: 4 warps
-  static constexpr int OUT0 = STATE0 + 4;             // scores and output group: 4 warps
+  static constexpr int OUT0 = STATE0 + 4;             // output group: 4 warps
   static constexpr int THREADS = (OUT0 + 4) * 32;
 };
-constexpr int kMaxSmem = 227 * 1024;
-constexpr uint32_t kTmemCols = 512;
-constexpr int kZRows = 16;  // extra key rows carrying z (row 0) in the causal K tile
-// causal items of at most this many chunks run on persistent CTAs
-constexpr int kPersistentCausalChunks = 32;
 
-template <int D, int MODE>
+template <int DK, int DV, int MODE>
 struct Cfg {
-  static constexpr int A = D / 64;          // 64-column atoms per [64][D] tile
-  static constexpr int TILE = A * kAtom;    // bytes of a bf16 [64][D] tile (Q, V)
+  static constexpr int AK = DK / 64;        // 64-column atoms per [64][DK] tile (Q, K)
+  static constexpr int AV = DV / 64;        // 64-column atoms per [64][DV] tile (V)
   static constexpr bool LQ = MODE != kState;
-  static constexpr bool LKV = MODE != kNoncausalOut;
-  // causal: each K atom carries 16 more rows after the 64 keys; row 64 holds z_<c, so the
-  // score MMA (N = 80) also yields phi(q_i).z_<c in its column 64.
-  static constexpr int KROWS = MODE == kCausalOut ? 64 + kZRows : 64;
-  static constexpr int KATOM = KROWS * 128;
-  static constexpr int KTILE = A * KATOM;
-  // a constant atom after each V tile whose column 0 is 1: the S MMA with N = D + 16 then
-  // also accumulates z = phi(K)^T 1 in its column D.
-  static constexpr int ONES = LKV ? kAtom : 0;
-  static constexpr int OFF_K = LQ ? TILE : 0;
-  static constexpr int OFF_V = OFF_K + (LKV ? KTILE : 0);
-  static constexpr int OFF_ONES = OFF_V + (LKV ? TILE : 0);
-  static constexpr int STAGE = OFF_ONES + ONES;
-  static constexpr int LOAD_BYTES = (LQ ? TILE : 0) + (LKV ? 2 * TILE : 0);
-  // bf16 S operand, MN-major [atoms][D rows][128 B]; non-causal adds an atom whose column 0
-  // is z, so O (N = D + 16) carries phi(q_i).z in its column D.
-  static constexpr int S_ATOMS = MODE == kState ? 0 : (MODE == kNoncausalOut ? A + 1 : A);
-  static constexpr int S_BUF = S_ATOMS * D * 128;  // one S operand
-  // non-causal: two S operands, so the next item's total is rounded while this one runs
-  static constexpr int S_BYTES = (MODE == kNoncausalOut ? 2 : 1) * S_BUF;
-  static constexpr int P_BYTES = MODE == kCausalOut ? kAtom : 0;  // bf16 [64][64], K-major
-  static constexpr int FIXED = S_BYTES + P_BYTES;
+  static constexpr bool LKV = MODE == kState;
+  // aggregate stage: K tile, V tile, then a constant atom whose column 0 is 1: the S MMA with
+  // N = DV + 16 then also accumulates z = phi(K)^T 1 in its column DV.
+  // non-causal stage: the Q tile.
+  static constexpr int OFF_V = AK * kAtom;
+  static constexpr int OFF_ONES = OFF_V + AV * kAtom;
+  static constexpr int STAGE = LQ ? AK * kAtom : OFF_ONES + kAtom;
+  static constexpr int LOAD_BYTES = LQ ? AK * kAtom : (AK + AV) * kAtom;
+  // non-causal: bf16 S operand, MN-major [atoms][DK rows][128 B] with one more atom whose
+  // column 0 is z, so O (N = DV + 16) carries phi(q_i).z in its column DV; two of them, so
+  // the next item's total is rounded while this one runs
+  static constexpr int S_ATOM = DK * 128;
+  static constexpr int S_BUF = LQ ? (AV + 1) * S_ATOM : 0;
+  static constexpr int S_BYTES = 2 * S_BUF;
   static constexpr int BAR_BYTES = 1024;
-  static constexpr int NS_FIT = (kMaxSmem - 1024 - BAR_BYTES - FIXED) / STAGE;
+  static constexpr int NS_FIT = (kMaxSmem - 1024 - BAR_BYTES - S_BYTES) / STAGE;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
-  static constexpr int OFF_STAGES = 0;
   static constexpr int OFF_S = NS * STAGE;
-  static constexpr int OFF_P = OFF_S + S_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_S + S_BYTES;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static_assert(NS >= 2, "at least two pipeline stages");
   static_assert(SMEM <= kMaxSmem, "shared memory budget");
-  static_assert(OFF_S % 1024 == 0 && OFF_P % 1024 == 0 && STAGE % 1024 == 0 &&
-                    OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_ONES % 1024 == 0 &&
-                    KATOM % 1024 == 0,
+  static_assert(OFF_S % 1024 == 0 && STAGE % 1024 == 0 && OFF_V % 1024 == 0 &&
+                    OFF_ONES % 1024 == 0 && S_ATOM % 1024 == 0,
                 "128B-swizzled operands need 1024-byte alignment");
 };
 
-// TMEM column map (32-column aligned): P (80 columns, causal), two O buffers (D columns,
-// plus the 16-column denominator block in the non-causal mode), S (D + 16 columns, z in
-// column D).  The state mode keeps two S accumulators, one per item parity, so one item's
-// aggregate is written out while the next one accumulates.
-template <int D, int MODE>
+// TMEM columns.  Aggregate: two [S | z] accumulators (DV + 16 columns each), one per item
+// parity, so one item's aggregate is written out while the next one accumulates.
+// Non-causal: two O buffers (DV + 16 columns, the denominator in column DV).
+template <int DV, int MODE>
 struct TmemMap {
-  static constexpr uint32_t P = 0;
-  static constexpr uint32_t OW = ((MODE == kNoncausalOut ? D + 16 : D) + 31) / 32 * 32;
-  static constexpr uint32_t O0 = MODE == kCausalOut ? 96 : 0;
-  static constexpr uint32_t O1 = O0 + OW;
-  static constexpr uint32_t S = MODE == kCausalOut ? O1 + OW : 0;  // unused when non-causal
-  static constexpr uint32_t S1 = MODE == kState ? kTmemCols / 2 : S;
-  static_assert((MODE == kNoncausalOut ? O1 + OW : S1 + D + 16) <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t OW = (DV + 16 + 31) / 32 * 32;
+  static constexpr uint32_t O0 = 0;
+  static constexpr uint32_t O1 = OW;
+  static constexpr uint32_t S = 0;
+  static constexpr uint32_t S1 = kTmemCols / 2;
+  static_assert((MODE == kNoncausalOut ? O1 + OW : S1 + DV + 16) <= kTmemCols, "TMEM budget");
 };
 
 struct Bars {
   uint64_t full[8], ready[8], empty[8];
-  uint64_t p_full, p_ready, s_full, s_ready, z_ready, rs_ready, o_full[2], o_empty[2], fin;
-  // per item parity: state mode, S accumulator complete (MMA -> state group) / written out
+  uint64_t o_full[2], o_empty[2], fin;
+  // per item parity: aggregate mode, S accumulator complete (MMA -> state group) / written out
   // (state group -> MMA); non-causal, S operand rounded (state group -> MMA) / no longer read
   // (MMA -> state group)
   uint64_t item_full[2], item_empty[2];
-  float rowsum[2][64];  // the state group's half of P's row sums, by chunk parity
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block");
-
-// Shared-memory descriptors are built once per operand base (make_sw128_desc) and then
-// stepped by adding (byte offset >> 4) to the 14-bit start-address field, which never
-// carries: shared addresses stay below 2^18 bytes.
-__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t byte_off) {
-  return desc + static_cast<uint64_t>(byte_off >> 4);
-}
-// K-major operand, K-step ks of a tile made of 64-column atoms of `atom_bytes` each: four
-// K-steps of 32 bytes inside one 128-byte swizzle row, then the next atom.
-__device__ __forceinline__ uint32_t kmajor_off(int ks, uint32_t atom_bytes) {
-  return (ks >> 2) * atom_bytes + (ks & 3) * 32;
-}
-// MN-major operand, K-step ks: 16 K-rows = two 8-row groups of 1024 bytes.
-__device__ __forceinline__ uint32_t mnmajor_off(int ks) { return ks * 2048; }
-__device__ __forceinline__ uint64_t kmajor_base(uint32_t addr) {
-  return make_sw128_desc(addr, 16, 1024);
-}
-__device__ __forceinline__ uint64_t mnmajor_base(uint32_t addr, uint32_t lbo) {
-  return make_sw128_desc(addr, lbo, 1024);
-}
-
-// phi on two packed bf16 values: exp(min(x, 0)) + max(x, 0), which is x + 1 above zero and
-// exp(x) at or below zero.  Everything is packed bf16 arithmetic:
-//   t = min(x, 0) * log2(e), with log2(e) split into a bf16 head and tail so that the product
-//       is rounded once (fma of the head onto the tail's product);
-//   e = 2^t with the packed bf16 exponential (one MUFU operation for two elements);
-//   phi = e + max(x, 0)  (above zero e = 1 exactly, so this is 1 + x rounded once).
-// The bf16 rounding of t perturbs exp(x) by at most |x| * 2^-9 relative; over the sums of
-// the method this stays far below the bf16 I/O tolerance (modelled and tested).
-__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t u) {
-  const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&u);
-  const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
-  const __nv_bfloat162 log2e_hi = __float2bfloat162_rn(1.4453125f);      // bf16(log2 e)
-  const __nv_bfloat162 log2e_lo = __float2bfloat162_rn(-0.0026174592f);  // log2 e - head
-  const __nv_bfloat162 m = __hmin2(x, zero);
-  const __nv_bfloat162 p = __hmax2(x, zero);
-  const __nv_bfloat162 t = __hfma2(m, log2e_hi, __hmul2(m, log2e_lo));
-  uint32_t e;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(*reinterpret_cast<const uint32_t *>(&t)));
-  const __nv_bfloat162 r = __hadd2(*reinterpret_cast<const __nv_bfloat162 *>(&e), p);
-  return *reinterpret_cast<const uint32_t *>(&r);
-}
-
-__device__ __forceinline__ uint4 pack8(const float *f) {
-  uint4 u;
-  u.x = pack_bf16x2(f[0], f[1]);
-  u.y = pack_bf16x2(f[2], f[3]);
-  u.z = pack_bf16x2(f[4], f[5]);
-  u.w = pack_bf16x2(f[6], f[7]);
-  return u;
-}
-// One 32-byte store (a full sector): 16 bf16 values.
-__device__ __forceinline__ void st_global_32B(void *p, uint4 a, uint4 b) {
-  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y),
-               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
-               : "memory");
-}
-
-// Columns [c0, c0 + 32) of the causal score row r64 (lanes < 16 of each warp hold rows of the
-// M = 64 accumulator): mask keys after the query (j > i), round to bf16 into the K-major
-// operand of P V, and return the row's partial sum (of the unrounded fp32 scores; it differs
-// from the sum of the rounded ones by at most 2^-9 relative).
-__device__ __forceinline__ float convert_P32(uint32_t taddr, uint8_t *sP, int r64, bool v64,
-                                             int c0) {
-  uint32_t p[32];
-  tmem_ld16_async(taddr + c0, p);
-  tmem_ld16_async(taddr + c0 + 16, p + 16);
-  tmem_ld_wait();
-  tmem_reg_fence<32>(p);
-  float sum = 0.f;
-  if (v64) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int g = c0 + 8 * j;  // first key of this group of 8
-      float f[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float x = __uint_as_float(p[8 * j + e]);
-        f[e] = (g + 7 <= r64 || g + e <= r64) ? x : 0.f;
-        sum += f[e];
-      }
-      *reinterpret_cast<uint4 *>(sP + sw128_offset(r64, g)) =
-          g > r64 ? make_uint4(0u, 0u, 0u, 0u) : pack8(f);
-    }
-  }
-  return sum;
-}
-
-// Lane-0 mbarrier wait whose outcome the whole warp shares (warp-uniform control flow).
-struct WarpWaiter {
-  volatile int *abort;
-  int *err;
-  int lane;
-  bool ok = true;
-  __device__ __forceinline__ bool operator()(uint64_t *b, uint32_t parity) {
-    int r = 1;
-    if (lane == 0) r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
-    r = __shfl_sync(0xffffffffu, r, 0);
-    ok = ok && (r != 0);
-    return ok;
-  }
-};
-
-// One work item: tokens [t_begin, t_end) of one head (one segment).
-struct Item {
-  int64_t head, seg, t_begin, t_end;
-  int nchunks;
-};
-__device__ __forceinline__ Item item_at(int64_t it, int64_t n, int64_t seg_len, int64_t nseg) {
-  Item I;
-  I.head = it / nseg;
-  I.seg = it % nseg;
-  I.t_begin = I.seg * seg_len;
-  I.t_end = n < I.t_begin + seg_len ? n : I.t_begin + seg_len;
-  I.nchunks = static_cast<int>((I.t_end - I.t_begin + C - 1) / C);
-  return I;
-}
 
 // CTA b takes the items b, b + gridDim.x, b + 2 gridDim.x, ... (one item when the grid
 // covers them all; several on persistent CTAs).  Every role walks the same sequence of
@@ -273,20 +129,22 @@ __device__ __forceinline__ Item item_at(int64_t it, int64_t n, int64_t seg_len, 
 // buffers run on from one item into the next: the loads of an item's first chunks overlap
 // the previous item's last ones.
 // PHI: apply phi = elu + 1 to Q and K (the method); false takes Q and K as given,
-// non-negative features (FAVOR+ features computed by favor_features_kernel).
-template <int D, int MODE, bool PHI>
+// non-negative features (FAVOR+ features computed by the feature kernels).
+// init_state (non-causal): the head's total [DK][DV] then z [DK], at init_state +
+// head * init_head_stride.  out_state (aggregate): [heads][nseg][DK*DV + DK].
+template <int DK, int DV, int MODE, bool PHI>
 __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
               const float *__restrict__ init_state, int64_t init_head_stride,
-              int64_t init_seg_stride, float *__restrict__ out_state, int64_t n, int64_t seg_len,
-              int64_t nseg, int64_t nitems, int *err) {
-  using G = Cfg<D, MODE>;
-  using TM = TmemMap<D, MODE>;
+              float *__restrict__ out_state, int64_t n, int64_t seg_len, int64_t nseg,
+              int64_t nitems, int *err) {
+  using G = Cfg<DK, DV, MODE>;
+  using TM = TmemMap<DV, MODE>;
   using W = Warps<MODE>;
   constexpr int NS = G::NS;
-  constexpr int KSD = D / 16;  // K-steps over the feature dimension
-  constexpr int KSC = C / 16;  // K-steps over the chunk's tokens
+  constexpr int KSD = DK / 16;  // K-steps over the feature dimension
+  constexpr int KSC = C / 16;   // K-steps over the chunk's tokens
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -304,12 +162,6 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
       mbar_init(&bar.ready[s], W::XTHREADS);
       mbar_init(&bar.empty[s], 1);
     }
-    mbar_init(&bar.p_full, 1);
-    mbar_init(&bar.p_ready, 2 * kGroupThreads);
-    mbar_init(&bar.rs_ready, kGroupThreads);
-    mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.s_ready, kGroupThreads);
-    mbar_init(&bar.z_ready, kGroupThreads);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.o_full[b], 1);
       mbar_init(&bar.o_empty[b], kGroupThreads);
@@ -320,29 +172,23 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     bar.abort = 0;
     fence_barrier_init();
   }
-  for (int s = 0; s < NS; ++s) {
-    uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
-    if (G::LKV) {
-      // ones atom: column 0 of every row is 1.0 (row r's column 0 sits in 16-byte chunk r & 7)
-      uint32_t *ones = reinterpret_cast<uint32_t *>(st + G::OFF_ONES);
+  if (G::LKV) {
+    // ones atom of every stage: column 0 of every row is 1.0 (row r's column 0 sits in 16-byte
+    // chunk r & 7)
+    for (int s = 0; s < NS; ++s) {
+      uint32_t *ones = reinterpret_cast<uint32_t *>(smem + s * G::STAGE + G::OFF_ONES);
       for (int i = threadIdx.x; i < kAtom / 4; i += W::THREADS) {
         const int row = i >> 5, word = i & 31;  // 32 words per 128-byte row
         ones[i] = (word == 4 * (row & 7)) ? 0x00003F80u : 0u;
-      }
-    }
-    if (MODE == kCausalOut) {
-      // z rows of the K tile start at zero (row 64 is rewritten before every chunk)
-      for (int a = 0; a < G::A; ++a) {
-        uint32_t *zr = reinterpret_cast<uint32_t *>(st + G::OFF_K + a * G::KATOM + 64 * 128);
-        for (int i = threadIdx.x; i < kZRows * 128 / 4; i += W::THREADS) zr[i] = 0u;
       }
     }
   }
   if (MODE == kNoncausalOut) {
     // the z atoms of the two S operands: zero except column 0 (rewritten with z per item)
     for (int b = 0; b < 2; ++b) {
-      uint32_t *za = reinterpret_cast<uint32_t *>(smem + G::OFF_S + b * G::S_BUF + G::A * D * 128);
-      for (int i = threadIdx.x; i < D * 128 / 4; i += W::THREADS) za[i] = 0u;
+      uint32_t *za =
+          reinterpret_cast<uint32_t *>(smem + G::OFF_S + b * G::S_BUF + G::AV * G::S_ATOM);
+      for (int i = threadIdx.x; i < G::S_ATOM / 4; i += W::THREADS) za[i] = 0u;
     }
   }
   fence_proxy_async_smem();
@@ -369,7 +215,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
       int g = 0;  // chunks issued
       bool ok = true;
       for (int64_t it = it0; ok && it < nitems; it += istep) {
-        const Item I = item_at(it, n, seg_len, nseg);
+        const Item I = item_at<C>(it, n, seg_len, nseg);
         const int zc = static_cast<int>(I.head);
         for (int c = 0; c < I.nchunks; ++c, ++g) {
           const int s = g % NS;
@@ -379,54 +225,47 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&bar.full[s], G::LOAD_BYTES);
-          uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+          uint8_t *st = smem + s * G::STAGE;
           const int y = static_cast<int>(I.t_begin + (int64_t)c * C);
           if (G::LQ) {
 #pragma unroll
-            for (int a = 0; a < G::A; ++a)
+            for (int a = 0; a < G::AK; ++a)
               tma_load_3d(st + a * kAtom, &tmQ, &bar.full[s], a * 64, y, zc, pol);
-          }
-          if (G::LKV) {
+          } else {
 #pragma unroll
-            for (int a = 0; a < G::A; ++a)
-              tma_load_3d(st + G::OFF_K + a * G::KATOM, &tmK, &bar.full[s], a * 64, y, zc, pol);
+            for (int a = 0; a < G::AK; ++a)
+              tma_load_3d(st + a * kAtom, &tmK, &bar.full[s], a * 64, y, zc, pol);
 #pragma unroll
-            for (int a = 0; a < G::A; ++a)
+            for (int a = 0; a < G::AV; ++a)
               tma_load_3d(st + G::OFF_V + a * kAtom, &tmV, &bar.full[s], a * 64, y, zc, pol);
           }
         }
       }
       // drain: every issued load has landed before the CTA may exit
       for (int gg = (g > NS ? g - NS : 0); gg < g; ++gg)
-        mbar_wait(&bar.full[gg % NS], (gg / NS) & 1, abort, err);
+        mbar_wait_drain(&bar.full[gg % NS], (gg / NS) & 1, err);
     }
   } else if (warp == kWarpMMA) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t I_P = make_idesc_bf16(64, 64 + kZRows, false, false);
-      constexpr uint32_t I_O = make_idesc_bf16(64, MODE == kNoncausalOut ? D + 16 : D, false, true);
-      constexpr uint32_t I_S = make_idesc_bf16(D, D + 16, true, true);
-      constexpr uint32_t I_OV = make_idesc_bf16(64, D, false, true);
-      uint64_t dVprev = 0;  // causal: [V | ones] of the previous chunk (its P V is still due)
-      int sprev = 0;        // and that chunk's stage
-      const uint32_t tP = tmem + TM::P;
-      const uint64_t dP = kmajor_base(smem_u32(smem + G::OFF_P));
-      const uint32_t st0 = smem_u32(smem + G::OFF_STAGES);
+      constexpr uint32_t I_O = make_idesc_bf16(64, DV + 16, false, true);
+      constexpr uint32_t I_S = make_idesc_bf16(DK, DV + 16, true, true);
+      const uint32_t st0 = smem_u32(smem);
       int g = 0;
       int j = 0;  // items of this CTA
       bool ok = true;
       for (int64_t it = it0; ok && it < nitems; it += istep, ++j) {
-        const Item I = item_at(it, n, seg_len, nseg);
+        const Item I = item_at<C>(it, n, seg_len, nseg);
         const int b = j & 1;
         const uint32_t tS = tmem + (b ? TM::S1 : TM::S);
-        const uint64_t dS =
-            mnmajor_base(smem_u32(smem + G::OFF_S + (MODE == kNoncausalOut ? b * G::S_BUF : 0)),
-                         D * 128);
-        // state mode: this S accumulator written out (item j - 2); non-causal: the head's
+        const uint64_t dS = mnmajor_base(smem_u32(smem + G::OFF_S + b * G::S_BUF), G::S_ATOM);
+        // aggregate: this S accumulator written out (item j - 2); non-causal: the head's
         // total rounded into this S operand
-        if (MODE == kState && j >= 2 && !mbar_wait(&bar.item_empty[b], ((j >> 1) - 1) & 1, abort, err))
+        if (MODE == kState && j >= 2 &&
+            !mbar_wait(&bar.item_empty[b], ((j >> 1) - 1) & 1, abort, err))
           break;
-        if (MODE == kNoncausalOut && !mbar_wait(&bar.item_full[b], (j >> 1) & 1, abort, err)) break;
+        if (MODE == kNoncausalOut && !mbar_wait(&bar.item_full[b], (j >> 1) & 1, abort, err))
+          break;
         for (int c = 0; c < I.nchunks; ++c, ++g) {
           const int s = g % NS;
           if (!mbar_wait(&bar.ready[s], (g / NS) & 1, abort, err)) {
@@ -434,12 +273,10 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
             break;
           }
           const uint32_t st = st0 + s * G::STAGE;
-          const uint64_t dQk = kmajor_base(st);                        // Q, K-major
-          const uint64_t dKk = kmajor_base(st + G::OFF_K);             // K (+z rows), K-major
-          const uint64_t dKm = mnmajor_base(st + G::OFF_K, G::KATOM);  // K, MN-major
-          const uint64_t dVm = mnmajor_base(st + G::OFF_V, kAtom);     // [V | ones], MN-major
-          tc_fence_after();
           if (MODE == kState) {
+            tc_fence_after();
+            const uint64_t dKm = mnmajor_base(st, kAtom);               // K, MN-major
+            const uint64_t dVm = mnmajor_base(st + G::OFF_V, kAtom);    // [V | ones], MN-major
 #pragma unroll
             for (int ks = 0; ks < KSC; ++ks)
               mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)),
@@ -449,64 +286,13 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
           }
           const int ob = g & 1;
           const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0);
-          if (MODE == kCausalOut) {
-            // The previous chunk's P V (its scores rounded by now) interleaved with this
-            // chunk's [scores | phi(q).z_<c]: different accumulators, so the tensor pipe
-            // overlaps the two chains instead of running them back to back.
-            if (!mbar_wait(&bar.z_ready, g & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            if (g >= 1 && !mbar_wait(&bar.p_ready, (g - 1) & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t tOp = tmem + (((g - 1) & 1) ? TM::O1 : TM::O0);  // O of chunk g - 1
-#pragma unroll
-            for (int ks = 0; ks < KSD; ++ks) {
-              if (g >= 1 && ks < KSC)
-                mma_bf16_ss(tOp, desc_add(dP, kmajor_off(ks, kAtom)),
-                            desc_add(dVprev, mnmajor_off(ks)), I_OV, 1u);
-              mma_bf16_ss(tP, desc_add(dQk, kmajor_off(ks, kAtom)),
-                          desc_add(dKk, kmajor_off(ks, G::KATOM)), I_P, ks > 0 ? 1u : 0u);
-              if (g >= 1 && ks == KSC - 1) {
-                mma_commit(&bar.o_full[(g - 1) & 1]);
-                mma_commit(&bar.empty[sprev]);
-              }
-            }
-            mma_commit(&bar.p_full);
-            // S_<c in the S operand; this O buffer drained
-            if (!mbar_wait(&bar.s_ready, g & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            // phi(Q_c) S_<c, then S += phi(K_c)^T [V_c | 1] (interleaving these two measured
-            // no faster)
-#pragma unroll
-            for (int ks = 0; ks < KSD; ++ks)
-              mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
-                          I_O, ks > 0 ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
-                          1u);
-            mma_commit(&bar.s_full);
-            dVprev = dVm;  // P V of this chunk goes with the next chunk's scores
-            sprev = s;
-            continue;
-          }
           // this O buffer drained
           if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const uint64_t dQk = kmajor_base(st);
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
@@ -518,68 +304,39 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
         if (MODE == kState) mma_commit(&bar.item_full[b]);        // aggregate complete
         if (MODE == kNoncausalOut) mma_commit(&bar.item_empty[b]);  // S operand no longer read
       }
-      if (MODE == kCausalOut && ok && g > 0) {
-        // the last chunk's P V
-        if (mbar_wait(&bar.p_ready, (g - 1) & 1, abort, err)) {
-          tc_fence_after();
-          const uint32_t tOp = tmem + (((g - 1) & 1) ? TM::O1 : TM::O0);
-#pragma unroll
-          for (int ks = 0; ks < KSC; ++ks)
-            mma_bf16_ss(tOp, desc_add(dP, kmajor_off(ks, kAtom)), desc_add(dVprev, mnmajor_off(ks)),
-                        I_OV, 1u);
-          mma_commit(&bar.o_full[(g - 1) & 1]);
-          mma_commit(&bar.empty[sprev]);
-        }
-      }
       // every MMA this CTA issued has finished before TMEM is released
       mma_commit(&bar.fin);
-      mbar_wait(&bar.fin, 0, abort, err);
+      mbar_wait_drain(&bar.fin, 0, err);
     }
   } else if (warp < W::STATE0) {
     // ================================================================ feature map
-    // phi in place on the Q tile and on the 64 key rows of each K atom; K rows past the
-    // item's end are zeroed (they must add nothing to S, z or the scores).
+    // phi in place on the Q tile (non-causal) or on the K tile (aggregate); K rows past the
+    // item's end are zeroed (they must add nothing to S or z).
     const int xt = threadIdx.x - kWarpXform0 * 32;
     int g = 0;
     bool ok = true;
     for (int64_t it = it0; ok && it < nitems; it += istep) {
-      const Item I = item_at(it, n, seg_len, nseg);
+      const Item I = item_at<C>(it, n, seg_len, nseg);
       for (int c = 0; c < I.nchunks; ++c, ++g) {
         const int s = g % NS;
         if (!mbar_wait(&bar.full[s], (g / NS) & 1, abort, err)) {
           ok = false;
           break;
         }
-        uint8_t *st = smem + G::OFF_STAGES + s * G::STAGE;
+        uint8_t *st = smem + s * G::STAGE;
         const int64_t left = I.t_end - (I.t_begin + (int64_t)c * C);
         const int valid = left < C ? static_cast<int>(left) : C;
-        if (G::LQ && PHI) {
-          uint4 *p = reinterpret_cast<uint4 *>(st);
 #pragma unroll 2
-          for (int i = xt; i < G::TILE / 16; i += W::XTHREADS) {
-            uint4 x = p[i];
-            x.x = phi_bf16x2(x.x);
-            x.y = phi_bf16x2(x.y);
-            x.z = phi_bf16x2(x.z);
-            x.w = phi_bf16x2(x.w);
-            p[i] = x;
-          }
-        }
-        if (G::LKV) {
-#pragma unroll 2
-          for (int i = xt; i < G::TILE / 16; i += W::XTHREADS) {
-            const int a = i / (kAtom / 16), within = i % (kAtom / 16);
-            const int row = within >> 3;  // 8 x 16 B per 128-byte row
-            uint4 *p = reinterpret_cast<uint4 *>(st + G::OFF_K + a * G::KATOM) + within;
+        for (int i = xt; i < G::AK * kAtom / 16; i += W::XTHREADS) {
+          uint4 *p = reinterpret_cast<uint4 *>(st) + i;
+          if (G::LQ) {
+            if (PHI) *p = phi_bf16x8(*p);
+          } else {
+            const int row = (i % (kAtom / 16)) >> 3;  // 8 x 16 B per 128-byte row
             uint4 x = make_uint4(0u, 0u, 0u, 0u);
             if (row < valid) {
               x = *p;
-              if (PHI) {
-                x.x = phi_bf16x2(x.x);
-                x.y = phi_bf16x2(x.y);
-                x.z = phi_bf16x2(x.z);
-                x.w = phi_bf16x2(x.w);
-              }
+              if (PHI) x = phi_bf16x8(x);
             }
             *p = x;
           }
@@ -590,153 +347,53 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     }
   } else if (warp < W::OUT0) {
     // ================================================================ state group
-    // Causal: half of each chunk's scores (columns 0..31) and their row sums; S_<c+1, z_<c+1
-    // -> bf16 operands of the next chunk (z into that chunk's K tile row 64); each item's
-    // starting state.  Non-causal: each item's head total -> one of the two S operands.
-    // State mode: each item's aggregate.  Control flow is warp-uniform: lane 0 waits and the
-    // warp shares the outcome.
+    // Aggregate: each item's aggregate out of TMEM.  Non-causal: each item's head total ->
+    // one of the two S operands.  Control flow is warp-uniform: lane 0 waits and the warp
+    // shares the outcome.
     const int sp = warp & 3;  // TMEM sub-partition of this warp
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
-    const bool v64 = lane < 16;                      // lanes holding rows of an M=64 tile
-    const int r64 = 16 * sp + lane;                  // row of an M=64 tile
-    const int rS = D == 128 ? 32 * sp + lane : r64;  // row of the S accumulator (M = D)
-    const bool vS = D == 128 ? true : v64;
+    // row rS of S (M = DK: lanes 0..127 at DK = 128; at DK = 64 rows 16 sp .. 16 sp + 15 sit
+    // in lanes 0..15 of sub-partition sp)
+    const int rS = DK == 128 ? 32 * sp + lane : 16 * sp + lane;
+    const bool vS = DK == 128 || lane < 16;
     WarpWaiter wait{abort, err, lane};
-
-    // 32 consecutive S columns [c0, c0+32) of row rS (fp32 in registers) -> bf16 operand sS
-    auto store_S32 = [&](uint8_t *sS, const uint32_t *r, int c0) {
-      if (!vS) return;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * j + e]);
-        *reinterpret_cast<uint4 *>(sS + (c0 >> 6) * (D * 128) +
-                                   sw128_offset(rS, (c0 & 63) + 8 * j)) = pack8(f);
-      }
-    };
-    // z_< for chunk gg: causal -> row 64 of that chunk's K atoms; non-causal -> column 0 of
-    // the z atom of the S operand sS
-    auto store_z = [&](uint8_t *sS, uint32_t zbits, int gg) {
-      if (!vS) return;
-      const __nv_bfloat16 zb = __float2bfloat16_rn(__uint_as_float(zbits));
-      if (MODE == kCausalOut) {
-        uint8_t *kt = smem + G::OFF_STAGES + (gg % NS) * G::STAGE + G::OFF_K;
-        *reinterpret_cast<__nv_bfloat16 *>(kt + (rS >> 6) * G::KATOM +
-                                           sw128_offset(64, rS & 63)) = zb;
-      } else {
-        *reinterpret_cast<__nv_bfloat16 *>(sS + G::A * D * 128 + sw128_offset(rS, 0)) = zb;
-      }
-    };
-    // an item's starting state (exclusive prefix, causal; the head's total, non-causal) ->
-    // TMEM S (causal) and the bf16 operand sS; z for the item's first chunk gg
-    auto load_start = [&](const Item &I, uint8_t *sS, int gg) {
-      const float *src = init_state + I.head * init_head_stride + I.seg * init_seg_stride;
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (vS) f = *reinterpret_cast<const float4 *>(src + (int64_t)rS * D + c0 + 4 * j);
-          r[4 * j + 0] = __float_as_uint(f.x);
-          r[4 * j + 1] = __float_as_uint(f.y);
-          r[4 * j + 2] = __float_as_uint(f.z);
-          r[4 * j + 3] = __float_as_uint(f.w);
-        }
-        if (MODE == kCausalOut) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tmem_st16(tmem + lane_off + TM::S + c0 + 16 * j,
-                      *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * j));
-        }
-        store_S32(sS, r, c0);
-      }
-      const uint32_t zb = vS ? __float_as_uint(src[(int64_t)D * D + rS]) : 0u;
-      if (MODE == kCausalOut) {
-        tmem_st1(tmem + lane_off + TM::S + D, zb);
-        tmem_st_wait();
-      }
-      store_z(sS, zb, gg);
-      fence_proxy_async_smem();
-    };
-
-    if (MODE == kCausalOut) {
-      // One flat loop over this CTA's chunks; only the chunk counter, the chunks left in
-      // the current item and the next item's index stay live across it.
-      uint8_t *sS = smem + G::OFF_S;
-      int64_t it = it0;
-      int left = 0;
-#pragma unroll 1
-      for (int g = 0;; ++g) {
-        if (left == 0) {
-          // ---- an item's starting state, once the previous item's last S and O products
-          // are done with TMEM S and the S operand
-          if (it >= nitems) break;
-          const Item I = item_at(it, n, seg_len, nseg);
-          it += istep;
-          left = I.nchunks;
-          if (g == 0 || wait(&bar.s_full, (g - 1) & 1)) {
-            tc_fence_after();
-            load_start(I, sS, g);
-            tc_fence_before();
-          }
-          mbar_arrive(&bar.z_ready);
-          mbar_arrive(&bar.s_ready);
-        }
-        // ---- this chunk's scores, columns 0..31 (the output group takes 32..63)
-        if (wait(&bar.p_full, g & 1)) {
-          tc_fence_after();
-          const float rs = convert_P32(tmem + lane_off + TM::P, smem + G::OFF_P, r64, v64, 0);
-          fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(&bar.p_ready);
-          if (v64) bar.rowsum[g & 1][r64] = rs;
-          mbar_arrive(&bar.rs_ready);
-        }
-        // ---- S_<c+1, z_<c+1: the operands of the item's next chunk
-        if (--left > 0 && wait(&bar.s_full, g & 1)) {
-          tc_fence_after();
-          // z_<c+1 first: the next chunk's score MMA needs only that
-          store_z(sS, tmem_ld1(tmem + lane_off + TM::S + D), g + 1);
-          fence_proxy_async_smem();
-          mbar_arrive(&bar.z_ready);
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 64) {
-            uint32_t r[64];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tmem_ld16_async(tmem + lane_off + TM::S + c0 + 16 * q, r + 16 * q);
-            tmem_ld_wait();
-            tmem_reg_fence<64>(r);
-            store_S32(sS, r, c0);
-            store_S32(sS, r + 32, c0 + 32);
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(&bar.s_ready);
-        }
-      }
-    } else if (MODE == kNoncausalOut) {
+    if (MODE == kNoncausalOut) {
       int j = 0;
       for (int64_t it = it0; it < nitems; it += istep, ++j) {
-        const Item I = item_at(it, n, seg_len, nseg);
+        const Item I = item_at<C>(it, n, seg_len, nseg);
         const int b = j & 1;
         uint8_t *sS = smem + G::OFF_S + b * G::S_BUF;
         // the MMAs of item j - 2 no longer read this S operand
-        if (j < 2 || wait(&bar.item_empty[b], ((j >> 1) - 1) & 1)) load_start(I, sS, 0);
+        if (j < 2 || wait(&bar.item_empty[b], ((j >> 1) - 1) & 1)) {
+          const float *src = init_state + I.head * init_head_stride;
+          if (vS) {
+            for (int c0 = 0; c0 < DV; c0 += 8) {
+              const float4 lo = *reinterpret_cast<const float4 *>(src + (int64_t)rS * DV + c0);
+              const float4 hi =
+                  *reinterpret_cast<const float4 *>(src + (int64_t)rS * DV + c0 + 4);
+              const float f[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+              *reinterpret_cast<uint4 *>(sS + (c0 >> 6) * G::S_ATOM +
+                                         sw128_offset(rS, c0 & 63)) = pack8(f);
+            }
+            // z_r in column 0 of the z atom
+            *reinterpret_cast<__nv_bfloat16 *>(sS + G::AV * G::S_ATOM + sw128_offset(rS, 0)) =
+                __float2bfloat16_rn(src[(int64_t)DK * DV + rS]);
+          }
+          fence_proxy_async_smem();
+        }
         mbar_arrive(&bar.item_full[b]);
       }
     } else {
-      // segment aggregates -> fp32 workspace [D][d] then z[D]
+      // segment aggregates -> fp32 workspace [DK][DV] then z[DK]
       int j = 0;
       for (int64_t it = it0; it < nitems; it += istep, ++j) {
-        const Item I = item_at(it, n, seg_len, nseg);
+        const Item I = item_at<C>(it, n, seg_len, nseg);
         const int b = j & 1;
         const uint32_t tS = tmem + lane_off + (b ? TM::S1 : TM::S);
         if (wait(&bar.item_full[b], (j >> 1) & 1)) {
           tc_fence_after();
-          float *dst = out_state + (I.head * nseg + I.seg) * (int64_t)(D * D + D);
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          float *dst = out_state + (I.head * nseg + I.seg) * ((int64_t)DK * DV + DK);
+          for (int c0 = 0; c0 < DV; c0 += 32) {
             uint32_t r[32];
 #pragma unroll
             for (int q = 0; q < 2; ++q) tmem_ld16_async(tS + c0 + 16 * q, r + 16 * q);
@@ -745,99 +402,58 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
             if (vS) {
 #pragma unroll
               for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4 *>(dst + (int64_t)rS * D + c0 + e) =
+                *reinterpret_cast<float4 *>(dst + (int64_t)rS * DV + c0 + e) =
                     make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
                                 __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
             }
           }
-          const uint32_t zr = tmem_ld1(tS + D);
-          if (vS) dst[(int64_t)D * D + rS] = __uint_as_float(zr);
+          const uint32_t zr = tmem_ld1(tS + DV);
+          if (vS) dst[(int64_t)DK * DV + rS] = __uint_as_float(zr);
         }
         tc_fence_before();
         mbar_arrive(&bar.item_empty[b]);
       }
     }
-  } else {
-    // ================================================================ scores and output
-    // P(c) columns 32..63 -> masked bf16 operand of P V (the state group takes 0..31), with
-    // phi(q).z_<c (column 64) and both groups' row sums -> the denominator of chunk c; then
-    // O(c-1) / den -> bf16 rows stored straight to global memory (32-byte stores; rows past
-    // the item's end are not written).
+  } else if (MODE == kNoncausalOut) {
+    // ================================================================ output
+    // O / den -> bf16 rows stored straight to global memory (32-byte stores; rows past the
+    // item's end are not written).  Lanes < 16 of each warp hold rows of the M = 64 tile.
     const int sp = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
     const bool v64 = lane < 16;
     const int r64 = 16 * sp + lane;
     WarpWaiter wait{abort, err, lane};
-
-    // Denominators of the chunks in flight, by parity.  The state group's half of the row sum
-    // is read BEFORE this group releases p_ready: the state group's next sums need this
-    // chunk's p_ready, so it never completes rs_ready's next phase (or rewrites that slot)
-    // before this wait has seen the current one.
-    float den0 = 1.f, den1 = 1.f;
-    auto convert_P = [&](int gg) {
-      if (!wait(&bar.p_full, gg & 1)) return;
-      tc_fence_after();
-      const float rs = convert_P32(tmem + lane_off + TM::P, smem + G::OFF_P, r64, v64, 32);
-      const float dz = __uint_as_float(tmem_ld1(tmem + lane_off + TM::P + 64));
-      const bool got = wait(&bar.rs_ready, gg & 1);
-      const float d = dz + rs + (got ? bar.rowsum[gg & 1][v64 ? r64 : 0] : 0.f);
-      if (gg & 1) den1 = d; else den0 = d;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bar.p_ready);
-    };
-
-    // O of chunk gg (chunk c of item I)
-    auto emit_O = [&](int gg, const Item &I, int c) {
-      const int ob = gg & 1;
-      const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
-      if (!wait(&bar.o_full[ob], (gg >> 1) & 1)) return;
-      tc_fence_after();
-      const float dd = MODE == kCausalOut ? (ob ? den1 : den0) : __uint_as_float(tmem_ld1(tO + D));
-      const float inv = 1.f / dd;
-      const int64_t t = I.t_begin + (int64_t)c * C + r64;
-      const bool live = v64 && t < I.t_end;
-      __nv_bfloat16 *orow = out + (I.head * n + (live ? t : 0)) * D;
+    int g = 0;
+    for (int64_t it = it0; it < nitems; it += istep) {
+      const Item I = item_at<C>(it, n, seg_len, nseg);
+      for (int c = 0; c < I.nchunks; ++c, ++g) {
+        const int ob = g & 1;
+        const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
+        if (!wait(&bar.o_full[ob], (g >> 1) & 1)) continue;
+        tc_fence_after();
+        const float inv = 1.f / __uint_as_float(tmem_ld1(tO + DV));
+        const int64_t t = I.t_begin + (int64_t)c * C + r64;
+        const bool live = v64 && t < I.t_end;
+        __nv_bfloat16 *orow = out + (I.head * n + (live ? t : 0)) * DV;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 64) {
-        uint32_t r[64];
+        for (int c0 = 0; c0 < DV; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld16_async(tO + c0, r);
+          tmem_ld16_async(tO + c0 + 16, r + 16);
+          tmem_ld_wait();
+          tmem_reg_fence<32>(r);
+          if (live) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16_async(tO + c0 + 16 * q, r + 16 * q);
-        tmem_ld_wait();
-        tmem_reg_fence<64>(r);
-        if (live) {
+            for (int q = 0; q < 2; ++q) {
+              float f[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float f[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
-            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8));
+              for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
+              st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8));
+            }
           }
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar.o_empty[ob]);
-    };
-
-    if (MODE == kCausalOut) {
-      int g = 0;
-      Item prev{};
-      int prev_c = 0;
-      for (int64_t it = it0; it < nitems; it += istep) {
-        const Item I = item_at(it, n, seg_len, nseg);
-        for (int c = 0; c < I.nchunks; ++c, ++g) {
-          convert_P(g);
-          if (g >= 1) emit_O(g - 1, prev, prev_c);
-          prev = I;
-          prev_c = c;
-        }
-      }
-      if (g > 0) emit_O(g - 1, prev, prev_c);
-    } else if (MODE == kNoncausalOut) {
-      int g = 0;
-      for (int64_t it = it0; it < nitems; it += istep) {
-        const Item I = item_at(it, n, seg_len, nseg);
-        for (int c = 0; c < I.nchunks; ++c, ++g) emit_O(g, I, c);
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty[ob]);
       }
     }
   }
@@ -849,6 +465,74 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
 }
 
 // ------------------------------------------------------------------ host side
+template <int DK, int DV, int MODE, bool PHI>
+cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                      void *out, const float *init, int64_t ihs, float *out_state,
+                      int64_t heads, int64_t n, int64_t seg, int64_t nseg, int *err,
+                      cudaStream_t st) {
+  using G = Cfg<DK, DV, MODE>;
+  auto kern = tc_kernel<DK, DV, MODE, PHI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+  if (e != cudaSuccess) return e;
+  // One CTA holds a whole SM's shared memory and TMEM; persistent CTAs (one per SM, items
+  // dealt round-robin) save each item the CTA start-up and pipeline fill and drain.
+  const int64_t nitems = heads * nseg;
+  const int64_t sms = sm_count();
+  const unsigned grid = static_cast<unsigned>(nitems < sms ? nitems : sms);
+  kern<<<grid, Warps<MODE>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out),
+                                                    init, ihs, out_state, n, seg, nseg, nitems,
+                                                    err);
+  count_launches(1);
+  record_launch_event(st);
+  return cudaGetLastError();
+}
+
+// The whole pass: K1 aggregates, K2 scan, K3 outputs.  q, k: [heads][n][DK]; v, out: [heads]
+// [n][DV].
+template <int DK, int DV, bool PHI>
+cudaError_t tc_forward_dims(const void *q, const void *k, const void *v, void *out,
+                            int64_t heads, int64_t n, int causal, int64_t seg, void *ws, int *err,
+                            const float *init_S, const float *init_z, cudaStream_t st) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  const int64_t per = (int64_t)DK * DV + DK;
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap_bf16(&tk, k, heads, n, DK, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tv, v, heads, n, DV, C)) != cudaSuccess) return e;
+  float *w = static_cast<float *>(ws);
+  // causal: one kernel, each segment's prefix by a look-back over the published states
+  if (causal) return tc_causal_fused(q, k, v, out, heads, n, DK, DV, seg, ws, init_S, init_z,
+                                     PHI ? 0 : 1, err, st);
+  e = launch_tc<DK, DV, kState, PHI>(tk, tk, tv, out, nullptr, 0, w, heads, n, seg, nseg, err,
+                                     st);
+  if (e != cudaSuccess) return e;
+  // per-head totals, packed as [heads][DK*DV + DK] (S row-major, then z)
+  float *tot = w + heads * nseg * per;
+  e = launch_scan_states(w, heads, nseg, DK, DV, 1, tot, per, tot + (int64_t)DK * DV, per, init_S,
+                         init_z, st);
+  if (e != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tq, q, heads, n, DK, C)) != cudaSuccess) return e;
+  return launch_tc<DK, DV, kNoncausalOut, PHI>(tq, tk, tv, out, tot, per, nullptr, heads, n, seg,
+                                               nseg, err, st);
+}
+
+template <int DK, int DV>
+cudaError_t tc_state_dims(const void *k, const void *v, float *S_out, float *z_out,
+                          int64_t heads, int64_t n, int64_t seg, void *ws, int *err,
+                          cudaStream_t st) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  CUtensorMap tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap_bf16(&tk, k, heads, n, DK, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tv, v, heads, n, DV, C)) != cudaSuccess) return e;
+  float *w = static_cast<float *>(ws);
+  e = launch_tc<DK, DV, kState, true>(tk, tk, tv, nullptr, nullptr, 0, w, heads, n, seg, nseg,
+                                      err, st);
+  if (e != cudaSuccess) return e;
+  return launch_scan_states(w, heads, nseg, DK, DV, 1, S_out, (int64_t)DK * DV, z_out, DK,
+                            nullptr, nullptr, st);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -863,14 +547,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [heads][n][d] bf16 as a 3-D tensor (d innermost), 64 x 64 boxes, 128-byte swizzle.
-// Rows beyond n read as zero and are never written.
-cudaError_t make_tmap(CUtensorMap *m, const void *ptr, int64_t heads, int64_t n, int d) {
+}  // namespace
+
+cudaError_t make_tmap_bf16(CUtensorMap *m, const void *ptr, int64_t heads, int64_t n, int d,
+                           int box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)heads};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)C, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -878,83 +563,11 @@ cudaError_t make_tmap(CUtensorMap *m, const void *ptr, int64_t heads, int64_t n,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Streaming multiprocessors of the current device (looked up once per device).
-int sm_count() {
-  constexpr int kMaxDev = 64;
-  static std::atomic<int> cache[kMaxDev];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
-  int v = cache[dev].load(std::memory_order_relaxed);
-  if (v <= 0) {
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-      v = 148;
-    cache[dev].store(v, std::memory_order_relaxed);
-  }
-  return v;
-}
-
-template <int D, int MODE, bool PHI = true>
-cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
-                      void *out, const float *init, int64_t ihs, int64_t iss,
-                      float *out_state, int64_t heads, int64_t n, int64_t seg, int64_t nseg,
-                      int *err, cudaStream_t st) {
-  using G = Cfg<D, MODE>;
-  auto kern = tc_kernel<D, MODE, PHI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
-  if (e != cudaSuccess) return e;
-  // One CTA holds a whole SM's shared memory and TMEM.  Persistent CTAs (one per SM, items
-  // dealt round-robin) save each item the CTA start-up and pipeline fill and drain; they
-  // pay off for the aggregate and non-causal kernels and for short causal items.  Long
-  // causal items run one CTA each: there the hardware's dynamic placement of CTAs on SMs
-  // evens out the few per cent by which SMs differ in speed, and a fresh CTA hides the load
-  // of its starting state behind its first TMA loads.
-  const int64_t nitems = heads * nseg;
-  const int64_t sms = sm_count();
-  const bool persistent = MODE != kCausalOut || seg <= kPersistentCausalChunks * C;
-  const int64_t want = persistent ? sms : nitems;
-  const unsigned grid = static_cast<unsigned>(nitems < want ? nitems : want);
-  kern<<<grid, Warps<MODE>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out), init, ihs,
-                                        iss, out_state, n, seg, nseg, nitems, err);
-  count_launches(1);
-  record_launch_event(st);
-  return cudaGetLastError();
-}
-
-template <int D, bool PHI>
-cudaError_t tc_forward_d(const void *q, const void *k, const void *v, void *out, int64_t heads,
-                         int64_t n, int causal, int64_t seg, void *ws, int *err,
-                         const float *init_S, const float *init_z, cudaStream_t st) {
-  const int64_t nseg = (n + seg - 1) / seg;
-  const int64_t per = (int64_t)D * D + D;
-  CUtensorMap tq, tk, tv;
-  cudaError_t e;
-  if ((e = make_tmap(&tq, q, heads, n, D)) != cudaSuccess) return e;
-  if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
-  if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
-  float *w = static_cast<float *>(ws);
-  e = launch_tc<D, kState, PHI>(tq, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
-  if (e != cudaSuccess) return e;
-  if (causal) {
-    e = launch_scan_states(w, heads, nseg, D, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
-    if (e != cudaSuccess) return e;
-    return launch_tc<D, kCausalOut, PHI>(tq, tk, tv, out, w, nseg * per, per, nullptr, heads, n,
-                                         seg, nseg, err, st);
-  }
-  // per-head totals, packed as [heads][D*D + D] (S row-major, then z)
-  float *tot = w + heads * nseg * per;
-  e = launch_scan_states(w, heads, nseg, D, 1, tot, per, tot + (int64_t)D * D, per, init_S,
-                         init_z, st);
-  if (e != cudaSuccess) return e;
-  return launch_tc<D, kNoncausalOut, PHI>(tq, tk, tv, out, tot, per, 0, nullptr, heads, n, seg,
-                                          nseg, err, st);
-}
-
-}  // namespace
-
 int64_t tc_default_segment(int64_t heads, int64_t n, int d) {
   (void)d;
-  // smallest tail loss over whole waves of 148 SMs (one CTA each), preferring long segments
-  const int64_t sms = 148;
+  // smallest tail loss over whole waves of the device's SMs (one CTA each), preferring long
+  // segments
+  const int64_t sms = sm_count();
   int64_t best = 64, best_score = -1;
   for (int64_t seg = 4096; seg >= 256; seg -= 256) {
     const int64_t nseg = (n + seg - 1) / seg;
@@ -967,51 +580,50 @@ int64_t tc_default_segment(int64_t heads, int64_t n, int d) {
       best = seg;
     }
   }
-  const int64_t nrounded = ((n + C - 1) / C) * C;
+  const int64_t nrounded = ((n + kTcCausalChunk - 1) / kTcCausalChunk) * kTcCausalChunk;
   return best > nrounded ? nrounded : best;
 }
 
-size_t tc_workspace_bytes(int64_t heads, int64_t n, int d, int64_t seg, int causal) {
+size_t tc_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg, int causal) {
+  if (causal) return tc_fused_workspace_bytes(heads, n, dk, dv, seg);
   const int64_t nseg = (n + seg - 1) / seg;
-  const int64_t per = (int64_t)d * d + d;
+  const int64_t per = (int64_t)dk * dv + dk;
   return (size_t)(heads * nseg * per + (causal ? 0 : heads * per)) * sizeof(float);
 }
 
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
-                       int64_t n, int d, int causal, int64_t seg, void *ws, int *err,
+                       int64_t n, int dk, int dv, int causal, int64_t seg, void *ws, int *err,
                        const float *init_S, const float *init_z, int features,
                        cudaStream_t st) {
-  if (features)
-    return d == 64 ? tc_forward_d<64, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                             init_z, st)
-                   : tc_forward_d<128, false>(q, k, v, out, heads, n, causal, seg, ws, err,
-                                              init_S, init_z, st);
-  return d == 64 ? tc_forward_d<64, true>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                          init_z, st)
-                 : tc_forward_d<128, true>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+  if (!features) {  // phi = elu + 1 keeps the dimension
+    if (dk == 64 && dv == 64)
+      return tc_forward_dims<64, 64, true>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
                                            init_z, st);
-}
-
-template <int D>
-cudaError_t tc_state_d(const void *k, const void *v, float *S_out, float *z_out, int64_t heads,
-                       int64_t n, int64_t seg, void *ws, int *err, cudaStream_t st) {
-  const int64_t nseg = (n + seg - 1) / seg;
-  CUtensorMap tk, tv;
-  cudaError_t e;
-  if ((e = make_tmap(&tk, k, heads, n, D)) != cudaSuccess) return e;
-  if ((e = make_tmap(&tv, v, heads, n, D)) != cudaSuccess) return e;
-  float *w = static_cast<float *>(ws);
-  e = launch_tc<D, kState>(tk, tk, tv, nullptr, nullptr, 0, 0, w, heads, n, seg, nseg, err, st);
-  if (e != cudaSuccess) return e;
-  return launch_scan_states(w, heads, nseg, D, 1, S_out, (int64_t)D * D, z_out, D, nullptr,
-                            nullptr, st);
+    if (dk == 128 && dv == 128)
+      return tc_forward_dims<128, 128, true>(q, k, v, out, heads, n, causal, seg, ws, err,
+                                             init_S, init_z, st);
+    return cudaErrorInvalidValue;
+  }
+  if (dk == 64 && dv == 64)
+    return tc_forward_dims<64, 64, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                          init_z, st);
+  if (dk == 128 && dv == 128)
+    return tc_forward_dims<128, 128, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                            init_z, st);
+  if (dk == 128 && dv == 64)
+    return tc_forward_dims<128, 64, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                           init_z, st);
+  if (dk == 64 && dv == 128)
+    return tc_forward_dims<64, 128, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
+                                           init_z, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
                              int64_t heads, int64_t n, int d, int64_t seg, void *ws, int *err,
                              cudaStream_t st) {
-  return d == 64 ? tc_state_d<64>(k, v, S_out, z_out, heads, n, seg, ws, err, st)
-                 : tc_state_d<128>(k, v, S_out, z_out, heads, n, seg, ws, err, st);
+  return d == 64 ? tc_state_dims<64, 64>(k, v, S_out, z_out, heads, n, seg, ws, err, st)
+                 : tc_state_dims<128, 128>(k, v, S_out, z_out, heads, n, seg, ws, err, st);
 }
 
 }  // namespace linattn

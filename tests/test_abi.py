@@ -78,6 +78,9 @@ def test_decode_and_state_argument_checks(lib):
         la.LINATTN_ERR_INVALID_ARG
     assert lib.linattn_forward_ex(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1, 1, -64, None) == \
         la.LINATTN_ERR_INVALID_ARG
+    # segments are whole 128-token chunks of the causal kernel
+    assert lib.linattn_forward_ex(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1, 1, 64, None) == \
+        la.LINATTN_ERR_INVALID_ARG
 
 
 def test_backward_init_and_sum_argument_checks(lib):

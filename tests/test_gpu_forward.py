@@ -38,7 +38,7 @@ def test_small_shapes(dtype, causal, d, B, H, n):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("seg", [0, 64, 128, 512, 1024])
+@pytest.mark.parametrize("seg", [0, 128, 256, 512, 1024])
 def test_segment_length_invariance(dtype, seg):
     B, H, n, d = 1, 2, 3000, 128
     q, k, v = inputs.forward_qkv(7, B, H, n, d, scaled=True)
@@ -120,39 +120,54 @@ def test_workload_causal_1x1x4096x64(dtype):
     assert max_row_rel_err(got, oracle.forward(q, k, v, True)) <= TOL[dtype]
 
 
-def _sample_rows(n, extra, seed):
+def _sample_rows(n, extra, seed, edge_step=0):
+    """Chunk edges, powers of two, the last rows and random rows; with edge_step, both sides of
+    every multiple of it (every segment edge the library can pick: its segments are multiples
+    of 128 tokens, chosen from multiples of 256)."""
     rng = np.random.default_rng(seed)
-    rows = {0, 1, 2, 63, 64, 65, 127, 128, n // 2, n - 2, n - 1}
+    rows = {0, 1, 2, 63, 64, 65, 127, 128, 129, 255, 256, n // 2, n - 2, n - 1}
     rows |= {r for m in (512, 1024, 2048, 4096) for r in (m - 1, m) if r < n}
+    if edge_step:
+        rows |= {r for m in range(edge_step, n, edge_step) for r in (m - 1, m)}
     rows |= set(rng.integers(0, n, size=extra).tolist())
     return np.array(sorted(r for r in rows if 0 <= r < n), dtype=np.int64)
 
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_workload_batched_8x16x8192x64_bf16(causal):
+    """Full size, as the benchmark runs it: every row of head (3, 7); on two more heads the
+    rows on both sides of every multiple of 128 tokens (every chunk and segment edge)."""
     w = inputs.WORKLOADS["batched_8x16x8192x64_bf16"]
     q, k, v = inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled)
     q, k, v = (inputs.round_bf16(x) for x in (q, k, v))
     got = _run(q, k, v, causal, "bf16")
-    heads = [(0, 0), (3, 7), (7, 15)]
-    rows = _sample_rows(w.n, 64, 1)
+    assert np.all(np.isfinite(got))
+    b, h = 3, 7
+    whole = oracle.forward(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], causal)
+    assert max_row_rel_err(got[b:b + 1, h:h + 1], whole) <= TOL["bf16"]
+    heads = [(0, 0), (7, 15)]
+    rows = _sample_rows(w.n, 64, 1, edge_step=128)
     qs = np.stack([q[b, h] for b, h in heads])
     ks = np.stack([k[b, h] for b, h in heads])
     vs = np.stack([v[b, h] for b, h in heads])
     ref = oracle.forward_rows(qs, ks, vs, rows, causal)
     gs = np.stack([got[b, h][rows] for b, h in heads])
     assert max_row_rel_err(gs, ref) <= TOL["bf16"]
-    assert np.all(np.isfinite(got))
 
 
 def test_workload_longctx_1x32x131072x128_bf16():
+    """Full size, as the benchmark runs it: every row of head 17; on heads 0 and 31 the rows on
+    both sides of every multiple of 256 tokens (every segment edge) plus random rows."""
     w = inputs.WORKLOADS["longctx_1x32x131072x128_bf16"]
     q, k, v = inputs.forward_qkv(w.seed, w.B, w.H, w.n, w.d, w.scaled)
     q, k, v = (inputs.round_bf16(x) for x in (q, k, v))
     got = _run(q, k, v, True, "bf16")
     assert np.all(np.isfinite(got))
-    heads = [0, 17, 31]
-    rows = _sample_rows(w.n, 48, 2)
+    h = 17
+    whole = oracle.forward(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], True)
+    assert max_row_rel_err(got[:, h:h + 1], whole) <= TOL["bf16"]
+    heads = [0, 31]
+    rows = _sample_rows(w.n, 48, 2, edge_step=256)
     ref = oracle.forward_rows(q[0, heads], k[0, heads], v[0, heads], rows, True)
     gs = np.stack([got[0, h][rows] for h in heads])
     assert max_row_rel_err(gs, ref) <= TOL["bf16"]

@@ -1,13 +1,12 @@
-"""linattn_forward_noalloc: the forward pass for callers that cannot allocate memory
-(graph capture with memory fixed up front, hosts that pre-reserve every byte, runtimes
-that own the device allocator).  It must give what linattn_forward gives, call after call,
-with its temporary state in the library's fixed device scratch block.
+"""linattn_forward_noalloc: the forward pass for callers that cannot allocate device memory
+(hosts that reserve all device memory up front, runtimes that own the allocator and forbid
+libraries from calling it).  It must give what linattn_forward gives, call after call, with
+its temporary state in the library's fixed device scratch block, allocate nothing, and
+report a kernel wait that gives up through linattn_device_error like every other entry point.
 
 This file is collected last on purpose: if it fails, a run that stops at the first
 failure has already run every other test.
 """
-import ctypes
-
 import numpy as np
 import pytest
 
@@ -41,10 +40,49 @@ def test_noalloc_matches_forward_on_two_calls(dtype, B, H, n, d, causal):
     for call in range(2):
         out = torch.full_like(qd, float("nan"))
         assert _noalloc(lib, qd, kd, vd, out, causal) == la.LINATTN_OK
-        torch.cuda.synchronize()
+        assert la.device_error() == la.LINATTN_OK, call
         got = to_host(out)
         assert np.all(np.isfinite(got)), call
         assert max_row_rel_err(got, ref) <= TOL[dtype], call
+
+
+def test_noalloc_calls_leave_free_device_memory_unchanged():
+    """After a first call (which looks the block's address up), further calls take no device
+    memory: the driver's count of free memory is the same before and after them."""
+    lib = la.load_library()
+    B, H, n, d = 2, 8, 3000, 128
+    q, k, v = inputs.forward_qkv(18, B, H, n, d, scaled=True)
+    qd, kd, vd = (to_dev(as_io(x, "bf16"), "bf16") for x in (q, k, v))
+    out = torch.empty_like(qd)
+    for causal in (True, False):
+        assert _noalloc(lib, qd, kd, vd, out, causal) == la.LINATTN_OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for causal in (True, False, True):
+        assert _noalloc(lib, qd, kd, vd, out, causal) == la.LINATTN_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert la.device_error() == la.LINATTN_OK
+
+
+def test_noalloc_wait_give_up_is_reported_once():
+    """A bounded wait that gives up writing into the static block's status word is reported by
+    linattn_device_error once (then cleared), and the next call still matches."""
+    lib = la.load_library()
+    st = torch.cuda.current_stream().cuda_stream
+    assert la.device_error() == la.LINATTN_OK
+    assert lib.linattn_selftest_noalloc_wait_timeout(st) == la.LINATTN_OK
+    assert la.device_error() == la.LINATTN_ERR_TIMEOUT
+    assert la.device_error() == la.LINATTN_OK
+    B, H, n, d = 1, 2, 500, 64
+    q, k, v = (as_io(x, "bf16") for x in inputs.forward_qkv(19, B, H, n, d, scaled=True))
+    qd, kd, vd = (to_dev(x, "bf16") for x in (q, k, v))
+    out = torch.empty_like(qd)
+    ref = to_host(la.forward(qd, kd, vd, True))
+    assert _noalloc(lib, qd, kd, vd, out, True) == la.LINATTN_OK
+    assert la.device_error() == la.LINATTN_OK
+    assert max_row_rel_err(to_host(out), ref) <= TOL["bf16"]
 
 
 def test_noalloc_rejects_work_beyond_the_scratch_block():
