@@ -225,14 +225,11 @@ def time_steps(fn, steps, warmup, world, clocks=None):
 def forward_launches(dtype: str, causal: bool, unit: int):
     """Names of the launches of one forward call, in order, and the algorithmic bytes of each
     (unit: the bytes of one [B,H,n,d] tensor)."""
-    if dtype == "bf16" and causal:
-        # the single pass: the look-back flags cleared, then one kernel reads q, k, v and
-        # writes out
-        return (["memset (look-back flags)",
-                 "tc_causal_kernel (single pass: aggregates, look-back, outputs)"], [0, 4 * unit])
     if dtype == "bf16":
-        return (["tc_kernel<state> (segment aggregates, K1)", "scan_states_kernel (totals, K2)",
-                 "tc_kernel<non-causal out> (K3)"], [2 * unit, 0, 2 * unit])
+        return (["tc_kernel<state> (segment aggregates, K1)",
+                 "scan_states_kernel (prefix, K2)" if causal else "scan_states_kernel (totals, K2)",
+                 "tc_kernel<causal out> (K3)" if causal else "tc_kernel<non-causal out> (K3)"],
+                [2 * unit, 0, 4 * unit if causal else 2 * unit])
     return (["simt_chunk_state_kernel (K1)", "scan_states_kernel (K2)",
              "simt_chunk_out_kernel (K3)"], [2 * unit, 0, 4 * unit if causal else 2 * unit])
 

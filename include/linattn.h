@@ -66,10 +66,8 @@ typedef enum {
  *             1 = query i sees keys j <= i (the recurrent view's running state).
  * Any n >= 1 is accepted.  Accumulation is fp32; the output is rounded once to `dtype`
  * (bf16: round to nearest even).  The causal mode runs as chunked prefix sums of (S, z):
- * with bf16 I/O in one pass, where each segment of a head publishes its aggregate state and
- * takes its prefix from the segments before it (a look-back); with fp32 I/O as per-chunk
- * aggregates, their scan, and the outputs.  Returns LINATTN_OK after enqueuing the work on
- * `stream`.
+ * per-segment aggregates, their exclusive scan, then the outputs of every segment from its
+ * prefix.  Returns LINATTN_OK after enqueuing the work on `stream`.
  */
 linattn_status linattn_forward(const void *q, const void *k, const void *v, void *out,
                                int64_t B, int64_t H, int64_t n, int64_t d, int causal,

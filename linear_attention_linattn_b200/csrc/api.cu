@@ -133,7 +133,7 @@ ForwardPlan plan_forward(int64_t heads, int64_t n, int dk, int d, int causal, in
   ForwardPlan p;
   if (is_bf16) {
     p.seg = seg_len > 0 ? seg_len
-                        : (causal ? tc_fused_segment(heads, n, dk, d) : tc_default_segment(heads, n, d));
+                        : tc_default_segment(heads, n, d);
     p.ws_bytes = tc_workspace_bytes(heads, n, dk, d, p.seg, causal);
     return p;
   }
@@ -210,7 +210,7 @@ linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, v
                                   linattn_stream_t stream) {
   linattn_status s = check_forward_args(q, k, v, out, B, H, n, d, causal, dtype);
   if (s != LINATTN_OK) return s;
-  if (segment_len < 0 || segment_len % kTcCausalChunk != 0) return LINATTN_ERR_INVALID_ARG;
+  if (segment_len < 0 || segment_len % kTcFeatureChunk != 0) return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   return forward_pooled(q, k, v, out, B * H, n, (int)d, (int)d, causal, dtype == LINATTN_BF16,

@@ -54,11 +54,6 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// `count` arrivals at once
-__device__ __forceinline__ void mbar_arrive_cnt(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
@@ -118,34 +113,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, 
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       atomicOr(err, kErrTimeout);
       return false;
-    }
-  }
-}
-
-// ------------------------------------------------------------------ flags in global memory
-__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_gpu(int *p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Waits until *p != 0 (another CTA's release store) and returns it.  Gives up after
-// kWaitLimitNs (or at once when *abort is set), sets *abort and the error word, returns 0.
-__device__ __forceinline__ int spin_flag(const int *p, volatile int *abort, int *err) {
-  int v = ld_acquire_gpu(p);
-  if (v != 0) return v;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (*abort) return 0;
-    __nanosleep(200);
-    v = ld_acquire_gpu(p);
-    if (v != 0) return v;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      atomicOr(err, kErrTimeout);
-      return 0;
     }
   }
 }
@@ -300,13 +267,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
       : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
-                   taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-               "r"(r[7])
-               : "memory");
 }
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r)

@@ -96,27 +96,18 @@ cudaError_t launch_decode_step(float *S, float *z, const void *q, const void *k,
 // ---- bf16 I/O, tensor cores (tc_forward.cu, tc_causal.cu) ---------------------------------
 // Chunk length of the tensor-core aggregate and non-causal kernels.
 constexpr int kTcChunk = 64;
-// Chunk length of the tensor-core causal output kernel; segments are multiples of it.
-constexpr int kTcCausalChunk = 128;
-// Causal outputs from the exclusive prefix state of every segment (prefix: [heads][segments]
-// [dk*dv + dk] fp32, S row-major then z).  q, k: [heads][n][dk]; v, out: [heads][n][dv];
-// dk = dv unless features != 0 (q and k are then non-negative features already).
-// seg: a multiple of kTcCausalChunk.
-cudaError_t tc_causal_out(const void *q, const void *k, const void *v, void *out, int64_t heads,
-                          int64_t n, int dk, int dv, int64_t seg, const float *prefix,
-                          int features, int *err, cudaStream_t st);
-// The causal pass in one kernel (each segment's aggregate, a look-back over the published
-// states of the earlier segments, then its outputs).  ws: tc_fused_workspace_bytes.
-// init_S [heads][dk][dv], init_z [heads][dk] (nullable): the state before each head's first
-// token.
-int64_t tc_fused_segment(int64_t heads, int64_t n, int dk, int dv);
-size_t tc_fused_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg);
-cudaError_t tc_causal_fused(const void *q, const void *k, const void *v, void *out,
-                            int64_t heads, int64_t n, int dk, int dv, int64_t seg, void *ws,
-                            const float *init_S, const float *init_z, int features, int *err,
-                            cudaStream_t st);
-// Default tokens per work item (segment) of the tensor-core path: the aggregate and
-// non-causal kernels (causal: tc_fused_segment).
+// Chunk length of the causal kernel on features of their own dimension (tc_causal.cu);
+// segments are multiples of it.
+constexpr int kTcFeatureChunk = 128;
+// Causal outputs on features whose dimension dk differs from the value dimension dv, from the
+// exclusive prefix state of every segment (prefix: [heads][segments][dk*dv + dk] fp32, S
+// row-major then z).  q, k: [heads][n][dk] features; v, out: [heads][n][dv].  seg: a multiple
+// of kTcFeatureChunk.
+cudaError_t tc_causal_features(const void *q, const void *k, const void *v, void *out,
+                               int64_t heads, int64_t n, int dk, int dv, int64_t seg,
+                               const float *prefix, int *err, cudaStream_t st);
+// Default tokens per work item (segment) of the tensor-core path (a multiple of 256, or the
+// whole head rounded up to kTcFeatureChunk).
 int64_t tc_default_segment(int64_t heads, int64_t n, int d);
 // Workspace bytes the tensor-core forward needs.
 size_t tc_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg, int causal);

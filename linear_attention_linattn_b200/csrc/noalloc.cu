@@ -97,16 +97,13 @@ extern "C" linattn_status linattn_forward_noalloc(const void *q, const void *k, 
   const size_t cap = kScratchBytes - kStatusBytes;
   ForwardPlan p = plan_forward(heads, n, di, di, causal, is_bf16, 0);
   if (p.ws_bytes > cap && is_bf16) {
-    // the tensor-core path: lengthen the segments until the per-segment states fit (causal:
-    // an aggregate, an inclusive state and a flag per segment; non-causal: one state per
-    // segment and a total per head)
+    // the tensor-core path: lengthen the segments until one state per segment (and, non-causal,
+    // a total per head) fits
     const int64_t per = (int64_t)(d * d + d) * (int64_t)sizeof(float);  // one (S, z) state
-    const int64_t per_seg = causal ? 2 * per + (int64_t)sizeof(int) : per;
-    const int64_t avail = (int64_t)cap - (causal ? 16 : heads * per);
-    const int64_t nseg_max = avail > 0 ? avail / per_seg / heads : 0;
+    const int64_t nseg_max = (int64_t)(cap / per) / heads - (causal ? 0 : 1);
     if (nseg_max < 1) return LINATTN_ERR_INVALID_ARG;
     const int64_t seg =
-        ((n + nseg_max - 1) / nseg_max + kTcCausalChunk - 1) / kTcCausalChunk * kTcCausalChunk;
+        ((n + nseg_max - 1) / nseg_max + kTcFeatureChunk - 1) / kTcFeatureChunk * kTcFeatureChunk;
     p = plan_forward(heads, n, di, di, causal, is_bf16, seg);
   }
   if (p.ws_bytes > cap) return LINATTN_ERR_INVALID_ARG;
