@@ -153,21 +153,38 @@ linattn_status linattn_forward_features(const void *phi_q, const void *phi_k, co
 /*
  * Backward pass: the gradients of a loss L with respect to q, k and v, given
  * dout = dL/dout for out = linattn_forward(q, k, v, causal).  All seven tensors are
- * [B][H][n][d] of type `dtype` (dq, dk, dv written in that type); accumulation is float32
- * on the CUDA cores.  The pages define the forward only; this is its chain rule: with
+ * [B][H][n][d] of type `dtype` (dq, dk, dv written in that type).  bf16: the products run
+ * on the tensor cores (bf16 operands, float32 accumulation), the rank-one terms on the CUDA
+ * cores in float32; float32: everything on the CUDA cores in float32.  The pages define the
+ * forward only ("Linear Attention > Memory Efficiency" notes that training keeps the forward's
+ * tensors for backpropagation); this is its chain rule: with
  * w_ij = phi(q_i).phi(k_j), den_i = sum_j w_ij and a_i = dout_i / den_i,
  * b_i = -(dout_i . out_i) / den_i,
  *     dL/dphi(q_i) = sum_j (v_j . a_i + b_i) phi(k_j),
  *     dL/dphi(k_j) = sum_i (v_j . a_i + b_i) phi(q_i),
  *     dL/dv_j      = sum_i w_ij a_i,
  * then through phi'(x) = 1 (x > 0), exp(x) (x <= 0); sums over j <= i (causal) or all.
- * Asynchronous on `stream`; takes a stream-ordered workspace of about
- * 2 (n/64) (d^2 + d) + n (d + 1) floats per head.  Errors as in linattn_forward.
+ * Asynchronous on `stream`; takes a stream-ordered workspace: per head, bf16: two records
+ * (d^2 + 3d + 4 floats) per segment of up to 4096 tokens plus n (d + 1) floats; float32:
+ * 2 (n/64) (d^2 + d) + n (d + 1) floats.  Errors as in linattn_forward; a bounded wait that
+ * gave up is reported by linattn_device_error.
  */
 linattn_status linattn_backward(const void *q, const void *k, const void *v, const void *dout,
                                 void *dq, void *dk, void *dv, int64_t B, int64_t H, int64_t n,
                                 int64_t d, int causal, linattn_dtype dtype,
                                 linattn_stream_t stream);
+
+/*
+ * linattn_backward with a chosen segment length for bf16 (the tokens of one work item of
+ * the two chunked walks: a multiple of 64; 0 picks the default; ignored for float32).  The
+ * result does not depend on it beyond rounding order; tests use it to move the segment
+ * boundaries.  Other arguments as in linattn_backward.
+ */
+linattn_status linattn_backward_ex(const void *q, const void *k, const void *v,
+                                   const void *dout, void *dq, void *dk, void *dv, int64_t B,
+                                   int64_t H, int64_t n, int64_t d, int causal,
+                                   linattn_dtype dtype, int64_t segment_len,
+                                   linattn_stream_t stream);
 
 /*
  * Per-head sum of gathered states.  states: float32 device memory laid out

@@ -58,6 +58,8 @@ SIGNATURES = {
     "linattn_sum_states": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
     "linattn_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                         _i64, ctypes.c_int, ctypes.c_int, _vp]),
+    "linattn_backward_ex": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                           _i64, _i64, ctypes.c_int, ctypes.c_int, _i64, _vp]),
     "linattn_favor_features": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int,
                                               _vp]),
     "linattn_selftest_wait_timeout": (ctypes.c_int, [_vp]),
@@ -244,9 +246,10 @@ def forward_favor(q, k, v, W, causal: bool, stream=None):
                             v, causal, stream=stream)
 
 
-def backward(q, k, v, dout, causal: bool, stream=None):
+def backward(q, k, v, dout, causal: bool, segment_len: int = 0, stream=None):
     """Gradients (dq, dk, dv) of a loss given dout = dL/dout for out = forward(q, k, v, causal);
-    all [B, H, n, d] CUDA tensors of one dtype (float32 or bfloat16)."""
+    all [B, H, n, d] CUDA tensors of one dtype (float32 or bfloat16).  segment_len (bf16, a
+    multiple of 64; 0 = default) sets the tokens of one work item."""
     import torch
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
         _dev(t, nm)
@@ -256,9 +259,10 @@ def backward(q, k, v, dout, causal: bool, stream=None):
     B, H, n, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     lib = load_library()
-    st = lib.linattn_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
-                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, n, d,
-                              int(bool(causal)), _dtype_code(q), _stream_ptr(stream))
+    st = lib.linattn_backward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, n, d,
+                                 int(bool(causal)), _dtype_code(q), int(segment_len),
+                                 _stream_ptr(stream))
     _check(st, "linattn_backward")
     return dq, dk, dv
 

@@ -267,8 +267,17 @@ linattn_status linattn_backward(const void *q, const void *k, const void *v, con
                                 void *dq, void *dk, void *dv, int64_t B, int64_t H, int64_t n,
                                 int64_t d, int causal, linattn_dtype dtype,
                                 linattn_stream_t stream) {
+  return linattn_backward_ex(q, k, v, dout, dq, dk, dv, B, H, n, d, causal, dtype, 0, stream);
+}
+
+linattn_status linattn_backward_ex(const void *q, const void *k, const void *v,
+                                   const void *dout, void *dq, void *dk, void *dv, int64_t B,
+                                   int64_t H, int64_t n, int64_t d, int causal,
+                                   linattn_dtype dtype, int64_t segment_len,
+                                   linattn_stream_t stream) {
   linattn_status s = check_forward_args(q, k, v, dout, B, H, n, d, causal, dtype);
   if (s != LINATTN_OK) return s;
+  if (segment_len < 0 || segment_len % kTcChunk != 0) return LINATTN_ERR_INVALID_ARG;
   if (!dq || !dk || !dv || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return LINATTN_ERR_INVALID_ARG;
   DeviceState *ds = nullptr;
@@ -277,11 +286,20 @@ linattn_status linattn_backward(const void *q, const void *k, const void *v, con
   const int64_t heads = B * H;
   Workspace ws;
   ws.st = st;
+  if (dtype == LINATTN_BF16) {  // tensor cores
+    const int64_t seg = segment_len > 0 ? segment_len : tc_backward_segment(heads, n, (int)d);
+    size_t bytes = 0;
+    tc_backward_layout(nullptr, heads, n, (int)d, seg, &bytes);
+    if (cudaMallocFromPoolAsync(&ws.ptr, bytes, ds->pool, st) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
+    return to_status(tc_backward(q, k, v, dout, dq, dk, dv, heads, n, (int)d, causal, seg,
+                                 ws.ptr, ds->err_word, st));
+  }
   const size_t bytes = backward_workspace_floats(heads, n, (int)d, causal) * sizeof(float);
   if (cudaMallocFromPoolAsync(&ws.ptr, bytes, ds->pool, st) != cudaSuccess)
     return LINATTN_ERR_CUDA;
-  return to_status(backward(q, k, v, dout, dq, dk, dv, heads, n, (int)d, causal,
-                            dtype == LINATTN_BF16, static_cast<float *>(ws.ptr), st));
+  return to_status(backward(q, k, v, dout, dq, dk, dv, heads, n, (int)d, causal, 0,
+                            static_cast<float *>(ws.ptr), st));
 }
 
 linattn_status linattn_sum_states(const float *states, int64_t count, int64_t skip, int64_t B,

@@ -117,6 +117,18 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, 
   }
 }
 
+// ------------------------------------------------------------------ programmatic launch
+// A kernel launched with programmatic stream serialization may start while the kernel before
+// it on the stream is finishing; it must pass grid_dependency_wait() before reading anything
+// that kernel writes.  grid_dependency_launch() lets the next such kernel start early.
+// Both are no-ops for a kernel launched the ordinary way.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

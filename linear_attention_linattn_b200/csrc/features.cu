@@ -152,6 +152,7 @@ template <int D, int M>
 __global__ void __launch_bounds__(kFThreads, 1)
     favor_tc_kernel(const __grid_constant__ CUtensorMap tmX, const float *__restrict__ W,
                     __nv_bfloat16 *__restrict__ out, int64_t rows, int *err) {
+  const bool a32 = aligned32(out);  // output rows take full-sector stores
   using G = FCfg<D, M>;
   constexpr int KS = D / 16;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
             float f[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) f[e] = expf(__uint_as_float(v[16 * q + e]) - half_sq) * scale;
-            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8));
+            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8), a32);
           }
         }
       }

@@ -1,6 +1,7 @@
 // Host-side declarations shared by the C-ABI layer and the kernel files.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -8,6 +9,25 @@
 #include "linattn.h"
 
 namespace linattn {
+
+// Launches `kern` on `st` with programmatic stream serialization: it may start while the
+// previous kernel on the stream finishes (it must call grid_dependency_wait() before reading
+// that kernel's results), so its set-up and its first loads of the inputs overlap that tail.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_programmatic(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t st, Args &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 // ---- forward dispatch shared by the entry points (api.cu) ---------------------------------
 // Checks shared by every forward entry point: pointers (non-null, 16-byte aligned), the causal
@@ -82,7 +102,7 @@ cudaError_t launch_simt_chunk_out(const void *q, const void *k, const void *v, v
 cudaError_t launch_favor_features(const void *x, const float *W, void *out, int64_t rows, int d,
                                   int m, int is_bf16, int *err, cudaStream_t st);
 
-// ---- backward pass (backward.cu), CUDA cores; is_bf16 selects bf16 I/O, else fp32 ------
+// ---- backward pass with fp32 I/O (backward.cu), CUDA cores; is_bf16 selects bf16 I/O ------
 // Workspace floats linattn_backward needs.
 size_t backward_workspace_floats(int64_t heads, int64_t n, int d, int causal);
 cudaError_t backward(const void *q, const void *k, const void *v, const void *g, void *dq,
@@ -121,5 +141,28 @@ cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, i
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
                              int64_t heads, int64_t n, int d, int64_t seg, void *ws, int *err,
                              cudaStream_t st);
+// Segment aggregates [S | z] = sum phi(k)^T [v | 1] of k, v: [heads][n][d] bf16 into
+// out: [heads][ceil(n / seg)][d*d + d] fp32 (one launch; seg a multiple of kTcChunk).
+cudaError_t tc_segment_aggregates(const void *k, const void *v, int64_t heads, int64_t n, int d,
+                                  int64_t seg, float *out, int *err, cudaStream_t st);
+
+// ---- bf16 I/O backward on the tensor cores (tc_backward.cu) --------------------------------
+struct TcBackwardLayout {
+  // [heads][segments][d*d + 3d + 4]: the forward records [Psi | zeta | vs | sigma | kappa] and
+  // the reverse records [Phi | rho | as | tau | bs] of the segments (tc_backward.cu)
+  float *s_rec, *r_rec;
+  float *s_tot, *r_tot;           // [heads][d*d + 3d + 4]: per-head totals (non-causal)
+  __nv_bfloat16 *a_hi, *a_lo;     // [heads][n][d]: a_i = g_i / den_i as a bf16 pair
+  float *b;                       // [heads][n]: -(a_i . out_i)
+};
+// Tokens per work item of the backward (a multiple of 256, or n rounded up to kTcChunk).
+int64_t tc_backward_segment(int64_t heads, int64_t n, int d);
+// The workspace's parts at ws (null: sizes only); *bytes = the workspace size.
+TcBackwardLayout tc_backward_layout(void *ws, int64_t heads, int64_t n, int d, int64_t seg,
+                                    size_t *bytes);
+// q, k, v, g, dq, dk, dv: [heads][n][d] bf16, d in {64, 128}.
+cudaError_t tc_backward(const void *q, const void *k, const void *v, const void *g, void *dq,
+                        void *dk, void *dv, int64_t heads, int64_t n, int d, int causal,
+                        int64_t seg, void *ws, int *err, cudaStream_t st);
 
 }  // namespace linattn

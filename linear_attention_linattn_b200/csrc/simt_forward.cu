@@ -120,6 +120,10 @@ __global__ void __launch_bounds__(256) scan_states_kernel(float *__restrict__ ws
                                                           float *__restrict__ z_out, int64_t z_hs,
                                                           const float *__restrict__ init_S,
                                                           const float *__restrict__ init_z) {
+  // launched programmatically: the next kernel may start now; this one reads the aggregates
+  // of the kernel before it only once that kernel has finished
+  grid_dependency_launch();
+  grid_dependency_wait();
   const int64_t per4 = ((int64_t)dk * dv + dk) / 4;
   const int64_t blocks_per_head = (per4 + blockDim.x - 1) / blockDim.x;
   const int64_t head = blockIdx.x / blocks_per_head;
@@ -359,8 +363,11 @@ cudaError_t launch_scan_states(float *ws, int64_t heads, int64_t nseg, int dk, i
                                float *S_out, int64_t S_hs, float *z_out, int64_t z_hs,
                                const float *init_S, const float *init_z, cudaStream_t st) {
   const int64_t per4 = ((int64_t)dk * dv + dk) / 4;
-  scan_states_kernel<<<(unsigned)(((per4 + 255) / 256) * heads), 256, 0, st>>>(
-      ws, nseg, dk, dv, mode, S_out, S_hs, z_out, z_hs, init_S, init_z);
+  cudaError_t e = launch_programmatic(scan_states_kernel,
+                                      dim3((unsigned)(((per4 + 255) / 256) * heads)), dim3(256), 0,
+                                      st, ws, nseg, dk, dv, mode, S_out, S_hs, z_out, z_hs, init_S,
+                                      init_z);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();

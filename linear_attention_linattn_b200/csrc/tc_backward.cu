@@ -1,0 +1,1397 @@
+// Backward pass with bf16 I/O on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// The pages define the forward only ("Efficient Transformers: Linear Attention and Flash
+// Attention", sections "Linear attention: reordering the matmuls, not shrinking them" and "The
+// recurrent view: attention as an RNN"; "Linear Attention", section "Memory Efficiency", notes
+// that training keeps the forward's tensors for backpropagation).  Its gradients follow by the
+// chain rule.  Per head, with w_ij = phi(q_i).phi(k_j) (j <= i when causal), den_i = sum_j w_ij,
+// out_i = sum_j w_ij v_j / den_i and g = dL/dout:
+//
+//   a_i = g_i / den_i,   b_i = -(a_i . out_i),   dW_ij = a_i . v_j + b_i
+//   dphi(q_i) = sum_j dW_ij phi(k_j),   dphi(k_j) = sum_i dW_ij phi(q_i),   dv_j = sum_i w_ij a_i
+//   dq = dphi(q) * phi'(q),  dk = dphi(k) * phi'(k),  phi'(x) = 1 above zero, exp(x) below.
+//
+// Precision.  With inputs of the usual scale phi(x) = 1 + psi(x) is 1 plus a small psi
+// (psi = elu: x above zero, exp(x) - 1 below), so w_ij is d plus a small varying part and the
+// gradients live in that part: rounded to bf16, phi itself would keep only a few bits of it.
+// So every tensor-core operand here is a psi quantity (small, kept to bf16's relative
+// precision) and the 1's are summed analytically in fp32 on the CUDA cores.  With
+// sq_i = sum_r psi(q_i)_r and sk_j likewise,
+//   w_ij = d + sq_i + sk_j + psi(q_i).psi(k_j)
+//   dphi(q_i) = C_i 1 + [ sum_j dW_ij psi(k_j) ],   C_i  = sum_j dW_ij
+//   dphi(k_j) = C'_j 1 + [ sum_i dW_ij psi(q_i) ],  C'_j = sum_i dW_ij
+// where C_i and C'_j, sums of terms that nearly cancel, are taken in fp32 from the exact a.
+// a itself enters the products as a bf16 pair (hi + lo), which keeps it to about 16 bits.
+//
+// The pass, per head; causal sums run over the chunks before (prefix) or after (suffix):
+//   K1  per segment, the forward record [Psi | zeta | vs | sigma | kappa] of the keys:
+//       Psi = sum psi(k_j) v_j^T, zeta = sum psi(k_j), vs = sum v_j, sigma = sum sk_j v_j,
+//       kappa = sum sk_j
+//   K2  its exclusive prefix over segments (causal) or the head's total
+//   B1  prefix walk: per segment, chunks in order, Psi in TMEM: den, out, a, b, dq; a (hi, lo)
+//       and b to the workspace; the segment's reverse record [Phi | rho | as | tau | bs]:
+//       Phi = sum psi(q_i) a_i^T, rho = sum psi(q_i) b_i, as = sum a_i, tau = sum sq_i a_i,
+//       bs = sum b_i
+//   K2  its exclusive suffix (causal) or the head's total
+//   B3  suffix walk: per segment, chunks in reverse order, Phi in TMEM: dk, dv
+//
+// Products of one 64-token chunk (tcgen05.mma kind::f16, bf16 operands, fp32 in TMEM):
+//   B1  P' = psi(Q) psi(K)^T;  Psi += psi(K)^T V;  LV = L V (L: the lower triangle of ones);
+//       O' = psi(Q) Psi + M V with M = mask(P' + sk);  dW = A V^T;  dQ' = A Psi^T + mask(dW + b)
+//       psi(K);  Phi += psi(Q)^T A  (A = [a_hi; a_lo] along the contraction)
+//   B3  P'^T = psi(K) psi(Q)^T;  dW^T = V A^T;  Phi += psi(Q)^T A;  dV' = psi(K) Phi +
+//       mask(w^T) A_hi;  dK' = V Phi^T + mask(dW^T + b) psi(Q)
+// and the fp32 rest, e.g. den_i = N_i (d + sq_i) + kappa + psi(q_i).zeta + rowsum(M)_i and
+// out_i = ((d + sq_i)(vs + LV_i) + sigma + O'_i) / den_i, N_i the keys row i sees.
+//
+// Each CTA runs 8 warps through a chunk's phases in step (warps w and w + 4 share TMEM
+// sub-partition w & 3 and split the columns), thread 0 issuing the TMA loads (one chunk ahead,
+// two stages) and the MMAs.  Two CTAs share an SM at d = 64, so one CTA's products run while
+// the other drains its accumulators.  Every wait is bounded (2 s); a CTA whose wait gave up lets
+// its copies and products land and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace linattn {
+namespace {
+
+using namespace tc;
+
+constexpr int C = kTcChunk;     // tokens per chunk (64)
+constexpr int kAtom = C * 128;  // one [64 rows][64 bf16] 128B-swizzled atom: 8 KB
+constexpr int kThreads = 256;   // 8 warps, two per TMEM sub-partition
+
+// A state record: [M (D x D, row-major) | three D-vectors | a scalar, three zeros].
+template <int D>
+__host__ __device__ constexpr int64_t rec_floats() {
+  return (int64_t)D * D + 3 * D + 4;
+}
+
+struct BwdShared {
+  uint64_t full[2];      // stage loaded (TMA transaction bytes)
+  uint64_t mma;          // the products issued since the last wait are done
+  uint64_t fin;          // drain at exit
+  float vec[3][128];     // the record's three vectors (current state)
+  float scal;            // the record's scalar
+  float sq[64], sk[64];  // row sums of psi(Q), psi(K) of the chunk
+  float part[2][64];     // per column half, per row: partial sums
+  float gd[2][64];
+  float cd[2][64];
+  float bv[64];          // b of the chunk's rows
+  float acc[3][128];     // column sums being gathered (atomically) for a chunk or an item
+  float racc[3][128];    // the prefix walk: the item's reverse-record vectors
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+struct BCfg {
+  static constexpr int AT = D / 64;        // 64-column atoms per [64][D] tile
+  static constexpr int TILE = AT * kAtom;  // one bf16 [64][D] tile
+  static constexpr int S_ATOM = D * 128;   // [D rows][64 columns] block of a D x D operand
+  static constexpr int STATE = AT * S_ATOM;
+  // prefix walk: stages of Q, G, K, V; the Psi operand; A hi, A lo; the M / dW operand; L
+  static constexpr int P_STAGE = 4 * TILE;
+  static constexpr int P_ST = 2 * P_STAGE;
+  static constexpr int P_A = P_ST + STATE;
+  static constexpr int P_AL = P_A + TILE;
+  static constexpr int P_W = P_AL + TILE;
+  static constexpr int P_L = P_W + kAtom;
+  static constexpr int P_SH = P_L + kAtom;
+  // suffix walk: stages of Q, A hi, A lo, K, V; the Phi operand; two [64][64] operands
+  static constexpr int S_STAGE = 5 * TILE;
+  static constexpr int S_ST = 2 * S_STAGE;
+  static constexpr int S_W0 = S_ST + STATE;
+  static constexpr int S_W1 = S_W0 + kAtom;
+  static constexpr int S_SH = S_W1 + kAtom;
+  // aggregate: stages of K, V
+  static constexpr int G_STAGE = 2 * TILE;
+  static constexpr int G_SH = 2 * G_STAGE;
+  static constexpr int SLACK = 1024;  // alignment of the dynamic shared memory base
+  static constexpr int P_SMEM = P_SH + (int)sizeof(BwdShared) + SLACK;
+  static constexpr int S_SMEM = S_SH + (int)sizeof(BwdShared) + SLACK;
+  static constexpr int G_SMEM = G_SH + (int)sizeof(BwdShared) + SLACK;
+  static constexpr uint32_t TCOLS = D == 64 ? 256 : 512;  // the walks' TMEM
+  static constexpr int CTAS = D == 64 ? 2 : 1;            // walk CTAs per SM
+  static constexpr int G_CTAS = D == 64 ? 4 : 2;          // aggregate CTAs per SM
+  static constexpr int kSmPerSm = 228 * 1024;             // an SM's shared memory
+  static_assert(P_SMEM <= kMaxSmem && S_SMEM <= kMaxSmem, "shared memory");
+  static_assert(CTAS * (P_SMEM + 1024) <= kSmPerSm && CTAS * (S_SMEM + 1024) <= kSmPerSm,
+                "CTAS walk CTAs fit on an SM");
+  static_assert(D == 128 || (3 * (P_SMEM + 1024) > kSmPerSm && 3 * (S_SMEM + 1024) > kSmPerSm),
+                "at most two walk CTAs per SM share its TMEM");
+  static_assert(P_ST % 1024 == 0 && P_A % 1024 == 0 && P_AL % 1024 == 0 && P_W % 1024 == 0 &&
+                    P_L % 1024 == 0 && S_ST % 1024 == 0 && S_W0 % 1024 == 0 &&
+                    S_W1 % 1024 == 0,
+                "128B-swizzled operands need 1024-byte alignment");
+};
+
+// ---------------------------------------------------------------- shared helpers
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tmem_row32(uint32_t taddr, float *f) {
+  uint32_t r[32];
+  tmem_ld16_async(taddr, r);
+  tmem_ld16_async(taddr + 16, r + 16);
+  tmem_ld_wait();
+  tmem_reg_fence<32>(r);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(r[e]);
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float *f) {
+  f[0] = bf16_lo(u.x);
+  f[1] = bf16_hi(u.x);
+  f[2] = bf16_lo(u.y);
+  f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z);
+  f[5] = bf16_hi(u.z);
+  f[6] = bf16_lo(u.w);
+  f[7] = bf16_hi(u.w);
+}
+// Byte offset of (row, col) in a token tile of 64-column atoms (col a multiple of 8 for
+// 16-byte accesses).
+__device__ __forceinline__ uint32_t tile_off(int row, int col) {
+  return (col >> 6) * kAtom + sw128_offset(row, col & 63);
+}
+__device__ __forceinline__ void tile_row8(const uint8_t *tile, int row, int col, float *f) {
+  unpack8(*reinterpret_cast<const uint4 *>(tile + tile_off(row, col)), f);
+}
+// phi'(x) from psi(x) = phi(x) - 1: 1 above zero, exp(x) = 1 + psi(x) at or below.
+__device__ __forceinline__ float dphi_from_psi(float p) { return p > 0.f ? 1.f : 1.f + p; }
+
+// psi in place on the 64 rows of a [64][D] token tile, in fp32 and rounded to bf16; rows at or
+// after `keep` zeroed.  rowsum (if not null) receives each row's sum of the rounded values.
+// Thread t takes rows t / 8 and 32 + t / 8 (16-byte chunk t % 8 of each atom), so the 8
+// threads of a row are 8 consecutive lanes.
+template <int D>
+__device__ __forceinline__ void psi_tile(uint8_t *tile, int keep, float *rowsum) {
+  uint4 *p = reinterpret_cast<uint4 *>(tile);
+  float s[2] = {0.f, 0.f};
+#pragma unroll
+  for (int m = 0; m < 2 * (D / 64); ++m) {
+    const int i = threadIdx.x + kThreads * m;
+    const int row = (i % (kAtom / 16)) >> 3;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (row < keep) {
+      float f[8];
+      unpack8(p[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = f[e] > 0.f ? f[e] : __expf(f[e]) - 1.f;
+      x = pack8(f);
+      unpack8(x, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[m & 1] += f[e];
+    }
+    p[i] = x;
+  }
+  if (rowsum != nullptr) {
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      s[0] += __shfl_xor_sync(0xffffffffu, s[0], o);
+      s[1] += __shfl_xor_sync(0xffffffffu, s[1], o);
+    }
+    if ((threadIdx.x & 7) == 0) {
+      rowsum[threadIdx.x >> 3] = s[0];
+      rowsum[32 + (threadIdx.x >> 3)] = s[1];
+    }
+  }
+}
+
+// Rows at or after `keep` of a [64][D] token tile zeroed.
+template <int D>
+__device__ __forceinline__ void zero_rows(uint8_t *tile, int keep) {
+  if (keep >= C) return;
+  uint4 *p = reinterpret_cast<uint4 *>(tile);
+#pragma unroll
+  for (int m = 0; m < 2 * (D / 64); ++m) {
+    const int i = threadIdx.x + kThreads * m;
+    if (((i % (kAtom / 16)) >> 3) >= keep) p[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Per-thread roles: warps w and w + 4 read TMEM sub-partition w & 3; the first four take the
+// low half of every accumulator's columns, the others the high half.
+struct Lanes {
+  int warp, lane, sp, hf;
+  uint32_t lane_off;  // TMEM lane field of this warp's sub-partition
+  bool v64;           // lane holds a row of an M = 64 accumulator (lanes 0..15)
+  int r64;            // that row (token within the chunk)
+  int rS;             // row of a D x D accumulator
+  bool vS;
+  template <int D>
+  __device__ __forceinline__ static Lanes make() {
+    Lanes L;
+    L.warp = threadIdx.x >> 5;
+    L.lane = threadIdx.x & 31;
+    L.sp = L.warp & 3;
+    L.hf = L.warp >> 2;
+    L.lane_off = static_cast<uint32_t>(32 * L.sp) << 16;
+    L.v64 = L.lane < 16;
+    L.r64 = 16 * L.sp + L.lane;
+    L.rS = D == 128 ? 32 * L.sp + L.lane : L.r64;
+    L.vS = D == 128 || L.v64;
+    return L;
+  }
+};
+
+// A record from global memory: M into the bf16 operand (and, when to_tmem, TMEM at tM), the
+// three vectors into sh.vec, the scalar into sh.scal.  Rows rS, this half's columns of M.
+template <int D>
+__device__ __forceinline__ void load_record(const float *src, uint8_t *sOp, uint32_t tM,
+                                            bool to_tmem, const Lanes &L, BwdShared &sh) {
+  constexpr int HD = D / 2;
+#pragma unroll 1
+  for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+    uint32_t r[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (L.vS) f = *reinterpret_cast<const float4 *>(src + (int64_t)L.rS * D + c0 + 4 * q);
+      r[4 * q + 0] = __float_as_uint(f.x);
+      r[4 * q + 1] = __float_as_uint(f.y);
+      r[4 * q + 2] = __float_as_uint(f.z);
+      r[4 * q + 3] = __float_as_uint(f.w);
+    }
+    if (to_tmem) {
+      tmem_st16(tM + c0, *reinterpret_cast<const uint32_t(*)[16]>(r));
+      tmem_st16(tM + c0 + 16, *reinterpret_cast<const uint32_t(*)[16]>(r + 16));
+    }
+    if (L.vS) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[8 * q + e]);
+        *reinterpret_cast<uint4 *>(sOp + (c0 >> 6) * (D * 128) +
+                                   sw128_offset(L.rS, (c0 & 63) + 8 * q)) = pack8(f);
+      }
+    }
+  }
+  if (to_tmem) tmem_st_wait();
+  if (threadIdx.x < D) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) sh.vec[k][threadIdx.x] = src[(int64_t)D * D + k * D + threadIdx.x];
+  }
+  if (threadIdx.x == 0) sh.scal = src[(int64_t)D * D + 3 * D];
+}
+
+// TMEM state (rows rS, this half's columns) -> its bf16 operand (warp-collective loads).
+template <int D>
+__device__ __forceinline__ void state_to_operand(uint32_t tM, uint8_t *sOp, const Lanes &L) {
+  constexpr int HD = D / 2;
+#pragma unroll 1
+  for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+    float f[32];
+    tmem_row32(tM + c0, f);
+    if (L.vS) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(sOp + (c0 >> 6) * (D * 128) +
+                                   sw128_offset(L.rS, (c0 & 63) + 8 * q)) = pack8(f + 8 * q);
+    }
+  }
+}
+
+// TMEM state (rows rS, this half's columns) -> fp32 row-major D x D at dst.
+template <int D>
+__device__ __forceinline__ void state_to_global(uint32_t tM, float *dst, const Lanes &L) {
+  constexpr int HD = D / 2;
+#pragma unroll 1
+  for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+    float f[32];
+    tmem_row32(tM + c0, f);
+    if (L.vS) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4 *>(dst + (int64_t)L.rS * D + c0 + e) =
+            make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+    }
+  }
+}
+
+// Adds to acc[0..2][col] the column sums over the chunk's 64 rows of three per-row terms:
+// terms(i, c, t) adds row i's terms for columns [c, c + 8) into t[0..2][0..7].  Warp w owns
+// D / 64 groups of 8 columns; the lanes of a group split its rows and then reduce-scatter their
+// 8 partial sums (each halving step sends half of them to the partner lane), so that every
+// column's total ends in one lane, which adds it to acc: no two lanes write the same column.
+template <int D, typename F>
+__device__ __forceinline__ void column_sums3(float (*acc)[128], F &&terms) {
+  constexpr int CPW = D / 64;    // column groups per warp
+  constexpr int LPG = 32 / CPW;  // lanes per column group
+  constexpr int RPL = C / LPG;   // rows per lane
+  const int lane = threadIdx.x & 31;
+  const int cg = (threadIdx.x >> 5) * CPW + lane / LPG;
+  float t[3][8];
+#pragma unroll
+  for (int k = 0; k < 3; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[k][e] = 0.f;
+#pragma unroll
+  for (int m = 0; m < RPL; ++m) terms(lane % LPG + m * LPG, 8 * cg, t);
+  int col = 0;
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    const int h = 4 >> r, o = LPG >> (r + 1);
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int j = 0; j < h; ++j) {
+        const float keep = up ? t[k][j + h] : t[k][j];
+        const float send = up ? t[k][j] : t[k][j + h];
+        t[k][j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    col += up ? h : 0;
+  }
+#pragma unroll
+  for (int o = LPG / 16; o >= 1; o >>= 1)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) t[k][0] += __shfl_xor_sync(0xffffffffu, t[k][0], o);
+  if ((lane & (LPG / 8 - 1)) == 0) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) acc[k][8 * cg + col] += t[k][0];
+  }
+}
+// Sum of x(i) over i in [0, 64), in every lane of the calling warp.
+template <typename F>
+__device__ __forceinline__ float warp_sum64(F &&x) {
+  const int l = threadIdx.x & 31;
+  float s = x(l) + x(l + 32);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+// The three vectors of acc into dst, and acc cleared (threads t < D, column t).
+template <int D>
+__device__ __forceinline__ void drain_acc(float (*acc)[128], float *dst, int64_t stride) {
+  if (threadIdx.x < D) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      dst[k * stride + threadIdx.x] = acc[k][threadIdx.x];
+      acc[k][threadIdx.x] = 0.f;
+    }
+  }
+}
+
+// Common set-up of the three kernels: barriers, TMEM, and the CTA-wide agreement on whether
+// every wait so far has succeeded.
+struct Sync {
+  BwdShared &sh;
+  WarpWaiter wait;
+  uint32_t mph = 0;  // commits to sh.mma waited for
+  __device__ __forceinline__ Sync(BwdShared &s, int *err, int lane)
+      : sh(s), wait{&s.abort, err, lane} {}
+  // CTA barrier; false (for every thread) once any thread's wait has given up
+  __device__ __forceinline__ bool barrier() {
+    tc_fence_before();
+    const int bad = __syncthreads_or(wait.ok ? 0 : 1);
+    tc_fence_after();
+    if (bad) wait.ok = false;
+    return bad == 0;
+  }
+  __device__ __forceinline__ void wait_mma() {
+    wait(&sh.mma, mph & 1);
+    ++mph;
+  }
+};
+
+__device__ __forceinline__ void init_barriers(BwdShared &sh) {
+  for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
+    sh.acc[i / 128][i % 128] = 0.f;
+    sh.racc[i / 128][i % 128] = 0.f;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&sh.full[0], 1);
+    mbar_init(&sh.full[1], 1);
+    mbar_init(&sh.mma, 1);
+    mbar_init(&sh.fin, 1);
+    sh.abort = 0;
+    fence_barrier_init();
+  }
+}
+
+// Lets every copy and product a CTA issued land (thread 0: `landed` of `issued` loads had
+// been waited for), then releases its TMEM.
+__device__ __forceinline__ void finish(BwdShared &sh, int landed, int issued, uint32_t tmem,
+                                       uint32_t cols, int *err) {
+  if (threadIdx.x == 0) {
+    for (int l = landed; l < issued; ++l) mbar_wait_drain(&sh.full[l & 1], (l >> 1) & 1, err);
+    mma_commit(&sh.fin);
+    mbar_wait_drain(&sh.fin, 0, err);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, cols);
+}
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t base, int ks, uint32_t atom) {
+  return desc_add(kmajor_base(base), kmajor_off(ks, atom));
+}
+__device__ __forceinline__ uint64_t mdesc(uint32_t base, int ks, uint32_t atom) {
+  return desc_add(mnmajor_base(base, atom), mnmajor_off(ks));
+}
+
+// ---------------------------------------------------------------- K1: forward records
+// k, v: [heads][n][D] via tmK, tmV.  Writes each item's record [Psi | zeta | vs | sigma |
+// kappa] to rec + (head * nseg + seg) * rec_floats<D>().
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    bwd_aggregate_kernel(const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, float *__restrict__ rec,
+                         int64_t n, int64_t seg_len, int64_t nseg, int64_t nitems, int *err) {
+  using G = BCfg<D>;
+  constexpr int AT = G::AT;
+  constexpr int KSC = C / 16;
+  constexpr int OK = 0, OV = G::TILE;
+  constexpr uint32_t LOAD = 2 * G::TILE;
+  constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~uintptr_t(1023));
+  BwdShared &sh = *reinterpret_cast<BwdShared *>(sm + G::G_SH);
+  const Lanes L = Lanes::make<D>();
+  const int64_t it0 = blockIdx.x, istep = gridDim.x;
+
+  init_barriers(sh);
+  if (L.warp == 0) {
+    tmem_alloc(&sh.tmem_base, D);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const uint64_t pol = policy_evict_first();
+  Sync S(sh, err, L.lane);
+
+  int issued = 0, landed = 0;
+  auto issue = [&](const Item &I, int c) {
+    uint64_t *fb = &sh.full[issued & 1];
+    uint8_t *st = sm + (issued & 1) * G::G_STAGE;
+    mbar_arrive_expect_tx(fb, LOAD);
+    const int y = static_cast<int>(I.t_begin + (int64_t)c * C), z = static_cast<int>(I.head);
+#pragma unroll
+    for (int a = 0; a < AT; ++a) {
+      tma_load_3d(st + OK + a * kAtom, &tmK, fb, 64 * a, y, z, pol);
+      tma_load_3d(st + OV + a * kAtom, &tmV, fb, 64 * a, y, z, pol);
+    }
+    ++issued;
+  };
+  if (threadIdx.x == 0) issue(item_at<C>(it0, n, seg_len, nseg), 0);
+
+  int g = 0;
+  for (int64_t it = it0; it < nitems && S.wait.ok; it += istep) {
+    const Item I = item_at<C>(it, n, seg_len, nseg);
+    float kap = 0.f;  // thread 0: kappa of the item (its vectors gather in sh.acc)
+    for (int c = 0; c < I.nchunks; ++c, ++g) {
+      uint8_t *st = sm + (g & 1) * G::G_STAGE;
+      const int64_t t0 = I.t_begin + (int64_t)c * C;
+      const int valid = I.t_end - t0 < C ? static_cast<int>(I.t_end - t0) : C;
+      if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
+        if (threadIdx.x == 0) landed = g + 1;
+        psi_tile<D>(st + OK, valid, sh.sk);
+      }
+      fence_proxy_async_smem();
+      if (!S.barrier()) break;
+      if (threadIdx.x == 0) {
+        if (c + 1 < I.nchunks)
+          issue(I, c + 1);
+        else if (it + istep < nitems)
+          issue(item_at<C>(it + istep, n, seg_len, nseg), 0);
+        const uint32_t k0 = smem_u32(st + OK), v0 = smem_u32(st + OV);
+        // Psi += psi(K)^T V
+#pragma unroll
+        for (int ks = 0; ks < KSC; ++ks)
+          mma_bf16_ss(tmem, mdesc(k0, ks, kAtom), mdesc(v0, ks, kAtom), I_S, (c > 0 || ks > 0));
+        mma_commit(&sh.mma);
+      }
+      // zeta, vs, sigma of the chunk's keys (rows past the item's end: psi(K) zero, V skipped)
+      column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
+        float kr[8], vr[8];
+        tile_row8(st + OK, i, c, kr);
+        tile_row8(st + OV, i, c, vr);
+        const float w = i < valid ? 1.f : 0.f, ski = sh.sk[i];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          t[0][e] += kr[e];
+          t[1][e] = fmaf(w, vr[e], t[1][e]);
+          t[2][e] = fmaf(w * ski, vr[e], t[2][e]);
+        }
+      });
+      if (L.warp == 0) {
+        const float ks = warp_sum64([&](int i) { return sh.sk[i]; });
+        if (threadIdx.x == 0) kap += ks;
+      }
+      S.wait_mma();
+      if (!S.barrier()) break;
+    }
+    if (!S.wait.ok) break;
+    float *dst = rec + (I.head * nseg + I.seg) * rec_floats<D>();
+    state_to_global<D>(tmem + L.lane_off, dst, L);
+    drain_acc<D>(sh.acc, dst + (int64_t)D * D, D);
+    if (threadIdx.x == 0) {
+      dst[(int64_t)D * D + 3 * D] = kap;
+      dst[(int64_t)D * D + 3 * D + 1] = 0.f;
+      dst[(int64_t)D * D + 3 * D + 2] = 0.f;
+      dst[(int64_t)D * D + 3 * D + 3] = 0.f;
+    }
+    if (!S.barrier()) break;
+  }
+  finish(sh, landed, issued, tmem, D, err);
+}
+
+// ---------------------------------------------------------------- B1: the prefix walk
+// q, dout: [heads][n][D] via tmQ, tmG; k, v via tmK, tmV (causal only).  start: each item's
+// forward record (causal: exclusive prefix at start + head * start_hs + seg * start_ss;
+// non-causal: the head's total).  Writes dq, a as a bf16 pair (a_hi, a_lo: [heads][n][D]),
+// b ([heads][n]) and each item's reverse record to r_rec + (head * nseg + seg) * rec_floats.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
+    bwd_prefix_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmG, __nv_bfloat16 *__restrict__ dq,
+                      __nv_bfloat16 *__restrict__ a_hi, __nv_bfloat16 *__restrict__ a_lo,
+                      float *__restrict__ b_out, const float *__restrict__ start,
+                      int64_t start_hs, int64_t start_ss, float *__restrict__ r_rec, int64_t n,
+                      int64_t seg_len, int64_t nseg, int64_t nitems, int *err) {
+  using G = BCfg<D>;
+  constexpr int AT = G::AT;
+  constexpr int KSD = D / 16;  // K-steps over D
+  constexpr int KSC = C / 16;  // K-steps over the chunk's tokens
+  constexpr int HD = D / 2;    // columns per half of a D-wide accumulator
+  constexpr int OQ = 0, OG = G::TILE, OK = 2 * G::TILE, OV = 3 * G::TILE;
+  constexpr uint32_t LOAD = (CAUSAL ? 4 : 2) * G::TILE;
+  constexpr uint32_t SA = G::S_ATOM;
+  constexpr uint32_t I_P = make_idesc_bf16(64, 64, false, false);  // P', dW
+  constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);      // Psi, Phi updates
+  constexpr uint32_t I_O = make_idesc_bf16(64, D, false, true);    // psi(Q) Psi, M V, L V, W psi(K)
+  constexpr uint32_t I_T = make_idesc_bf16(64, D, false, false);   // A Psi^T
+  constexpr float kD = static_cast<float>(D);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~uintptr_t(1023));
+  BwdShared &sh = *reinterpret_cast<BwdShared *>(sm + G::P_SH);
+  uint8_t *sST = sm + G::P_ST;  // bf16 Psi (rows: features; 64-column blocks of values)
+  uint8_t *sA = sm + G::P_A, *sAL = sm + G::P_AL, *sW = sm + G::P_W, *sL = sm + G::P_L;
+  const bool a32 = aligned32(dq);  // the gradient rows take full-sector stores
+  const Lanes L = Lanes::make<D>();
+  const int64_t it0 = blockIdx.x, istep = gridDim.x;
+
+  init_barriers(sh);
+  // L: [64][64] lower triangle of ones (j <= i), the K-major operand of the prefix sums of V
+  for (int i = threadIdx.x; i < kAtom / 16; i += kThreads) {
+    const int row = i >> 3, c8 = 8 * (i & 7);
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      w[e] = (c8 + 2 * e <= row ? 0x3F80u : 0u) | (c8 + 2 * e + 1 <= row ? 0x3F800000u : 0u);
+    *reinterpret_cast<uint4 *>(sL + sw128_offset(row, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  fence_proxy_async_smem();
+  if (L.warp == 0) {
+    tmem_alloc(&sh.tmem_base, G::TCOLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmG);
+    if (CAUSAL) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const uint32_t tX = tmem, tY = tmem + D, tR = tmem + 2 * D, tS = tmem + 3 * D;
+  const uint32_t myX = tX + L.lane_off, myY = tY + L.lane_off, myR = tR + L.lane_off,
+                 myS = tS + L.lane_off;
+  const uint64_t pol = policy_evict_first();
+  Sync S(sh, err, L.lane);
+
+  int issued = 0, landed = 0;
+  auto issue = [&](const Item &I, int c) {
+    uint64_t *fb = &sh.full[issued & 1];
+    uint8_t *st = sm + (issued & 1) * G::P_STAGE;
+    mbar_arrive_expect_tx(fb, LOAD);
+    const int y = static_cast<int>(I.t_begin + (int64_t)c * C), z = static_cast<int>(I.head);
+#pragma unroll
+    for (int a = 0; a < AT; ++a) {
+      tma_load_3d(st + OQ + a * kAtom, &tmQ, fb, 64 * a, y, z, pol);
+      tma_load_3d(st + OG + a * kAtom, &tmG, fb, 64 * a, y, z, pol);
+      if (CAUSAL) {
+        tma_load_3d(st + OK + a * kAtom, &tmK, fb, 64 * a, y, z, pol);
+        tma_load_3d(st + OV + a * kAtom, &tmV, fb, 64 * a, y, z, pol);
+      }
+    }
+    ++issued;
+  };
+  if (threadIdx.x == 0) issue(item_at<C>(it0, n, seg_len, nseg), 0);
+
+  const uint32_t uA = smem_u32(sA), uAL = smem_u32(sAL), uST = smem_u32(sST);
+  const uint32_t uW = smem_u32(sW), uL = smem_u32(sL);
+  int g = 0;  // steps of this CTA's walk
+  for (int64_t it = it0; it < nitems && S.wait.ok; it += istep) {
+    const Item I = item_at<C>(it, n, seg_len, nseg);
+    // ---- the item's starting forward record: Psi (TMEM, causal) and its operand; vectors
+    load_record<D>(start + I.head * start_hs + I.seg * start_ss, sST, myS, CAUSAL, L, sh);
+    float bs_acc = 0.f;  // thread 0: bs of the item (its vectors gather in sh.racc)
+    for (int c = 0; c < I.nchunks; ++c, ++g) {
+      uint8_t *st = sm + (g & 1) * G::P_STAGE;
+      const uint32_t uQ = smem_u32(st + OQ), uK = smem_u32(st + OK), uV = smem_u32(st + OV);
+      const int64_t t0 = I.t_begin + (int64_t)c * C;
+      const int valid = I.t_end - t0 < C ? static_cast<int>(I.t_end - t0) : C;
+      const bool more = CAUSAL && c + 1 < I.nchunks;  // the record after this chunk is needed
+      const bool live = L.v64 && L.r64 < valid;
+      const int64_t row = I.head * n + t0 + L.r64;  // global row of this thread (when live)
+      // keys row i sees: every key up to it (causal), all n (non-causal)
+      const float Ni = CAUSAL ? static_cast<float>(t0 + L.r64 + 1) : static_cast<float>(n);
+
+      // ---- (a) psi on Q and K (K rows past the item's end zeroed), with row sums
+      if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
+        if (threadIdx.x == 0) landed = g + 1;
+        psi_tile<D>(st + OQ, C, sh.sq);
+        if (CAUSAL) psi_tile<D>(st + OK, valid, sh.sk);
+      }
+      fence_proxy_async_smem();
+      if (!S.barrier()) break;
+      if (threadIdx.x == 0) {
+        // the next step's tiles into the other stage (its last reader, step g - 1, is done)
+        if (c + 1 < I.nchunks)
+          issue(I, c + 1);
+        else if (it + istep < nitems)
+          issue(item_at<C>(it + istep, n, seg_len, nseg), 0);
+        if (CAUSAL) {
+          // P' = psi(Q) psi(K)^T;  LV = L V;  Psi += psi(K)^T V
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uQ, ks, kAtom), kdesc(uK, ks, kAtom), I_P, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tY, kdesc(uL, ks, kAtom), mdesc(uV, ks, kAtom), I_O, ks > 0);
+          if (more) {
+#pragma unroll
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tS, mdesc(uK, ks, kAtom), mdesc(uV, ks, kAtom), I_S, 1u);
+          }
+        } else {
+          // O' = psi(Q) Psi
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uQ, ks, kAtom), mdesc(uST, ks, SA), I_O, ks > 0);
+        }
+        mma_commit(&sh.mma);
+      }
+      // psi(q_i) . zeta over this half's features
+      float dpart = 0.f;
+      if (L.v64) {
+#pragma unroll 2
+        for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 8) {
+          float f[8];
+          tile_row8(st + OQ, L.r64, c0, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dpart = fmaf(f[e], sh.vec[0][c0 + e], dpart);
+        }
+      }
+      float kap_chunk = 0.f;  // thread 0: kappa of this chunk's keys
+      if (CAUSAL) {
+        // ---- (c) M = mask(P' + sk) (j <= i) rounded into its operand; row sums of M
+        S.wait_mma();
+        if (S.wait.ok) {
+          float p[32];
+          tmem_row32(myX + 32 * L.hf, p);
+          if (L.v64) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int j0 = 32 * L.hf + 8 * q;
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = j0 + e <= L.r64 ? p[8 * q + e] + sh.sk[j0 + e] : 0.f;
+              const uint4 u = pack8(f);
+              unpack8(u, f);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) dpart += f[e];
+              *reinterpret_cast<uint4 *>(sW + sw128_offset(L.r64, j0)) = u;
+            }
+          }
+        }
+        if (L.v64) sh.part[L.hf][L.r64] = dpart;
+        fence_proxy_async_smem();
+        if (!S.barrier()) break;
+        if (threadIdx.x == 0) {
+          // O' = psi(Q) Psi + M V
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uQ, ks, kAtom), mdesc(uST, ks, SA), I_O, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tX, kdesc(uW, ks, kAtom), mdesc(uV, ks, kAtom), I_O, 1u);
+          mma_commit(&sh.mma);
+        }
+        // this chunk's part of the next chunk's forward record: zeta, vs, sigma (sh.acc), kappa
+        if (more) {
+          column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
+            float kr[8], vr[8];
+            tile_row8(st + OK, i, c, kr);
+            tile_row8(st + OV, i, c, vr);
+            const float w = i < valid ? 1.f : 0.f, ski = sh.sk[i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              t[0][e] += kr[e];
+              t[1][e] = fmaf(w, vr[e], t[1][e]);
+              t[2][e] = fmaf(w * ski, vr[e], t[2][e]);
+            }
+          });
+          if (L.warp == 0) {
+            const float ks = warp_sum64([&](int i) { return sh.sk[i]; });
+            if (threadIdx.x == 0) kap_chunk = ks;
+          }
+        }
+      } else {
+        if (L.v64) sh.part[L.hf][L.r64] = dpart;
+        S.wait_mma();
+        if (!S.barrier()) break;
+      }
+      const float sq_i = L.v64 ? sh.sq[L.r64] : 0.f;
+      const float den =
+          L.v64 ? Ni * (kD + sq_i) + sh.scal + sh.part[0][L.r64] + sh.part[1][L.r64] : 1.f;
+
+      // ---- (e) out_i, a_i = g_i / den_i (the bf16 pair into its operands and the
+      //     workspace); partial a_i . out_i and a_i . (vs + LV_i)
+      if (CAUSAL) S.wait_mma();
+      float gdot = 0.f, cdot = 0.f;
+      if (S.wait.ok) {
+        const float inv = 1.f / den;
+#pragma unroll 1
+        for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+          float o[32], lv[32];
+          tmem_row32(myX + c0, o);
+          if (CAUSAL) {
+            tmem_row32(myY + c0, lv);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) lv[e] = 0.f;
+          }
+          if (L.v64) {
+            uint4 hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float gv[8], av[8], rv[8];
+              tile_row8(st + OG, L.r64, c0 + 8 * q, gv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int col = c0 + 8 * q + e;
+                const float vsum = sh.vec[1][col] + lv[8 * q + e];
+                const float out = ((kD + sq_i) * vsum + sh.vec[2][col] + o[8 * q + e]) * inv;
+                const float a = live ? gv[e] * inv : 0.f;
+                gdot = fmaf(a, out, gdot);
+                cdot = fmaf(a, vsum, cdot);
+                av[e] = a;
+              }
+              hi[q] = pack8(av);
+              unpack8(hi[q], rv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) rv[e] = av[e] - rv[e];
+              lo[q] = pack8(rv);
+              *reinterpret_cast<uint4 *>(sA + tile_off(L.r64, c0 + 8 * q)) = hi[q];
+              *reinterpret_cast<uint4 *>(sAL + tile_off(L.r64, c0 + 8 * q)) = lo[q];
+            }
+            if (live) {
+              st_global_32B(a_hi + row * D + c0, hi[0], hi[1], true);
+              st_global_32B(a_hi + row * D + c0 + 16, hi[2], hi[3], true);
+              st_global_32B(a_lo + row * D + c0, lo[0], lo[1], true);
+              st_global_32B(a_lo + row * D + c0 + 16, lo[2], lo[3], true);
+            }
+          }
+        }
+      }
+      if (L.v64) {
+        sh.gd[L.hf][L.r64] = gdot;
+        sh.cd[L.hf][L.r64] = cdot;
+      }
+      fence_proxy_async_smem();
+      if (!S.barrier()) break;
+      // b_i = -(a_i . out_i);  C_i = sum_{j seen} dW_ij = a_i . (vs + LV_i) + N_i b_i
+      const float b = live ? -(sh.gd[0][L.r64] + sh.gd[1][L.r64]) : 0.f;
+      const float Ci = live ? sh.cd[0][L.r64] + sh.cd[1][L.r64] + Ni * b : 0.f;
+      if (live && L.hf == 0) b_out[row] = b;
+      if (threadIdx.x == 0) {
+        if (CAUSAL) {
+          // dW = A V^T  (a_hi, then a_lo, along the contraction)
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uA, ks, kAtom), kdesc(uV, ks, kAtom), I_P, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uAL, ks, kAtom), kdesc(uV, ks, kAtom), I_P, 1u);
+        }
+        // dQ' = A Psi^T
+#pragma unroll
+        for (int ks = 0; ks < KSD; ++ks)
+          mma_bf16_ss(tY, kdesc(uA, ks, kAtom), kdesc(uST, ks, SA), I_T, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < KSD; ++ks)
+          mma_bf16_ss(tY, kdesc(uAL, ks, kAtom), kdesc(uST, ks, SA), I_T, 1u);
+        // Phi += psi(Q)^T A
+#pragma unroll
+        for (int ks = 0; ks < KSC; ++ks)
+          mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uA, ks, kAtom), I_S, (c > 0 || ks > 0));
+#pragma unroll
+        for (int ks = 0; ks < KSC; ++ks)
+          mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uAL, ks, kAtom), I_S, 1u);
+        mma_commit(&sh.mma);
+      }
+      // this chunk's part of the item's reverse record: rho, as, tau (sh.racc), bs; b of each
+      // row from the exchanged partial dot products, zero past the item's end (so is a)
+      column_sums3<D>(sh.racc, [&](int i, int c, float (*t)[8]) {
+        float qr[8], ar[8], lr[8];
+        tile_row8(st + OQ, i, c, qr);
+        tile_row8(sA, i, c, ar);
+        tile_row8(sAL, i, c, lr);
+        const float bi = i < valid ? -(sh.gd[0][i] + sh.gd[1][i]) : 0.f, sqi = sh.sq[i];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float aa = ar[e] + lr[e];
+          t[0][e] = fmaf(qr[e], bi, t[0][e]);
+          t[1][e] += aa;
+          t[2][e] = fmaf(sqi, aa, t[2][e]);
+        }
+      });
+      if (L.warp == 0) {
+        const float bsum =
+            warp_sum64([&](int i) { return i < valid ? -(sh.gd[0][i] + sh.gd[1][i]) : 0.f; });
+        if (threadIdx.x == 0) bs_acc += bsum;
+      }
+      S.wait_mma();
+      if (CAUSAL) {
+        // ---- (g) mask(dW + b) (j <= i) rounded into the M operand's buffer (M V is done);
+        //     the record after this chunk: Psi (TMEM) -> operand (A Psi^T is done)
+        if (S.wait.ok) {
+          float w[32];
+          tmem_row32(myX + 32 * L.hf, w);
+          if (L.v64) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int j0 = 32 * L.hf + 8 * q;
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = j0 + e <= L.r64 ? w[8 * q + e] + b : 0.f;
+              *reinterpret_cast<uint4 *>(sW + sw128_offset(L.r64, j0)) = pack8(f);
+            }
+          }
+          if (more) state_to_operand<D>(myS, sST, L);
+        }
+        fence_proxy_async_smem();
+        if (!S.barrier()) break;
+        if (threadIdx.x == 0) {
+          // dQ' += mask(dW + b) psi(K)
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tY, kdesc(uW, ks, kAtom), mdesc(uK, ks, kAtom), I_O, 1u);
+          mma_commit(&sh.mma);
+        }
+        S.wait_mma();
+      }
+      // ---- (i) dq_i = (dQ'_i + zeta b_i + C_i) * phi'(q_i)
+      if (S.wait.ok) {
+#pragma unroll 1
+        for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+          float f[32];
+          tmem_row32(myY + c0, f);
+          if (live) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float ps[8];
+              tile_row8(st + OQ, L.r64, c0 + 8 * q, ps);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int col = c0 + 8 * q + e;
+                f[8 * q + e] =
+                    (f[8 * q + e] + fmaf(sh.vec[0][col], b, Ci)) * dphi_from_psi(ps[e]);
+              }
+            }
+            st_global_32B(dq + row * D + c0, pack8(f), pack8(f + 8), a32);
+            st_global_32B(dq + row * D + c0 + 16, pack8(f + 16), pack8(f + 24), a32);
+          }
+        }
+      }
+      if (!S.barrier()) break;
+      if (more) {
+        // the forward record after this chunk
+        if (threadIdx.x < D) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            sh.vec[k][threadIdx.x] += sh.acc[k][threadIdx.x];
+            sh.acc[k][threadIdx.x] = 0.f;
+          }
+        }
+        if (threadIdx.x == 0) sh.scal += kap_chunk;
+      }
+    }
+    if (!S.wait.ok) break;
+    // ---- the item's reverse record [Phi | rho | as | tau | bs]
+    float *dst = r_rec + (I.head * nseg + I.seg) * rec_floats<D>();
+    state_to_global<D>(myR, dst, L);
+    drain_acc<D>(sh.racc, dst + (int64_t)D * D, D);
+    if (threadIdx.x == 0) {
+      dst[(int64_t)D * D + 3 * D] = bs_acc;
+      dst[(int64_t)D * D + 3 * D + 1] = 0.f;
+      dst[(int64_t)D * D + 3 * D + 2] = 0.f;
+      dst[(int64_t)D * D + 3 * D + 3] = 0.f;
+    }
+    if (!S.barrier()) break;
+  }
+  finish(sh, landed, issued, tmem, G::TCOLS, err);
+}
+
+// ---------------------------------------------------------------- B3: the suffix walk
+// q, a_hi, a_lo: [heads][n][D] via tmQ, tmA, tmAL, and b_in: [heads][n] (causal only); k, v
+// via tmK, tmV.  start: each item's reverse record (causal: exclusive suffix at start +
+// head * start_hs + seg * start_ss; non-causal: the head's total).  Writes dk, dv.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
+    bwd_suffix_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmAL,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const float *__restrict__ b_in,
+                      __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
+                      const float *__restrict__ start, int64_t start_hs, int64_t start_ss,
+                      int64_t n, int64_t seg_len, int64_t nseg, int64_t nitems, int *err) {
+  using G = BCfg<D>;
+  constexpr int AT = G::AT;
+  constexpr int KSD = D / 16;
+  constexpr int KSC = C / 16;
+  constexpr int HD = D / 2;
+  constexpr int OQ = 0, OA = G::TILE, OAL = 2 * G::TILE, OK = 3 * G::TILE, OV = 4 * G::TILE;
+  constexpr uint32_t LOAD = (CAUSAL ? 5 : 2) * G::TILE;
+  constexpr uint32_t SA = G::S_ATOM;
+  constexpr uint32_t I_P = make_idesc_bf16(64, 64, false, false);  // P'^T, dW^T
+  constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);      // Phi update
+  constexpr uint32_t I_O = make_idesc_bf16(64, D, false, true);    // psi(K) Phi, W A, W psi(Q)
+  constexpr uint32_t I_T = make_idesc_bf16(64, D, false, false);   // V Phi^T
+  constexpr float kD = static_cast<float>(D);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~uintptr_t(1023));
+  BwdShared &sh = *reinterpret_cast<BwdShared *>(sm + G::S_SH);
+  uint8_t *sFT = sm + G::S_ST;  // bf16 Phi (rows: features; 64-column blocks of values)
+  uint8_t *sW0 = sm + G::S_W0;  // mask(w^T): the weights of the chunk's keys
+  uint8_t *sW1 = sm + G::S_W1;  // mask(dW^T + b)
+  const bool a32v = aligned32(dv), a32k = aligned32(dk);  // full-sector stores
+  const Lanes L = Lanes::make<D>();
+  const int64_t it0 = blockIdx.x, istep = gridDim.x;
+
+  init_barriers(sh);
+  if (L.warp == 0) {
+    tmem_alloc(&sh.tmem_base, G::TCOLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    if (CAUSAL) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmAL);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const uint32_t tX = tmem, tR = tmem + 2 * D;  // X: P'^T | dW^T, then dV' | dK'
+  const uint32_t myX = tX + L.lane_off, myR = tR + L.lane_off;
+  const uint64_t pol = policy_evict_first();
+  Sync S(sh, err, L.lane);
+  // walk step w of an item -> its chunk (the causal walk runs from the item's last chunk)
+  auto chunk_of = [](int w, int nchunks) { return CAUSAL ? nchunks - 1 - w : w; };
+
+  int issued = 0, landed = 0;
+  auto issue = [&](const Item &I, int w) {
+    uint64_t *fb = &sh.full[issued & 1];
+    uint8_t *st = sm + (issued & 1) * G::S_STAGE;
+    mbar_arrive_expect_tx(fb, LOAD);
+    const int y = static_cast<int>(I.t_begin + (int64_t)chunk_of(w, I.nchunks) * C);
+    const int z = static_cast<int>(I.head);
+#pragma unroll
+    for (int a = 0; a < AT; ++a) {
+      tma_load_3d(st + OK + a * kAtom, &tmK, fb, 64 * a, y, z, pol);
+      tma_load_3d(st + OV + a * kAtom, &tmV, fb, 64 * a, y, z, pol);
+      if (CAUSAL) {
+        tma_load_3d(st + OQ + a * kAtom, &tmQ, fb, 64 * a, y, z, pol);
+        tma_load_3d(st + OA + a * kAtom, &tmA, fb, 64 * a, y, z, pol);
+        tma_load_3d(st + OAL + a * kAtom, &tmAL, fb, 64 * a, y, z, pol);
+      }
+    }
+    ++issued;
+  };
+  if (threadIdx.x == 0) issue(item_at<C>(it0, n, seg_len, nseg), 0);
+
+  const uint32_t uFT = smem_u32(sFT), uW0 = smem_u32(sW0), uW1 = smem_u32(sW1);
+  int g = 0;
+  for (int64_t it = it0; it < nitems && S.wait.ok; it += istep) {
+    const Item I = item_at<C>(it, n, seg_len, nseg);
+    // ---- the item's starting reverse record: Phi (TMEM, causal) and its operand; vectors
+    load_record<D>(start + I.head * start_hs + I.seg * start_ss, sFT, myR, CAUSAL, L, sh);
+    for (int w = 0; w < I.nchunks; ++w, ++g) {
+      uint8_t *st = sm + (g & 1) * G::S_STAGE;
+      const uint32_t uQ = smem_u32(st + OQ), uA = smem_u32(st + OA), uAL = smem_u32(st + OAL);
+      const uint32_t uK = smem_u32(st + OK), uV = smem_u32(st + OV);
+      const int64_t t0 = I.t_begin + (int64_t)chunk_of(w, I.nchunks) * C;
+      const int valid = I.t_end - t0 < C ? static_cast<int>(I.t_end - t0) : C;
+      const bool more = CAUSAL && w + 1 < I.nchunks;  // the record before this chunk is needed
+      const bool live = L.v64 && L.r64 < valid;
+      const int64_t row = I.head * n + t0 + L.r64;
+
+      // b of the chunk's rows, fetched while the tiles land (zero past the item's end)
+      float bload = 0.f;
+      if (CAUSAL && threadIdx.x < valid) bload = b_in[I.head * n + t0 + threadIdx.x];
+      // ---- (a) psi on K (row sums); causal: psi on Q (row sums) and the rows of Q and A past
+      //     the item's end zeroed
+      if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
+        if (threadIdx.x == 0) landed = g + 1;
+        psi_tile<D>(st + OK, C, sh.sk);
+        if (CAUSAL) {
+          psi_tile<D>(st + OQ, valid, sh.sq);
+          zero_rows<D>(st + OA, valid);
+          zero_rows<D>(st + OAL, valid);
+        }
+      }
+      if (CAUSAL && threadIdx.x < C) sh.bv[threadIdx.x] = bload;
+      fence_proxy_async_smem();
+      if (!S.barrier()) break;
+      if (threadIdx.x == 0) {
+        if (w + 1 < I.nchunks)
+          issue(I, w + 1);
+        else if (it + istep < nitems)
+          issue(item_at<C>(it + istep, n, seg_len, nseg), 0);
+        if (CAUSAL) {
+          // P'^T = psi(K) psi(Q)^T;  dW^T = V A^T (a_hi, then a_lo);  Phi += psi(Q)^T A
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uK, ks, kAtom), kdesc(uQ, ks, kAtom), I_P, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX + 64, kdesc(uV, ks, kAtom), kdesc(uA, ks, kAtom), I_P, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX + 64, kdesc(uV, ks, kAtom), kdesc(uAL, ks, kAtom), I_P, 1u);
+          if (more) {
+#pragma unroll
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uA, ks, kAtom), I_S, 1u);
+#pragma unroll
+            for (int ks = 0; ks < KSC; ++ks)
+              mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uAL, ks, kAtom), I_S, 1u);
+          }
+        } else {
+          // dV' = psi(K) Phi;  dK' = V Phi^T  (Phi the head's total)
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks) {
+            mma_bf16_ss(tX, kdesc(uK, ks, kAtom), mdesc(uFT, ks, SA), I_O, ks > 0);
+            mma_bf16_ss(tX + D, kdesc(uV, ks, kAtom), kdesc(uFT, ks, SA), I_T, ks > 0);
+          }
+        }
+        mma_commit(&sh.mma);
+      }
+      // v_j . as over this half's columns (as: the record after this chunk, read after the
+      // barrier above, which orders it after the record's load or last update)
+      if (L.v64) {
+        float vdot = 0.f;
+#pragma unroll 2
+        for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 8) {
+          float f[8];
+          tile_row8(st + OV, L.r64, c0, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vdot = fmaf(f[e], sh.vec[1][c0 + e], vdot);
+        }
+        sh.gd[L.hf][L.r64] = vdot;
+      }
+      float bs_chunk = 0.f;  // thread 0: bs of this chunk's rows
+      if (CAUSAL) {
+        // ---- (c) row j: the weights w_ji = d + sq_i + sk_j + P'^T_ji and dW^T_ji + b_i, kept
+        //     for i >= j and rounded into their operands; C'_j's part from this chunk
+        S.wait_mma();
+        float cin = 0.f;
+        if (S.wait.ok) {
+          float p[32];
+          tmem_row32(myX + 32 * L.hf, p);
+          if (L.v64) {
+            const float skj = kD + sh.sk[L.r64];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int i0 = 32 * L.hf + 8 * q;
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                f[e] = i0 + e >= L.r64 ? p[8 * q + e] + sh.sq[i0 + e] + skj : 0.f;
+              *reinterpret_cast<uint4 *>(sW0 + sw128_offset(L.r64, i0)) = pack8(f);
+            }
+          }
+          tmem_row32(myX + 64 + 32 * L.hf, p);
+          if (L.v64) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int i0 = 32 * L.hf + 8 * q;
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                f[e] = i0 + e >= L.r64 ? p[8 * q + e] + sh.bv[i0 + e] : 0.f;
+                cin += f[e];
+              }
+              *reinterpret_cast<uint4 *>(sW1 + sw128_offset(L.r64, i0)) = pack8(f);
+            }
+          }
+        }
+        if (L.v64) sh.part[L.hf][L.r64] = cin;
+        fence_proxy_async_smem();
+        if (!S.barrier()) break;
+        if (threadIdx.x == 0) {
+          // dV' = psi(K) Phi + mask(w^T) a_hi;  dK' = V Phi^T + mask(dW^T + b) psi(Q)
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks) {
+            mma_bf16_ss(tX, kdesc(uK, ks, kAtom), mdesc(uFT, ks, SA), I_O, ks > 0);
+            mma_bf16_ss(tX + D, kdesc(uV, ks, kAtom), kdesc(uFT, ks, SA), I_T, ks > 0);
+          }
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks) {
+            mma_bf16_ss(tX, kdesc(uW0, ks, kAtom), mdesc(uA, ks, kAtom), I_O, 1u);
+            mma_bf16_ss(tX + D, kdesc(uW1, ks, kAtom), mdesc(uQ, ks, kAtom), I_O, 1u);
+          }
+          mma_commit(&sh.mma);
+        }
+        // this chunk's part of the record before it: rho, as, tau (sh.acc), bs
+        if (more) {
+          column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
+            float qr[8], ar[8], lr[8];
+            tile_row8(st + OQ, i, c, qr);
+            tile_row8(st + OA, i, c, ar);
+            tile_row8(st + OAL, i, c, lr);
+            const float bi = sh.bv[i], sqi = sh.sq[i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float aa = ar[e] + lr[e];
+              t[0][e] = fmaf(qr[e], bi, t[0][e]);
+              t[1][e] += aa;
+              t[2][e] = fmaf(sqi, aa, t[2][e]);
+            }
+          });
+          if (L.warp == 0) {
+            const float bsum = warp_sum64([&](int i) { return sh.bv[i]; });
+            if (threadIdx.x == 0) bs_chunk = bsum;
+          }
+        }
+      }
+      // ---- (e) dv_j = (d + sk_j) as + tau + dV'_j;  dk_j = (dK'_j + rho + C'_j) phi'(k_j),
+      //     C'_j = v_j . as + bs + (this chunk's sum_{i >= j} dW_ij);  Phi -> operand
+      S.wait_mma();
+      if (!CAUSAL && !S.barrier()) break;  // both halves of v_j . as are in sh.gd
+      if (S.wait.ok) {
+        const float skj = L.v64 ? kD + sh.sk[L.r64] : 0.f;
+        const float cpj =
+            L.v64 ? sh.gd[0][L.r64] + sh.gd[1][L.r64] + sh.scal +
+                        (CAUSAL ? sh.part[0][L.r64] + sh.part[1][L.r64] : 0.f)
+                  : 0.f;
+#pragma unroll 1
+        for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+          float f[32];
+          tmem_row32(myX + c0, f);
+          if (live) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              f[e] = fmaf(skj, sh.vec[1][c0 + e], sh.vec[2][c0 + e] + f[e]);
+            st_global_32B(dv + row * D + c0, pack8(f), pack8(f + 8), a32v);
+            st_global_32B(dv + row * D + c0 + 16, pack8(f + 16), pack8(f + 24), a32v);
+          }
+          tmem_row32(myX + D + c0, f);
+          if (live) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float ps[8];
+              tile_row8(st + OK, L.r64, c0 + 8 * q, ps);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int col = c0 + 8 * q + e;
+                f[8 * q + e] = (f[8 * q + e] + sh.vec[0][col] + cpj) * dphi_from_psi(ps[e]);
+              }
+            }
+            st_global_32B(dk + row * D + c0, pack8(f), pack8(f + 8), a32k);
+            st_global_32B(dk + row * D + c0 + 16, pack8(f + 16), pack8(f + 24), a32k);
+          }
+        }
+        if (more) state_to_operand<D>(myR, sFT, L);
+      }
+      fence_proxy_async_smem();
+      if (!S.barrier()) break;
+      if (more) {
+        if (threadIdx.x < D) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            sh.vec[k][threadIdx.x] += sh.acc[k][threadIdx.x];
+            sh.acc[k][threadIdx.x] = 0.f;
+          }
+        }
+        if (threadIdx.x == 0) sh.scal += bs_chunk;
+      }
+    }
+  }
+  finish(sh, landed, issued, tmem, G::TCOLS, err);
+}
+
+// ------------------------------------------------------------------ host side
+template <typename K>
+cudaError_t prepare(K kern, int smem) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+template <int D, bool CAUSAL>
+cudaError_t backward_dims(const void *q, const void *k, const void *v, const void *g, void *dq,
+                          void *dk, void *dv, int64_t heads, int64_t n, int64_t seg,
+                          const TcBackwardLayout &W, int *err, cudaStream_t st) {
+  using G = BCfg<D>;
+  const int64_t nseg = (n + seg - 1) / seg;
+  const int64_t rec = rec_floats<D>();
+  const int64_t nitems = heads * nseg;
+  const int64_t sms = sm_count();
+  const unsigned grid = static_cast<unsigned>(nitems < sms * G::CTAS ? nitems : sms * G::CTAS);
+  const unsigned grid_agg =
+      static_cast<unsigned>(nitems < sms * G::G_CTAS ? nitems : sms * G::G_CTAS);
+  CUtensorMap tq, tk, tv, tg, ta, tal;
+  cudaError_t e;
+  if ((e = make_tmap_bf16(&tq, q, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tk, k, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tv, v, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tg, g, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&ta, W.a_hi, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tal, W.a_lo, heads, n, D, C)) != cudaSuccess) return e;
+  // the scans treat a record as 4 x (rec / 4 - 1) + 4 floats: element by element
+  const int sdk = 4, sdv = static_cast<int>(rec / 4 - 1);
+
+  // K1 + K2: the forward record before every segment (causal) or of the head (non-causal)
+  auto kg = bwd_aggregate_kernel<D>;
+  if ((e = prepare(kg, G::G_SMEM)) != cudaSuccess) return e;
+  kg<<<grid_agg, kThreads, G::G_SMEM, st>>>(tk, tv, W.s_rec, n, seg, nseg, nitems, err);
+  count_launches(1);
+  record_launch_event(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const float *s_start = W.s_rec;
+  int64_t s_hs = nseg * rec, s_ss = rec;
+  if (CAUSAL) {
+    e = launch_scan_states(W.s_rec, heads, nseg, sdk, sdv, 0, nullptr, 0, nullptr, 0, nullptr,
+                           nullptr, st);
+  } else {
+    e = launch_scan_states(W.s_rec, heads, nseg, sdk, sdv, 1, W.s_tot, rec, W.s_tot + rec - 4,
+                           rec, nullptr, nullptr, st);
+    s_start = W.s_tot;
+    s_hs = rec;
+    s_ss = 0;
+  }
+  if (e != cudaSuccess) return e;
+
+  // B1: dq, a (hi, lo), b and the reverse record of every segment
+  auto k1 = bwd_prefix_kernel<D, CAUSAL>;
+  if ((e = prepare(k1, G::P_SMEM)) != cudaSuccess) return e;
+  k1<<<grid, kThreads, G::P_SMEM, st>>>(tq, tk, tv, tg, static_cast<__nv_bfloat16 *>(dq),
+                                        W.a_hi, W.a_lo, W.b, s_start, s_hs, s_ss, W.r_rec, n,
+                                        seg, nseg, nitems, err);
+  count_launches(1);
+  record_launch_event(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // K2: the reverse record after every segment (causal) or of the head (non-causal)
+  const float *r_start = W.r_rec;
+  int64_t r_hs = nseg * rec, r_ss = rec;
+  if (CAUSAL) {
+    e = launch_scan_states(W.r_rec, heads, nseg, sdk, sdv, 2, nullptr, 0, nullptr, 0, nullptr,
+                           nullptr, st);
+  } else {
+    e = launch_scan_states(W.r_rec, heads, nseg, sdk, sdv, 1, W.r_tot, rec, W.r_tot + rec - 4,
+                           rec, nullptr, nullptr, st);
+    r_start = W.r_tot;
+    r_hs = rec;
+    r_ss = 0;
+  }
+  if (e != cudaSuccess) return e;
+
+  // B3: dk, dv
+  auto k3 = bwd_suffix_kernel<D, CAUSAL>;
+  if ((e = prepare(k3, G::S_SMEM)) != cudaSuccess) return e;
+  k3<<<grid, kThreads, G::S_SMEM, st>>>(tq, ta, tal, tk, tv, W.b,
+                                        static_cast<__nv_bfloat16 *>(dk),
+                                        static_cast<__nv_bfloat16 *>(dv), r_start, r_hs, r_ss,
+                                        n, seg, nseg, nitems, err);
+  count_launches(1);
+  record_launch_event(st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int64_t tc_backward_segment(int64_t heads, int64_t n, int d) {
+  // the segment (a multiple of 256 tokens, at most 4096) with the smallest loss to partial
+  // waves over every walk CTA slot of the device, preferring long segments (fewer records)
+  const int64_t slots = (int64_t)sm_count() * (d == 64 ? BCfg<64>::CTAS : BCfg<128>::CTAS);
+  int64_t best = 256, best_score = -1;
+  for (int64_t seg = 4096; seg >= 256; seg -= 256) {
+    const int64_t items = heads * ((n + seg - 1) / seg);
+    const int64_t waves = (items + slots - 1) / slots;
+    const int64_t eff = items * 1000 / (waves * slots);
+    if (best_score < 0 || eff > best_score + 30) {
+      best_score = eff;
+      best = seg;
+    }
+  }
+  const int64_t nrounded = (n + C - 1) / C * C;
+  return best > nrounded ? nrounded : best;
+}
+
+TcBackwardLayout tc_backward_layout(void *ws, int64_t heads, int64_t n, int d, int64_t seg,
+                                    size_t *bytes) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  const int64_t rec = (int64_t)d * d + 3 * d + 4;
+  size_t off = 0;
+  char *base = static_cast<char *>(ws);
+  auto take = [&](size_t nbytes) {
+    char *p = base ? base + off : nullptr;
+    off += (nbytes + 255) / 256 * 256;
+    return p;
+  };
+  TcBackwardLayout W;
+  W.s_rec = reinterpret_cast<float *>(take(heads * nseg * rec * sizeof(float)));
+  W.r_rec = reinterpret_cast<float *>(take(heads * nseg * rec * sizeof(float)));
+  W.s_tot = reinterpret_cast<float *>(take(heads * rec * sizeof(float)));
+  W.r_tot = reinterpret_cast<float *>(take(heads * rec * sizeof(float)));
+  W.a_hi = reinterpret_cast<__nv_bfloat16 *>(take(heads * n * d * sizeof(__nv_bfloat16)));
+  W.a_lo = reinterpret_cast<__nv_bfloat16 *>(take(heads * n * d * sizeof(__nv_bfloat16)));
+  W.b = reinterpret_cast<float *>(take(heads * n * sizeof(float)));
+  if (bytes) *bytes = off;
+  return W;
+}
+
+cudaError_t tc_backward(const void *q, const void *k, const void *v, const void *g, void *dq,
+                        void *dk, void *dv, int64_t heads, int64_t n, int d, int causal,
+                        int64_t seg, void *ws, int *err, cudaStream_t st) {
+  const TcBackwardLayout W = tc_backward_layout(ws, heads, n, d, seg, nullptr);
+  if (d == 64)
+    return causal ? backward_dims<64, true>(q, k, v, g, dq, dk, dv, heads, n, seg, W, err, st)
+                  : backward_dims<64, false>(q, k, v, g, dq, dk, dv, heads, n, seg, W, err, st);
+  if (d == 128)
+    return causal ? backward_dims<128, true>(q, k, v, g, dq, dk, dv, heads, n, seg, W, err, st)
+                  : backward_dims<128, false>(q, k, v, g, dq, dk, dv, heads, n, seg, W, err, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace linattn

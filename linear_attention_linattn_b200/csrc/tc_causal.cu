@@ -171,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *qz = reinterpret_cast<float *>(smem + G::OFF_QZ);
   volatile int *abort = &bar.abort;
   const int warp = threadIdx.x >> 5;
+  const bool a32 = aligned32(out);  // output rows take full-sector stores
   const int lane = threadIdx.x & 31;
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
@@ -318,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cg = (t & 7) ^ (r0 & 7);
     const int vec_off = r0 * 128 + (t & 7) * 16;  // byte offset of row r0's vector in an atom
     WarpWaiter wait{abort, err, lane};
+    grid_dependency_wait();  // the prefix states come from the scan before this kernel
     float zr[G::AK][8];
     int g = 0;
     for (int64_t it = it0; it < nitems; it += istep) {
@@ -433,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool vS = DK == 128 || lane < 16;
     uint8_t *sS = smem + G::OFF_S;
     WarpWaiter wait{abort, err, lane};
+    grid_dependency_wait();  // the prefix states come from the scan before this kernel
     // 32 consecutive columns [c0, c0 + 32) of row rS (fp32 bits) -> the bf16 S operand
     auto store_S32 = [&](const uint32_t *r, int c0) {
       if (!vS) return;
@@ -563,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float f[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
-            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8));
+            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8), a32);
           }
         }
       }
@@ -618,8 +621,11 @@ cudaError_t launch_causal(const void *q, const void *k, const void *v, void *out
   // hardware's placement of CTAs evens out the SMs' speed differences.
   const int64_t want = seg <= kPersistentTokens ? (int64_t)sm_count() : nitems;
   const unsigned grid = static_cast<unsigned>(nitems < want ? nitems : want);
-  kern<<<grid, kThreads, G::SMEM, st>>>(tq, tk, tv, static_cast<__nv_bfloat16 *>(out), prefix,
-                                        nseg * per, per, n, seg, nseg, nitems, err);
+  // follows the scan: launched so that its set-up and first loads overlap the scan's tail
+  e = launch_programmatic(kern, dim3(grid), dim3(kThreads), G::SMEM, st, tq, tk, tv,
+                          static_cast<__nv_bfloat16 *>(out), prefix, nseg * per, per, n, seg,
+                          nseg, nitems, err);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();

@@ -71,11 +71,23 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
   u.w = pack_bf16x2(f[6], f[7]);
   return u;
 }
-// One 32-byte store (a full sector): 16 bf16 values.
-__device__ __forceinline__ void st_global_32B(void *p, uint4 a, uint4 b) {
-  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y),
-               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
-               : "memory");
+// 32 bytes (16 bf16 values) to global memory: one full-sector store where the buffer is
+// 32-byte aligned (a32), else two 16-byte stores.  Callers promise only 16-byte aligned
+// buffers; a row's alignment is its buffer's (rows are 128 or 256 bytes long), so kernels
+// test their output pointer once and pass the result, uniform over the launch.
+__device__ __forceinline__ bool aligned32(const void *p) {
+  return (reinterpret_cast<uintptr_t>(p) & 31u) == 0;
+}
+__device__ __forceinline__ void st_global_32B(void *p, uint4 a, uint4 b, bool a32) {
+  if (a32) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x),
+                 "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+  } else {
+    uint4 *q = static_cast<uint4 *>(p);
+    q[0] = a;
+    q[1] = b;
+  }
 }
 
 // Lane-0 mbarrier wait whose outcome the whole warp shares (warp-uniform control flow).

@@ -181,43 +181,6 @@ __device__ __forceinline__ float convert_P32(uint32_t taddr, uint8_t *sP, int r6
   return sum;
 }
 
-// phi on the 16-byte vectors of a tile in place, NB vectors per thread at a time (loaded
-// together, transformed, stored: the shared-memory latency is paid once per group, not once
-// per vector).  Vector i of the tile sits at base + (i / 512) * atom_stride + (i % 512) * 16
-// (512 vectors per 64-row atom); with mask_rows, rows at or past `valid` become zero instead.
-template <int NV, bool PHI, int NB>
-__device__ __forceinline__ void phi_tile(uint8_t *base, uint32_t atom_stride, int xt,
-                                         int nthreads, bool mask_rows, int valid) {
-  const uint32_t b0 = smem_u32(base);
-  for (int i0 = xt; i0 < NV; i0 += NB * nthreads) {
-    uint4 x[NB];
-    uint32_t live = 0;  // bit u: vector u holds data (else it is outside the tile or masked)
-#pragma unroll
-    for (int u = 0; u < NB; ++u) {
-      const int i = i0 + u * nthreads;
-      const int within = i % (kAtom / 16);
-      const bool ok = i < NV && (!mask_rows || (within >> 3) < valid);  // 8 x 16 B per row
-      live |= ok ? 1u << u : 0u;
-      x[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (ok)
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(x[u].x), "=r"(x[u].y), "=r"(x[u].z), "=r"(x[u].w)
-                     : "r"(b0 + (i / (kAtom / 16)) * atom_stride + within * 16));
-    }
-#pragma unroll
-    for (int u = 0; u < NB; ++u) {
-      const int i = i0 + u * nthreads;
-      if (i < NV && (PHI || mask_rows)) {
-        if (PHI && (live >> u & 1u)) x[u] = phi_bf16x8(x[u]);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(
-                         b0 + (i / (kAtom / 16)) * atom_stride + (i % (kAtom / 16)) * 16),
-                     "r"(x[u].x), "r"(x[u].y), "r"(x[u].z), "r"(x[u].w)
-                     : "memory");
-      }
-    }
-  }
-}
-
 // CTA b takes the items b, b + gridDim.x, b + 2 gridDim.x, ... (one item when the grid
 // covers them all; several on persistent CTAs).  Every role walks the same sequence of
 // chunks, and g counts them across items, so the stage ring, the barrier phases and the O
@@ -248,6 +211,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
   volatile int *abort = &bar.abort;
 
   const int warp = threadIdx.x >> 5;
+  const bool a32 = aligned32(out);  // output rows take full-sector stores
   const int lane = threadIdx.x & 31;
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
@@ -510,13 +474,25 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
         uint8_t *st = smem + s * G::STAGE;
         const int64_t left = I.t_end - (I.t_begin + (int64_t)c * C);
         const int valid = left < C ? static_cast<int>(left) : C;
-        // batches of 4 vectors where registers allow (the aggregate mode runs 22 warps: 2)
-        constexpr int NB = MODE == kState ? 2 : 4;
-        if (G::LQ && PHI)
-          phi_tile<G::AK * kAtom / 16, PHI, NB>(st, kAtom, xt, W::XTHREADS, false, C);
-        if (G::LKV)
-          phi_tile<G::AK * kAtom / 16, PHI, NB>(st + G::OFF_K, G::KATOM, xt, W::XTHREADS, true,
-                                                valid);
+        if (G::LQ && PHI) {
+          uint4 *p = reinterpret_cast<uint4 *>(st);
+#pragma unroll 2
+          for (int i = xt; i < G::AK * kAtom / 16; i += W::XTHREADS) p[i] = phi_bf16x8(p[i]);
+        }
+        if (G::LKV) {
+#pragma unroll 2
+          for (int i = xt; i < G::AK * kAtom / 16; i += W::XTHREADS) {
+            const int a = i / (kAtom / 16), within = i % (kAtom / 16);
+            const int row = within >> 3;  // 8 x 16 B per 128-byte row
+            uint4 *p = reinterpret_cast<uint4 *>(st + G::OFF_K + a * G::KATOM) + within;
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);
+            if (row < valid) {
+              x = *p;
+              if (PHI) x = phi_bf16x8(x);
+            }
+            *p = x;
+          }
+        }
         fence_proxy_async_smem();
         mbar_arrive(&bar.ready[s]);
       }
@@ -535,6 +511,9 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     const int rS = DK == 128 ? 32 * sp + lane : r64;  // row of the S accumulator (M = DK)
     const bool vS = DK == 128 ? true : v64;
     WarpWaiter wait{abort, err, lane};
+    // the output kernels start while the scan before them finishes (a programmatic launch):
+    // the starting states it writes are read only once it is done
+    if (MODE != kState) grid_dependency_wait();
 
     // 32 consecutive S columns [c0, c0+32) of row rS (fp32 in registers) -> bf16 operand sS
     auto store_S32 = [&](uint8_t *sS, const uint32_t *r, int c0) {
@@ -680,7 +659,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
               for (int e = 0; e < 32; e += 8)
                 st_global_32B(dst + (int64_t)rS * DV + c0 + e,
                               make_uint4(r[e], r[e + 1], r[e + 2], r[e + 3]),
-                              make_uint4(r[e + 4], r[e + 5], r[e + 6], r[e + 7]));
+                              make_uint4(r[e + 4], r[e + 5], r[e + 6], r[e + 7]), true);
             }
           }
           const uint32_t zr = tmem_ld1(tS + DV);
@@ -745,7 +724,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
             float f[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
-            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8));
+            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8), a32);
           }
         }
       }
@@ -803,9 +782,18 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
   const bool persistent = MODE != kCausalOut || seg <= kPersistentCausalChunks * C;
   const int64_t want = persistent ? sms : nitems;
   const unsigned grid = static_cast<unsigned>(nitems < want ? nitems : want);
-  kern<<<grid, Warps<MODE>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out),
-                                                    init, ihs, iss, out_state, n, seg, nseg,
-                                                    nitems, err);
+  if (MODE == kState) {
+    kern<<<grid, Warps<MODE>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out),
+                                                      init, ihs, iss, out_state, n, seg, nseg,
+                                                      nitems, err);
+  } else {
+    // the output kernels follow the scan: launched so that their set-up and first loads of
+    // q, k, v overlap the scan's tail (the state group waits for the scan's results)
+    e = launch_programmatic(kern, dim3(grid), dim3(Warps<MODE>::THREADS), G::SMEM, st, q, k, v,
+                            static_cast<__nv_bfloat16 *>(out), init, ihs, iss, out_state, n, seg,
+                            nseg, nitems, err);
+    if (e != cudaSuccess) return e;
+  }
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();
@@ -947,6 +935,22 @@ cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, i
   if (dk == 64 && dv == 128)
     return tc_forward_dims<64, 128, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
                                            init_z, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t tc_segment_aggregates(const void *k, const void *v, int64_t heads, int64_t n, int d,
+                                  int64_t seg, float *out, int *err, cudaStream_t st) {
+  const int64_t nseg = (n + seg - 1) / seg;
+  CUtensorMap tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap_bf16(&tk, k, heads, n, d, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tv, v, heads, n, d, C)) != cudaSuccess) return e;
+  if (d == 64)
+    return launch_tc<64, 64, kState, true>(tk, tk, tv, nullptr, nullptr, 0, 0, out, heads, n, seg,
+                                           nseg, err, st);
+  if (d == 128)
+    return launch_tc<128, 128, kState, true>(tk, tk, tv, nullptr, nullptr, 0, 0, out, heads, n,
+                                             seg, nseg, err, st);
   return cudaErrorInvalidValue;
 }
 

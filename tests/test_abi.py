@@ -94,6 +94,10 @@ def test_backward_init_and_sum_argument_checks(lib):
                                 None) == bad
     assert lib.linattn_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 1, 0,
                                 None) == la.LINATTN_ERR_UNSUPPORTED
+    # backward segments: whole 64-token chunks, not negative
+    for seg in (-64, 100):
+        assert lib.linattn_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1,
+                                       1, seg, None) == bad
     # forward from a state: the state pointers are required
     assert lib.linattn_forward_init(FAKE, FAKE, FAKE, FAKE, 0, FAKE, 1, 1, 8, 64, 1, 1,
                                     None) == bad

@@ -61,6 +61,66 @@ def test_backward_longer_sequence(dtype, causal):
     _check(1, 2, 4096, 64, causal, dtype, 7)
 
 
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("segment_len", [64, 128, 320, 1024])
+def test_backward_bf16_segment_edges(causal, d, segment_len):
+    """The bf16 backward walks segments (work items) chunk by chunk, forwards for dq and
+    backwards for dk and dv, carrying [S | z] and [R | r] across chunks in TMEM and across
+    segments through the scans: moving the segment edges, ragged n included, changes nothing
+    beyond rounding."""
+    B, H, n = 2, 3, 1000
+    dtype = "bf16"
+    q, k, v = (as_io(x, dtype) for x in inputs.forward_qkv(41, B, H, n, d, scaled=True))
+    g = as_io(inputs.forward_qkv(42, B, H, n, d, scaled=True)[0], dtype)
+    dq, dk, dv = la.backward(*(to_dev(x, dtype) for x in (q, k, v, g)), causal,
+                             segment_len=segment_len)
+    assert la.device_error() == la.LINATTN_OK
+    ref = oracle.backward(q, k, v, g, causal)
+    errs = [grad_err(to_host(a), b) for a, b in zip((dq, dk, dv), ref)]
+    assert max(errs) <= TOL[dtype], errs
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_bf16_many_items_per_cta(causal):
+    """More segments than CTA slots (each CTA walks several items, its loads running one chunk
+    ahead across item boundaries), at the shape of the batched benchmark's heads (d = 64)."""
+    B, H, n, d = 2, 16, 2048, 64
+    dtype = "bf16"
+    q, k, v = (as_io(x, dtype) for x in inputs.forward_qkv(43, B, H, n, d, scaled=True))
+    g = as_io(inputs.forward_qkv(44, B, H, n, d, scaled=True)[0], dtype)
+    dq, dk, dv = la.backward(*(to_dev(x, dtype) for x in (q, k, v, g)), causal, segment_len=64)
+    assert la.device_error() == la.LINATTN_OK
+    ref = oracle.backward(q, k, v, g, causal)
+    errs = [grad_err(to_host(a), b) for a, b in zip((dq, dk, dv), ref)]
+    assert max(errs) <= TOL[dtype], errs
+
+
+def test_backward_bf16_unaligned_outputs():
+    """Buffers only 16-byte aligned (the interface's promise): the gradient rows are written
+    with 16-byte stores there."""
+    B, H, n, d = 1, 2, 300, 64
+    dtype = "bf16"
+    q, k, v = (as_io(x, dtype) for x in inputs.forward_qkv(45, B, H, n, d, scaled=True))
+    g = as_io(inputs.forward_qkv(46, B, H, n, d, scaled=True)[0], dtype)
+    qd, kd, vd, gd = (to_dev(x, dtype) for x in (q, k, v, g))
+    numel = B * H * n * d
+    bufs = [torch.full((numel + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+            for _ in range(3)]
+    outs = [b_[8:].view(B, H, n, d) for b_ in bufs]
+    assert all(o.data_ptr() % 32 == 16 for o in outs)
+    lib = la.load_library()
+    st = lib.linattn_backward(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), gd.data_ptr(),
+                              outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(), B, H,
+                              n, d, 1, la.LINATTN_BF16, torch.cuda.current_stream().cuda_stream)
+    assert st == la.LINATTN_OK
+    assert la.device_error() == la.LINATTN_OK
+    ref = oracle.backward(q, k, v, g, True)
+    errs = [grad_err(to_host(a), b) for a, b in zip(outs, ref)]
+    assert max(errs) <= TOL[dtype], errs
+    assert all(torch.isnan(b_[:8].float()).all() for b_ in bufs)
+
+
 def test_value_gradients_sum_to_output_gradients_on_gpu():
     """sum_j dL/dv_j = sum_i dL/dout_i: each output row is a convex combination of values."""
     B, H, n, d = 2, 2, 700, 64

@@ -86,6 +86,22 @@ def test_output_canary_untouched():
             assert bool((buf[:pad] == 12345.0).all()) and bool((buf[-pad:] == 12345.0).all())
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_outputs_only_16_byte_aligned(causal):
+    """The interface promises 16-byte aligned buffers, not 32: an output that starts 16 bytes
+    past a 32-byte boundary is written with 16-byte stores, and matches."""
+    B, H, n, d = 2, 3, 700, 64
+    q, k, v = (as_io(x, "bf16") for x in inputs.forward_qkv(21, B, H, n, d, scaled=True))
+    qd, kd, vd = (to_dev(x, "bf16") for x in (q, k, v))
+    buf = torch.full((qd.numel() + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(qd.shape)
+    assert out.data_ptr() % 32 == 16
+    la.forward(qd, kd, vd, causal, out=out)
+    assert la.device_error() == la.LINATTN_OK
+    assert max_row_rel_err(to_host(out), oracle.forward(q, k, v, causal)) <= TOL["bf16"]
+    assert bool(torch.isnan(buf[:8].float()).all())
+
+
 def test_forward_state_matches_oracle():
     for dtype in ("f32", "bf16"):
         for d in (64, 128):
