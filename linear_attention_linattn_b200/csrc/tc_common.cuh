@@ -90,21 +90,34 @@ __device__ __forceinline__ void st_global_32B(void *p, uint4 a, uint4 b, bool a3
   }
 }
 
-// Lane-0 mbarrier wait whose outcome the whole warp shares (warp-uniform control flow).
-struct WarpWaiter {
+// mbarrier wait of a whole warp whose outcome the lanes share (warp-uniform control flow);
+// a lane whose bounded wait gave up makes the warp give up.  Two forms, chosen per kernel by
+// measurement (the faster one differs with the shape of the work between waits):
+//   LANE0 = false  every lane waits on the barrier itself;
+//   LANE0 = true   lane 0 waits (suspending while the phase is pending), then every lane
+//                  tests the completed phase once, which orders its later reads after the
+//                  barrier like its own wait would.
+template <bool LANE0>
+struct WarpWaiterT {
   volatile int *abort;
   int *err;
   int lane;
   bool ok = true;
   __device__ __forceinline__ bool operator()(uint64_t *b, uint32_t parity) {
-    int r = 1;
-    if (lane == 0) r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
-    r = __shfl_sync(0xffffffffu, r, 0);
-    __syncwarp();  // the other lanes' reads are ordered after lane 0's wait
-    ok = ok && (r != 0);
+    if (LANE0) {
+      int r = 1;
+      if (lane == 0) r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r) mbar_try_wait(b, parity);
+      ok = ok && (r != 0);
+    } else {
+      const int r = (ok && mbar_wait(b, parity, abort, err)) ? 1 : 0;
+      ok = __all_sync(0xffffffffu, r) != 0;
+    }
     return ok;
   }
 };
+using WarpWaiter = WarpWaiterT<false>;
 
 // One work item: tokens [t_begin, t_end) of one head (one segment), in chunks of CH tokens.
 struct Item {

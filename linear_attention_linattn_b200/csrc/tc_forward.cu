@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     const int r64 = 16 * sp + lane;                   // row of an M=64 tile
     const int rS = DK == 128 ? 32 * sp + lane : r64;  // row of the S accumulator (M = DK)
     const bool vS = DK == 128 ? true : v64;
-    WarpWaiter wait{abort, err, lane};
+    WarpWaiterT<(DV >= 128)> wait{abort, err, lane};  // measured per value width
     // the output kernels start while the scan before them finishes (a programmatic launch):
     // the starting states it writes are read only once it is done
     if (MODE != kState) grid_dependency_wait();
@@ -679,7 +679,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(32 * sp) << 16;
     const bool v64 = lane < 16;
     const int r64 = 16 * sp + lane;
-    WarpWaiter wait{abort, err, lane};
+    WarpWaiterT<(DV >= 128)> wait{abort, err, lane};  // measured per value width
 
     // Denominators of the chunks in flight, by parity.  The state group's half of the row sum
     // is read BEFORE this group releases p_ready: the state group's next sums need this
