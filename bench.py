@@ -234,6 +234,18 @@ def forward_launches(dtype: str, causal: bool, unit: int):
              "simt_chunk_out_kernel (K3)"], [2 * unit, 0, 4 * unit if causal else 2 * unit])
 
 
+def backward_launches(causal: bool, unit: int):
+    """Names of the launches of one bf16 backward call, in order, and the algorithmic bytes of
+    each (unit: the bytes of one [B,H,n,d] tensor): K1 reads k, v; B1 reads q, k, v, dout and
+    writes dq (and a, b for the suffix walk); B3 reads q, k, v (and a, b) and writes dk, dv."""
+    return (["bwd_aggregate_kernel (forward records, K1)",
+             "scan_states_kernel (prefix, K2)" if causal else "scan_states_kernel (totals, K2)",
+             "bwd_prefix_kernel (dq, B1)",
+             "scan_states_kernel (suffix, K2)" if causal else "scan_states_kernel (totals, K2)",
+             "bwd_suffix_kernel (dk, dv, B3)"],
+            [2 * unit, 0, 5 * unit, 0, 5 * unit if causal else 4 * unit])
+
+
 def time_launches(fn, steps, warmup, names):
     """Per-launch device times of a multi-kernel call: before each timed call the library is
     given events (linattn_profile_events) that it records after each of its launches on the
@@ -373,9 +385,17 @@ def main_forward(args, world, rank, local):
     del q, k, v
     qd, kd, vd = qh.cuda(), kh.cuda(), vh.cuda()
     out = torch.empty_like(qd)
+    backward = args.pass_ == "backward"
+    if backward:
+        if seq or dtype != "bf16":
+            raise SystemExit("--pass backward times the bf16 backward on whole heads")
+        gd = torch.from_numpy(inputs.forward_qkv(w.seed + 1, w.B, w.H, shape[2], w.d,
+                                                 w.scaled)[0]).to(tdt).cuda()
 
     def step():
-        if seq:
+        if backward:
+            la.backward(qd, kd, vd, gd, causal)
+        elif seq:
             seqshard.forward_sequence_sharded(qd, kd, vd, causal)
         else:
             la.forward(qd, kd, vd, causal, out=out)
@@ -392,7 +412,10 @@ def main_forward(args, world, rank, local):
     pk = peaks()
     alg = forward_bytes(w.B, w.H, shape[2], w.d, elem)  # this rank's share
     unit = w.B * w.H * shape[2] * w.d * elem  # one [B,H,n,d] tensor (this rank's share)
-    names, kbytes = forward_launches(dtype, causal, unit)
+    names, kbytes = (backward_launches(causal, unit) if backward
+                     else forward_launches(dtype, causal, unit))
+    if backward:
+        alg = 7 * unit  # reads q, k, v, dout; writes dq, dk, dv
     if seq:
         # block state (aggregates, total), the start state, then the forward from it
         names = ["block state: aggregates (K1)", "block state: total (K2)",
@@ -416,7 +439,7 @@ def main_forward(args, world, rank, local):
         outh.copy_(o, non_blocking=True)
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not backward:
         e2e_steps = max(1, min(args.steps, 3))
         e2e_ms, _ = time_steps(e2e_step, e2e_steps, 1, world)
         e2e = {"value": tokens_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
@@ -435,13 +458,15 @@ def main_forward(args, world, rank, local):
         del tmp
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC + (" (backward pass)" if backward else ""), "value": value,
+        "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "strong" if seq else "weak", "vs_baseline": None,
         "dtype": dtype,
         "data": "synthetic (per head default_rng([seed, b, h]) draws q, k, v N(0,1), times 1/sqrt(d); bf16-rounded)",
         "config": {"workload": args.workload + (f" (first {w.H} heads)" if args.max_heads else "")
-                   + (f" [{args.mode}]" if args.mode else ""),
+                   + (f" [{args.mode}]" if args.mode else "")
+                   + (" [backward]" if backward else ""),
                    "B": w.B, "H": w.H, "n": w.n, "d": w.d,
                    "causal": causal, "global_batch": w.B if seq else w.B * world,
                    "seq_len": w.n,
@@ -551,14 +576,18 @@ def extras(args):
         res[f"{name}_{'causal' if causal else 'noncausal'}"] = {
             "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
             "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
-    # backward pass on the same shape (causal): reads q, k, v, dout and writes dq, dk, dv
+    # backward pass on the same shape: reads q, k, v, dout and writes dq, dk, dv
     dout = torch.randn_like(o)
-    ms, _ = time_steps(lambda: la.backward(q, k, v, dout, True), 5, 3, 1)
-    alg = 7 * w.B * w.H * w.n * w.d * 2
-    res[f"backward_{name}_causal"] = {
-        "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
-        "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
-        "path": "CUDA cores (float32 FFMA), 6 launches"}
+    for causal in (True, False):
+        fn = lambda: la.backward(q, k, v, dout, causal)  # noqa: E731
+        ms, _ = time_steps(fn, 10, 3, 1)
+        alg = 7 * w.B * w.H * w.n * w.d * 2
+        names = backward_launches(causal, 0)[0]
+        res[f"backward_{name}_{'causal' if causal else 'noncausal'}"] = {
+            "ms": ms, "tokens_per_s": w.B * w.n / (ms * 1e-3), "gbs": alg / (ms * 1e-3) / 1e9,
+            "frac_hbm": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": alg,
+            "launch_ms": time_launches(fn, 5, 2, names),
+            "path": "tensor cores (tcgen05, TMEM, TMA), 5 launches"}
     # FAVOR+ (Performer's positive random features) on the same shape, causal: the features of
     # q and k (m of them), then the pass on them; m = d and m = 2 d
     for m in (w.d, 2 * w.d):
@@ -607,6 +636,8 @@ def main():
                     help="for a workload that has both modes (default: causal)")
     ap.add_argument("--max-heads", type=int, default=0,
                     help="profiling aid: run only the first N heads of the workload")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
+                    help="backward: time the bf16 backward pass (dq, dk, dv) on the workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
