@@ -154,6 +154,9 @@ struct TcBackwardLayout {
   float *s_tot, *r_tot;           // [heads][d*d + 3d + 4]: per-head totals (non-causal)
   __nv_bfloat16 *a_hi, *a_lo;     // [heads][n][d]: a_i = g_i / den_i as a bf16 pair
   float *b;                       // [heads][n]: -(a_i . out_i)
+  // [heads][chunks][3d + 4]: per chunk, the vectors of the forward record before it within
+  // its segment, and the chunk's own reverse-record vectors
+  float *s_vec, *r_vec;
 };
 // Tokens per work item of the backward (a multiple of 256, or n rounded up to kTcChunk).
 int64_t tc_backward_segment(int64_t heads, int64_t n, int d);

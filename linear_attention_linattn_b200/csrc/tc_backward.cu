@@ -70,6 +70,12 @@ __host__ __device__ constexpr int64_t rec_floats() {
   return (int64_t)D * D + 3 * D + 4;
 }
 
+// A chunk's vectors: [three D-vectors | a scalar, three zeros] (the vector part of a record).
+template <int D>
+__host__ __device__ constexpr int64_t vec_floats() {
+  return 3 * D + 4;
+}
+
 struct BwdShared {
   uint64_t full[2];      // stage loaded (TMA transaction bytes)
   uint64_t mma;          // the products issued since the last wait are done
@@ -442,13 +448,15 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     bwd_aggregate_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, float *__restrict__ rec,
-                         int64_t n, int64_t seg_len, int64_t nseg, int64_t nitems, int *err) {
+                         float *__restrict__ chunk_vec, int64_t n, int64_t seg_len, int64_t nseg,
+                         int64_t nitems, int *err) {
   using G = BCfg<D>;
   constexpr int AT = G::AT;
   constexpr int KSC = C / 16;
   constexpr int OK = 0, OV = G::TILE;
   constexpr uint32_t LOAD = 2 * G::TILE;
   constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);
+  const int64_t nck = (n + C - 1) / C;  // chunks per head
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
@@ -532,6 +540,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       S.wait_mma();
       if (!S.barrier()) break;
+      // the item's vectors before its next chunk (exclusive within the item), for the walk
+      if (c + 1 < I.nchunks) {
+        float *cv = chunk_vec + (I.head * nck + I.t_begin / C + c + 1) * vec_floats<D>();
+        if (threadIdx.x < D) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) cv[k * D + threadIdx.x] = sh.acc[k][threadIdx.x];
+        }
+        if (threadIdx.x == 0) cv[3 * D] = kap;
+      }
     }
     if (!S.wait.ok) break;
     float *dst = rec + (I.head * nseg + I.seg) * rec_floats<D>();
@@ -561,7 +578,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
                       const __grid_constant__ CUtensorMap tmG, __nv_bfloat16 *__restrict__ dq,
                       __nv_bfloat16 *__restrict__ a_hi, __nv_bfloat16 *__restrict__ a_lo,
                       float *__restrict__ b_out, const float *__restrict__ start,
-                      int64_t start_hs, int64_t start_ss, float *__restrict__ r_rec, int64_t n,
+                      int64_t start_hs, int64_t start_ss, const float *__restrict__ s_vec,
+                      float *__restrict__ r_rec, float *__restrict__ r_vec, int64_t n,
                       int64_t seg_len, int64_t nseg, int64_t nitems, int *err) {
   using G = BCfg<D>;
   constexpr int AT = G::AT;
@@ -576,6 +594,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   constexpr uint32_t I_O = make_idesc_bf16(64, D, false, true);    // psi(Q) Psi, M V, L V, W psi(K)
   constexpr uint32_t I_T = make_idesc_bf16(64, D, false, false);   // A Psi^T
   constexpr float kD = static_cast<float>(D);
+  constexpr int64_t VF = vec_floats<D>();
+  const int64_t nck = (n + C - 1) / C;  // chunks per head
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -645,7 +665,16 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   for (int64_t it = it0; it < nitems && S.wait.ok; it += istep) {
     const Item I = item_at<C>(it, n, seg_len, nseg);
     // ---- the item's starting forward record: Psi (TMEM, causal) and its operand; vectors
-    load_record<D>(start + I.head * start_hs + I.seg * start_ss, sST, myS, CAUSAL, L, sh);
+    const float *rec0 = start + I.head * start_hs + I.seg * start_ss;
+    load_record<D>(rec0, sST, myS, CAUSAL, L, sh);
+    // the record's vectors (threads t < D, column t) and scalar (thread 0), to which each
+    // chunk's exclusive sums within the item (from the aggregate kernel) are added
+    float base[3] = {0.f, 0.f, 0.f}, base_s = 0.f;
+    if (CAUSAL && threadIdx.x < D) {
+#pragma unroll
+      for (int k = 0; k < 3; ++k) base[k] = rec0[(int64_t)D * D + k * D + threadIdx.x];
+    }
+    if (CAUSAL && threadIdx.x == 0) base_s = rec0[(int64_t)D * D + 3 * D];
     float bs_acc = 0.f;  // thread 0: bs of the item (its vectors gather in sh.racc)
     for (int c = 0; c < I.nchunks; ++c, ++g) {
       uint8_t *st = sm + (g & 1) * G::P_STAGE;
@@ -657,12 +686,30 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       const int64_t row = I.head * n + t0 + L.r64;  // global row of this thread (when live)
       // keys row i sees: every key up to it (causal), all n (non-causal)
       const float Ni = CAUSAL ? static_cast<float>(t0 + L.r64 + 1) : static_cast<float>(n);
+      const int64_t slot = I.head * nck + t0 / C;  // this chunk's per-chunk vectors
+      // causal: the forward record before this chunk = the item's record + the item's chunks
+      // before this one; fetched now, stored once the stage has landed
+      float fv[3] = {0.f, 0.f, 0.f}, fs = 0.f;
+      if (CAUSAL && c > 0) {
+        if (threadIdx.x < D) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) fv[k] = s_vec[slot * VF + k * D + threadIdx.x];
+        }
+        if (threadIdx.x == 0) fs = s_vec[slot * VF + 3 * D];
+      }
 
       // ---- (a) psi on Q and K (K rows past the item's end zeroed), with row sums
       if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
         if (threadIdx.x == 0) landed = g + 1;
         psi_tile<D>(st + OQ, C, sh.sq);
         if (CAUSAL) psi_tile<D>(st + OK, valid, sh.sk);
+      }
+      if (CAUSAL && c > 0) {
+        if (threadIdx.x < D) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) sh.vec[k][threadIdx.x] = base[k] + fv[k];
+        }
+        if (threadIdx.x == 0) sh.scal = base_s + fs;
       }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
@@ -704,7 +751,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           for (int e = 0; e < 8; ++e) dpart = fmaf(f[e], sh.vec[0][c0 + e], dpart);
         }
       }
-      float kap_chunk = 0.f;  // thread 0: kappa of this chunk's keys
       if (CAUSAL) {
         // ---- (c) M = mask(P' + sk) (j <= i) rounded into its operand; row sums of M
         S.wait_mma();
@@ -738,25 +784,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           for (int ks = 0; ks < KSC; ++ks)
             mma_bf16_ss(tX, kdesc(uW, ks, kAtom), mdesc(uV, ks, kAtom), I_O, 1u);
           mma_commit(&sh.mma);
-        }
-        // this chunk's part of the next chunk's forward record: zeta, vs, sigma (sh.acc), kappa
-        if (more) {
-          column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
-            float kr[8], vr[8];
-            tile_row8(st + OK, i, c, kr);
-            tile_row8(st + OV, i, c, vr);
-            const float w = i < valid ? 1.f : 0.f, ski = sh.sk[i];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              t[0][e] += kr[e];
-              t[1][e] = fmaf(w, vr[e], t[1][e]);
-              t[2][e] = fmaf(w * ski, vr[e], t[2][e]);
-            }
-          });
-          if (L.warp == 0) {
-            const float ks = warp_sum64([&](int i) { return sh.sk[i]; });
-            if (threadIdx.x == 0) kap_chunk = ks;
-          }
         }
       } else {
         if (L.v64) sh.part[L.hf][L.r64] = dpart;
@@ -854,7 +881,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       }
       // this chunk's part of the item's reverse record: rho, as, tau (sh.racc), bs; b of each
       // row from the exchanged partial dot products, zero past the item's end (so is a)
-      column_sums3<D>(sh.racc, [&](int i, int c, float (*t)[8]) {
+      column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
         float qr[8], ar[8], lr[8];
         tile_row8(st + OQ, i, c, qr);
         tile_row8(sA, i, c, ar);
@@ -868,10 +895,11 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           t[2][e] = fmaf(sqi, aa, t[2][e]);
         }
       });
+      float bs_chunk = 0.f;  // thread 0: bs of this chunk's rows
       if (L.warp == 0) {
         const float bsum =
             warp_sum64([&](int i) { return i < valid ? -(sh.gd[0][i] + sh.gd[1][i]) : 0.f; });
-        if (threadIdx.x == 0) bs_acc += bsum;
+        if (threadIdx.x == 0) bs_chunk = bsum;
       }
       S.wait_mma();
       if (CAUSAL) {
@@ -927,16 +955,19 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         }
       }
       if (!S.barrier()) break;
-      if (more) {
-        // the forward record after this chunk
-        if (threadIdx.x < D) {
+      // this chunk's reverse sums: into the item's record, and (causal) to the suffix walk
+      if (threadIdx.x < D) {
 #pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            sh.vec[k][threadIdx.x] += sh.acc[k][threadIdx.x];
-            sh.acc[k][threadIdx.x] = 0.f;
-          }
+        for (int k = 0; k < 3; ++k) {
+          const float x = sh.acc[k][threadIdx.x];
+          sh.racc[k][threadIdx.x] += x;
+          sh.acc[k][threadIdx.x] = 0.f;
+          if (CAUSAL) r_vec[slot * VF + k * D + threadIdx.x] = x;
         }
-        if (threadIdx.x == 0) sh.scal += kap_chunk;
+      }
+      if (threadIdx.x == 0) {
+        bs_acc += bs_chunk;
+        if (CAUSAL) r_vec[slot * VF + 3 * D] = bs_chunk;
       }
     }
     if (!S.wait.ok) break;
@@ -968,7 +999,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
                       const __grid_constant__ CUtensorMap tmV, const float *__restrict__ b_in,
                       __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
                       const float *__restrict__ start, int64_t start_hs, int64_t start_ss,
-                      int64_t n, int64_t seg_len, int64_t nseg, int64_t nitems, int *err) {
+                      const float *__restrict__ r_vec, int64_t n, int64_t seg_len, int64_t nseg,
+                      int64_t nitems, int *err) {
   using G = BCfg<D>;
   constexpr int AT = G::AT;
   constexpr int KSD = D / 16;
@@ -982,6 +1014,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   constexpr uint32_t I_O = make_idesc_bf16(64, D, false, true);    // psi(K) Phi, W A, W psi(Q)
   constexpr uint32_t I_T = make_idesc_bf16(64, D, false, false);   // V Phi^T
   constexpr float kD = static_cast<float>(D);
+  constexpr int64_t VF = vec_floats<D>();
+  const int64_t nck = (n + C - 1) / C;  // chunks per head
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1056,9 +1090,19 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       const bool live = L.v64 && L.r64 < valid;
       const int64_t row = I.head * n + t0 + L.r64;
 
-      // b of the chunk's rows, fetched while the tiles land (zero past the item's end)
+      // b of the chunk's rows, fetched while the tiles land (zero past the item's end), and
+      // this chunk's reverse sums (from the prefix walk), added to the record after it
       float bload = 0.f;
       if (CAUSAL && threadIdx.x < valid) bload = b_in[I.head * n + t0 + threadIdx.x];
+      float rv[3] = {0.f, 0.f, 0.f}, rs = 0.f;
+      if (more) {
+        const float *src = r_vec + (I.head * nck + t0 / C) * VF;
+        if (threadIdx.x < D) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) rv[k] = src[k * D + threadIdx.x];
+        }
+        if (threadIdx.x == 0) rs = src[3 * D];
+      }
       // ---- (a) psi on K (row sums); causal: psi on Q (row sums) and the rows of Q and A past
       //     the item's end zeroed
       if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
@@ -1120,7 +1164,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         }
         sh.gd[L.hf][L.r64] = vdot;
       }
-      float bs_chunk = 0.f;  // thread 0: bs of this chunk's rows
       if (CAUSAL) {
         // ---- (c) row j: the weights w_ji = d + sq_i + sk_j + P'^T_ji and dW^T_ji + b_i, kept
         //     for i >= j and rounded into their operands; C'_j's part from this chunk
@@ -1173,27 +1216,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           }
           mma_commit(&sh.mma);
         }
-        // this chunk's part of the record before it: rho, as, tau (sh.acc), bs
-        if (more) {
-          column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
-            float qr[8], ar[8], lr[8];
-            tile_row8(st + OQ, i, c, qr);
-            tile_row8(st + OA, i, c, ar);
-            tile_row8(st + OAL, i, c, lr);
-            const float bi = sh.bv[i], sqi = sh.sq[i];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float aa = ar[e] + lr[e];
-              t[0][e] = fmaf(qr[e], bi, t[0][e]);
-              t[1][e] += aa;
-              t[2][e] = fmaf(sqi, aa, t[2][e]);
-            }
-          });
-          if (L.warp == 0) {
-            const float bsum = warp_sum64([&](int i) { return sh.bv[i]; });
-            if (threadIdx.x == 0) bs_chunk = bsum;
-          }
-        }
       }
       // ---- (e) dv_j = (d + sk_j) as + tau + dV'_j;  dk_j = (dK'_j + rho + C'_j) phi'(k_j),
       //     C'_j = v_j . as + bs + (this chunk's sum_{i >= j} dW_ij);  Phi -> operand
@@ -1237,14 +1259,12 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       fence_proxy_async_smem();
       if (!S.barrier()) break;
       if (more) {
+        // the record before this chunk
         if (threadIdx.x < D) {
 #pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            sh.vec[k][threadIdx.x] += sh.acc[k][threadIdx.x];
-            sh.acc[k][threadIdx.x] = 0.f;
-          }
+          for (int k = 0; k < 3; ++k) sh.vec[k][threadIdx.x] += rv[k];
         }
-        if (threadIdx.x == 0) sh.scal += bs_chunk;
+        if (threadIdx.x == 0) sh.scal += rs;
       }
     }
   }
@@ -1283,7 +1303,8 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   // K1 + K2: the forward record before every segment (causal) or of the head (non-causal)
   auto kg = bwd_aggregate_kernel<D>;
   if ((e = prepare(kg, G::G_SMEM)) != cudaSuccess) return e;
-  kg<<<grid_agg, kThreads, G::G_SMEM, st>>>(tk, tv, W.s_rec, n, seg, nseg, nitems, err);
+  kg<<<grid_agg, kThreads, G::G_SMEM, st>>>(tk, tv, W.s_rec, W.s_vec, n, seg, nseg, nitems,
+                                            err);
   count_launches(1);
   record_launch_event(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1305,8 +1326,8 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   auto k1 = bwd_prefix_kernel<D, CAUSAL>;
   if ((e = prepare(k1, G::P_SMEM)) != cudaSuccess) return e;
   k1<<<grid, kThreads, G::P_SMEM, st>>>(tq, tk, tv, tg, static_cast<__nv_bfloat16 *>(dq),
-                                        W.a_hi, W.a_lo, W.b, s_start, s_hs, s_ss, W.r_rec, n,
-                                        seg, nseg, nitems, err);
+                                        W.a_hi, W.a_lo, W.b, s_start, s_hs, s_ss, W.s_vec,
+                                        W.r_rec, W.r_vec, n, seg, nseg, nitems, err);
   count_launches(1);
   record_launch_event(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1332,7 +1353,7 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   k3<<<grid, kThreads, G::S_SMEM, st>>>(tq, ta, tal, tk, tv, W.b,
                                         static_cast<__nv_bfloat16 *>(dk),
                                         static_cast<__nv_bfloat16 *>(dv), r_start, r_hs, r_ss,
-                                        n, seg, nseg, nitems, err);
+                                        W.r_vec, n, seg, nseg, nitems, err);
   count_launches(1);
   record_launch_event(st);
   return cudaGetLastError();
@@ -1377,6 +1398,9 @@ TcBackwardLayout tc_backward_layout(void *ws, int64_t heads, int64_t n, int d, i
   W.a_hi = reinterpret_cast<__nv_bfloat16 *>(take(heads * n * d * sizeof(__nv_bfloat16)));
   W.a_lo = reinterpret_cast<__nv_bfloat16 *>(take(heads * n * d * sizeof(__nv_bfloat16)));
   W.b = reinterpret_cast<float *>(take(heads * n * sizeof(float)));
+  const int64_t nck = (n + C - 1) / C;
+  W.s_vec = reinterpret_cast<float *>(take(heads * nck * (3 * d + 4) * sizeof(float)));
+  W.r_vec = reinterpret_cast<float *>(take(heads * nck * (3 * d + 4) * sizeof(float)));
   if (bytes) *bytes = off;
   return W;
 }
