@@ -445,7 +445,7 @@ __device__ __forceinline__ uint64_t mdesc(uint32_t base, int ks, uint32_t atom) 
 // k, v: [heads][n][D] via tmK, tmV.  Writes each item's record [Psi | zeta | vs | sigma |
 // kappa] to rec + (head * nseg + seg) * rec_floats<D>().
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
     bwd_aggregate_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, float *__restrict__ rec,
                          float *__restrict__ chunk_vec, int64_t n, int64_t seg_len, int64_t nseg,
