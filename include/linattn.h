@@ -119,6 +119,32 @@ linattn_status linattn_forward_init(const void *q, const void *k, const void *v,
                                     linattn_dtype dtype, linattn_stream_t stream);
 
 /*
+ * The two calls of a sequence-sharded block that read its k, v once: linattn_forward_state_keep
+ * is linattn_forward_state that also leaves the block's aggregates in `aggregates` (caller-
+ * owned device memory of linattn_block_aggregates_bytes(B, H, n, d, dtype) bytes, 16-byte
+ * aligned); linattn_forward_init_from is linattn_forward_init that takes them from there
+ * instead of recomputing them from k, v.  The pair must see the same B, H, n, d, dtype and
+ * device, with nothing between them writing k, v or the buffer; linattn_forward_init_from
+ * overwrites the buffer (causal: its exclusive prefixes).  linattn_block_aggregates_bytes
+ * returns 0 for arguments linattn_forward_state would reject.  Other arguments, layouts and
+ * errors as in linattn_forward_state and linattn_forward_init.  (Pages: "Efficient
+ * Transformers: Linear Attention and Flash Attention", section "The recurrent view: attention
+ * as an RNN": a block's state is the sum of its tokens' contributions, so the sums the state
+ * needs are the ones the block's own pass starts from.)
+ */
+size_t linattn_block_aggregates_bytes(int64_t B, int64_t H, int64_t n, int64_t d,
+                                      linattn_dtype dtype);
+linattn_status linattn_forward_state_keep(const void *k, const void *v, float *state_S,
+                                          float *state_z, float *aggregates, int64_t B,
+                                          int64_t H, int64_t n, int64_t d, linattn_dtype dtype,
+                                          linattn_stream_t stream);
+linattn_status linattn_forward_init_from(const void *q, const void *k, const void *v,
+                                         void *out, const float *state_S, const float *state_z,
+                                         float *aggregates, int64_t B, int64_t H, int64_t n,
+                                         int64_t d, int causal, linattn_dtype dtype,
+                                         linattn_stream_t stream);
+
+/*
  * Performer's FAVOR+ positive random features (named on the page "Efficient Transformers:
  * Linear Attention and Flash Attention", section "Linear attention: reordering the matmuls,
  * not shrinking them", as features whose dot products approximate the softmax kernel

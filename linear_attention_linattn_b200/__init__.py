@@ -60,6 +60,11 @@ SIGNATURES = {
                                         _i64, ctypes.c_int, ctypes.c_int, _vp]),
     "linattn_backward_ex": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
                                            _i64, _i64, ctypes.c_int, ctypes.c_int, _i64, _vp]),
+    "linattn_block_aggregates_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, ctypes.c_int]),
+    "linattn_forward_state_keep": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                  _i64, ctypes.c_int, _vp]),
+    "linattn_forward_init_from": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                                 _i64, _i64, ctypes.c_int, ctypes.c_int, _vp]),
     "linattn_favor_features": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int,
                                               _vp]),
     "linattn_selftest_wait_timeout": (ctypes.c_int, [_vp]),
@@ -152,10 +157,11 @@ def forward(q, k, v, causal: bool, out=None, segment_len: int = 0, stream=None):
     return out
 
 
-def forward_init(q, k, v, S0, z0, causal: bool, out=None, stream=None):
+def forward_init(q, k, v, S0, z0, causal: bool, out=None, aggregates=None, stream=None):
     """forward continued from a state: S0 [B, H, d, d] and z0 [B, H, d] (float32) hold what
     the tokens before this block (causal) or the rest of the sequence (non-causal)
-    contribute."""
+    contribute.  aggregates: the buffer forward_state(k, v, keep=True) returned for the same
+    k, v (its sums are reused instead of recomputed, and the buffer is overwritten)."""
     import torch
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (S0, "S0"), (z0, "z0")):
         _dev(t, nm)
@@ -169,6 +175,17 @@ def forward_init(q, k, v, S0, z0, causal: bool, out=None, stream=None):
         out = torch.empty_like(q)
     _dev(out, "out")
     lib = load_library()
+    if aggregates is not None:
+        _dev(aggregates, "aggregates")
+        if aggregates.numel() * aggregates.element_size() < lib.linattn_block_aggregates_bytes(
+                B, H, n, d, _dtype_code(q)):
+            raise ValueError("aggregates is smaller than this block's aggregates")
+        st = lib.linattn_forward_init_from(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           out.data_ptr(), S0.data_ptr(), z0.data_ptr(),
+                                           aggregates.data_ptr(), B, H, n, d, int(bool(causal)),
+                                           _dtype_code(q), _stream_ptr(stream))
+        _check(st, "linattn_forward_init_from")
+        return out
     st = lib.linattn_forward_init(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                   S0.data_ptr(), z0.data_ptr(), B, H, n, d, int(bool(causal)),
                                   _dtype_code(q), _stream_ptr(stream))
@@ -267,8 +284,10 @@ def backward(q, k, v, dout, causal: bool, segment_len: int = 0, stream=None):
     return dq, dk, dv
 
 
-def forward_state(k, v, S=None, z=None, stream=None):
-    """Final causal state of k, v [B, H, n, d]: S [B, H, d, d] and z [B, H, d] (float32)."""
+def forward_state(k, v, S=None, z=None, keep: bool = False, stream=None):
+    """Final causal state of k, v [B, H, n, d]: S [B, H, d, d] and z [B, H, d] (float32).
+    keep=True also returns the block's aggregates (a float32 device buffer) for
+    forward_init(..., aggregates=...), which then skips summing k, v again."""
     import torch
     _dev(k, "k")
     _dev(v, "v")
@@ -278,6 +297,16 @@ def forward_state(k, v, S=None, z=None, stream=None):
     if z is None:
         z = torch.empty((B, H, d), dtype=torch.float32, device=k.device)
     lib = load_library()
+    if keep:
+        nbytes = lib.linattn_block_aggregates_bytes(B, H, n, d, _dtype_code(k))
+        if nbytes == 0:
+            raise ValueError("unsupported shape or dtype for the block's aggregates")
+        agg = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=k.device)
+        st = lib.linattn_forward_state_keep(k.data_ptr(), v.data_ptr(), S.data_ptr(),
+                                            z.data_ptr(), agg.data_ptr(), B, H, n, d,
+                                            _dtype_code(k), _stream_ptr(stream))
+        _check(st, "linattn_forward_state_keep")
+        return S, z, agg
     st = lib.linattn_forward_state(k.data_ptr(), v.data_ptr(), S.data_ptr(), z.data_ptr(),
                                    B, H, n, d, _dtype_code(k), _stream_ptr(stream))
     _check(st, "linattn_forward_state")

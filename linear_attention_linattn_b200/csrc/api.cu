@@ -147,15 +147,16 @@ ForwardPlan plan_forward(int64_t heads, int64_t n, int dk, int d, int causal, in
 cudaError_t run_forward(const ForwardPlan &p, const void *q, const void *k, const void *v,
                         void *out, int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
                         const float *init_S, const float *init_z, int features, void *ws,
-                        int *err, cudaStream_t st) {
+                        int *err, cudaStream_t st, float *aggregates) {
   if (is_bf16)
     return tc_forward(q, k, v, out, heads, n, dk, d, causal, p.seg, ws, err, init_S, init_z,
-                      features, st);
+                      features, st, aggregates);
   if (dk != d) return cudaErrorInvalidValue;  // the CUDA-core kernels keep one dimension
   const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
   const int64_t per = (int64_t)d * d + d;
-  float *w = static_cast<float *>(ws);
-  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, d, 0, features, st);
+  float *w = aggregates ? aggregates : static_cast<float *>(ws);
+  cudaError_t e = cudaSuccess;
+  if (!aggregates) e = launch_simt_chunk_state(k, v, w, heads, n, d, 0, features, st);
   if (e != cudaSuccess) return e;
   if (causal) {
     e = launch_scan_states(w, heads, nchunks, d, d, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
@@ -163,7 +164,7 @@ cudaError_t run_forward(const ForwardPlan &p, const void *q, const void *k, cons
     return launch_simt_chunk_out(q, k, v, out, w, w + (int64_t)d * d, per, nchunks * per, per,
                                  nchunks * per, heads, n, d, 1, 0, features, st);
   }
-  float *tot = w + heads * nchunks * per;
+  float *tot = aggregates ? static_cast<float *>(ws) : w + heads * nchunks * per;
   float *tot_z = tot + heads * (int64_t)d * d;
   e = launch_scan_states(w, heads, nchunks, d, d, 1, tot, (int64_t)d * d, tot_z, d, init_S, init_z,
                          st);
@@ -324,6 +325,31 @@ linattn_status linattn_forward(const void *q, const void *k, const void *v, void
   return linattn_forward_ex(q, k, v, out, B, H, n, d, causal, dtype, 0, stream);
 }
 
+// The block state of k, v into state_S / state_z, its aggregates left in agg (bf16: per
+// segment, fp32: per 64-token chunk; [heads][..][d*d + d] fp32).
+static cudaError_t forward_state_into(const void *k, const void *v, float *state_S,
+                                      float *state_z, int64_t heads, int64_t n, int64_t d,
+                                      int is_bf16, float *agg, int *err, cudaStream_t st) {
+  if (is_bf16) {
+    const int64_t seg = tc_default_segment(heads, n, (int)d);
+    return tc_forward_state(k, v, state_S, state_z, heads, n, (int)d, seg, agg, err, st);
+  }
+  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
+  cudaError_t e = launch_simt_chunk_state(k, v, agg, heads, n, (int)d, 0, 0, st);
+  if (e == cudaSuccess)
+    e = launch_scan_states(agg, heads, nchunks, (int)d, (int)d, 1, state_S, d * d, state_z, d,
+                           nullptr, nullptr, st);
+  return e;
+}
+
+static size_t block_aggregate_bytes(int64_t heads, int64_t n, int64_t d, int is_bf16) {
+  const int64_t per = d * d + d;
+  const int64_t units = is_bf16 ? (n + tc_default_segment(heads, n, (int)d) - 1) /
+                                      tc_default_segment(heads, n, (int)d)
+                                : (n + kSimtChunk - 1) / kSimtChunk;
+  return (size_t)(heads * units * per) * sizeof(float);
+}
+
 linattn_status linattn_forward_state(const void *k, const void *v, float *state_S,
                                      float *state_z, int64_t B, int64_t H, int64_t n, int64_t d,
                                      linattn_dtype dtype, linattn_stream_t stream) {
@@ -334,27 +360,64 @@ linattn_status linattn_forward_state(const void *k, const void *v, float *state_
   if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t heads = B * H;
+  const int is_bf16 = dtype == LINATTN_BF16;
   Workspace ws;
   ws.st = st;
-  if (dtype == LINATTN_BF16) {
-    const int64_t seg = tc_default_segment(heads, n, (int)d);
-    if (cudaMallocFromPoolAsync(&ws.ptr, tc_workspace_bytes(heads, n, (int)d, (int)d, seg, 0), ds->pool,
-                                st) != cudaSuccess)
-      return LINATTN_ERR_CUDA;
-    return to_status(tc_forward_state(k, v, state_S, state_z, heads, n, (int)d, seg, ws.ptr,
-                                      ds->err_word, st));
-  }
-  const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
-  const int64_t per = d * d + d;
-  if (cudaMallocFromPoolAsync(&ws.ptr, (size_t)(heads * nchunks * per) * 4, ds->pool, st) !=
-      cudaSuccess)
+  if (cudaMallocFromPoolAsync(&ws.ptr, block_aggregate_bytes(heads, n, d, is_bf16), ds->pool,
+                              st) != cudaSuccess)
     return LINATTN_ERR_CUDA;
-  float *w = static_cast<float *>(ws.ptr);
-  cudaError_t e = launch_simt_chunk_state(k, v, w, heads, n, (int)d, 0, 0, st);
-  if (e == cudaSuccess)
-    e = launch_scan_states(w, heads, nchunks, (int)d, (int)d, 1, state_S, d * d, state_z, d, nullptr,
-                           nullptr, st);
-  return to_status(e);
+  return to_status(forward_state_into(k, v, state_S, state_z, heads, n, d, is_bf16,
+                                      static_cast<float *>(ws.ptr), ds->err_word, st));
+}
+
+size_t linattn_block_aggregates_bytes(int64_t B, int64_t H, int64_t n, int64_t d,
+                                      linattn_dtype dtype) {
+  if (B <= 0 || H <= 0 || n <= 0 || B > (1 << 24) || H > (1 << 24) || B * H > (1 << 24) ||
+      n >= (int64_t(1) << 31) || (d != 64 && d != 128) ||
+      (dtype != LINATTN_F32 && dtype != LINATTN_BF16))
+    return 0;
+  return block_aggregate_bytes(B * H, n, d, dtype == LINATTN_BF16);
+}
+
+linattn_status linattn_forward_state_keep(const void *k, const void *v, float *state_S,
+                                          float *state_z, float *aggregates, int64_t B,
+                                          int64_t H, int64_t n, int64_t d, linattn_dtype dtype,
+                                          linattn_stream_t stream) {
+  linattn_status s = check_forward_args(k, k, v, state_S, B, H, n, d, 0, dtype);
+  if (s != LINATTN_OK) return s;
+  if (!state_z || !aligned16(state_z) || !aggregates || !aligned16(aggregates))
+    return LINATTN_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  return to_status(forward_state_into(k, v, state_S, state_z, B * H, n, d,
+                                      dtype == LINATTN_BF16, aggregates, ds->err_word,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+linattn_status linattn_forward_init_from(const void *q, const void *k, const void *v,
+                                         void *out, const float *state_S, const float *state_z,
+                                         float *aggregates, int64_t B, int64_t H, int64_t n,
+                                         int64_t d, int causal, linattn_dtype dtype,
+                                         linattn_stream_t stream) {
+  linattn_status s = check_forward_args(q, k, v, out, B, H, n, d, causal, dtype);
+  if (s != LINATTN_OK) return s;
+  if (!state_S || !state_z || !aligned16(state_S) || !aligned16(state_z) || !aggregates ||
+      !aligned16(aggregates))
+    return LINATTN_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t heads = B * H;
+  const int is_bf16 = dtype == LINATTN_BF16;
+  const ForwardPlan p = plan_forward(heads, n, (int)d, (int)d, causal, is_bf16, 0);
+  // the aggregates are given: the workspace holds only the non-causal per-head totals
+  Workspace ws;
+  ws.st = st;
+  if (!causal && cudaMallocFromPoolAsync(&ws.ptr, (size_t)(heads * (d * d + d)) * sizeof(float),
+                                         ds->pool, st) != cudaSuccess)
+    return LINATTN_ERR_CUDA;
+  return to_status(run_forward(p, q, k, v, out, heads, n, (int)d, (int)d, causal, is_bf16,
+                               state_S, state_z, 0, ws.ptr, ds->err_word, st, aggregates));
 }
 
 linattn_status linattn_decode_step(float *state_S, float *state_z, const void *q, const void *k,

@@ -49,10 +49,13 @@ ForwardPlan plan_forward(int64_t heads, int64_t n, int dk, int d, int causal, in
 // and the word that bounded waits report a give-up in.  init_S / init_z (nullable): the state
 // before each head's first token (causal) or what the rest of the sequence contributes
 // (non-causal).  features != 0: q and k are non-negative features already.
+// aggregates (nullable): the pass's per-segment (bf16) or per-chunk (fp32) aggregates as
+// linattn_forward_state_keep left them; the aggregate launch is then skipped, the causal scan
+// rewrites them in place, and ws needs only the per-head totals (non-causal).
 cudaError_t run_forward(const ForwardPlan &p, const void *q, const void *k, const void *v,
                         void *out, int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
                         const float *init_S, const float *init_z, int features, void *ws,
-                        int *err, cudaStream_t st);
+                        int *err, cudaStream_t st, float *aggregates = nullptr);
 // The no-allocation entry point's status word (noalloc.cu): reads it for the current device
 // into *word and clears it.  *word = 0 when that entry point has not run on this device.
 cudaError_t noalloc_take_status(int *word);
@@ -137,7 +140,7 @@ size_t tc_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg,
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
                        int64_t n, int dk, int dv, int causal, int64_t seg, void *ws, int *err,
                        const float *init_S, const float *init_z, int features,
-                       cudaStream_t st);
+                       cudaStream_t st, float *aggregates = nullptr);
 cudaError_t tc_forward_state(const void *k, const void *v, float *S_out, float *z_out,
                              int64_t heads, int64_t n, int d, int64_t seg, void *ws, int *err,
                              cudaStream_t st);

@@ -804,7 +804,8 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
 template <int DK, int DV, bool PHI>
 cudaError_t tc_forward_dims(const void *q, const void *k, const void *v, void *out,
                             int64_t heads, int64_t n, int causal, int64_t seg, void *ws, int *err,
-                            const float *init_S, const float *init_z, cudaStream_t st) {
+                            const float *init_S, const float *init_z, cudaStream_t st,
+                            float *aggregates) {
   const int64_t nseg = (n + seg - 1) / seg;
   const int64_t per = (int64_t)DK * DV + DK;
   CUtensorMap tq, tk, tv;
@@ -812,10 +813,13 @@ cudaError_t tc_forward_dims(const void *q, const void *k, const void *v, void *o
   if ((e = make_tmap_bf16(&tq, q, heads, n, DK, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tk, k, heads, n, DK, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tv, v, heads, n, DV, C)) != cudaSuccess) return e;
-  float *w = static_cast<float *>(ws);
-  e = launch_tc<DK, DV, kState, PHI>(tk, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg, err,
-                                     st);
-  if (e != cudaSuccess) return e;
+  // the segment aggregates: computed here (K1), or given
+  float *w = aggregates ? aggregates : static_cast<float *>(ws);
+  if (!aggregates) {
+    e = launch_tc<DK, DV, kState, PHI>(tk, tk, tv, out, nullptr, 0, 0, w, heads, n, seg, nseg,
+                                       err, st);
+    if (e != cudaSuccess) return e;
+  }
   if (causal) {
     e = launch_scan_states(w, heads, nseg, DK, DV, 0, nullptr, 0, nullptr, 0, init_S, init_z, st);
     if (e != cudaSuccess) return e;
@@ -828,7 +832,7 @@ cudaError_t tc_forward_dims(const void *q, const void *k, const void *v, void *o
       return tc_causal_features(q, k, v, out, heads, n, DK, DV, seg, w, err, st);
   }
   // per-head totals, packed as [heads][DK*DV + DK] (S row-major, then z)
-  float *tot = w + heads * nseg * per;
+  float *tot = aggregates ? static_cast<float *>(ws) : w + heads * nseg * per;
   e = launch_scan_states(w, heads, nseg, DK, DV, 1, tot, per, tot + (int64_t)DK * DV, per, init_S,
                          init_z, st);
   if (e != cudaSuccess) return e;
@@ -913,28 +917,28 @@ size_t tc_workspace_bytes(int64_t heads, int64_t n, int dk, int dv, int64_t seg,
 cudaError_t tc_forward(const void *q, const void *k, const void *v, void *out, int64_t heads,
                        int64_t n, int dk, int dv, int causal, int64_t seg, void *ws, int *err,
                        const float *init_S, const float *init_z, int features,
-                       cudaStream_t st) {
+                       cudaStream_t st, float *aggregates) {
   if (!features) {  // phi = elu + 1 keeps the dimension
     if (dk == 64 && dv == 64)
       return tc_forward_dims<64, 64, true>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                           init_z, st);
+                                           init_z, st, aggregates);
     if (dk == 128 && dv == 128)
       return tc_forward_dims<128, 128, true>(q, k, v, out, heads, n, causal, seg, ws, err,
-                                             init_S, init_z, st);
+                                             init_S, init_z, st, aggregates);
     return cudaErrorInvalidValue;
   }
   if (dk == 64 && dv == 64)
     return tc_forward_dims<64, 64, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                          init_z, st);
+                                          init_z, st, aggregates);
   if (dk == 128 && dv == 128)
     return tc_forward_dims<128, 128, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                            init_z, st);
+                                            init_z, st, aggregates);
   if (dk == 128 && dv == 64)
     return tc_forward_dims<128, 64, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                           init_z, st);
+                                           init_z, st, aggregates);
   if (dk == 64 && dv == 128)
     return tc_forward_dims<64, 128, false>(q, k, v, out, heads, n, causal, seg, ws, err, init_S,
-                                           init_z, st);
+                                           init_z, st, aggregates);
   return cudaErrorInvalidValue;
 }
 

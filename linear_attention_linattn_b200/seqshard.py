@@ -4,12 +4,14 @@ The recurrent view of linear attention (page "Efficient Transformers: Linear Att
 Flash Attention", section "The recurrent view: attention as an RNN") carries everything the
 earlier tokens contribute in one fixed-size state (S, z).  So the blocks need one exchange:
 
-  1. this rank's block state   (S_r, z_r) = linattn_forward_state(k_r, v_r)
+  1. this rank's block state   (S_r, z_r) = linattn_forward_state_keep(k_r, v_r), which also
+     keeps the block's sums of k_r, v_r for step 4
   2. one all-gather of every rank's packed state, B*H*(d*d + d)*4 bytes per rank
   3. the state the block starts from, with linattn_sum_states:
        causal:     the sum over ranks r' < r  (the tokens before this block)
        non-causal: the sum over ranks r' != r (the rest of the sequence)
-  4. out_r = linattn_forward_init(q_r, k_r, v_r, S0, z0)
+  4. out_r = linattn_forward_init_from(q_r, k_r, v_r, S0, z0, kept sums)  (k_r, v_r are read
+     once in all)
 
 Rank r of G holds tokens [r*n/G, (r+1)*n/G) of a length-n sequence (ranks in group order).
 Steps 1, 3 and 4 run in this library's kernels; step 2 is the process group's all-gather
@@ -24,8 +26,9 @@ class DeviceOps:
 
     @staticmethod
     def state(k, v):
+        """(S, z, carry): the block state and what forward_init may reuse."""
         from . import forward_state
-        return forward_state(k, v)
+        return forward_state(k, v, keep=True)
 
     @staticmethod
     def sum(states, count: int, skip: int):
@@ -33,9 +36,9 @@ class DeviceOps:
         return sum_states(states, count, skip)
 
     @staticmethod
-    def forward_init(q, k, v, S0, z0, causal: bool):
+    def forward_init(q, k, v, S0, z0, causal: bool, carry=None):
         from . import forward_init
-        return forward_init(q, k, v, S0, z0, causal)
+        return forward_init(q, k, v, S0, z0, causal, aggregates=carry)
 
 
 def pack_state(S, z):
@@ -66,7 +69,7 @@ def forward_sequence_sharded(q, k, v, causal: bool, group=None, ops=None):
     single = not dist.is_available() or not dist.is_initialized()
     G = 1 if single else dist.get_world_size(group)
     r = 0 if single else dist.get_rank(group)
-    S, z = ops.state(k, v)
+    S, z, carry = ops.state(k, v)
     packed = pack_state(S, z)
     if G == 1:
         gathered = packed[None]
@@ -75,4 +78,4 @@ def forward_sequence_sharded(q, k, v, causal: bool, group=None, ops=None):
         dist.all_gather(parts, packed, group=group)
         gathered = torch.stack(parts)
     S0, z0 = start_state(gathered, r, causal, ops)
-    return ops.forward_init(q, k, v, S0, z0, causal)
+    return ops.forward_init(q, k, v, S0, z0, causal, carry)

@@ -98,6 +98,15 @@ def test_backward_init_and_sum_argument_checks(lib):
     for seg in (-64, 100):
         assert lib.linattn_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1,
                                        1, seg, None) == bad
+    # block aggregates: the buffer is required; sizes for unsupported shapes are 0
+    assert lib.linattn_forward_state_keep(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 8, 64, 1,
+                                          None) == bad
+    assert lib.linattn_forward_init_from(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 1, 1, 8,
+                                         64, 1, 1, None) == bad
+    assert lib.linattn_block_aggregates_bytes(1, 1, 8, 96, 1) == 0
+    assert lib.linattn_block_aggregates_bytes(1, 1, 0, 64, 1) == 0
+    # fp32: one (d*d + d)-float state per 64-token chunk
+    assert lib.linattn_block_aggregates_bytes(2, 3, 130, 64, 0) == 2 * 3 * 3 * (64 * 64 + 64) * 4
     # forward from a state: the state pointers are required
     assert lib.linattn_forward_init(FAKE, FAKE, FAKE, FAKE, 0, FAKE, 1, 1, 8, 64, 1, 1,
                                     None) == bad

@@ -32,7 +32,7 @@ class NumpyOps:
         fk = _phi(k.double().numpy())
         vv = v.double().numpy()
         S = np.einsum("bhnr,bhnc->bhrc", fk, vv)
-        return torch.from_numpy(S), torch.from_numpy(fk.sum(axis=2))
+        return torch.from_numpy(S), torch.from_numpy(fk.sum(axis=2)), None
 
     @staticmethod
     def sum(states, count, skip):
@@ -47,7 +47,7 @@ class NumpyOps:
                 torch.from_numpy(acc[..., d * d:].copy()))
 
     @staticmethod
-    def forward_init(q, k, v, S0, z0, causal):
+    def forward_init(q, k, v, S0, z0, causal, carry=None):
         fq, fk = _phi(q.double().numpy()), _phi(k.double().numpy())
         vv = v.double().numpy()
         S0, z0 = S0.double().numpy(), z0.double().numpy()
@@ -138,6 +138,56 @@ def test_blocks_on_one_gpu_match_oracle(dtype, causal, d):
     assert la.device_error() == la.LINATTN_OK
     got = np.concatenate(outs, axis=2)
     assert max_row_rel_err(got, oracle.forward(q, k, v, causal)) <= TOL[dtype]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+def test_blocks_reusing_their_sums_match_oracle(dtype, causal, d):
+    """The same four blocks through the calls that read k, v once per block: the state call
+    keeps the block's sums (linattn_forward_state_keep) and the block's pass reuses them
+    (linattn_forward_init_from), as forward_sequence_sharded does."""
+    import linear_attention_linattn_b200 as la
+    from tests.helpers import to_dev, to_host
+    B, H, G, blk = 1, 3, 4, 1100
+    n = G * blk
+    q, k, v = (as_io(x, dtype) for x in inputs.forward_qkv(43, B, H, n, d, scaled=True))
+    blocks = [[to_dev(np.ascontiguousarray(x[:, :, r * blk:(r + 1) * blk]), dtype)
+               for x in (q, k, v)] for r in range(G)]
+    kept = [la.forward_state(bk, bv, keep=True) for _, bk, bv in blocks]
+    # the kept call's state is the plain call's
+    for (_, bk, bv), (S, z, _) in zip(blocks, kept):
+        S1, z1 = la.forward_state(bk, bv)
+        assert torch.equal(S, S1) and torch.equal(z, z1)
+    gathered = torch.stack([seqshard.pack_state(S, z) for S, z, _ in kept])
+    outs = []
+    for r, (bq, bk, bv) in enumerate(blocks):
+        S0, z0 = seqshard.start_state(gathered, r, causal)
+        outs.append(to_host(la.forward_init(bq, bk, bv, S0, z0, causal, aggregates=kept[r][2])))
+    assert la.device_error() == la.LINATTN_OK
+    got = np.concatenate(outs, axis=2)
+    assert max_row_rel_err(got, oracle.forward(q, k, v, causal)) <= TOL[dtype]
+
+
+@pytest.mark.gpu
+def test_sharded_forward_reads_each_block_once():
+    """forward_sequence_sharded without a process group (one block = the whole sequence)
+    launches the aggregates once: the state call's, reused by the block's pass."""
+    import linear_attention_linattn_b200 as la
+    from tests.helpers import to_dev, to_host
+    B, H, n, d = 1, 2, 3000, 64
+    q, k, v = (as_io(x, "bf16") for x in inputs.forward_qkv(44, B, H, n, d, scaled=True))
+    qd, kd, vd = (to_dev(x, "bf16") for x in (q, k, v))
+    for causal in (True, False):
+        got = to_host(seqshard.forward_sequence_sharded(qd, kd, vd, causal))
+        assert max_row_rel_err(got, oracle.forward(q, k, v, causal)) <= TOL["bf16"]
+    lib = la.load_library()
+    l0 = lib.linattn_launch_count()
+    seqshard.forward_sequence_sharded(qd, kd, vd, True)
+    torch.cuda.synchronize()
+    # state: aggregates + total; sum of states; pass: prefix + outputs (no second aggregate)
+    assert lib.linattn_launch_count() - l0 == 5
 
 
 @pytest.mark.gpu
