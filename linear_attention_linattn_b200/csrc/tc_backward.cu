@@ -63,6 +63,10 @@ using namespace tc;
 constexpr int C = kTcChunk;     // tokens per chunk (64)
 constexpr int kAtom = C * 128;  // one [64 rows][64 bf16] 128B-swizzled atom: 8 KB
 constexpr int kThreads = 256;   // 8 warps, two per TMEM sub-partition
+// The walks' products of one phase go to different accumulators and are issued by lane 0 of
+// warps 0, 1 and 2 in parallel: one thread issues a tcgen05.mma about every 55 cycles, slower
+// than the tensor pipe runs these small products.
+constexpr int kIssuers = 3;
 
 // A state record: [M (D x D, row-major) | three D-vectors | a scalar, three zeros].
 template <int D>
@@ -404,7 +408,9 @@ struct Sync {
   }
 };
 
-__device__ __forceinline__ void init_barriers(BwdShared &sh) {
+// issuers: the threads (lane 0 of the first warps) that issue MMAs; sh.mma and sh.fin take
+// one arrival from each.
+__device__ __forceinline__ void init_barriers(BwdShared &sh, int issuers) {
   for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
     sh.acc[i / 128][i % 128] = 0.f;
     sh.racc[i / 128][i % 128] = 0.f;
@@ -412,22 +418,31 @@ __device__ __forceinline__ void init_barriers(BwdShared &sh) {
   if (threadIdx.x == 0) {
     mbar_init(&sh.full[0], 1);
     mbar_init(&sh.full[1], 1);
-    mbar_init(&sh.mma, 1);
-    mbar_init(&sh.fin, 1);
+    mbar_init(&sh.mma, issuers);
+    mbar_init(&sh.fin, issuers);
     sh.abort = 0;
     fence_barrier_init();
   }
 }
 
+// An issuer's end of an MMA phase: its products of the phase committed to `bar`, or (none
+// issued) an arrival at once.
+__device__ __forceinline__ void phase_done(uint64_t *bar, bool issued_any) {
+  if (issued_any)
+    mma_commit(bar);
+  else
+    mbar_arrive(bar);
+}
+
 // Lets every copy and product a CTA issued land (thread 0: `landed` of `issued` loads had
-// been waited for), then releases its TMEM.
+// been waited for; each of the `issuers` MMA-issuing threads: my_mma, whether it issued any),
+// then releases its TMEM.
 __device__ __forceinline__ void finish(BwdShared &sh, int landed, int issued, uint32_t tmem,
-                                       uint32_t cols, int *err) {
-  if (threadIdx.x == 0) {
+                                       uint32_t cols, int *err, int issuers, bool my_mma) {
+  if (threadIdx.x == 0)
     for (int l = landed; l < issued; ++l) mbar_wait_drain(&sh.full[l & 1], (l >> 1) & 1, err);
-    mma_commit(&sh.fin);
-    mbar_wait_drain(&sh.fin, 0, err);
-  }
+  if ((threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < issuers) phase_done(&sh.fin, my_mma);
+  if (threadIdx.x == 0) mbar_wait_drain(&sh.fin, 0, err);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
   const Lanes L = Lanes::make<D>();
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
-  init_barriers(sh);
+  init_barriers(sh, 1);
   if (L.warp == 0) {
     tmem_alloc(&sh.tmem_base, D);
     tmem_relinquish();
@@ -481,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
   Sync S(sh, err, L.lane);
 
   int issued = 0, landed = 0;
+  bool my_mma = false;  // thread 0 issued products
   auto issue = [&](const Item &I, int c) {
     uint64_t *fb = &sh.full[issued & 1];
     uint8_t *st = sm + (issued & 1) * G::G_STAGE;
@@ -520,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
         for (int ks = 0; ks < KSC; ++ks)
           mma_bf16_ss(tmem, mdesc(k0, ks, kAtom), mdesc(v0, ks, kAtom), I_S, (c > 0 || ks > 0));
         mma_commit(&sh.mma);
+        my_mma = true;
       }
       // zeta, vs, sigma of the chunk's keys (rows past the item's end: psi(K) zero, V skipped)
       column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
@@ -562,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
     }
     if (!S.barrier()) break;
   }
-  finish(sh, landed, issued, tmem, D, err);
+  finish(sh, landed, issued, tmem, D, err, 1, my_mma);
 }
 
 // ---------------------------------------------------------------- B1: the prefix walk
@@ -607,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   const Lanes L = Lanes::make<D>();
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
-  init_barriers(sh);
+  init_barriers(sh, kIssuers);
   // L: [64][64] lower triangle of ones (j <= i), the K-major operand of the prefix sums of V
   for (int i = threadIdx.x; i < kAtom / 16; i += kThreads) {
     const int row = i >> 3, c8 = 8 * (i & 7);
@@ -641,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   Sync S(sh, err, L.lane);
 
   int issued = 0, landed = 0;
+  bool my_mma = false;  // this thread (an issuer) issued products
   auto issue = [&](const Item &I, int c) {
     uint64_t *fb = &sh.full[issued & 1];
     uint8_t *st = sm + (issued & 1) * G::P_STAGE;
@@ -720,18 +738,10 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         else if (it + istep < nitems)
           issue(item_at<C>(it + istep, n, seg_len, nseg), 0);
         if (CAUSAL) {
-          // P' = psi(Q) psi(K)^T;  LV = L V;  Psi += psi(K)^T V
+          // P' = psi(Q) psi(K)^T
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX, kdesc(uQ, ks, kAtom), kdesc(uK, ks, kAtom), I_P, ks > 0);
-#pragma unroll
-          for (int ks = 0; ks < KSC; ++ks)
-            mma_bf16_ss(tY, kdesc(uL, ks, kAtom), mdesc(uV, ks, kAtom), I_O, ks > 0);
-          if (more) {
-#pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tS, mdesc(uK, ks, kAtom), mdesc(uV, ks, kAtom), I_S, 1u);
-          }
         } else {
           // O' = psi(Q) Psi
 #pragma unroll
@@ -739,6 +749,25 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
             mma_bf16_ss(tX, kdesc(uQ, ks, kAtom), mdesc(uST, ks, SA), I_O, ks > 0);
         }
         mma_commit(&sh.mma);
+        my_mma = true;
+      } else if (threadIdx.x == 32) {
+        if (CAUSAL) {
+          // LV = L V
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tY, kdesc(uL, ks, kAtom), mdesc(uV, ks, kAtom), I_O, ks > 0);
+        }
+        phase_done(&sh.mma, CAUSAL);
+        my_mma = my_mma || CAUSAL;
+      } else if (threadIdx.x == 64) {
+        if (more) {
+          // Psi += psi(K)^T V
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tS, mdesc(uK, ks, kAtom), mdesc(uV, ks, kAtom), I_S, 1u);
+        }
+        phase_done(&sh.mma, more);
+        my_mma = my_mma || more;
       }
       // psi(q_i) . zeta over this half's features
       float dpart = 0.f;
@@ -784,6 +813,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           for (int ks = 0; ks < KSC; ++ks)
             mma_bf16_ss(tX, kdesc(uW, ks, kAtom), mdesc(uV, ks, kAtom), I_O, 1u);
           mma_commit(&sh.mma);
+        } else if (threadIdx.x == 32 || threadIdx.x == 64) {
+          mbar_arrive(&sh.mma);
         }
       } else {
         if (L.v64) sh.part[L.hf][L.r64] = dpart;
@@ -863,6 +894,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX, kdesc(uAL, ks, kAtom), kdesc(uV, ks, kAtom), I_P, 1u);
         }
+        phase_done(&sh.mma, CAUSAL);
+      } else if (threadIdx.x == 32) {
         // dQ' = A Psi^T
 #pragma unroll
         for (int ks = 0; ks < KSD; ++ks)
@@ -870,6 +903,9 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
 #pragma unroll
         for (int ks = 0; ks < KSD; ++ks)
           mma_bf16_ss(tY, kdesc(uAL, ks, kAtom), kdesc(uST, ks, SA), I_T, 1u);
+        mma_commit(&sh.mma);
+        my_mma = true;
+      } else if (threadIdx.x == 64) {
         // Phi += psi(Q)^T A
 #pragma unroll
         for (int ks = 0; ks < KSC; ++ks)
@@ -878,6 +914,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         for (int ks = 0; ks < KSC; ++ks)
           mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uAL, ks, kAtom), I_S, 1u);
         mma_commit(&sh.mma);
+        my_mma = true;
       }
       // this chunk's part of the item's reverse record: rho, as, tau (sh.racc), bs; b of each
       // row from the exchanged partial dot products, zero past the item's end (so is a)
@@ -928,6 +965,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           for (int ks = 0; ks < KSC; ++ks)
             mma_bf16_ss(tY, kdesc(uW, ks, kAtom), mdesc(uK, ks, kAtom), I_O, 1u);
           mma_commit(&sh.mma);
+        } else if (threadIdx.x == 32 || threadIdx.x == 64) {
+          mbar_arrive(&sh.mma);
         }
         S.wait_mma();
       }
@@ -983,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
     }
     if (!S.barrier()) break;
   }
-  finish(sh, landed, issued, tmem, G::TCOLS, err);
+  finish(sh, landed, issued, tmem, G::TCOLS, err, kIssuers, my_mma);
 }
 
 // ---------------------------------------------------------------- B3: the suffix walk
@@ -1028,7 +1067,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   const Lanes L = Lanes::make<D>();
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
-  init_barriers(sh);
+  init_barriers(sh, kIssuers);
   if (L.warp == 0) {
     tmem_alloc(&sh.tmem_base, G::TCOLS);
     tmem_relinquish();
@@ -1054,6 +1093,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   auto chunk_of = [](int w, int nchunks) { return CAUSAL ? nchunks - 1 - w : w; };
 
   int issued = 0, landed = 0;
+  bool my_mma = false;  // this thread (an issuer) issued products
   auto issue = [&](const Item &I, int w) {
     uint64_t *fb = &sh.full[issued & 1];
     uint8_t *st = sm + (issued & 1) * G::S_STAGE;
@@ -1123,33 +1163,47 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         else if (it + istep < nitems)
           issue(item_at<C>(it + istep, n, seg_len, nseg), 0);
         if (CAUSAL) {
-          // P'^T = psi(K) psi(Q)^T;  dW^T = V A^T (a_hi, then a_lo);  Phi += psi(Q)^T A
+          // P'^T = psi(K) psi(Q)^T
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX, kdesc(uK, ks, kAtom), kdesc(uQ, ks, kAtom), I_P, ks > 0);
+        } else {
+          // dV' = psi(K) Phi  (Phi the head's total)
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX, kdesc(uK, ks, kAtom), mdesc(uFT, ks, SA), I_O, ks > 0);
+        }
+        mma_commit(&sh.mma);
+        my_mma = true;
+      } else if (threadIdx.x == 32) {
+        if (CAUSAL) {
+          // dW^T = V A^T (a_hi, then a_lo)
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX + 64, kdesc(uV, ks, kAtom), kdesc(uA, ks, kAtom), I_P, ks > 0);
 #pragma unroll
           for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX + 64, kdesc(uV, ks, kAtom), kdesc(uAL, ks, kAtom), I_P, 1u);
-          if (more) {
-#pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uA, ks, kAtom), I_S, 1u);
-#pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uAL, ks, kAtom), I_S, 1u);
-          }
         } else {
-          // dV' = psi(K) Phi;  dK' = V Phi^T  (Phi the head's total)
+          // dK' = V Phi^T
 #pragma unroll
-          for (int ks = 0; ks < KSD; ++ks) {
-            mma_bf16_ss(tX, kdesc(uK, ks, kAtom), mdesc(uFT, ks, SA), I_O, ks > 0);
+          for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX + D, kdesc(uV, ks, kAtom), kdesc(uFT, ks, SA), I_T, ks > 0);
-          }
         }
         mma_commit(&sh.mma);
+        my_mma = true;
+      } else if (threadIdx.x == 64) {
+        if (more) {
+          // Phi += psi(Q)^T A
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uA, ks, kAtom), I_S, 1u);
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tR, mdesc(uQ, ks, kAtom), mdesc(uAL, ks, kAtom), I_S, 1u);
+        }
+        phase_done(&sh.mma, more);
+        my_mma = my_mma || more;
       }
       // v_j . as over this half's columns (as: the record after this chunk, read after the
       // barrier above, which orders it after the record's load or last update)
@@ -1203,18 +1257,25 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         fence_proxy_async_smem();
         if (!S.barrier()) break;
         if (threadIdx.x == 0) {
-          // dV' = psi(K) Phi + mask(w^T) a_hi;  dK' = V Phi^T + mask(dW^T + b) psi(Q)
+          // dV' = psi(K) Phi + mask(w^T) a_hi
 #pragma unroll
-          for (int ks = 0; ks < KSD; ++ks) {
+          for (int ks = 0; ks < KSD; ++ks)
             mma_bf16_ss(tX, kdesc(uK, ks, kAtom), mdesc(uFT, ks, SA), I_O, ks > 0);
-            mma_bf16_ss(tX + D, kdesc(uV, ks, kAtom), kdesc(uFT, ks, SA), I_T, ks > 0);
-          }
 #pragma unroll
-          for (int ks = 0; ks < KSC; ++ks) {
+          for (int ks = 0; ks < KSC; ++ks)
             mma_bf16_ss(tX, kdesc(uW0, ks, kAtom), mdesc(uA, ks, kAtom), I_O, 1u);
-            mma_bf16_ss(tX + D, kdesc(uW1, ks, kAtom), mdesc(uQ, ks, kAtom), I_O, 1u);
-          }
           mma_commit(&sh.mma);
+        } else if (threadIdx.x == 32) {
+          // dK' = V Phi^T + mask(dW^T + b) psi(Q)
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tX + D, kdesc(uV, ks, kAtom), kdesc(uFT, ks, SA), I_T, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tX + D, kdesc(uW1, ks, kAtom), mdesc(uQ, ks, kAtom), I_O, 1u);
+          mma_commit(&sh.mma);
+        } else if (threadIdx.x == 64) {
+          mbar_arrive(&sh.mma);
         }
       }
       // ---- (e) dv_j = (d + sk_j) as + tau + dV'_j;  dk_j = (dK'_j + rho + C'_j) phi'(k_j),
@@ -1268,7 +1329,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       }
     }
   }
-  finish(sh, landed, issued, tmem, G::TCOLS, err);
+  finish(sh, landed, issued, tmem, G::TCOLS, err, kIssuers, my_mma);
 }
 
 // ------------------------------------------------------------------ host side

@@ -62,18 +62,24 @@ enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
 
 constexpr int kWarpTMA = 0;
 constexpr int kWarpMMA = 1;
-constexpr int kWarpXform0 = 2;
 constexpr int kGroupThreads = 128;
-// Warps per mode (measured on the benchmark shapes).  Causal: 6 feature-map warps, 16 warps
-// in all, so each SM sub-partition holds 4 warps and a thread may use 128 registers (the
-// score, state and output drains keep 64-column batches in registers).  Aggregate: the
-// feature map on K bounds the chunk rate, so 12 feature-map warps (22 warps, 80 registers).
-// Non-causal: 8 feature-map warps (18 warps, 96 registers).
-template <int MODE>
+// Warps per mode and feature width (measured on the benchmark shapes).  Causal: 16 warps, so
+// each SM sub-partition holds 4 warps and a thread may use 128 registers (the score, state and
+// output drains keep 64-column batches in registers).  At d = 64 two warps issue the MMAs (one
+// thread issues a tcgen05.mma about every 55 cycles, slower than the tensor pipe runs these
+// small products; issuers in different warps proceed in parallel), with 5 feature-map warps;
+// at d = 128 the feature map is the tighter bound, so one issuer and 6 feature-map warps.
+// Aggregate: the feature map on K bounds the chunk rate, so 12 feature-map warps (22 warps,
+// 80 registers).  Non-causal: 8 feature-map warps (18 warps, 96 registers).
+template <int MODE, int DK>
 struct Warps {
-  static constexpr int XFORM = MODE == kCausalOut ? 6 : (MODE == kState ? 12 : 8);
+  static constexpr bool TWO_ISSUERS = MODE == kCausalOut && DK == 64;
+  static constexpr int MMA2 = 2;                      // the second issuer
+  static constexpr int XFORM0 = TWO_ISSUERS ? 3 : 2;  // first feature-map warp
+  static constexpr int XFORM =
+      MODE == kCausalOut ? (TWO_ISSUERS ? 5 : 6) : (MODE == kState ? 12 : 8);
   static constexpr int XTHREADS = XFORM * 32;
-  static constexpr int STATE0 = kWarpXform0 + XFORM;  // state group: 4 warps
+  static constexpr int STATE0 = XFORM0 + XFORM;  // state group: 4 warps
   static constexpr int OUT0 = STATE0 + 4;             // scores and output group: 4 warps
   static constexpr int THREADS = (OUT0 + 4) * 32;
 };
@@ -140,7 +146,7 @@ struct TmemMap {
 
 struct Bars {
   uint64_t full[8], ready[8], empty[8];
-  uint64_t p_full, p_ready, s_full, s_ready, z_ready, rs_ready, o_full[2], o_empty[2], fin;
+  uint64_t p_full, p_ready, s_full, s_ready, z_ready, rs_ready, o_full[2], o_empty[2], fin, fin2;
   // per item parity: aggregate mode, S accumulator complete (MMA -> state group) / written out
   // (state group -> MMA); non-causal, S operand rounded (state group -> MMA) / no longer read
   // (MMA -> state group)
@@ -192,7 +198,7 @@ __device__ __forceinline__ float convert_P32(uint32_t taddr, uint8_t *sP, int r6
 // exclusive prefix, at init_state + head * init_head_stride + seg * init_seg_stride;
 // non-causal: the head's total).  out_state (aggregate): [heads][nseg][DK*DV + DK].
 template <int DK, int DV, int MODE, bool PHI>
-__global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
+__global__ void __launch_bounds__(Warps<MODE, DK>::THREADS, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
               const float *__restrict__ init_state, int64_t init_head_stride,
@@ -200,7 +206,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
               int64_t nseg, int64_t nitems, int *err) {
   using G = Cfg<DK, DV, MODE>;
   using TM = TmemMap<DV, MODE>;
-  using W = Warps<MODE>;
+  using W = Warps<MODE, DK>;
   constexpr int NS = G::NS;
   constexpr int KSD = DK / 16;  // K-steps over the feature dimension
   constexpr int KSC = C / 16;   // K-steps over the chunk's tokens
@@ -235,6 +241,7 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
       mbar_init(&bar.item_empty[b], MODE == kState ? kGroupThreads : 1);
     }
     mbar_init(&bar.fin, 1);
+    mbar_init(&bar.fin2, 1);
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -373,7 +380,10 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
           if (MODE == kCausalOut) {
             // The previous chunk's P V (its scores rounded by now) interleaved with this
             // chunk's [scores | phi(q).z_<c]: different accumulators, so the tensor pipe
-            // overlaps the two chains instead of running them back to back.
+            // overlaps the two chains instead of running them back to back.  With a second
+            // issuer, its products of the previous chunk (phi(Q) S_<c onto which P V adds, and
+            // the S update, both reading its stage) are done by z_ready: the state group
+            // reads z after their commit.
             if (!mbar_wait(&bar.z_ready, g & 1, abort, err)) {
               ok = false;
               break;
@@ -397,27 +407,29 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
               }
             }
             mma_commit(&bar.p_full);
-            // S_<c in the S operand; this O buffer drained
-            if (!mbar_wait(&bar.s_ready, g & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            // phi(Q_c) S_<c, then S += phi(K_c)^T [V_c | 1] (interleaving these two measured
-            // no faster)
+            if (!W::TWO_ISSUERS) {
+              // S_<c in the S operand; this O buffer drained
+              if (!mbar_wait(&bar.s_ready, g & 1, abort, err)) {
+                ok = false;
+                break;
+              }
+              if (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              // phi(Q_c) S_<c, then S += phi(K_c)^T [V_c | 1] (interleaving these two
+              // measured no faster)
 #pragma unroll
-            for (int ks = 0; ks < KSD; ++ks)
-              mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
-                          I_O, ks > 0 ? 1u : 0u);
+              for (int ks = 0; ks < KSD; ++ks)
+                mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)),
+                            desc_add(dS, mnmajor_off(ks)), I_O, ks > 0 ? 1u : 0u);
 #pragma unroll
-            for (int ks = 0; ks < KSC; ++ks)
-              mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
-                          1u);
-            mma_commit(&bar.s_full);
+              for (int ks = 0; ks < KSC; ++ks)
+                mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)),
+                            I_S, 1u);
+              mma_commit(&bar.s_full);
+            }
             dVprev = dVm;  // P V of this chunk goes with the next chunk's scores
             sprev = s;
             continue;
@@ -440,8 +452,10 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
         if (MODE == kNoncausalOut) mma_commit(&bar.item_empty[b]);  // S operand no longer read
       }
       if (MODE == kCausalOut && ok && g > 0) {
-        // the last chunk's P V
-        if (mbar_wait(&bar.p_ready, (g - 1) & 1, abort, err)) {
+        // the last chunk's P V, once a second issuer's products of that chunk are done
+        // (nothing else waits for that s_full phase)
+        if ((!W::TWO_ISSUERS || mbar_wait(&bar.s_full, (g - 1) & 1, abort, err)) &&
+            mbar_wait(&bar.p_ready, (g - 1) & 1, abort, err)) {
           tc_fence_after();
           const uint32_t tOp = tmem + (((g - 1) & 1) ? TM::O1 : TM::O0);
 #pragma unroll
@@ -452,15 +466,63 @@ __global__ void __launch_bounds__(Warps<MODE>::THREADS, 1)
           mma_commit(&bar.empty[sprev]);
         }
       }
-      // every MMA this CTA issued has finished before TMEM is released
+      // every MMA this thread issued has finished before TMEM is released
       mma_commit(&bar.fin);
       mbar_wait_drain(&bar.fin, 0, err);
+    }
+  } else if (W::TWO_ISSUERS && warp == W::MMA2) {
+    // ================================================================ second MMA issuer
+    // Causal, per chunk c: O = phi(Q_c) S_<c into the chunk's O buffer, then
+    // [S | z] += phi(K_c)^T [V_c | 1] (interleaving these two measured no faster).  These are
+    // issued as soon as their inputs are ready, not after the first issuer's scores of the
+    // chunk: holding them back for the scores measured 10% slower (the S update ends the
+    // chain that gives the next chunk its z).
+    if (lane == 0) {
+      constexpr uint32_t I_O = make_idesc_bf16(64, DV, false, true);
+      constexpr uint32_t I_S = make_idesc_bf16(DK, DV + 16, true, true);
+      const uint32_t tS = tmem + TM::S;
+      const uint64_t dS = mnmajor_base(smem_u32(smem + G::OFF_S), G::S_ATOM);
+      const uint32_t st0 = smem_u32(smem);
+      int g = 0;
+      bool ok = true;
+      for (int64_t it = it0; ok && it < nitems; it += istep) {
+        const Item I = item_at<C>(it, n, seg_len, nseg);
+        for (int c = 0; c < I.nchunks; ++c, ++g) {
+          const int s = g % NS;
+          const int ob = g & 1;
+          // the chunk's features; S_<c in the S operand (and TMEM S read out); this O
+          // buffer drained
+          if (!mbar_wait(&bar.ready[s], (g / NS) & 1, abort, err) ||
+              !mbar_wait(&bar.s_ready, g & 1, abort, err) ||
+              (g >= 2 && !mbar_wait(&bar.o_empty[ob], ((g >> 1) - 1) & 1, abort, err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = st0 + s * G::STAGE;
+          const uint32_t tO = tmem + (ob ? TM::O1 : TM::O0);
+          const uint64_t dQk = kmajor_base(st);                        // Q, K-major
+          const uint64_t dKm = mnmajor_base(st + G::OFF_K, G::KATOM);  // K, MN-major
+          const uint64_t dVm = mnmajor_base(st + G::OFF_V, kAtom);     // [V | ones], MN-major
+#pragma unroll
+          for (int ks = 0; ks < KSD; ++ks)
+            mma_bf16_ss(tO, desc_add(dQk, kmajor_off(ks, kAtom)), desc_add(dS, mnmajor_off(ks)),
+                        I_O, ks > 0 ? 1u : 0u);
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tS, desc_add(dKm, mnmajor_off(ks)), desc_add(dVm, mnmajor_off(ks)), I_S,
+                        1u);
+          mma_commit(&bar.s_full);
+        }
+      }
+      mma_commit(&bar.fin2);
+      mbar_wait_drain(&bar.fin2, 0, err);
     }
   } else if (warp < W::STATE0) {
     // ================================================================ feature map
     // phi in place on the Q tile and on the 64 key rows of each K atom; K rows past the
     // item's end are zeroed (they must add nothing to S, z or the scores).
-    const int xt = threadIdx.x - kWarpXform0 * 32;
+    const int xt = threadIdx.x - W::XFORM0 * 32;
     int g = 0;
     bool ok = true;
     for (int64_t it = it0; ok && it < nitems; it += istep) {
@@ -783,13 +845,13 @@ cudaError_t launch_tc(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
   const int64_t want = persistent ? sms : nitems;
   const unsigned grid = static_cast<unsigned>(nitems < want ? nitems : want);
   if (MODE == kState) {
-    kern<<<grid, Warps<MODE>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out),
+    kern<<<grid, Warps<MODE, DK>::THREADS, G::SMEM, st>>>(q, k, v, static_cast<__nv_bfloat16 *>(out),
                                                       init, ihs, iss, out_state, n, seg, nseg,
                                                       nitems, err);
   } else {
     // the output kernels follow the scan: launched so that their set-up and first loads of
     // q, k, v overlap the scan's tail (the state group waits for the scan's results)
-    e = launch_programmatic(kern, dim3(grid), dim3(Warps<MODE>::THREADS), G::SMEM, st, q, k, v,
+    e = launch_programmatic(kern, dim3(grid), dim3(Warps<MODE, DK>::THREADS), G::SMEM, st, q, k, v,
                             static_cast<__nv_bfloat16 *>(out), init, ihs, iss, out_state, n, seg,
                             nseg, nitems, err);
     if (e != cudaSuccess) return e;

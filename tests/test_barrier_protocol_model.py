@@ -3,7 +3,8 @@
 Every warp role (TMA producer, feature map, MMA issuer, state group, scores/output group) is
 written as the sequence of mbarrier waits (with the phase index it waits for) and arrivals it
 performs, for the three modes of tc_forward.cu (0 aggregate, 1 causal output, 2 non-causal
-output) and the causal kernel on features of their own dimension, tc_causal.cu (mode 3), and
+output; 4 is the causal output with two MMA-issuing warps, as run at d = 64) and the causal
+kernel on features of their own dimension, tc_causal.cu (mode 3), and
 any list of work items of 1..16 chunks walked by one CTA.  A random scheduler interleaves the roles. The
 test fails on a deadlock (no role can move) or on parity aliasing (a wait for a phase two or more
 phases behind its barrier, which the hardware's parity test cannot tell from a pending one).
@@ -21,7 +22,7 @@ class Barrier:
         self.count, self.pending, self.completed = count, 0, 0
 
 
-def roles_forward(mode, NS, items):
+def roles_forward(mode, NS, items, two=False):
     """Generators of ('w', barrier, phase) and ('a', barrier) events, one per warp role."""
 
     def tma():
@@ -65,10 +66,11 @@ def roles_forward(mode, NS, items):
                         yield ("a", f"o_full[{(g - 1) & 1}]")
                         yield ("a", f"empty[{(g - 1) % NS}]")
                     yield ("a", "p_full")
-                    yield ("w", "s_ready", g)
-                    if g >= 2:
-                        yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
-                    yield ("a", "s_full")
+                    if not two:  # else phi(Q) S_<c and the S update go to the second issuer
+                        yield ("w", "s_ready", g)
+                        if g >= 2:
+                            yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
+                        yield ("a", "s_full")
                 else:
                     if g >= 2:
                         yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
@@ -79,12 +81,27 @@ def roles_forward(mode, NS, items):
                 yield ("a", f"item_full[{b}]")
             if mode == 2:
                 yield ("a", f"item_empty[{b}]")
-        if mode == 1 and g > 0:  # the last chunk's P V
+        if mode == 1 and g > 0:  # the last chunk's P V (after a second issuer's products)
+            if two:
+                yield ("w", "s_full", g - 1)
             yield ("w", "p_ready", g - 1)
             yield ("a", f"o_full[{(g - 1) & 1}]")
             yield ("a", f"empty[{(g - 1) % NS}]")
         yield ("a", "fin")
         yield ("w", "fin", 0)
+
+    def mma2():  # causal: the second issuer, phi(Q) S_<c and the S update
+        g = 0
+        for nc in items:
+            for _ in range(nc):
+                yield ("w", f"ready[{g % NS}]", g // NS)
+                yield ("w", "s_ready", g)
+                if g >= 2:
+                    yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
+                yield ("a", "s_full")
+                g += 1
+        yield ("a", "fin2")
+        yield ("w", "fin2", 0)
 
     def state_group():
         if mode == 1:
@@ -137,7 +154,8 @@ def roles_forward(mode, NS, items):
                     yield ("a", f"o_empty[{g & 1}]")
                     g += 1
 
-    return [tma(), feature_map(), mma(), state_group(), output_group()]
+    roles = [tma(), feature_map(), mma(), state_group(), output_group()]
+    return roles + [mma2()] if two else roles
 
 
 def roles_features(NS, items):
@@ -216,12 +234,16 @@ def roles_features(NS, items):
 
 
 def roles(mode, NS, items):
-    return roles_features(NS, items) if mode == 3 else roles_forward(mode, NS, items)
+    if mode == 3:
+        return roles_features(NS, items)
+    if mode == 4:
+        return roles_forward(1, NS, items, two=True)
+    return roles_forward(mode, NS, items)
 
 
 def run(mode, NS, items, rng):
     # arrivals per phase; tc_forward.cu's causal mode: both drain groups release p_ready
-    counts = {"p_ready": 2} if mode == 1 else {}
+    counts = {"p_ready": 2} if mode in (1, 4) else {}
     bars = {}
 
     def bar(name):
@@ -255,7 +277,7 @@ def run(mode, NS, items, rng):
         cur[r] = next(gens[r], None)
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 def test_protocol_has_no_deadlock_or_aliasing(mode):
     rng = random.Random(1000 + mode)
     for _ in range(1500):
