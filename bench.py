@@ -236,8 +236,9 @@ def forward_launches(dtype: str, causal: bool, unit: int):
 
 def backward_launches(causal: bool, unit: int):
     """Names of the launches of one bf16 backward call, in order, and the algorithmic bytes of
-    each (unit: the bytes of one [B,H,n,d] tensor): K1 reads k, v; B1 reads q, k, v, dout and
-    writes dq (and a, b for the suffix walk); B3 reads q, k, v (and a, b) and writes dk, dv."""
+    each (unit: the bytes of one [B,H,n,d] tensor): K1 reads k, v (and stores psi(k) to the
+    workspace); B1 reads q, psi(k), v, dout and writes dq (and a, b and psi(q) for the suffix
+    walk); B3 reads psi(q), psi(k), v (and a, b) and writes dk, dv."""
     return (["bwd_aggregate_kernel (forward records, K1)",
              "scan_states_kernel (prefix, K2)" if causal else "scan_states_kernel (totals, K2)",
              "bwd_prefix_kernel (dq, B1)",

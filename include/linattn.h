@@ -191,7 +191,7 @@ linattn_status linattn_forward_features(const void *phi_q, const void *phi_k, co
  *     dL/dv_j      = sum_i w_ij a_i,
  * then through phi'(x) = 1 (x > 0), exp(x) (x <= 0); sums over j <= i (causal) or all.
  * Asynchronous on `stream`; takes a stream-ordered workspace: per head, bf16: two records
- * (d^2 + 3d + 4 floats) per segment of up to 4096 tokens plus about n (1.1 d + 1.2) floats;
+ * (d^2 + 3d + 4 floats) per segment of up to 4096 tokens plus about n (2.1 d + 3.2) floats;
  * float32:
  * 2 (n/64) (d^2 + d) + n (d + 1) floats.  Errors as in linattn_forward; a bounded wait that
  * gave up is reported by linattn_device_error.

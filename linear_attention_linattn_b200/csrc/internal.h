@@ -160,6 +160,8 @@ struct TcBackwardLayout {
   // [heads][chunks][3d + 4]: per chunk, the vectors of the forward record before it within
   // its segment, and the chunk's own reverse-record vectors
   float *s_vec, *r_vec;
+  __nv_bfloat16 *psi_q, *psi_k;  // [heads][n][d]: psi = phi - 1 of q and k, rounded to bf16
+  float *sq, *sk;                // [heads][n]: their row sums
 };
 // Tokens per work item of the backward (a multiple of 256, or n rounded up to kTcChunk).
 int64_t tc_backward_segment(int64_t heads, int64_t n, int d);

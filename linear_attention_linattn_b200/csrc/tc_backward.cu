@@ -26,14 +26,16 @@
 // The pass, per head; causal sums run over the chunks before (prefix) or after (suffix):
 //   K1  per segment, the forward record [Psi | zeta | vs | sigma | kappa] of the keys:
 //       Psi = sum psi(k_j) v_j^T, zeta = sum psi(k_j), vs = sum v_j, sigma = sum sk_j v_j,
-//       kappa = sum sk_j
+//       kappa = sum sk_j; psi(k) (rounded to bf16) and its row sums sk to the workspace
 //   K2  its exclusive prefix over segments (causal) or the head's total
-//   B1  prefix walk: per segment, chunks in order, Psi in TMEM: den, out, a, b, dq; a (hi, lo)
-//       and b to the workspace; the segment's reverse record [Phi | rho | as | tau | bs]:
+//   B1  prefix walk: per segment, chunks in order, Psi in TMEM: den, out, a, b, dq; a (hi, lo),
+//       b and (causal) psi(q) with its row sums sq to the workspace; the segment's reverse record [Phi | rho | as | tau | bs]:
 //       Phi = sum psi(q_i) a_i^T, rho = sum psi(q_i) b_i, as = sum a_i, tau = sum sq_i a_i,
 //       bs = sum b_i
 //   K2  its exclusive suffix (causal) or the head's total
 //   B3  suffix walk: per segment, chunks in reverse order, Phi in TMEM: dk, dv
+// psi(q) and psi(k) are each computed once: B1 and B3 read psi(k) from K1, B3 psi(q) from B1
+// (tile stores by TMA from the shared-memory tiles the kernel computed them in).
 //
 // Products of one 64-token chunk (tcgen05.mma kind::f16, bf16 operands, fp32 in TMEM):
 //   B1  P' = psi(Q) psi(K)^T;  Psi += psi(K)^T V;  LV = L V (L: the lower triangle of ones);
@@ -46,7 +48,7 @@
 //
 // Each CTA runs 8 warps through a chunk's phases in step (warps w and w + 4 share TMEM
 // sub-partition w & 3 and split the columns), thread 0 issuing the TMA loads (one chunk ahead,
-// two stages) and the MMAs.  Two CTAs share an SM at d = 64, so one CTA's products run while
+// two stages) and lane 0 of warps 0-2 the MMAs of each phase.  Two CTAs share an SM at d = 64, so one CTA's products run while
 // the other drains its accumulators.  Every wait is bounded (2 s); a CTA whose wait gave up lets
 // its copies and products land and exits.
 #include <cuda.h>
@@ -458,11 +460,14 @@ __device__ __forceinline__ uint64_t mdesc(uint32_t base, int ks, uint32_t atom) 
 
 // ---------------------------------------------------------------- K1: forward records
 // k, v: [heads][n][D] via tmK, tmV.  Writes each item's record [Psi | zeta | vs | sigma |
-// kappa] to rec + (head * nseg + seg) * rec_floats<D>().
+// kappa] to rec + (head * nseg + seg) * rec_floats<D>(), and psi(k) (rounded to bf16, via the
+// store map tmPK) with its row sums (skg, [heads][n]) for the walks.
 template <int D>
 __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
     bwd_aggregate_kernel(const __grid_constant__ CUtensorMap tmK,
-                         const __grid_constant__ CUtensorMap tmV, float *__restrict__ rec,
+                         const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmPK, float *__restrict__ skg,
+                         float *__restrict__ rec,
                          float *__restrict__ chunk_vec, int64_t n, int64_t seg_len, int64_t nseg,
                          int64_t nitems, int *err) {
   using G = BCfg<D>;
@@ -525,7 +530,16 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
       }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
+      // psi(k) and its row sums to the workspace (rows past n are not stored)
+      if (threadIdx.x < valid) skg[I.head * n + t0 + threadIdx.x] = sh.sk[threadIdx.x];
       if (threadIdx.x == 0) {
+#pragma unroll
+        for (int a = 0; a < AT; ++a)
+          tma_store_3d(&tmPK, st + OK + a * kAtom, 64 * a, static_cast<int>(t0),
+                       static_cast<int>(I.head), pol);
+        tma_store_commit();
+        // the other stage's tile has been read by its store before the next load lands there
+        tma_store_wait_read<1>();
         if (c + 1 < I.nchunks)
           issue(I, c + 1);
         else if (it + istep < nitems)
@@ -579,12 +593,14 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
     }
     if (!S.barrier()) break;
   }
+  if (threadIdx.x == 0) tma_store_wait_all<0>();  // the stores are done with shared memory
   finish(sh, landed, issued, tmem, D, err, 1, my_mma);
 }
 
 // ---------------------------------------------------------------- B1: the prefix walk
-// q, dout: [heads][n][D] via tmQ, tmG; k, v via tmK, tmV (causal only).  start: each item's
-// forward record (causal: exclusive prefix at start + head * start_hs + seg * start_ss;
+// q, dout: [heads][n][D] via tmQ, tmG; psi(k), v via tmK, tmV and skg (psi(k)'s row sums,
+// [heads][n]) (causal only).  Causal: stores psi(q) via tmPQ with its row sums to sqg, for the
+// suffix walk.  start: each item's forward record (causal: exclusive prefix at start + head * start_hs + seg * start_ss;
 // non-causal: the head's total).  Writes dq, a as a bf16 pair (a_hi, a_lo: [heads][n][D]),
 // b ([heads][n]) and each item's reverse record to r_rec + (head * nseg + seg) * rec_floats.
 template <int D, bool CAUSAL>
@@ -592,7 +608,9 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
     bwd_prefix_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
-                      const __grid_constant__ CUtensorMap tmG, __nv_bfloat16 *__restrict__ dq,
+                      const __grid_constant__ CUtensorMap tmG,
+                      const __grid_constant__ CUtensorMap tmPQ, float *__restrict__ sqg,
+                      const float *__restrict__ skg, __nv_bfloat16 *__restrict__ dq,
                       __nv_bfloat16 *__restrict__ a_hi, __nv_bfloat16 *__restrict__ a_lo,
                       float *__restrict__ b_out, const float *__restrict__ start,
                       int64_t start_hs, int64_t start_ss, const float *__restrict__ s_vec,
@@ -715,13 +733,16 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         }
         if (threadIdx.x == 0) fs = s_vec[slot * VF + 3 * D];
       }
+      // causal: psi(k)'s row sums of the chunk (zero past the item's end, where the tile's
+      // rows, past n, read as zero)
+      const float skv = CAUSAL && threadIdx.x < valid ? skg[I.head * n + t0 + threadIdx.x] : 0.f;
 
-      // ---- (a) psi on Q and K (K rows past the item's end zeroed), with row sums
+      // ---- (a) psi on Q, with row sums (causal: psi(K) and its row sums come from K1)
       if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
         if (threadIdx.x == 0) landed = g + 1;
         psi_tile<D>(st + OQ, C, sh.sq);
-        if (CAUSAL) psi_tile<D>(st + OK, valid, sh.sk);
       }
+      if (CAUSAL && threadIdx.x < C) sh.sk[threadIdx.x] = skv;
       if (CAUSAL && c > 0) {
         if (threadIdx.x < D) {
 #pragma unroll
@@ -731,7 +752,19 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
+      // causal: psi(q) and its row sums to the workspace for the suffix walk (rows past n are
+      // not stored)
+      if (CAUSAL && threadIdx.x < valid) sqg[I.head * n + t0 + threadIdx.x] = sh.sq[threadIdx.x];
       if (threadIdx.x == 0) {
+        if (CAUSAL) {
+#pragma unroll
+          for (int a = 0; a < AT; ++a)
+            tma_store_3d(&tmPQ, st + OQ + a * kAtom, 64 * a, static_cast<int>(t0),
+                         static_cast<int>(I.head), pol);
+          tma_store_commit();
+          // the other stage's tile has been read by its store before the next load lands there
+          tma_store_wait_read<1>();
+        }
         // the next step's tiles into the other stage (its last reader, step g - 1, is done)
         if (c + 1 < I.nchunks)
           issue(I, c + 1);
@@ -1022,12 +1055,13 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
     }
     if (!S.barrier()) break;
   }
+  if (CAUSAL && threadIdx.x == 0) tma_store_wait_all<0>();  // done with shared memory
   finish(sh, landed, issued, tmem, G::TCOLS, err, kIssuers, my_mma);
 }
 
 // ---------------------------------------------------------------- B3: the suffix walk
-// q, a_hi, a_lo: [heads][n][D] via tmQ, tmA, tmAL, and b_in: [heads][n] (causal only); k, v
-// via tmK, tmV.  start: each item's reverse record (causal: exclusive suffix at start +
+// psi(q), a_hi, a_lo: [heads][n][D] via tmQ, tmA, tmAL, and b_in: [heads][n] (causal only);
+// psi(k), v via tmK, tmV; sqg, skg: the row sums of psi(q), psi(k) ([heads][n]).  start: each item's reverse record (causal: exclusive suffix at start +
 // head * start_hs + seg * start_ss; non-causal: the head's total).  Writes dk, dv.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
@@ -1035,7 +1069,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
                       const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmAL,
                       const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const float *__restrict__ b_in,
+                      const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sqg,
+                      const float *__restrict__ skg, const float *__restrict__ b_in,
                       __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
                       const float *__restrict__ start, int64_t start_hs, int64_t start_ss,
                       const float *__restrict__ r_vec, int64_t n, int64_t seg_len, int64_t nseg,
@@ -1143,18 +1178,27 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         }
         if (threadIdx.x == 0) rs = src[3 * D];
       }
-      // ---- (a) psi on K (row sums); causal: psi on Q (row sums) and the rows of Q and A past
-      //     the item's end zeroed
+      // the row sums of psi(k), psi(q) of the chunk (zero past the item's end, where the
+      // tiles' rows, past n, read as zero)
+      float skv = 0.f, sqv = 0.f;
+      if (threadIdx.x < valid) {
+        skv = skg[I.head * n + t0 + threadIdx.x];
+        if (CAUSAL) sqv = sqg[I.head * n + t0 + threadIdx.x];
+      }
+      // ---- (a) the stage (psi(K), V; causal psi(Q), a_hi, a_lo: the rows of A past the
+      //     item's end zeroed) and the row sums
       if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
         if (threadIdx.x == 0) landed = g + 1;
-        psi_tile<D>(st + OK, C, sh.sk);
         if (CAUSAL) {
-          psi_tile<D>(st + OQ, valid, sh.sq);
           zero_rows<D>(st + OA, valid);
           zero_rows<D>(st + OAL, valid);
         }
       }
-      if (CAUSAL && threadIdx.x < C) sh.bv[threadIdx.x] = bload;
+      if (threadIdx.x < C) {
+        sh.sk[threadIdx.x] = skv;
+        sh.sq[threadIdx.x] = sqv;
+        if (CAUSAL) sh.bv[threadIdx.x] = bload;
+      }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
       if (threadIdx.x == 0) {
@@ -1350,10 +1394,13 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   const unsigned grid = static_cast<unsigned>(nitems < sms * G::CTAS ? nitems : sms * G::CTAS);
   const unsigned grid_agg =
       static_cast<unsigned>(nitems < sms * G::G_CTAS ? nitems : sms * G::G_CTAS);
-  CUtensorMap tq, tk, tv, tg, ta, tal;
+  CUtensorMap tq, tk, tv, tg, ta, tal, tpq, tpk;
   cudaError_t e;
   if ((e = make_tmap_bf16(&tq, q, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tk, k, heads, n, D, C)) != cudaSuccess) return e;
+  // psi(q), psi(k) in the workspace: stored by B1 and K1, read by the walks
+  if ((e = make_tmap_bf16(&tpq, W.psi_q, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tpk, W.psi_k, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tv, v, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tg, g, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&ta, W.a_hi, heads, n, D, C)) != cudaSuccess) return e;
@@ -1364,8 +1411,8 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   // K1 + K2: the forward record before every segment (causal) or of the head (non-causal)
   auto kg = bwd_aggregate_kernel<D>;
   if ((e = prepare(kg, G::G_SMEM)) != cudaSuccess) return e;
-  kg<<<grid_agg, kThreads, G::G_SMEM, st>>>(tk, tv, W.s_rec, W.s_vec, n, seg, nseg, nitems,
-                                            err);
+  kg<<<grid_agg, kThreads, G::G_SMEM, st>>>(tk, tv, tpk, W.sk, W.s_rec, W.s_vec, n, seg, nseg,
+                                            nitems, err);
   count_launches(1);
   record_launch_event(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1386,7 +1433,8 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   // B1: dq, a (hi, lo), b and the reverse record of every segment
   auto k1 = bwd_prefix_kernel<D, CAUSAL>;
   if ((e = prepare(k1, G::P_SMEM)) != cudaSuccess) return e;
-  k1<<<grid, kThreads, G::P_SMEM, st>>>(tq, tk, tv, tg, static_cast<__nv_bfloat16 *>(dq),
+  k1<<<grid, kThreads, G::P_SMEM, st>>>(tq, tpk, tv, tg, tpq, W.sq, W.sk,
+                                        static_cast<__nv_bfloat16 *>(dq),
                                         W.a_hi, W.a_lo, W.b, s_start, s_hs, s_ss, W.s_vec,
                                         W.r_rec, W.r_vec, n, seg, nseg, nitems, err);
   count_launches(1);
@@ -1411,7 +1459,7 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   // B3: dk, dv
   auto k3 = bwd_suffix_kernel<D, CAUSAL>;
   if ((e = prepare(k3, G::S_SMEM)) != cudaSuccess) return e;
-  k3<<<grid, kThreads, G::S_SMEM, st>>>(tq, ta, tal, tk, tv, W.b,
+  k3<<<grid, kThreads, G::S_SMEM, st>>>(tpq, ta, tal, tpk, tv, W.sq, W.sk, W.b,
                                         static_cast<__nv_bfloat16 *>(dk),
                                         static_cast<__nv_bfloat16 *>(dv), r_start, r_hs, r_ss,
                                         W.r_vec, n, seg, nseg, nitems, err);
@@ -1462,6 +1510,10 @@ TcBackwardLayout tc_backward_layout(void *ws, int64_t heads, int64_t n, int d, i
   const int64_t nck = (n + C - 1) / C;
   W.s_vec = reinterpret_cast<float *>(take(heads * nck * (3 * d + 4) * sizeof(float)));
   W.r_vec = reinterpret_cast<float *>(take(heads * nck * (3 * d + 4) * sizeof(float)));
+  W.psi_q = reinterpret_cast<__nv_bfloat16 *>(take(heads * n * d * sizeof(__nv_bfloat16)));
+  W.psi_k = reinterpret_cast<__nv_bfloat16 *>(take(heads * n * d * sizeof(__nv_bfloat16)));
+  W.sq = reinterpret_cast<float *>(take(heads * n * sizeof(float)));
+  W.sk = reinterpret_cast<float *>(take(heads * n * sizeof(float)));
   if (bytes) *bytes = off;
   return W;
 }
