@@ -87,7 +87,6 @@ struct BwdShared {
   uint64_t mma;          // the products issued since the last wait are done
   uint64_t fin;          // drain at exit
   float vec[3][128];     // the record's three vectors (current state)
-  float scal;            // the record's scalar
   float sq[64], sk[64];  // row sums of psi(Q), psi(K) of the chunk
   float part[2][64];     // per column half, per row: partial sums
   float gd[2][64];
@@ -95,9 +94,14 @@ struct BwdShared {
   float bv[64];          // b of the chunk's rows
   float acc[3][128];     // column sums being gathered (atomically) for a chunk or an item
   float racc[3][128];    // the prefix walk: the item's reverse-record vectors
+  float scal;            // the record's scalar
   uint32_t tmem_base;
   int abort;
 };
+// pairs of columns are read as float2
+static_assert(offsetof(BwdShared, vec) % 8 == 0 && offsetof(BwdShared, sq) % 8 == 0 &&
+                  offsetof(BwdShared, sk) % 8 == 0 && offsetof(BwdShared, bv) % 8 == 0,
+              "float2 reads of the shared vectors");
 
 template <int D>
 struct BCfg {
@@ -151,6 +155,26 @@ __device__ __forceinline__ void tmem_row32(uint32_t taddr, float *f) {
   tmem_reg_fence<32>(r);
 #pragma unroll
   for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(r[e]);
+}
+
+// 16 lanes x 32 consecutive fp32 columns of an M = 64 accumulator (lanes 0..15 of the calling
+// warp's sub-partition; taddr: that lane base and the first column), read by all 32 threads
+// (warp-collective): thread t gets rows t/4 and 8 + t/4 of the 16, columns 8k + 2(t%4) + {0, 1}
+// for k = 0..3, as f[4k + {0, 1}] (first row) and f[4k + {2, 3}] (second row).
+__device__ __forceinline__ void tmem_quad32(uint32_t taddr, float *f) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  tmem_ld_wait();
+  tmem_reg_fence<16>(r);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[e]);
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float *f) {
@@ -233,6 +257,8 @@ struct Lanes {
   int r64;            // that row (token within the chunk)
   int rS;             // row of a D x D accumulator
   bool vS;
+  int qa, qb;         // rows of an M = 64 accumulator this thread gets from tmem_quad32
+  int cq;             // its first column within each group of 8 (2 (lane % 4))
   template <int D>
   __device__ __forceinline__ static Lanes make() {
     Lanes L;
@@ -245,6 +271,9 @@ struct Lanes {
     L.r64 = 16 * L.sp + L.lane;
     L.rS = D == 128 ? 32 * L.sp + L.lane : L.r64;
     L.vS = D == 128 || L.v64;
+    L.qa = 16 * L.sp + (L.lane >> 2);
+    L.qb = L.qa + 8;
+    L.cq = 2 * (L.lane & 3);
     return L;
   }
 };
@@ -291,18 +320,32 @@ __device__ __forceinline__ void load_record(const float *src, uint8_t *sOp, uint
 }
 
 // TMEM state (rows rS, this half's columns) -> its bf16 operand (warp-collective loads).
+// D = 64: the state is an M = 64 accumulator, read by all 32 lanes (tmem_quad32).
 template <int D>
 __device__ __forceinline__ void state_to_operand(uint32_t tM, uint8_t *sOp, const Lanes &L) {
   constexpr int HD = D / 2;
-#pragma unroll 1
-  for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
-    float f[32];
-    tmem_row32(tM + c0, f);
-    if (L.vS) {
+  if constexpr (D == 64) {
+    float f[16];
+    tmem_quad32(tM + L.hf * HD, f);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4 *>(sOp + (c0 >> 6) * (D * 128) +
-                                   sw128_offset(L.rS, (c0 & 63) + 8 * q)) = pack8(f + 8 * q);
+    for (int q = 0; q < 4; ++q) {
+      const int c = L.hf * HD + 8 * q + L.cq;
+      *reinterpret_cast<uint32_t *>(sOp + sw128_offset(L.qa, c)) =
+          pack_bf16x2(f[4 * q], f[4 * q + 1]);
+      *reinterpret_cast<uint32_t *>(sOp + sw128_offset(L.qb, c)) =
+          pack_bf16x2(f[4 * q + 2], f[4 * q + 3]);
+    }
+  } else {
+#pragma unroll 1
+    for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
+      float f[32];
+      tmem_row32(tM + c0, f);
+      if (L.vS) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4 *>(sOp + (c0 >> 6) * (D * 128) +
+                                     sw128_offset(L.rS, (c0 & 63) + 8 * q)) = pack8(f + 8 * q);
+      }
     }
   }
 }
@@ -638,7 +681,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   BwdShared &sh = *reinterpret_cast<BwdShared *>(sm + G::P_SH);
   uint8_t *sST = sm + G::P_ST;  // bf16 Psi (rows: features; 64-column blocks of values)
   uint8_t *sA = sm + G::P_A, *sAL = sm + G::P_AL, *sW = sm + G::P_W, *sL = sm + G::P_L;
-  const bool a32 = aligned32(dq);  // the gradient rows take full-sector stores
   const Lanes L = Lanes::make<D>();
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
@@ -718,10 +760,12 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       const int64_t t0 = I.t_begin + (int64_t)c * C;
       const int valid = I.t_end - t0 < C ? static_cast<int>(I.t_end - t0) : C;
       const bool more = CAUSAL && c + 1 < I.nchunks;  // the record after this chunk is needed
-      const bool live = L.v64 && L.r64 < valid;
-      const int64_t row = I.head * n + t0 + L.r64;  // global row of this thread (when live)
+      // every lane takes two rows i (qa, qb) and a quarter of each group of 8 columns
+      const bool la = L.qa < valid, lb = L.qb < valid;
+      const int64_t rowa = I.head * n + t0 + L.qa, rowb = rowa + 8;  // global rows
       // keys row i sees: every key up to it (causal), all n (non-causal)
-      const float Ni = CAUSAL ? static_cast<float>(t0 + L.r64 + 1) : static_cast<float>(n);
+      const float Na = CAUSAL ? static_cast<float>(t0 + L.qa + 1) : static_cast<float>(n);
+      const float Nb = CAUSAL ? static_cast<float>(t0 + L.qb + 1) : static_cast<float>(n);
       const int64_t slot = I.head * nck + t0 / C;  // this chunk's per-chunk vectors
       // causal: the forward record before this chunk = the item's record + the item's chunks
       // before this one; fetched now, stored once the stage has landed
@@ -802,39 +846,47 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         phase_done(&sh.mma, more);
         my_mma = my_mma || more;
       }
-      // psi(q_i) . zeta over this half's features
-      float dpart = 0.f;
-      if (L.v64) {
-#pragma unroll 2
-        for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 8) {
-          float f[8];
-          tile_row8(st + OQ, L.r64, c0, f);
+      // psi(q_i) . zeta over this half's features (this lane's quarter of them)
+      float dpa = 0.f, dpb = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dpart = fmaf(f[e], sh.vec[0][c0 + e], dpart);
-        }
+      for (int f = L.hf * HD + L.cq; f < L.hf * HD + HD; f += 8) {
+        const float2 z = *reinterpret_cast<const float2 *>(&sh.vec[0][f]);
+        const uint32_t ua = *reinterpret_cast<const uint32_t *>(st + OQ + tile_off(L.qa, f));
+        const uint32_t ub = *reinterpret_cast<const uint32_t *>(st + OQ + tile_off(L.qb, f));
+        dpa = fmaf(bf16_lo(ua), z.x, fmaf(bf16_hi(ua), z.y, dpa));
+        dpb = fmaf(bf16_lo(ub), z.x, fmaf(bf16_hi(ub), z.y, dpb));
       }
       if (CAUSAL) {
         // ---- (c) M = mask(P' + sk) (j <= i) rounded into its operand; row sums of M
         S.wait_mma();
         if (S.wait.ok) {
-          float p[32];
-          tmem_row32(myX + 32 * L.hf, p);
-          if (L.v64) {
+          float p[16];
+          tmem_quad32(myX + 32 * L.hf, p);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int j0 = 32 * L.hf + 8 * q;
-              float f[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = j0 + e <= L.r64 ? p[8 * q + e] + sh.sk[j0 + e] : 0.f;
-              const uint4 u = pack8(f);
-              unpack8(u, f);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) dpart += f[e];
-              *reinterpret_cast<uint4 *>(sW + sw128_offset(L.r64, j0)) = u;
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int j = 32 * L.hf + 8 * q + L.cq;  // columns j, j + 1
+            const float2 skj = *reinterpret_cast<const float2 *>(&sh.sk[j]);
+            const uint32_t ua = pack_bf16x2(j <= L.qa ? p[4 * q] + skj.x : 0.f,
+                                            j + 1 <= L.qa ? p[4 * q + 1] + skj.y : 0.f);
+            const uint32_t ub = pack_bf16x2(j <= L.qb ? p[4 * q + 2] + skj.x : 0.f,
+                                            j + 1 <= L.qb ? p[4 * q + 3] + skj.y : 0.f);
+            dpa += bf16_lo(ua) + bf16_hi(ua);
+            dpb += bf16_lo(ub) + bf16_hi(ub);
+            *reinterpret_cast<uint32_t *>(sW + sw128_offset(L.qa, j)) = ua;
+            *reinterpret_cast<uint32_t *>(sW + sw128_offset(L.qb, j)) = ub;
           }
         }
-        if (L.v64) sh.part[L.hf][L.r64] = dpart;
+      }
+      // each row's partial denominator over the four lanes that hold it
+      dpa += __shfl_xor_sync(0xffffffffu, dpa, 1);
+      dpb += __shfl_xor_sync(0xffffffffu, dpb, 1);
+      dpa += __shfl_xor_sync(0xffffffffu, dpa, 2);
+      dpb += __shfl_xor_sync(0xffffffffu, dpb, 2);
+      if ((L.lane & 3) == 0) {
+        sh.part[L.hf][L.qa] = dpa;
+        sh.part[L.hf][L.qb] = dpb;
+      }
+      if (CAUSAL) {
         fence_proxy_async_smem();
         if (!S.barrier()) break;
         if (threadIdx.x == 0) {
@@ -850,73 +902,85 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           mbar_arrive(&sh.mma);
         }
       } else {
-        if (L.v64) sh.part[L.hf][L.r64] = dpart;
         S.wait_mma();
         if (!S.barrier()) break;
       }
-      const float sq_i = L.v64 ? sh.sq[L.r64] : 0.f;
-      const float den =
-          L.v64 ? Ni * (kD + sq_i) + sh.scal + sh.part[0][L.r64] + sh.part[1][L.r64] : 1.f;
+      const float sqa = sh.sq[L.qa], sqb = sh.sq[L.qb];
+      const float dena = Na * (kD + sqa) + sh.scal + sh.part[0][L.qa] + sh.part[1][L.qa];
+      const float denb = Nb * (kD + sqb) + sh.scal + sh.part[0][L.qb] + sh.part[1][L.qb];
 
       // ---- (e) out_i, a_i = g_i / den_i (the bf16 pair into its operands and the
       //     workspace); partial a_i . out_i and a_i . (vs + LV_i)
       if (CAUSAL) S.wait_mma();
-      float gdot = 0.f, cdot = 0.f;
+      float gda = 0.f, gdb = 0.f, cda = 0.f, cdb = 0.f;
       if (S.wait.ok) {
-        const float inv = 1.f / den;
+        const float inva = 1.f / dena, invb = 1.f / denb;
+        const float wa = kD + sqa, wb = kD + sqb;
+        // a_i, its bf16 pair and the partial dot products, for columns c, c + 1 of one row
+        auto emit = [&](int64_t grow, bool lv_ok, int row, int c, float o0, float o1, float l0,
+                        float l1, float w, float inv, float g0, float g1, float &gd, float &cd) {
+          const float2 vs = *reinterpret_cast<const float2 *>(&sh.vec[1][c]);
+          const float2 sg = *reinterpret_cast<const float2 *>(&sh.vec[2][c]);
+          const float v0 = vs.x + l0, v1 = vs.y + l1;
+          const float a0 = lv_ok ? g0 * inv : 0.f, a1 = lv_ok ? g1 * inv : 0.f;
+          gd = fmaf(a0, (w * v0 + sg.x + o0) * inv, fmaf(a1, (w * v1 + sg.y + o1) * inv, gd));
+          cd = fmaf(a0, v0, fmaf(a1, v1, cd));
+          const uint32_t hi = pack_bf16x2(a0, a1);
+          const uint32_t lo = pack_bf16x2(a0 - bf16_lo(hi), a1 - bf16_hi(hi));
+          *reinterpret_cast<uint32_t *>(sA + tile_off(row, c)) = hi;
+          *reinterpret_cast<uint32_t *>(sAL + tile_off(row, c)) = lo;
+          if (lv_ok) {
+            *reinterpret_cast<uint32_t *>(a_hi + grow * D + c) = hi;
+            *reinterpret_cast<uint32_t *>(a_lo + grow * D + c) = lo;
+          }
+        };
 #pragma unroll 1
         for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
-          float o[32], lv[32];
-          tmem_row32(myX + c0, o);
+          float o[16], lv[16];
+          tmem_quad32(myX + c0, o);
           if (CAUSAL) {
-            tmem_row32(myY + c0, lv);
+            tmem_quad32(myY + c0, lv);
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) lv[e] = 0.f;
+            for (int e = 0; e < 16; ++e) lv[e] = 0.f;
           }
-          if (L.v64) {
-            uint4 hi[4], lo[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float gv[8], av[8], rv[8];
-              tile_row8(st + OG, L.r64, c0 + 8 * q, gv);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int col = c0 + 8 * q + e;
-                const float vsum = sh.vec[1][col] + lv[8 * q + e];
-                const float out = ((kD + sq_i) * vsum + sh.vec[2][col] + o[8 * q + e]) * inv;
-                const float a = live ? gv[e] * inv : 0.f;
-                gdot = fmaf(a, out, gdot);
-                cdot = fmaf(a, vsum, cdot);
-                av[e] = a;
-              }
-              hi[q] = pack8(av);
-              unpack8(hi[q], rv);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) rv[e] = av[e] - rv[e];
-              lo[q] = pack8(rv);
-              *reinterpret_cast<uint4 *>(sA + tile_off(L.r64, c0 + 8 * q)) = hi[q];
-              *reinterpret_cast<uint4 *>(sAL + tile_off(L.r64, c0 + 8 * q)) = lo[q];
-            }
-            if (live) {
-              st_global_32B(a_hi + row * D + c0, hi[0], hi[1], true);
-              st_global_32B(a_hi + row * D + c0 + 16, hi[2], hi[3], true);
-              st_global_32B(a_lo + row * D + c0, lo[0], lo[1], true);
-              st_global_32B(a_lo + row * D + c0 + 16, lo[2], lo[3], true);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int c = c0 + 8 * q + L.cq;
+            const uint32_t ga = *reinterpret_cast<const uint32_t *>(st + OG + tile_off(L.qa, c));
+            const uint32_t gb = *reinterpret_cast<const uint32_t *>(st + OG + tile_off(L.qb, c));
+            emit(rowa, la, L.qa, c, o[4 * q], o[4 * q + 1], lv[4 * q], lv[4 * q + 1], wa, inva,
+                 bf16_lo(ga), bf16_hi(ga), gda, cda);
+            emit(rowb, lb, L.qb, c, o[4 * q + 2], o[4 * q + 3], lv[4 * q + 2], lv[4 * q + 3],
+                 wb, invb, bf16_lo(gb), bf16_hi(gb), gdb, cdb);
           }
         }
       }
-      if (L.v64) {
-        sh.gd[L.hf][L.r64] = gdot;
-        sh.cd[L.hf][L.r64] = cdot;
+      // each row's partial dot products over the four lanes that hold it
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        gda += __shfl_xor_sync(0xffffffffu, gda, o);
+        gdb += __shfl_xor_sync(0xffffffffu, gdb, o);
+        cda += __shfl_xor_sync(0xffffffffu, cda, o);
+        cdb += __shfl_xor_sync(0xffffffffu, cdb, o);
+      }
+      if ((L.lane & 3) == 0) {
+        sh.gd[L.hf][L.qa] = gda;
+        sh.gd[L.hf][L.qb] = gdb;
+        sh.cd[L.hf][L.qa] = cda;
+        sh.cd[L.hf][L.qb] = cdb;
       }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
       // b_i = -(a_i . out_i);  C_i = sum_{j seen} dW_ij = a_i . (vs + LV_i) + N_i b_i
-      const float b = live ? -(sh.gd[0][L.r64] + sh.gd[1][L.r64]) : 0.f;
-      const float Ci = live ? sh.cd[0][L.r64] + sh.cd[1][L.r64] + Ni * b : 0.f;
-      if (live && L.hf == 0) b_out[row] = b;
+      const float ba = la ? -(sh.gd[0][L.qa] + sh.gd[1][L.qa]) : 0.f;
+      const float bb = lb ? -(sh.gd[0][L.qb] + sh.gd[1][L.qb]) : 0.f;
+      const float Ca = la ? sh.cd[0][L.qa] + sh.cd[1][L.qa] + Na * ba : 0.f;
+      const float Cb = lb ? sh.cd[0][L.qb] + sh.cd[1][L.qb] + Nb * bb : 0.f;
+      if (L.hf == 0 && (L.lane & 3) == 0) {
+        if (la) b_out[rowa] = ba;
+        if (lb) b_out[rowb] = bb;
+      }
       if (threadIdx.x == 0) {
         if (CAUSAL) {
           // dW = A V^T  (a_hi, then a_lo, along the contraction)
@@ -976,17 +1040,16 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         // ---- (g) mask(dW + b) (j <= i) rounded into the M operand's buffer (M V is done);
         //     the record after this chunk: Psi (TMEM) -> operand (A Psi^T is done)
         if (S.wait.ok) {
-          float w[32];
-          tmem_row32(myX + 32 * L.hf, w);
-          if (L.v64) {
+          float w[16];
+          tmem_quad32(myX + 32 * L.hf, w);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int j0 = 32 * L.hf + 8 * q;
-              float f[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = j0 + e <= L.r64 ? w[8 * q + e] + b : 0.f;
-              *reinterpret_cast<uint4 *>(sW + sw128_offset(L.r64, j0)) = pack8(f);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int j = 32 * L.hf + 8 * q + L.cq;  // columns j, j + 1
+            *reinterpret_cast<uint32_t *>(sW + sw128_offset(L.qa, j)) =
+                pack_bf16x2(j <= L.qa ? w[4 * q] + ba : 0.f, j + 1 <= L.qa ? w[4 * q + 1] + ba : 0.f);
+            *reinterpret_cast<uint32_t *>(sW + sw128_offset(L.qb, j)) =
+                pack_bf16x2(j <= L.qb ? w[4 * q + 2] + bb : 0.f,
+                            j + 1 <= L.qb ? w[4 * q + 3] + bb : 0.f);
           }
           if (more) state_to_operand<D>(myS, sST, L);
         }
@@ -1007,22 +1070,22 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       if (S.wait.ok) {
 #pragma unroll 1
         for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
-          float f[32];
-          tmem_row32(myY + c0, f);
-          if (live) {
+          float f[16];
+          tmem_quad32(myY + c0, f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float ps[8];
-              tile_row8(st + OQ, L.r64, c0 + 8 * q, ps);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int col = c0 + 8 * q + e;
-                f[8 * q + e] =
-                    (f[8 * q + e] + fmaf(sh.vec[0][col], b, Ci)) * dphi_from_psi(ps[e]);
-              }
-            }
-            st_global_32B(dq + row * D + c0, pack8(f), pack8(f + 8), a32);
-            st_global_32B(dq + row * D + c0 + 16, pack8(f + 16), pack8(f + 24), a32);
+          for (int q = 0; q < 4; ++q) {
+            const int c = c0 + 8 * q + L.cq;  // columns c, c + 1
+            const float2 z = *reinterpret_cast<const float2 *>(&sh.vec[0][c]);
+            const uint32_t pa = *reinterpret_cast<const uint32_t *>(st + OQ + tile_off(L.qa, c));
+            const uint32_t pb = *reinterpret_cast<const uint32_t *>(st + OQ + tile_off(L.qb, c));
+            if (la)
+              *reinterpret_cast<uint32_t *>(dq + rowa * D + c) =
+                  pack_bf16x2((f[4 * q] + fmaf(z.x, ba, Ca)) * dphi_from_psi(bf16_lo(pa)),
+                              (f[4 * q + 1] + fmaf(z.y, ba, Ca)) * dphi_from_psi(bf16_hi(pa)));
+            if (lb)
+              *reinterpret_cast<uint32_t *>(dq + rowb * D + c) =
+                  pack_bf16x2((f[4 * q + 2] + fmaf(z.x, bb, Cb)) * dphi_from_psi(bf16_lo(pb)),
+                              (f[4 * q + 3] + fmaf(z.y, bb, Cb)) * dphi_from_psi(bf16_hi(pb)));
           }
         }
       }
@@ -1098,7 +1161,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
   uint8_t *sFT = sm + G::S_ST;  // bf16 Phi (rows: features; 64-column blocks of values)
   uint8_t *sW0 = sm + G::S_W0;  // mask(w^T): the weights of the chunk's keys
   uint8_t *sW1 = sm + G::S_W1;  // mask(dW^T + b)
-  const bool a32v = aligned32(dv), a32k = aligned32(dk);  // full-sector stores
   const Lanes L = Lanes::make<D>();
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
@@ -1162,8 +1224,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       const int64_t t0 = I.t_begin + (int64_t)chunk_of(w, I.nchunks) * C;
       const int valid = I.t_end - t0 < C ? static_cast<int>(I.t_end - t0) : C;
       const bool more = CAUSAL && w + 1 < I.nchunks;  // the record before this chunk is needed
-      const bool live = L.v64 && L.r64 < valid;
-      const int64_t row = I.head * n + t0 + L.r64;
 
       // b of the chunk's rows, fetched while the tiles land (zero past the item's end), and
       // this chunk's reverse sums (from the prefix walk), added to the record after it
@@ -1266,38 +1326,47 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         // ---- (c) row j: the weights w_ji = d + sq_i + sk_j + P'^T_ji and dW^T_ji + b_i, kept
         //     for i >= j and rounded into their operands; C'_j's part from this chunk
         S.wait_mma();
-        float cin = 0.f;
+        // every lane takes two rows j (qa, qb) and 16 of this half's columns i (tmem_quad32)
+        float cina = 0.f, cinb = 0.f;
         if (S.wait.ok) {
-          float p[32];
-          tmem_row32(myX + 32 * L.hf, p);
-          if (L.v64) {
-            const float skj = kD + sh.sk[L.r64];
+          float p[16];
+          tmem_quad32(myX + 32 * L.hf, p);
+          const float ska = kD + sh.sk[L.qa], skb = kD + sh.sk[L.qb];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int i0 = 32 * L.hf + 8 * q;
-              float f[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                f[e] = i0 + e >= L.r64 ? p[8 * q + e] + sh.sq[i0 + e] + skj : 0.f;
-              *reinterpret_cast<uint4 *>(sW0 + sw128_offset(L.r64, i0)) = pack8(f);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int i = 32 * L.hf + 8 * q + L.cq;  // columns i, i + 1
+            const float2 sqi = *reinterpret_cast<const float2 *>(&sh.sq[i]);
+            const float a0 = i >= L.qa ? p[4 * q] + sqi.x + ska : 0.f;
+            const float a1 = i + 1 >= L.qa ? p[4 * q + 1] + sqi.y + ska : 0.f;
+            const float b0 = i >= L.qb ? p[4 * q + 2] + sqi.x + skb : 0.f;
+            const float b1 = i + 1 >= L.qb ? p[4 * q + 3] + sqi.y + skb : 0.f;
+            *reinterpret_cast<uint32_t *>(sW0 + sw128_offset(L.qa, i)) = pack_bf16x2(a0, a1);
+            *reinterpret_cast<uint32_t *>(sW0 + sw128_offset(L.qb, i)) = pack_bf16x2(b0, b1);
           }
-          tmem_row32(myX + 64 + 32 * L.hf, p);
-          if (L.v64) {
+          tmem_quad32(myX + 64 + 32 * L.hf, p);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int i0 = 32 * L.hf + 8 * q;
-              float f[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                f[e] = i0 + e >= L.r64 ? p[8 * q + e] + sh.bv[i0 + e] : 0.f;
-                cin += f[e];
-              }
-              *reinterpret_cast<uint4 *>(sW1 + sw128_offset(L.r64, i0)) = pack8(f);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int i = 32 * L.hf + 8 * q + L.cq;
+            const float2 bi = *reinterpret_cast<const float2 *>(&sh.bv[i]);
+            const float a0 = i >= L.qa ? p[4 * q] + bi.x : 0.f;
+            const float a1 = i + 1 >= L.qa ? p[4 * q + 1] + bi.y : 0.f;
+            const float b0 = i >= L.qb ? p[4 * q + 2] + bi.x : 0.f;
+            const float b1 = i + 1 >= L.qb ? p[4 * q + 3] + bi.y : 0.f;
+            cina += a0 + a1;
+            cinb += b0 + b1;
+            *reinterpret_cast<uint32_t *>(sW1 + sw128_offset(L.qa, i)) = pack_bf16x2(a0, a1);
+            *reinterpret_cast<uint32_t *>(sW1 + sw128_offset(L.qb, i)) = pack_bf16x2(b0, b1);
           }
         }
-        if (L.v64) sh.part[L.hf][L.r64] = cin;
+        // each row's sum over the four lanes that hold it
+        cina += __shfl_xor_sync(0xffffffffu, cina, 1);
+        cinb += __shfl_xor_sync(0xffffffffu, cinb, 1);
+        cina += __shfl_xor_sync(0xffffffffu, cina, 2);
+        cinb += __shfl_xor_sync(0xffffffffu, cinb, 2);
+        if ((L.lane & 3) == 0) {
+          sh.part[L.hf][L.qa] = cina;
+          sh.part[L.hf][L.qb] = cinb;
+        }
         fence_proxy_async_smem();
         if (!S.barrier()) break;
         if (threadIdx.x == 0) {
@@ -1327,36 +1396,47 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       S.wait_mma();
       if (!CAUSAL && !S.barrier()) break;  // both halves of v_j . as are in sh.gd
       if (S.wait.ok) {
-        const float skj = L.v64 ? kD + sh.sk[L.r64] : 0.f;
-        const float cpj =
-            L.v64 ? sh.gd[0][L.r64] + sh.gd[1][L.r64] + sh.scal +
-                        (CAUSAL ? sh.part[0][L.r64] + sh.part[1][L.r64] : 0.f)
-                  : 0.f;
+        // every lane takes two rows j (qa, qb) and 16 of each 32 columns (tmem_quad32)
+        const bool la = L.qa < valid, lb = L.qb < valid;
+        const int64_t rowa = I.head * n + t0 + L.qa, rowb = rowa + 8;
+        const float ska = kD + sh.sk[L.qa], skb = kD + sh.sk[L.qb];
+        const float cpa = sh.gd[0][L.qa] + sh.gd[1][L.qa] + sh.scal +
+                          (CAUSAL ? sh.part[0][L.qa] + sh.part[1][L.qa] : 0.f);
+        const float cpb = sh.gd[0][L.qb] + sh.gd[1][L.qb] + sh.scal +
+                          (CAUSAL ? sh.part[0][L.qb] + sh.part[1][L.qb] : 0.f);
 #pragma unroll 1
         for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
-          float f[32];
-          tmem_row32(myX + c0, f);
-          if (live) {
+          float f[16];
+          tmem_quad32(myX + c0, f);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              f[e] = fmaf(skj, sh.vec[1][c0 + e], sh.vec[2][c0 + e] + f[e]);
-            st_global_32B(dv + row * D + c0, pack8(f), pack8(f + 8), a32v);
-            st_global_32B(dv + row * D + c0 + 16, pack8(f + 16), pack8(f + 24), a32v);
+          for (int q = 0; q < 4; ++q) {
+            const int c = c0 + 8 * q + L.cq;  // columns c, c + 1
+            const float2 as = *reinterpret_cast<const float2 *>(&sh.vec[1][c]);
+            const float2 tau = *reinterpret_cast<const float2 *>(&sh.vec[2][c]);
+            if (la)
+              *reinterpret_cast<uint32_t *>(dv + rowa * D + c) =
+                  pack_bf16x2(fmaf(ska, as.x, tau.x + f[4 * q]),
+                              fmaf(ska, as.y, tau.y + f[4 * q + 1]));
+            if (lb)
+              *reinterpret_cast<uint32_t *>(dv + rowb * D + c) =
+                  pack_bf16x2(fmaf(skb, as.x, tau.x + f[4 * q + 2]),
+                              fmaf(skb, as.y, tau.y + f[4 * q + 3]));
           }
-          tmem_row32(myX + D + c0, f);
-          if (live) {
+          tmem_quad32(myX + D + c0, f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float ps[8];
-              tile_row8(st + OK, L.r64, c0 + 8 * q, ps);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int col = c0 + 8 * q + e;
-                f[8 * q + e] = (f[8 * q + e] + sh.vec[0][col] + cpj) * dphi_from_psi(ps[e]);
-              }
-            }
-            st_global_32B(dk + row * D + c0, pack8(f), pack8(f + 8), a32k);
-            st_global_32B(dk + row * D + c0 + 16, pack8(f + 16), pack8(f + 24), a32k);
+          for (int q = 0; q < 4; ++q) {
+            const int c = c0 + 8 * q + L.cq;
+            const float2 rho = *reinterpret_cast<const float2 *>(&sh.vec[0][c]);
+            const uint32_t pa = *reinterpret_cast<const uint32_t *>(st + OK + tile_off(L.qa, c));
+            const uint32_t pb = *reinterpret_cast<const uint32_t *>(st + OK + tile_off(L.qb, c));
+            if (la)
+              *reinterpret_cast<uint32_t *>(dk + rowa * D + c) =
+                  pack_bf16x2((f[4 * q] + rho.x + cpa) * dphi_from_psi(bf16_lo(pa)),
+                              (f[4 * q + 1] + rho.y + cpa) * dphi_from_psi(bf16_hi(pa)));
+            if (lb)
+              *reinterpret_cast<uint32_t *>(dk + rowb * D + c) =
+                  pack_bf16x2((f[4 * q + 2] + rho.x + cpb) * dphi_from_psi(bf16_lo(pb)),
+                              (f[4 * q + 3] + rho.y + cpb) * dphi_from_psi(bf16_hi(pb)));
           }
         }
         if (more) state_to_operand<D>(myR, sFT, L);
