@@ -157,26 +157,6 @@ __device__ __forceinline__ void tmem_row32(uint32_t taddr, float *f) {
   for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(r[e]);
 }
 
-// 16 lanes x 32 consecutive fp32 columns of an M = 64 accumulator (lanes 0..15 of the calling
-// warp's sub-partition; taddr: that lane base and the first column), read by all 32 threads
-// (warp-collective): thread t gets rows t/4 and 8 + t/4 of the 16, columns 8k + 2(t%4) + {0, 1}
-// for k = 0..3, as f[4k + {0, 1}] (first row) and f[4k + {2, 3}] (second row).
-__device__ __forceinline__ void tmem_quad32(uint32_t taddr, float *f) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-  tmem_ld_wait();
-  tmem_reg_fence<16>(r);
-#pragma unroll
-  for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[e]);
-}
-
 __device__ __forceinline__ void unpack8(uint4 u, float *f) {
   f[0] = bf16_lo(u.x);
   f[1] = bf16_hi(u.x);

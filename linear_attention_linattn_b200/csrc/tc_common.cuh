@@ -1,6 +1,7 @@
-// Pieces shared by the tensor-core kernels (tc_forward.cu, tc_causal.cu): shared-memory
-// matrix descriptors, the packed-bf16 feature map, 32-byte global stores, warp-uniform
-// waits, the (head, segment) work items, and the TMA tensor maps of [heads][n][d] bf16.
+// Pieces shared by the tensor-core kernels (tc_forward.cu, tc_causal.cu, tc_backward.cu):
+// shared-memory matrix descriptors, the packed-bf16 feature map, 32-byte global stores, the
+// all-lane read of M = 64 accumulators, warp-uniform waits, the (head, segment) work items, and
+// the TMA tensor maps of [heads][n][d] bf16.
 #pragma once
 
 #include <cuda.h>
@@ -88,6 +89,27 @@ __device__ __forceinline__ void st_global_32B(void *p, uint4 a, uint4 b, bool a3
     q[0] = a;
     q[1] = b;
   }
+}
+
+// 16 lanes x 32 consecutive fp32 columns of an M = 64 accumulator (it lives in lanes 0..15 of
+// each TMEM sub-partition; taddr: the calling warp's lane base and the first column), read by
+// all 32 threads (warp-collective), where the 32x32b loads would leave half the warp idle:
+// thread t gets rows t/4 and 8 + t/4 of the 16, columns 8k + 2(t%4) + {0, 1} for k = 0..3, as
+// f[4k + {0, 1}] (first row) and f[4k + {2, 3}] (second row).
+__device__ __forceinline__ void tmem_quad32(uint32_t taddr, float *f) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  tmem_ld_wait();
+  tmem_reg_fence<16>(r);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[e]);
 }
 
 // mbarrier wait of a whole warp whose outcome the lanes share (warp-uniform control flow);
