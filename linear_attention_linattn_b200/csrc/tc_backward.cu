@@ -1197,6 +1197,23 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
     const Item I = item_at<C>(it, n, seg_len, nseg);
     // ---- the item's starting reverse record: Phi (TMEM, causal) and its operand; vectors
     load_record<D>(start + I.head * start_hs + I.seg * start_ss, sFT, myR, CAUSAL, L, sh);
+    // b and the row sums of psi(k), psi(q) of a chunk's rows (zero past the item's end, where
+    // the tiles' rows, past n, read as zero), fetched a chunk ahead of their use
+    float nb = 0.f, nsk = 0.f, nsq = 0.f;
+    auto fetch = [&](int ww) {
+      const int64_t tt = I.t_begin + (int64_t)chunk_of(ww, I.nchunks) * C;
+      if (threadIdx.x < I.t_end - tt && threadIdx.x < C) {
+        const int64_t at = I.head * n + tt + threadIdx.x;
+        nsk = skg[at];
+        if (CAUSAL) {
+          nb = b_in[at];
+          nsq = sqg[at];
+        }
+      } else {
+        nb = nsk = nsq = 0.f;
+      }
+    };
+    fetch(0);
     for (int w = 0; w < I.nchunks; ++w, ++g) {
       uint8_t *st = sm + (g & 1) * G::S_STAGE;
       const uint32_t uQ = smem_u32(st + OQ), uA = smem_u32(st + OA), uAL = smem_u32(st + OAL);
@@ -1205,10 +1222,9 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       const int valid = I.t_end - t0 < C ? static_cast<int>(I.t_end - t0) : C;
       const bool more = CAUSAL && w + 1 < I.nchunks;  // the record before this chunk is needed
 
-      // b of the chunk's rows, fetched while the tiles land (zero past the item's end), and
+      const float bload = nb, skv = nsk, sqv = nsq;
+      if (w + 1 < I.nchunks) fetch(w + 1);
       // this chunk's reverse sums (from the prefix walk), added to the record after it
-      float bload = 0.f;
-      if (CAUSAL && threadIdx.x < valid) bload = b_in[I.head * n + t0 + threadIdx.x];
       float rv[3] = {0.f, 0.f, 0.f}, rs = 0.f;
       if (more) {
         const float *src = r_vec + (I.head * nck + t0 / C) * VF;
@@ -1217,13 +1233,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           for (int k = 0; k < 3; ++k) rv[k] = src[k * D + threadIdx.x];
         }
         if (threadIdx.x == 0) rs = src[3 * D];
-      }
-      // the row sums of psi(k), psi(q) of the chunk (zero past the item's end, where the
-      // tiles' rows, past n, read as zero)
-      float skv = 0.f, sqv = 0.f;
-      if (threadIdx.x < valid) {
-        skv = skg[I.head * n + t0 + threadIdx.x];
-        if (CAUSAL) sqv = sqg[I.head * n + t0 + threadIdx.x];
       }
       // ---- (a) the stage (psi(K), V; causal psi(Q), a_hi, a_lo: the rows of A past the
       //     item's end zeroed) and the row sums
