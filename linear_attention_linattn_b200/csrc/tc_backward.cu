@@ -623,7 +623,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
 // ---------------------------------------------------------------- B1: the prefix walk
 // q, dout: [heads][n][D] via tmQ, tmG; psi(k), v via tmK, tmV and skg (psi(k)'s row sums,
 // [heads][n]) (causal only).  Causal: stores psi(q) via tmPQ with its row sums to sqg, for the
-// suffix walk.  start: each item's forward record (causal: exclusive prefix at start + head * start_hs + seg * start_ss;
+// suffix walk.  dq, and (causal) a as a bf16 pair, are stored through tile stores (tmDQ,
+// tmAH, tmAL: [heads][n][D]).  start: each item's forward record (causal: exclusive prefix at start + head * start_hs + seg * start_ss;
 // non-causal: the head's total).  Writes dq, a as a bf16 pair (a_hi, a_lo: [heads][n][D]),
 // b ([heads][n]) and each item's reverse record to r_rec + (head * nseg + seg) * rec_floats.
 template <int D, bool CAUSAL>
@@ -633,8 +634,9 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
                       const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmG,
                       const __grid_constant__ CUtensorMap tmPQ, float *__restrict__ sqg,
-                      const float *__restrict__ skg, __nv_bfloat16 *__restrict__ dq,
-                      __nv_bfloat16 *__restrict__ a_hi, __nv_bfloat16 *__restrict__ a_lo,
+                      const float *__restrict__ skg, const __grid_constant__ CUtensorMap tmDQ,
+                      const __grid_constant__ CUtensorMap tmAH,
+                      const __grid_constant__ CUtensorMap tmAL,
                       float *__restrict__ b_out, const float *__restrict__ start,
                       int64_t start_hs, int64_t start_ss, const float *__restrict__ s_vec,
                       float *__restrict__ r_rec, float *__restrict__ r_vec, int64_t n,
@@ -786,8 +788,11 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
             tma_store_3d(&tmPQ, st + OQ + a * kAtom, 64 * a, static_cast<int>(t0),
                          static_cast<int>(I.head), pol);
           tma_store_commit();
-          // the other stage's tile has been read by its store before the next load lands there
+          // every earlier tile store (the other stage's psi(q), the last chunk's a pair and dq)
+          // has read its tile before the next load, or this chunk's a pair, lands there
           tma_store_wait_read<1>();
+        } else {
+          tma_store_wait_read<0>();  // the last chunk's dq has been read from sA
         }
         // the next step's tiles into the other stage (its last reader, step g - 1, is done)
         if (c + 1 < I.nchunks)
@@ -897,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
         const float inva = 1.f / dena, invb = 1.f / denb;
         const float wa = kD + sqa, wb = kD + sqb;
         // a_i, its bf16 pair and the partial dot products, for columns c, c + 1 of one row
-        auto emit = [&](int64_t grow, bool lv_ok, int row, int c, float o0, float o1, float l0,
+        auto emit = [&](bool lv_ok, int row, int c, float o0, float o1, float l0,
                         float l1, float w, float inv, float g0, float g1, float &gd, float &cd) {
           const float2 vs = *reinterpret_cast<const float2 *>(&sh.vec[1][c]);
           const float2 sg = *reinterpret_cast<const float2 *>(&sh.vec[2][c]);
@@ -909,10 +914,6 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           const uint32_t lo = pack_bf16x2(a0 - bf16_lo(hi), a1 - bf16_hi(hi));
           *reinterpret_cast<uint32_t *>(sA + tile_off(row, c)) = hi;
           *reinterpret_cast<uint32_t *>(sAL + tile_off(row, c)) = lo;
-          if (lv_ok) {
-            *reinterpret_cast<uint32_t *>(a_hi + grow * D + c) = hi;
-            *reinterpret_cast<uint32_t *>(a_lo + grow * D + c) = lo;
-          }
         };
 #pragma unroll 1
         for (int c0 = L.hf * HD; c0 < L.hf * HD + HD; c0 += 32) {
@@ -929,10 +930,10 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
             const int c = c0 + 8 * q + L.cq;
             const uint32_t ga = *reinterpret_cast<const uint32_t *>(st + OG + tile_off(L.qa, c));
             const uint32_t gb = *reinterpret_cast<const uint32_t *>(st + OG + tile_off(L.qb, c));
-            emit(rowa, la, L.qa, c, o[4 * q], o[4 * q + 1], lv[4 * q], lv[4 * q + 1], wa, inva,
+            emit(la, L.qa, c, o[4 * q], o[4 * q + 1], lv[4 * q], lv[4 * q + 1], wa, inva,
                  bf16_lo(ga), bf16_hi(ga), gda, cda);
-            emit(rowb, lb, L.qb, c, o[4 * q + 2], o[4 * q + 3], lv[4 * q + 2], lv[4 * q + 3],
-                 wb, invb, bf16_lo(gb), bf16_hi(gb), gdb, cdb);
+            emit(lb, L.qb, c, o[4 * q + 2], o[4 * q + 3], lv[4 * q + 2], lv[4 * q + 3], wb, invb,
+                 bf16_lo(gb), bf16_hi(gb), gdb, cdb);
           }
         }
       }
@@ -960,6 +961,17 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       if (L.hf == 0 && (L.lane & 3) == 0) {
         if (la) b_out[rowa] = ba;
         if (lb) b_out[rowb] = bb;
+      }
+      if (CAUSAL && threadIdx.x == 0) {
+        // a as a bf16 pair to the workspace for the suffix walk (rows past n are not stored)
+#pragma unroll
+        for (int a = 0; a < AT; ++a) {
+          tma_store_3d(&tmAH, sA + a * kAtom, 64 * a, static_cast<int>(t0),
+                       static_cast<int>(I.head), pol);
+          tma_store_3d(&tmAL, sAL + a * kAtom, 64 * a, static_cast<int>(t0),
+                       static_cast<int>(I.head), pol);
+        }
+        tma_store_commit();
       }
       if (threadIdx.x == 0) {
         if (CAUSAL) {
@@ -1033,6 +1045,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
           }
           if (more) state_to_operand<D>(myS, sST, L);
         }
+        // (i) stages dq in sA: the tile stores of the pair have read it by the barrier below
+        if (threadIdx.x == 0) tma_store_wait_read<0>();
         fence_proxy_async_smem();
         if (!S.barrier()) break;
         if (threadIdx.x == 0) {
@@ -1058,18 +1072,25 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
             const float2 z = *reinterpret_cast<const float2 *>(&sh.vec[0][c]);
             const uint32_t pa = *reinterpret_cast<const uint32_t *>(st + OQ + tile_off(L.qa, c));
             const uint32_t pb = *reinterpret_cast<const uint32_t *>(st + OQ + tile_off(L.qb, c));
-            if (la)
-              *reinterpret_cast<uint32_t *>(dq + rowa * D + c) =
-                  pack_bf16x2((f[4 * q] + fmaf(z.x, ba, Ca)) * dphi_from_psi(bf16_lo(pa)),
-                              (f[4 * q + 1] + fmaf(z.y, ba, Ca)) * dphi_from_psi(bf16_hi(pa)));
-            if (lb)
-              *reinterpret_cast<uint32_t *>(dq + rowb * D + c) =
-                  pack_bf16x2((f[4 * q + 2] + fmaf(z.x, bb, Cb)) * dphi_from_psi(bf16_lo(pb)),
-                              (f[4 * q + 3] + fmaf(z.y, bb, Cb)) * dphi_from_psi(bf16_hi(pb)));
+            *reinterpret_cast<uint32_t *>(sA + tile_off(L.qa, c)) =
+                pack_bf16x2((f[4 * q] + fmaf(z.x, ba, Ca)) * dphi_from_psi(bf16_lo(pa)),
+                            (f[4 * q + 1] + fmaf(z.y, ba, Ca)) * dphi_from_psi(bf16_hi(pa)));
+            *reinterpret_cast<uint32_t *>(sA + tile_off(L.qb, c)) =
+                pack_bf16x2((f[4 * q + 2] + fmaf(z.x, bb, Cb)) * dphi_from_psi(bf16_lo(pb)),
+                            (f[4 * q + 3] + fmaf(z.y, bb, Cb)) * dphi_from_psi(bf16_hi(pb)));
           }
         }
       }
+      fence_proxy_async_smem();
       if (!S.barrier()) break;
+      if (threadIdx.x == 0) {
+        // the chunk's dq rows, staged in sA (rows past n are not stored)
+#pragma unroll
+        for (int a = 0; a < AT; ++a)
+          tma_store_3d(&tmDQ, sA + a * kAtom, 64 * a, static_cast<int>(t0),
+                       static_cast<int>(I.head), pol);
+        tma_store_commit();
+      }
       // this chunk's reverse sums: into the item's record, and (causal) to the suffix walk
       if (threadIdx.x < D) {
 #pragma unroll
@@ -1098,13 +1119,14 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
     }
     if (!S.barrier()) break;
   }
-  if (CAUSAL && threadIdx.x == 0) tma_store_wait_all<0>();  // done with shared memory
+  if (threadIdx.x == 0) tma_store_wait_all<0>();  // the tile stores are done
   finish(sh, landed, issued, tmem, G::TCOLS, err, kIssuers, my_mma);
 }
 
 // ---------------------------------------------------------------- B3: the suffix walk
 // psi(q), a_hi, a_lo: [heads][n][D] via tmQ, tmA, tmAL, and b_in: [heads][n] (causal only);
-// psi(k), v via tmK, tmV; sqg, skg: the row sums of psi(q), psi(k) ([heads][n]).  start: each item's reverse record (causal: exclusive suffix at start +
+// psi(k), v via tmK, tmV; sqg, skg: the row sums of psi(q), psi(k) ([heads][n]).  dk, dv leave
+// through tile stores (tmDK, tmDV: [heads][n][D]), staged in the stage's A slots.  start: each item's reverse record (causal: exclusive suffix at start +
 // head * start_hs + seg * start_ss; non-causal: the head's total).  Writes dk, dv.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
@@ -1114,7 +1136,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sqg,
                       const float *__restrict__ skg, const float *__restrict__ b_in,
-                      __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
+                      const __grid_constant__ CUtensorMap tmDK,
+                      const __grid_constant__ CUtensorMap tmDV,
                       const float *__restrict__ start, int64_t start_hs, int64_t start_ss,
                       const float *__restrict__ r_vec, int64_t n, int64_t seg_len, int64_t nseg,
                       int64_t nitems, int *err) {
@@ -1251,6 +1274,9 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       fence_proxy_async_smem();
       if (!S.barrier()) break;
       if (threadIdx.x == 0) {
+        // the other stage's dk, dv (the last chunk's) have been read by their tile stores
+        // before the next load lands there
+        tma_store_wait_read<0>();
         if (w + 1 < I.nchunks)
           issue(I, w + 1);
         else if (it + istep < nitems)
@@ -1385,9 +1411,9 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       S.wait_mma();
       if (!CAUSAL && !S.barrier()) break;  // both halves of v_j . as are in sh.gd
       if (S.wait.ok) {
-        // every lane takes two rows j (qa, qb) and 16 of each 32 columns (tmem_quad32)
-        const bool la = L.qa < valid, lb = L.qb < valid;
-        const int64_t rowa = I.head * n + t0 + L.qa, rowb = rowa + 8;
+        // every lane takes two rows j (qa, qb) and 16 of each 32 columns (tmem_quad32); dv
+        // and dk go to the stage's A and A-lo slots (the products that read them are done)
+        uint8_t *sDV = st + OA, *sDK = st + OAL;
         const float ska = kD + sh.sk[L.qa], skb = kD + sh.sk[L.qb];
         const float cpa = sh.gd[0][L.qa] + sh.gd[1][L.qa] + sh.scal +
                           (CAUSAL ? sh.part[0][L.qa] + sh.part[1][L.qa] : 0.f);
@@ -1402,14 +1428,11 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
             const int c = c0 + 8 * q + L.cq;  // columns c, c + 1
             const float2 as = *reinterpret_cast<const float2 *>(&sh.vec[1][c]);
             const float2 tau = *reinterpret_cast<const float2 *>(&sh.vec[2][c]);
-            if (la)
-              *reinterpret_cast<uint32_t *>(dv + rowa * D + c) =
-                  pack_bf16x2(fmaf(ska, as.x, tau.x + f[4 * q]),
-                              fmaf(ska, as.y, tau.y + f[4 * q + 1]));
-            if (lb)
-              *reinterpret_cast<uint32_t *>(dv + rowb * D + c) =
-                  pack_bf16x2(fmaf(skb, as.x, tau.x + f[4 * q + 2]),
-                              fmaf(skb, as.y, tau.y + f[4 * q + 3]));
+            *reinterpret_cast<uint32_t *>(sDV + tile_off(L.qa, c)) =
+                pack_bf16x2(fmaf(ska, as.x, tau.x + f[4 * q]), fmaf(ska, as.y, tau.y + f[4 * q + 1]));
+            *reinterpret_cast<uint32_t *>(sDV + tile_off(L.qb, c)) =
+                pack_bf16x2(fmaf(skb, as.x, tau.x + f[4 * q + 2]),
+                            fmaf(skb, as.y, tau.y + f[4 * q + 3]));
           }
           tmem_quad32(myX + D + c0, f);
 #pragma unroll
@@ -1418,20 +1441,29 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
             const float2 rho = *reinterpret_cast<const float2 *>(&sh.vec[0][c]);
             const uint32_t pa = *reinterpret_cast<const uint32_t *>(st + OK + tile_off(L.qa, c));
             const uint32_t pb = *reinterpret_cast<const uint32_t *>(st + OK + tile_off(L.qb, c));
-            if (la)
-              *reinterpret_cast<uint32_t *>(dk + rowa * D + c) =
-                  pack_bf16x2((f[4 * q] + rho.x + cpa) * dphi_from_psi(bf16_lo(pa)),
-                              (f[4 * q + 1] + rho.y + cpa) * dphi_from_psi(bf16_hi(pa)));
-            if (lb)
-              *reinterpret_cast<uint32_t *>(dk + rowb * D + c) =
-                  pack_bf16x2((f[4 * q + 2] + rho.x + cpb) * dphi_from_psi(bf16_lo(pb)),
-                              (f[4 * q + 3] + rho.y + cpb) * dphi_from_psi(bf16_hi(pb)));
+            *reinterpret_cast<uint32_t *>(sDK + tile_off(L.qa, c)) =
+                pack_bf16x2((f[4 * q] + rho.x + cpa) * dphi_from_psi(bf16_lo(pa)),
+                            (f[4 * q + 1] + rho.y + cpa) * dphi_from_psi(bf16_hi(pa)));
+            *reinterpret_cast<uint32_t *>(sDK + tile_off(L.qb, c)) =
+                pack_bf16x2((f[4 * q + 2] + rho.x + cpb) * dphi_from_psi(bf16_lo(pb)),
+                            (f[4 * q + 3] + rho.y + cpb) * dphi_from_psi(bf16_hi(pb)));
           }
         }
         if (more) state_to_operand<D>(myR, sFT, L);
       }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
+      if (threadIdx.x == 0) {
+        // the chunk's dk, dv rows (rows past n are not stored)
+#pragma unroll
+        for (int a = 0; a < AT; ++a) {
+          tma_store_3d(&tmDV, st + OA + a * kAtom, 64 * a, static_cast<int>(t0),
+                       static_cast<int>(I.head), pol);
+          tma_store_3d(&tmDK, st + OAL + a * kAtom, 64 * a, static_cast<int>(t0),
+                       static_cast<int>(I.head), pol);
+        }
+        tma_store_commit();
+      }
       if (more) {
         // the record before this chunk
         if (threadIdx.x < D) {
@@ -1442,6 +1474,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::CTAS)
       }
     }
   }
+  if (threadIdx.x == 0) tma_store_wait_all<0>();  // the tile stores are done
   finish(sh, landed, issued, tmem, G::TCOLS, err, kIssuers, my_mma);
 }
 
@@ -1463,7 +1496,7 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   const unsigned grid = static_cast<unsigned>(nitems < sms * G::CTAS ? nitems : sms * G::CTAS);
   const unsigned grid_agg =
       static_cast<unsigned>(nitems < sms * G::G_CTAS ? nitems : sms * G::G_CTAS);
-  CUtensorMap tq, tk, tv, tg, ta, tal, tpq, tpk;
+  CUtensorMap tq, tk, tv, tg, ta, tal, tpq, tpk, tdq, tdk, tdv;
   cudaError_t e;
   if ((e = make_tmap_bf16(&tq, q, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tk, k, heads, n, D, C)) != cudaSuccess) return e;
@@ -1474,6 +1507,10 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   if ((e = make_tmap_bf16(&tg, g, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&ta, W.a_hi, heads, n, D, C)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tal, W.a_lo, heads, n, D, C)) != cudaSuccess) return e;
+  // the gradients leave through tile stores
+  if ((e = make_tmap_bf16(&tdq, dq, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tdk, dk, heads, n, D, C)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tdv, dv, heads, n, D, C)) != cudaSuccess) return e;
   // the scans treat a record as 4 x (rec / 4 - 1) + 4 floats: element by element
   const int sdk = 4, sdv = static_cast<int>(rec / 4 - 1);
 
@@ -1502,9 +1539,8 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   // B1: dq, a (hi, lo), b and the reverse record of every segment
   auto k1 = bwd_prefix_kernel<D, CAUSAL>;
   if ((e = prepare(k1, G::P_SMEM)) != cudaSuccess) return e;
-  k1<<<grid, kThreads, G::P_SMEM, st>>>(tq, tpk, tv, tg, tpq, W.sq, W.sk,
-                                        static_cast<__nv_bfloat16 *>(dq),
-                                        W.a_hi, W.a_lo, W.b, s_start, s_hs, s_ss, W.s_vec,
+  k1<<<grid, kThreads, G::P_SMEM, st>>>(tq, tpk, tv, tg, tpq, W.sq, W.sk, tdq, ta, tal,
+                                        W.b, s_start, s_hs, s_ss, W.s_vec,
                                         W.r_rec, W.r_vec, n, seg, nseg, nitems, err);
   count_launches(1);
   record_launch_event(st);
@@ -1528,9 +1564,8 @@ cudaError_t backward_dims(const void *q, const void *k, const void *v, const voi
   // B3: dk, dv
   auto k3 = bwd_suffix_kernel<D, CAUSAL>;
   if ((e = prepare(k3, G::S_SMEM)) != cudaSuccess) return e;
-  k3<<<grid, kThreads, G::S_SMEM, st>>>(tpq, ta, tal, tpk, tv, W.sq, W.sk, W.b,
-                                        static_cast<__nv_bfloat16 *>(dk),
-                                        static_cast<__nv_bfloat16 *>(dv), r_start, r_hs, r_ss,
+  k3<<<grid, kThreads, G::S_SMEM, st>>>(tpq, ta, tal, tpk, tv, W.sq, W.sk, W.b, tdk, tdv,
+                                        r_start, r_hs, r_ss,
                                         W.r_vec, n, seg, nseg, nitems, err);
   count_launches(1);
   record_launch_event(st);
