@@ -123,9 +123,13 @@ struct BCfg {
   static constexpr int S_W0 = S_ST + STATE;
   static constexpr int S_W1 = S_W0 + kAtom;
   static constexpr int S_SH = S_W1 + kAtom;
-  // aggregate: stages of K, V
+  // aggregate: stages of K, V; D = 64: the E atom and the ones atom of the extended product
+  static constexpr bool G_XT = D == 64;
   static constexpr int G_STAGE = 2 * TILE;
-  static constexpr int G_SH = 2 * G_STAGE;
+  static constexpr int G_E = 2 * G_STAGE;
+  static constexpr int G_ONES = G_E + kAtom;
+  static constexpr int G_SH = G_XT ? G_ONES + kAtom : 2 * G_STAGE;
+  static constexpr uint32_t G_TCOLS = G_XT ? 128 : D;  // the aggregate's TMEM
   static constexpr int SLACK = 1024;  // alignment of the dynamic shared memory base
   static constexpr int P_SMEM = P_SH + (int)sizeof(BwdShared) + SLACK;
   static constexpr int S_SMEM = S_SH + (int)sizeof(BwdShared) + SLACK;
@@ -139,6 +143,8 @@ struct BCfg {
                 "CTAS walk CTAs fit on an SM");
   static_assert(D == 128 || (3 * (P_SMEM + 1024) > kSmPerSm && 3 * (S_SMEM + 1024) > kSmPerSm),
                 "at most two walk CTAs per SM share its TMEM");
+  static_assert(G_CTAS * (G_SMEM + 1024) <= kSmPerSm && G_CTAS * G_TCOLS <= 512,
+                "G_CTAS aggregate CTAs fit on an SM");
   static_assert(P_ST % 1024 == 0 && P_A % 1024 == 0 && P_AL % 1024 == 0 && P_W % 1024 == 0 &&
                     P_L % 1024 == 0 && S_ST % 1024 == 0 && S_W0 % 1024 == 0 &&
                     S_W1 % 1024 == 0,
@@ -483,8 +489,14 @@ __device__ __forceinline__ uint64_t mdesc(uint32_t base, int ks, uint32_t atom) 
 
 // ---------------------------------------------------------------- K1: forward records
 // k, v: [heads][n][D] via tmK, tmV.  Writes each item's record [Psi | zeta | vs | sigma |
-// kappa] to rec + (head * nseg + seg) * rec_floats<D>(), and psi(k) (rounded to bf16, via the
-// store map tmPK) with its row sums (skg, [heads][n]) for the walks.
+// kappa] to rec + (head * nseg + seg) * rec_floats<D>(), the item's vectors before each of its
+// chunks to chunk_vec, and psi(k) (rounded to bf16, via the store map tmPK) with its row sums
+// (skg, [heads][n]) for the walks.
+// D = 64: the whole record comes from one product per K-step, A = [psi(K) | E] (M = 128, E's row
+// j = [1, hi(sk_j), lo(sk_j), 0 ...], sk_j split into two bf16) times B = [V | 1] (N = 80):
+// accumulator rows 0..63 hold [Psi | zeta], row 64 [vs | count], rows 65 and 66 the two halves
+// of [sigma | kappa].  D = 128 (M would pass 128): Psi from the product, the vectors by column
+// sums on the CUDA cores.
 template <int D>
 __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
     bwd_aggregate_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -499,6 +511,8 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
   constexpr int OK = 0, OV = G::TILE;
   constexpr uint32_t LOAD = 2 * G::TILE;
   constexpr uint32_t I_S = make_idesc_bf16(D, D, true, true);
+  constexpr bool XT = G::G_XT;
+  constexpr uint32_t I_X = make_idesc_bf16(128, D + 16, true, true);  // the extended product
   const int64_t nck = (n + C - 1) / C;  // chunks per head
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -507,9 +521,21 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
   const Lanes L = Lanes::make<D>();
   const int64_t it0 = blockIdx.x, istep = gridDim.x;
 
+  uint8_t *sE = sm + G::G_E, *sOnes = sm + G::G_ONES;
   init_barriers(sh, 1);
+  if (XT) {
+    // E starts at zero (each chunk rewrites the first 16 bytes of its rows); the ones atom's
+    // column 0 is 1 in every row (row r's column 0 sits in 16-byte chunk r & 7)
+    uint32_t *e = reinterpret_cast<uint32_t *>(sE), *o = reinterpret_cast<uint32_t *>(sOnes);
+    for (int i = threadIdx.x; i < kAtom / 4; i += kThreads) {
+      const int row = i >> 5, word = i & 31;
+      e[i] = 0u;
+      o[i] = (word == 4 * (row & 7)) ? 0x00003F80u : 0u;
+    }
+    fence_proxy_async_smem();
+  }
   if (L.warp == 0) {
-    tmem_alloc(&sh.tmem_base, D);
+    tmem_alloc(&sh.tmem_base, G::G_TCOLS);
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
@@ -550,6 +576,18 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
       if (S.wait(&sh.full[g & 1], (g >> 1) & 1)) {
         if (threadIdx.x == 0) landed = g + 1;
         psi_tile<D>(st + OK, valid, sh.sk);
+        if (XT && (threadIdx.x & 7) == 0) {
+          // E's rows for the two rows whose sums this thread made (psi_tile's mapping); rows
+          // past the item's end are zero
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = 32 * h + (threadIdx.x >> 3);
+            const float skr = sh.sk[r];
+            const uint32_t w0 = pack_bf16x2(r < valid ? 1.f : 0.f, skr);
+            *reinterpret_cast<uint4 *>(sE + sw128_offset(r, 0)) =
+                make_uint4(w0, pack_bf16x2(skr - bf16_hi(w0), 0.f), 0u, 0u);
+          }
+        }
       }
       fence_proxy_async_smem();
       if (!S.barrier()) break;
@@ -568,15 +606,28 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
         else if (it + istep < nitems)
           issue(item_at<C>(it + istep, n, seg_len, nseg), 0);
         const uint32_t k0 = smem_u32(st + OK), v0 = smem_u32(st + OV);
-        // Psi += psi(K)^T V
+        if (XT) {
+          // [Psi | zeta; vs | count; sigma | kappa] += [psi(K) | E]^T [V | 1]: the second
+          // 64-wide block of each operand (E, ones) is one atom shared by both stages, reached
+          // through the descriptor's block stride
+          const uint64_t dA = mnmajor_base(k0, smem_u32(sE) - k0);
+          const uint64_t dB = mnmajor_base(v0, smem_u32(sOnes) - v0);
 #pragma unroll
-        for (int ks = 0; ks < KSC; ++ks)
-          mma_bf16_ss(tmem, mdesc(k0, ks, kAtom), mdesc(v0, ks, kAtom), I_S, (c > 0 || ks > 0));
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tmem, desc_add(dA, mnmajor_off(ks)), desc_add(dB, mnmajor_off(ks)), I_X,
+                        (c > 0 || ks > 0));
+        } else {
+          // Psi += psi(K)^T V
+#pragma unroll
+          for (int ks = 0; ks < KSC; ++ks)
+            mma_bf16_ss(tmem, mdesc(k0, ks, kAtom), mdesc(v0, ks, kAtom), I_S, (c > 0 || ks > 0));
+        }
         mma_commit(&sh.mma);
         my_mma = true;
       }
-      // zeta, vs, sigma of the chunk's keys (rows past the item's end: psi(K) zero, V skipped)
-      column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
+      // D = 128: zeta, vs, sigma of the chunk's keys (rows past the item's end: psi(K) zero, V
+      // skipped)
+      if (!XT) column_sums3<D>(sh.acc, [&](int i, int c, float (*t)[8]) {
         float kr[8], vr[8];
         tile_row8(st + OK, i, c, kr);
         tile_row8(st + OV, i, c, vr);
@@ -588,26 +639,75 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
           t[2][e] = fmaf(w * ski, vr[e], t[2][e]);
         }
       });
-      if (L.warp == 0) {
+      if (!XT && L.warp == 0) {
         const float ks = warp_sum64([&](int i) { return sh.sk[i]; });
         if (threadIdx.x == 0) kap += ks;
       }
       S.wait_mma();
+      if (XT && S.wait.ok) {
+        // the item's vectors so far, from the accumulator: zeta (column D of rows 0..63:
+        // warps 0, 1) into sh.racc[0]; rows 64..66 (warp 2, lanes 0..2), columns 0..D, into
+        // sh.acc[0..2]
+        tc_fence_after();
+        if (L.warp < 2) {
+          sh.racc[0][32 * L.warp + L.lane] = __uint_as_float(tmem_ld1(tmem + L.lane_off + D));
+        } else if (L.warp == 2) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float f[32];
+            tmem_row32(tmem + L.lane_off + c0, f);
+            if (L.lane < 3) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) sh.acc[L.lane][c0 + e] = f[e];
+            }
+          }
+          const float last = __uint_as_float(tmem_ld1(tmem + L.lane_off + D));
+          if (L.lane < 3) sh.acc[L.lane][D] = last;
+        }
+      }
       if (!S.barrier()) break;
       // the item's vectors before its next chunk (exclusive within the item), for the walk
       if (c + 1 < I.nchunks) {
         float *cv = chunk_vec + (I.head * nck + I.t_begin / C + c + 1) * vec_floats<D>();
-        if (threadIdx.x < D) {
+        if (XT) {
+          if (threadIdx.x < D) {
+            cv[threadIdx.x] = sh.racc[0][threadIdx.x];
+            cv[D + threadIdx.x] = sh.acc[0][threadIdx.x];
+            cv[2 * D + threadIdx.x] = sh.acc[1][threadIdx.x] + sh.acc[2][threadIdx.x];
+          }
+          if (threadIdx.x == 0) cv[3 * D] = sh.acc[1][D] + sh.acc[2][D];
+        } else {
+          if (threadIdx.x < D) {
 #pragma unroll
-          for (int k = 0; k < 3; ++k) cv[k * D + threadIdx.x] = sh.acc[k][threadIdx.x];
+            for (int k = 0; k < 3; ++k) cv[k * D + threadIdx.x] = sh.acc[k][threadIdx.x];
+          }
+          if (threadIdx.x == 0) cv[3 * D] = kap;
         }
-        if (threadIdx.x == 0) cv[3 * D] = kap;
       }
     }
     if (!S.wait.ok) break;
     float *dst = rec + (I.head * nseg + I.seg) * rec_floats<D>();
-    state_to_global<D>(tmem + L.lane_off, dst, L);
-    drain_acc<D>(sh.acc, dst + (int64_t)D * D, D);
+    if (XT) {
+      // Psi: rows 0..63 are lanes 0..63 (warps 0, 1; 4, 5 take the other half of the columns);
+      // the vectors from the last chunk's read-out
+      if (L.sp < 2) {
+        float f[32];
+        tmem_row32(tmem + L.lane_off + L.hf * 32, f);
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4 *>(dst + (int64_t)(32 * L.sp + L.lane) * D + L.hf * 32 + e) =
+              make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+      }
+      if (threadIdx.x < D) {
+        dst[(int64_t)D * D + threadIdx.x] = sh.racc[0][threadIdx.x];
+        dst[(int64_t)D * D + D + threadIdx.x] = sh.acc[0][threadIdx.x];
+        dst[(int64_t)D * D + 2 * D + threadIdx.x] = sh.acc[1][threadIdx.x] + sh.acc[2][threadIdx.x];
+      }
+      if (threadIdx.x == 0) kap = sh.acc[1][D] + sh.acc[2][D];
+    } else {
+      state_to_global<D>(tmem + L.lane_off, dst, L);
+      drain_acc<D>(sh.acc, dst + (int64_t)D * D, D);
+    }
     if (threadIdx.x == 0) {
       dst[(int64_t)D * D + 3 * D] = kap;
       dst[(int64_t)D * D + 3 * D + 1] = 0.f;
@@ -617,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, BCfg<D>::G_CTAS)
     if (!S.barrier()) break;
   }
   if (threadIdx.x == 0) tma_store_wait_all<0>();  // the stores are done with shared memory
-  finish(sh, landed, issued, tmem, D, err, 1, my_mma);
+  finish(sh, landed, issued, tmem, G::G_TCOLS, err, 1, my_mma);
 }
 
 // ---------------------------------------------------------------- B1: the prefix walk
