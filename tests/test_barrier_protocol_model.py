@@ -113,8 +113,9 @@ def roles_forward(mode, NS, items, two=False):
                 yield ("a", "s_ready")
                 for c in range(nc):
                     yield ("w", "p_full", g)
-                    yield ("a", "p_ready")
-                    yield ("a", "rs_ready")
+                    if not two:  # with two issuers the output group takes all the scores
+                        yield ("a", "p_ready")
+                        yield ("a", "rs_ready")
                     if c + 1 < nc:
                         yield ("w", "s_full", g)
                         yield ("a", "z_ready")
@@ -138,7 +139,8 @@ def roles_forward(mode, NS, items, two=False):
             for nc in items:
                 for _ in range(nc):
                     yield ("w", "p_full", g)
-                    yield ("w", "rs_ready", g)
+                    if not two:
+                        yield ("w", "rs_ready", g)
                     yield ("a", "p_ready")
                     if g >= 1:
                         yield ("w", f"o_full[{(g - 1) & 1}]", (g - 1) >> 1)
@@ -243,7 +245,7 @@ def roles(mode, NS, items):
 
 def run(mode, NS, items, rng):
     # arrivals per phase; tc_forward.cu's causal mode: both drain groups release p_ready
-    counts = {"p_ready": 2} if mode in (1, 4) else {}
+    counts = {"p_ready": 2} if mode == 1 else {}
     bars = {}
 
     def bar(name):
