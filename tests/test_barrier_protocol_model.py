@@ -8,8 +8,11 @@ kernel on features of their own dimension, tc_causal.cu (mode 3), and
 any list of work items of 1..16 chunks walked by one CTA.  A random scheduler interleaves the roles. The
 test fails on a deadlock (no role can move) or on parity aliasing (a wait for a phase two or more
 phases behind its barrier, which the hardware's parity test cannot tell from a pending one).
-Each role's arrivals count as one (the kernel's thread counts are per role).  This model mirrors
-the kernel's code by hand: change both together.
+Each role's arrivals count as one (the kernel's thread counts are per role).  TMA loads and
+tcgen05.commit arrivals ('i' events) are asynchronous: they land later, in any order, each as a
+step of its own.  A wait may target only its barrier's pending phase or the one just completed
+(the hardware tests a phase's parity): waiting further behind, or ahead, fails the test.  This
+model mirrors the kernel's code by hand: change both together.
 """
 import random
 import sys
@@ -32,18 +35,19 @@ def roles_forward(mode, NS, items, two=False):
                 s = g % NS
                 if g >= NS:
                     yield ("w", f"empty[{s}]", g // NS - 1)
-                yield ("a", f"full[{s}]")
+                yield ("i", f"full[{s}]")
                 g += 1
         for gg in range(max(0, g - NS), g):  # drain: every load has landed
             yield ("w", f"full[{gg % NS}]", gg // NS)
 
-    def feature_map():
+    def feature_map(team=0, teams=1):  # teams take alternate chunks
         g = 0
         for nc in items:
             for _ in range(nc):
                 s = g % NS
-                yield ("w", f"full[{s}]", g // NS)
-                yield ("a", f"ready[{s}]")
+                if g % teams == team:
+                    yield ("w", f"full[{s}]", g // NS)
+                    yield ("a", f"ready[{s}]")
                 g += 1
 
     def mma():
@@ -58,36 +62,36 @@ def roles_forward(mode, NS, items, two=False):
                 s = g % NS
                 yield ("w", f"ready[{s}]", g // NS)
                 if mode == 0:
-                    yield ("a", f"empty[{s}]")
+                    yield ("i", f"empty[{s}]")
                 elif mode == 1:
                     yield ("w", "z_ready", g)
                     if g >= 1:  # the previous chunk's P V, interleaved with this chunk's scores
                         yield ("w", "p_ready", g - 1)
-                        yield ("a", f"o_full[{(g - 1) & 1}]")
-                        yield ("a", f"empty[{(g - 1) % NS}]")
-                    yield ("a", "p_full")
+                        yield ("i", f"o_full[{(g - 1) & 1}]")
+                        yield ("i", f"empty[{(g - 1) % NS}]")
+                    yield ("i", "p_full")
                     if not two:  # else phi(Q) S_<c and the S update go to the second issuer
                         yield ("w", "s_ready", g)
                         if g >= 2:
                             yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
-                        yield ("a", "s_full")
+                        yield ("i", "s_full")
                 else:
                     if g >= 2:
                         yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
-                    yield ("a", f"o_full[{g & 1}]")
-                    yield ("a", f"empty[{s}]")
+                    yield ("i", f"o_full[{g & 1}]")
+                    yield ("i", f"empty[{s}]")
                 g += 1
             if mode == 0:
-                yield ("a", f"item_full[{b}]")
+                yield ("i", f"item_full[{b}]")
             if mode == 2:
-                yield ("a", f"item_empty[{b}]")
+                yield ("i", f"item_empty[{b}]")
         if mode == 1 and g > 0:  # the last chunk's P V (after a second issuer's products)
             if two:
                 yield ("w", "s_full", g - 1)
             yield ("w", "p_ready", g - 1)
-            yield ("a", f"o_full[{(g - 1) & 1}]")
-            yield ("a", f"empty[{(g - 1) % NS}]")
-        yield ("a", "fin")
+            yield ("i", f"o_full[{(g - 1) & 1}]")
+            yield ("i", f"empty[{(g - 1) % NS}]")
+        yield ("i", "fin")
         yield ("w", "fin", 0)
 
     def mma2():  # causal: the second issuer, phi(Q) S_<c and the S update
@@ -98,9 +102,9 @@ def roles_forward(mode, NS, items, two=False):
                 yield ("w", "s_ready", g)
                 if g >= 2:
                     yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
-                yield ("a", "s_full")
+                yield ("i", "s_full")
                 g += 1
-        yield ("a", "fin2")
+        yield ("i", "fin2")
         yield ("w", "fin2", 0)
 
     def state_group():
@@ -156,7 +160,11 @@ def roles_forward(mode, NS, items, two=False):
                     yield ("a", f"o_empty[{g & 1}]")
                     g += 1
 
-    roles = [tma(), feature_map(), mma(), state_group(), output_group()]
+    # the aggregate kernel splits its feature map into two teams when the stages divide evenly
+    teams = 2 if mode == 0 and NS % 2 == 0 else 1
+    roles = [tma(), feature_map(0, teams), mma(), state_group(), output_group()]
+    if teams == 2:
+        roles.append(feature_map(1, 2))
     return roles + [mma2()] if two else roles
 
 
@@ -171,7 +179,7 @@ def roles_features(NS, items):
                 s = g % NS
                 if g >= NS:
                     yield ("w", f"empty[{s}]", g // NS - 1)
-                yield ("a", f"full[{s}]")
+                yield ("i", f"full[{s}]")
                 g += 1
         for gg in range(max(0, g - NS), g):
             yield ("w", f"full[{gg % NS}]", gg // NS)
@@ -196,13 +204,13 @@ def roles_features(NS, items):
                 yield ("w", "s_ready", g)
                 if g >= 2:
                     yield ("w", f"o_empty[{g & 1}]", (g >> 1) - 1)
-                yield ("a", "p_full")  # the scores
-                yield ("a", "s_full")  # F(Q) S_<c and the state update
+                yield ("i", "p_full")  # the scores
+                yield ("i", "s_full")  # F(Q) S_<c and the state update
                 yield ("w", "p_ready", g)
-                yield ("a", f"o_full[{g & 1}]")  # P V
-                yield ("a", f"empty[{s}]")
+                yield ("i", f"o_full[{g & 1}]")  # P V
+                yield ("i", f"empty[{s}]")
                 g += 1
-        yield ("a", "fin")
+        yield ("i", "fin")
         yield ("w", "fin", 0)
 
     def state_group():
@@ -255,27 +263,40 @@ def run(mode, NS, items, rng):
 
     gens = roles(mode, NS, items)
     cur = [next(gen, None) for gen in gens]
+    inflight = []  # asynchronous arrivals issued and not yet landed
+
+    def arrive(name):
+        b = bar(name)
+        b.pending += 1
+        if b.pending == b.count:
+            b.pending, b.completed = 0, b.completed + 1
+
     while True:
         runnable = []
         for r, ev in enumerate(cur):
             if ev is None:
                 continue
-            if ev[0] == "a":
+            if ev[0] in ("a", "i"):
                 runnable.append(r)
                 continue
             b, phase = bar(ev[1]), ev[2]
             assert b.completed < phase + 2, f"parity aliasing: {ev}, mode {mode}, items {items}"
+            # the hardware tests a phase's parity, so a wait may only target the pending phase
+            # or the one just completed: a wait two phases ahead would pass at once
+            assert phase <= b.completed, f"wait ahead of its barrier: {ev}, mode {mode}, items {items}"
             if b.completed > phase:  # the waited-for phase has completed
                 runnable.append(r)
-        if not runnable:
+        if not runnable and not inflight:
             assert all(ev is None for ev in cur), f"deadlock at {cur}, mode {mode}, items {items}"
             return True
+        if inflight and (not runnable or rng.random() < 0.3):
+            arrive(inflight.pop(rng.randrange(len(inflight))))  # one landing, in any order
+            continue
         r = rng.choice(runnable)
         if cur[r][0] == "a":
-            b = bar(cur[r][1])
-            b.pending += 1
-            if b.pending == b.count:
-                b.pending, b.completed = 0, b.completed + 1
+            arrive(cur[r][1])
+        elif cur[r][0] == "i":
+            inflight.append(cur[r][1])
         cur[r] = next(gens[r], None)
 
 
