@@ -299,6 +299,43 @@ __global__ void __launch_bounds__(Warps<MODE, DK>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
 
+  // O of chunk gg (chunk c of item I) over its denominator -> bf16 rows of out, by the four
+  // output warps (one per TMEM sub-partition; lanes < 16 hold the rows of the M = 64 product).
+  // den: the causal denominator; the non-causal one is column DV of the accumulator.
+  auto emit_O = [&](auto &wait, int gg, const Item &I, int c, float den) {
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const bool v64 = lane < 16;
+    const int r64 = 16 * (warp & 3) + lane;
+    const int ob = gg & 1;
+    const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
+    if (!wait(&bar.o_full[ob], (gg >> 1) & 1)) return;
+    tc_fence_after();
+    const float dd = MODE == kCausalOut ? den : __uint_as_float(tmem_ld1(tO + DV));
+    const float inv = 1.f / dd;
+    const int64_t t = I.t_begin + (int64_t)c * C + r64;
+    const bool live = v64 && t < I.t_end;
+    __nv_bfloat16 *orow = out + (I.head * n + (live ? t : 0)) * DV;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DV; c0 += 64) {
+      uint32_t r[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld16_async(tO + c0 + 16 * q, r + 16 * q);
+      tmem_ld_wait();
+      tmem_reg_fence<64>(r);
+      if (live) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float f[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
+          st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8), a32);
+        }
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(&bar.o_empty[ob]);
+  };
+
   if (warp == kWarpTMA) {
     // ================================================================ TMA producer
     if (lane == 0) {
@@ -787,38 +824,6 @@ __global__ void __launch_bounds__(Warps<MODE, DK>::THREADS, 1)
       mbar_arrive(&bar.p_ready);
     };
 
-    // O of chunk gg (chunk c of item I)
-    auto emit_O = [&](int gg, const Item &I, int c) {
-      const int ob = gg & 1;
-      const uint32_t tO = tmem + lane_off + (ob ? TM::O1 : TM::O0);
-      if (!wait(&bar.o_full[ob], (gg >> 1) & 1)) return;
-      tc_fence_after();
-      const float dd =
-          MODE == kCausalOut ? (ob ? den1 : den0) : __uint_as_float(tmem_ld1(tO + DV));
-      const float inv = 1.f / dd;
-      const int64_t t = I.t_begin + (int64_t)c * C + r64;
-      const bool live = v64 && t < I.t_end;
-      __nv_bfloat16 *orow = out + (I.head * n + (live ? t : 0)) * DV;
-#pragma unroll 1
-      for (int c0 = 0; c0 < DV; c0 += 64) {
-        uint32_t r[64];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16_async(tO + c0 + 16 * q, r + 16 * q);
-        tmem_ld_wait();
-        tmem_reg_fence<64>(r);
-        if (live) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float f[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[16 * q + e]) * inv;
-            st_global_32B(orow + c0 + 16 * q, pack8(f), pack8(f + 8), a32);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar.o_empty[ob]);
-    };
 
     if (MODE == kCausalOut) {
       int g = 0;
@@ -828,17 +833,17 @@ __global__ void __launch_bounds__(Warps<MODE, DK>::THREADS, 1)
         const Item I = item_at<C>(it, n, seg_len, nseg);
         for (int c = 0; c < I.nchunks; ++c, ++g) {
           convert_P(g);
-          if (g >= 1) emit_O(g - 1, prev, prev_c);
+          if (g >= 1) emit_O(wait, g - 1, prev, prev_c, ((g - 1) & 1) ? den1 : den0);
           prev = I;
           prev_c = c;
         }
       }
-      if (g > 0) emit_O(g - 1, prev, prev_c);
+      if (g > 0) emit_O(wait, g - 1, prev, prev_c, ((g - 1) & 1) ? den1 : den0);
     } else if (MODE == kNoncausalOut) {
       int g = 0;
       for (int64_t it = it0; it < nitems; it += istep) {
         const Item I = item_at<C>(it, n, seg_len, nseg);
-        for (int c = 0; c < I.nchunks; ++c, ++g) emit_O(g, I, c);
+        for (int c = 0; c < I.nchunks; ++c, ++g) emit_O(wait, g, I, c, 0.f);
       }
     }
   }
