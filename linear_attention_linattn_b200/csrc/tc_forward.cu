@@ -67,8 +67,10 @@ constexpr int kGroupThreads = 128;
 // each SM sub-partition holds 4 warps and a thread may use 128 registers (the score, state and
 // output drains keep 64-column batches in registers).  At d = 64 two warps issue the MMAs (one
 // thread issues a tcgen05.mma about every 55 cycles, slower than the tensor pipe runs these
-// small products; issuers in different warps proceed in parallel), with 5 feature-map warps;
-// at d = 128 the feature map is the tighter bound, so one issuer and 6 feature-map warps.
+// small products; issuers in different warps proceed in parallel), with 4 feature-map warps,
+// one per SM sub-partition (0.167 ms with 5, 0.156 with 4, 0.194 with 3 on the batched
+// workload); at d = 128 the feature map is the tighter bound, so one issuer and 6 feature-map
+// warps (1.00 ms; 1.05 with 4).
 // Aggregate: the feature map on K bounds the chunk rate, so 12 feature-map warps (22 warps,
 // 80 registers), in two teams of 6 taking alternate stages where the stage count is even (at
 // d = 64: 0.069 -> 0.060 ms on the batched workload).  Non-causal: 8 feature-map warps (18
@@ -79,7 +81,7 @@ struct Warps {
   static constexpr int MMA2 = 2;                      // the second issuer
   static constexpr int XFORM0 = TWO_ISSUERS ? 3 : 2;  // first feature-map warp
   static constexpr int XFORM =
-      MODE == kCausalOut ? (TWO_ISSUERS ? 5 : 6) : (MODE == kState ? 12 : 8);
+      MODE == kCausalOut ? (TWO_ISSUERS ? 4 : 6) : (MODE == kState ? 12 : 8);
   static constexpr int XTHREADS = XFORM * 32;
   // feature-map teams wanted: the warps split into groups that take alternate chunks, so
   // several chunks are in flight instead of all warps waiting on one (the kernel keeps one
