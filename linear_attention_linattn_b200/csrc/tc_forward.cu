@@ -28,11 +28,13 @@
 // DK is the feature dimension of phi(q), phi(k), DV the value dimension; the causal mode here
 // keeps DK = DV = D.
 //
-// Warp roles (one CTA per SM; 16, 22 or 18 warps in the causal, aggregate, non-causal modes):
+// Warp roles (one CTA per SM; 16 or 15 warps in the causal mode at d = 128 or 64, 22 in the
+// aggregate mode, 18 in the non-causal mode):
 //   warp 0     TMA producer: 3-D tiled loads (128-byte swizzle) of Q/K/V chunks into a
 //              ring of stages; no multicast.
-//   warp 1     TMEM allocation and the single MMA-issuing thread.
-//   next 6-12  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
+//   warp 1     TMEM allocation and the MMA-issuing thread (warp 2 holds a second one in the
+//              causal mode at d = 64).
+//   next 4-12  feature map: phi applied in place to the Q and K tiles (bf16), K rows beyond
 //              the item's end zeroed, then handed to the tensor cores.
 //   next 4     state: round S_<c+1 and z into the next chunk's operands; the starting
 //              state; the segment aggregate.
@@ -63,9 +65,9 @@ enum Mode : int { kState = 0, kCausalOut = 1, kNoncausalOut = 2 };
 constexpr int kWarpTMA = 0;
 constexpr int kWarpMMA = 1;
 constexpr int kGroupThreads = 128;
-// Warps per mode and feature width (measured on the benchmark shapes).  Causal: 16 warps, so
-// each SM sub-partition holds 4 warps and a thread may use 128 registers (the score, state and
-// output drains keep 64-column batches in registers).  At d = 64 two warps issue the MMAs (one
+// Warps per mode and feature width (measured on the benchmark shapes).  Causal: 16 or 15
+// warps, so each SM sub-partition holds about 4 and a thread may use 128 registers (the score,
+// state and output drains keep 64-column batches in registers).  At d = 64 two warps issue the MMAs (one
 // thread issues a tcgen05.mma about every 55 cycles, slower than the tensor pipe runs these
 // small products; issuers in different warps proceed in parallel), with 4 feature-map warps,
 // one per SM sub-partition (0.167 ms with 5, 0.156 with 4, 0.194 with 3 on the batched
