@@ -432,12 +432,14 @@ def main_forward(args, world, rank, local):
     outh = torch.empty_like(qh).pin_memory()
 
     def e2e_step():
-        a, b_, c = (x.to("cuda", non_blocking=True) for x in (qh, kh, vh))
         if seq:
+            a, b_, c = (x.to("cuda", non_blocking=True) for x in (qh, kh, vh))
             o = seqshard.forward_sequence_sharded(a, b_, c, causal)
+            outh.copy_(o, non_blocking=True)
         else:
-            o = la.forward(a, b_, c, causal)
-        outh.copy_(o, non_blocking=True)
+            # the C entry point on host buffers: head groups copied in, run and copied out
+            # on the library's streams, the copies of one group overlapping the others' work
+            la.forward_host(qh, kh, vh, causal, out=outh)
 
     e2e = None
     if not args.no_e2e and not backward:
@@ -445,7 +447,10 @@ def main_forward(args, world, rank, local):
         e2e_ms, _ = time_steps(e2e_step, e2e_steps, 1, world)
         e2e = {"value": tokens_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": 3 * qh.numel() * elem,
-               "d2h_bytes_per_step": outh.numel() * elem}
+               "d2h_bytes_per_step": outh.numel() * elem,
+               "path": ("to device, sequence-sharded forward, to host" if seq else
+                        "linattn_forward_host: head groups copied in, run and copied out on "
+                        "three streams")}
         # the host link's own rate on one input tensor, for context
         t0, t1, t2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         t0.record()

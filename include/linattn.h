@@ -237,6 +237,23 @@ linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, v
                                   linattn_dtype dtype, int64_t segment_len,
                                   linattn_stream_t stream);
 
+/*
+ * linattn_forward with q, k, v and out in HOST memory: the same result as copying q, k, v to
+ * the device, calling linattn_forward and copying out back.  The heads run in groups (about
+ * eight, each at most 1 GiB of the four tensors) on three internal streams, so the copies of
+ * one group overlap the copies and kernels of the others.  Page-locked (pinned) buffers let
+ * the copies run asynchronously and concurrently; pageable ones are accepted and copied by the
+ * runtime's staging.  The groups start after the work already enqueued on `stream`, and
+ * `stream` waits for all of them: once it is synchronised, `out` holds the result and the
+ * inputs may be reused.  Device memory: the pool holds three groups' buffers (and their
+ * workspaces) while the call runs.  Returns after enqueuing; LINATTN_ERR_INVALID_ARG for a
+ * null pointer or a bad shape (as linattn_forward; no alignment is required of host
+ * buffers), LINATTN_ERR_CUDA if a copy, an allocation or a launch fails.
+ */
+linattn_status linattn_forward_host(const void *q, const void *k, const void *v, void *out,
+                                    int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                    linattn_dtype dtype, linattn_stream_t stream);
+
 /* Bytes of one head's state, D*d*4 + D*4 (fp32 S and z), independent of n
  * (page "Linear Attention > Memory Efficiency": 16,640 bytes at d = D = 64). */
 size_t linattn_state_bytes(int64_t d);

@@ -42,6 +42,8 @@ SIGNATURES = {
                                        ctypes.c_int, _vp]),
     "linattn_forward_ex": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                           ctypes.c_int, ctypes.c_int, _i64, _vp]),
+    "linattn_forward_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                            ctypes.c_int, ctypes.c_int, _vp]),
     "linattn_forward_state": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                              ctypes.c_int, _vp]),
     "linattn_decode_step": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
@@ -154,6 +156,32 @@ def forward(q, k, v, causal: bool, out=None, segment_len: int = 0, stream=None):
                                 B, H, n, d, int(bool(causal)), _dtype_code(q), int(segment_len),
                                 _stream_ptr(stream))
     _check(st, "linattn_forward")
+    return out
+
+
+def forward_host(q, k, v, causal: bool, out=None, stream=None):
+    """forward on host tensors: q, k, v [B, H, n, d] contiguous CPU tensors (float32 or
+    bfloat16; pinned ones let the library overlap the copies with the work).  The library
+    copies head groups in, runs them and copies the outputs back on its own streams; this
+    waits for `stream` (default: the current CUDA stream) before returning out, a CPU tensor
+    (pinned when q is)."""
+    import torch
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous CPU tensor")
+    if not (q.shape == k.shape == v.shape and q.dim() == 4 and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share one [B, H, n, d] shape and dtype")
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    if out.is_cuda or not out.is_contiguous() or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must be a contiguous CPU tensor of q's shape and dtype")
+    B, H, n, d = q.shape
+    s = stream if stream is not None else torch.cuda.current_stream()
+    st = load_library().linattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                             out.data_ptr(), B, H, n, d, int(bool(causal)),
+                                             _dtype_code(q), int(s.cuda_stream))
+    _check(st, "linattn_forward_host")
+    s.synchronize()
     return out
 
 

@@ -21,6 +21,10 @@ struct DeviceState {
   cudaError_t init_err = cudaSuccess;
   int *err_word = nullptr;     // kernels' error word (device memory)
   cudaMemPool_t pool = nullptr;  // stream-ordered workspace pool
+  // linattn_forward_host: the streams its head groups run on (created on its first call)
+  std::once_flag streams_once;
+  cudaError_t streams_err = cudaSuccess;
+  cudaStream_t group_streams[3] = {nullptr, nullptr, nullptr};
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -108,12 +112,9 @@ __global__ void wait_timeout_selftest_kernel(int *err) {
 
 }  // namespace
 
-linattn_status check_forward_args(const void *q, const void *k, const void *v, const void *out,
-                                  int64_t B, int64_t H, int64_t n, int64_t d, int causal,
-                                  linattn_dtype dtype) {
-  if (!q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return LINATTN_ERR_INVALID_ARG;
+// The forward's shape, mode and type checks (the pointers are checked by the callers).
+linattn_status check_forward_shape(int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                   linattn_dtype dtype) {
   if (causal != 0 && causal != 1) return LINATTN_ERR_INVALID_ARG;
   if (dtype != LINATTN_F32 && dtype != LINATTN_BF16) return LINATTN_ERR_INVALID_ARG;
   // n < 2^31, B*H < 2^24, total elements < 2^40
@@ -126,6 +127,15 @@ linattn_status check_forward_args(const void *q, const void *k, const void *v, c
   const int64_t nchunks = (n + kSimtChunk - 1) / kSimtChunk;
   if (nchunks * heads >= (int64_t(1) << 31)) return LINATTN_ERR_INVALID_ARG;
   return LINATTN_OK;
+}
+
+linattn_status check_forward_args(const void *q, const void *k, const void *v, const void *out,
+                                  int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                  linattn_dtype dtype) {
+  if (!q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return LINATTN_ERR_INVALID_ARG;
+  return check_forward_shape(B, H, n, d, causal, dtype);
 }
 
 ForwardPlan plan_forward(int64_t heads, int64_t n, int dk, int d, int causal, int is_bf16,
@@ -217,6 +227,86 @@ linattn_status linattn_forward_ex(const void *q, const void *k, const void *v, v
   return forward_pooled(q, k, v, out, B * H, n, (int)d, (int)d, causal, dtype == LINATTN_BF16,
                         segment_len, nullptr, nullptr, 0, ds,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+linattn_status linattn_forward_host(const void *q, const void *k, const void *v, void *out,
+                                    int64_t B, int64_t H, int64_t n, int64_t d, int causal,
+                                    linattn_dtype dtype, linattn_stream_t stream) {
+  if (!q || !k || !v || !out) return LINATTN_ERR_INVALID_ARG;  // host buffers: any alignment
+  linattn_status s = check_forward_shape(B, H, n, d, causal, dtype);
+  if (s != LINATTN_OK) return s;
+  DeviceState *ds = nullptr;
+  if (device_state(&ds) != cudaSuccess) return LINATTN_ERR_CUDA;
+  std::call_once(ds->streams_once, [&]() {
+    for (cudaStream_t &gs : ds->group_streams) {
+      ds->streams_err = cudaStreamCreateWithFlags(&gs, cudaStreamNonBlocking);
+      if (ds->streams_err != cudaSuccess) break;
+    }
+  });
+  if (ds->streams_err != cudaSuccess) return LINATTN_ERR_CUDA;
+  const cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
+  constexpr int kSlots = 3;  // head groups in flight, one per stream
+  const int64_t heads = B * H;
+  const size_t head_bytes = static_cast<size_t>(n) * d * (dtype == LINATTN_BF16 ? 2 : 4);
+  // about eight groups, so that all but one group's copies overlap others' work, each at most
+  // 1 GiB of the four tensors
+  int64_t g = (heads + 7) / 8;
+  const int64_t g_cap = static_cast<int64_t>((size_t(1) << 30) / (4 * head_bytes));
+  if (g > g_cap) g = g_cap > 0 ? g_cap : 1;
+  const int64_t ngroups = (heads + g - 1) / g;
+  const size_t group_bytes = static_cast<size_t>(g) * head_bytes;
+  const auto *hq = static_cast<const unsigned char *>(q);
+  const auto *hk = static_cast<const unsigned char *>(k);
+  const auto *hv = static_cast<const unsigned char *>(v);
+  auto *ho = static_cast<unsigned char *>(out);
+
+  // the group streams start after the work enqueued on the caller's stream so far
+  cudaEvent_t start = nullptr, done[kSlots] = {nullptr, nullptr, nullptr};
+  cudaError_t e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventRecord(start, user);
+  for (int i = 0; i < kSlots && e == cudaSuccess; ++i)
+    e = cudaStreamWaitEvent(ds->group_streams[i], start, 0);
+  // per stream: device buffers for one group's q, k, v, out
+  unsigned char *buf[kSlots] = {nullptr, nullptr, nullptr};
+  const int used = static_cast<int>(ngroups < kSlots ? ngroups : kSlots);
+  for (int i = 0; i < used && e == cudaSuccess; ++i)
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf[i]), 4 * group_bytes, ds->pool,
+                                ds->group_streams[i]);
+  // group j on stream j % kSlots: copy in, forward, copy out (the stream orders the reuse of
+  // its buffers; the copies of one group overlap the work of the others)
+  linattn_status st = e == cudaSuccess ? LINATTN_OK : LINATTN_ERR_CUDA;
+  for (int64_t j = 0; j < ngroups && st == LINATTN_OK; ++j) {
+    const int i = static_cast<int>(j % kSlots);
+    const cudaStream_t gs = ds->group_streams[i];
+    const int64_t h0 = j * g, gh = heads - h0 < g ? heads - h0 : g;
+    const size_t off = static_cast<size_t>(h0) * head_bytes, bytes = gh * head_bytes;
+    unsigned char *dq = buf[i], *dk = dq + group_bytes, *dv = dk + group_bytes,
+                  *dout = dv + group_bytes;
+    if (cudaMemcpyAsync(dq, hq + off, bytes, cudaMemcpyHostToDevice, gs) != cudaSuccess ||
+        cudaMemcpyAsync(dk, hk + off, bytes, cudaMemcpyHostToDevice, gs) != cudaSuccess ||
+        cudaMemcpyAsync(dv, hv + off, bytes, cudaMemcpyHostToDevice, gs) != cudaSuccess) {
+      st = LINATTN_ERR_CUDA;
+      break;
+    }
+    st = forward_pooled(dq, dk, dv, dout, gh, n, (int)d, (int)d, causal, dtype == LINATTN_BF16,
+                        0, nullptr, nullptr, 0, ds, gs);
+    if (st == LINATTN_OK &&
+        cudaMemcpyAsync(ho + off, dout, bytes, cudaMemcpyDeviceToHost, gs) != cudaSuccess)
+      st = LINATTN_ERR_CUDA;
+  }
+  // release the buffers in stream order; the caller's stream waits for every group
+  for (int i = 0; i < kSlots; ++i) {
+    if (buf[i] && cudaFreeAsync(buf[i], ds->group_streams[i]) != cudaSuccess)
+      st = LINATTN_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&done[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventRecord(done[i], ds->group_streams[i]) != cudaSuccess ||
+        cudaStreamWaitEvent(user, done[i], 0) != cudaSuccess)
+      st = LINATTN_ERR_CUDA;
+  }
+  for (cudaEvent_t ev : done)
+    if (ev) cudaEventDestroy(ev);
+  if (start) cudaEventDestroy(start);
+  return st;
 }
 
 linattn_status linattn_forward_init(const void *q, const void *k, const void *v, void *out,

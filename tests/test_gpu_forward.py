@@ -232,3 +232,33 @@ def test_fewer_items_than_sms(causal):
     q, k, v = (inputs.round_bf16(x) for x in inputs.forward_qkv(23, B, H, n, d, scaled=True))
     got = _run(q, k, v, causal, "bf16", segment_len=384)
     assert max_row_rel_err(got, oracle.forward(q, k, v, causal)) <= TOL["bf16"]
+
+
+# Host buffers in, host buffers out: the library copies head groups in, runs them and copies
+# them back on its own streams.  24 heads make 8 groups of 3 on 3 streams (each stream's
+# buffers reused), 5 heads make 5 groups of 1.
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H,n,d,pinned", [(2, 12, 777, 128, True), (1, 5, 1000, 64, False)])
+def test_forward_host_buffers(dtype, causal, B, H, n, d, pinned):
+    q, k, v = inputs.forward_qkv(31 + n, B, H, n, d, scaled=True)
+    q, k, v = as_io(q, dtype), as_io(k, dtype), as_io(v, dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    qh, kh, vh = (torch.from_numpy(x.astype(np.float32)).to(tdt).contiguous() for x in (q, k, v))
+    if pinned:
+        qh, kh, vh = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
+    out = la.forward_host(qh, kh, vh, causal)
+    assert la.device_error() == la.LINATTN_OK
+    assert not out.is_cuda and out.is_pinned() == pinned
+    got = out.float().numpy()
+    ref = oracle.forward(q, k, v, causal)
+    assert max_row_rel_err(got, ref) <= TOL[dtype]
+    # the same result as the device entry point (up to the segment lengths its head count picks)
+    dev = _run(q, k, v, causal, dtype)
+    assert max_row_rel_err(got, dev) <= TOL[dtype]
+
+
+def test_forward_host_rejects_device_tensors():
+    q = torch.zeros((1, 1, 64, 64), device="cuda")
+    with pytest.raises(ValueError):
+        la.forward_host(q, q, q, True)
