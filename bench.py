@@ -17,6 +17,10 @@ value = all ranks' tokens / the max over ranks of the device time ("scaling": "w
 block's state, the ranks all-gather the block states once, and each continues its block
 from the states before it ("scaling": "strong"; linear_attention_linattn_b200.seqshard).
 
+"e2e" is the same step through the C entry point on pinned host buffers
+(linattn_forward_host): every step copies q, k, v in and the output back, in head groups whose
+copies overlap one another's work; the host link bounds it.
+
 At N=1 the line also carries the decode step (256 x 32 states, d = 128, 512 steps), the
 batched 8x16x8192x64 forward (both modes) and the small latency cases under "extras", and
 the oracle's throughput on a bounded sample under "cpu_baseline".
