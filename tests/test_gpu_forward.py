@@ -239,7 +239,8 @@ def test_fewer_items_than_sms(causal):
 # buffers reused), 5 heads make 5 groups of 1.
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("B,H,n,d,pinned", [(2, 12, 777, 128, True), (1, 5, 1000, 64, False)])
+@pytest.mark.parametrize("B,H,n,d,pinned", [(2, 12, 777, 128, True), (1, 5, 1000, 64, False),
+                                             (1, 1, 5, 64, True)])
 def test_forward_host_buffers(dtype, causal, B, H, n, d, pinned):
     q, k, v = inputs.forward_qkv(31 + n, B, H, n, d, scaled=True)
     q, k, v = as_io(q, dtype), as_io(k, dtype), as_io(v, dtype)
@@ -262,3 +263,28 @@ def test_forward_host_rejects_device_tensors():
     q = torch.zeros((1, 1, 64, 64), device="cuda")
     with pytest.raises(ValueError):
         la.forward_host(q, q, q, True)
+
+
+def test_forward_host_calls_on_two_streams():
+    """Two calls enqueued back to back on different streams share the library's group streams;
+    each result is its own."""
+    outs, refs = [], []
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for seed, st in ((41, s1), (42, s2)):
+        q, k, v = inputs.forward_qkv(seed, 1, 6, 700, 64, scaled=True)
+        q, k, v = as_io(q, "bf16"), as_io(k, "bf16"), as_io(v, "bf16")
+        qh, kh, vh = (torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).pin_memory()
+                      for x in (q, k, v))
+        out = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+        st_ = la.load_library().linattn_forward_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(),
+                                                     out.data_ptr(), 1, 6, 700, 64, 1,
+                                                     la.LINATTN_BF16, st.cuda_stream)
+        assert st_ == la.LINATTN_OK
+        outs.append((out, qh, kh, vh))
+        refs.append(oracle.forward(q, k, v, True))
+    s1.synchronize()
+    s2.synchronize()
+    assert la.device_error() == la.LINATTN_OK
+    for (out, *_), ref in zip(outs, refs):
+        assert max_row_rel_err(out.float().numpy(), ref) <= TOL["bf16"]
+
