@@ -117,6 +117,18 @@ def test_backward_init_and_sum_argument_checks(lib):
         la.LINATTN_ERR_UNSUPPORTED
 
 
+def test_forward_host_argument_checks(lib):
+    """Host buffers need no alignment; null pointers and bad shapes are rejected before any
+    device call."""
+    bad = la.LINATTN_ERR_INVALID_ARG
+    assert lib.linattn_forward_host(0, FAKE, FAKE, FAKE, 1, 1, 8, 64, 1, 1, None) == bad
+    assert lib.linattn_forward_host(FAKE, FAKE, FAKE, 0, 1, 1, 8, 64, 1, 1, None) == bad
+    assert lib.linattn_forward_host(FAKE + 2, FAKE, FAKE, FAKE, 1, 0, 8, 64, 1, 1, None) == bad
+    assert lib.linattn_forward_host(FAKE + 2, FAKE, FAKE, FAKE, 1, 1, 8, 64, 3, 1, None) == bad
+    assert lib.linattn_forward_host(FAKE + 2, FAKE, FAKE, FAKE, 1, 1, 8, 96, 1, 1, None) == \
+        la.LINATTN_ERR_UNSUPPORTED
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError):
         la.load_library(str(tmp_path / "nope.so"))
